@@ -1,0 +1,447 @@
+#!/usr/bin/env python
+"""Throughput of the routed MoE layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    torchrun --nproc-per-node N bench.py --gpus N ...   (one process per GPU)
+
+A step is one pass of the whole layer (router + top-k, dispatch permutation,
+expert input gather, gate/up + SwiGLU, down projection, combine) over one
+batch of the workload's tokens, run through the library's C ABI. Inputs are
+resident in HBM when the timed region starts. Multi-GPU runs are replicas
+(weak scaling): every rank holds all experts and runs its own batch; there is
+no data-path collective, only a barrier and a max over ranks of the timing.
+
+Prints one JSON line on rank 0 (fields documented in the repository design
+notes). ``--impl reference`` times the float64 CPU oracle instead, on a bounded
+sample of the same workload per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s on 1 B200; % of HBM roofline (decode) / tensor peak (prefill)"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = "k2_decode_bf16"
+L2_FLUSH_BYTES = 256 << 20  # > 2x the 126 MB L2
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNELS_PER_STEP = 9  # router gemm, top-k, 3 permute, gather, gate/up, down, combine
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--tokens", type=int, default=None, help="override T (profiling runs)")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="override the routed expert count (small profiling runs)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--cpu-sample-tokens", type=int, default=24)
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, dev_index: int, enabled: bool = True):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", "clocks_rank%d.csv" % dev_index)
+        if not enabled:
+            return
+        import torch
+        p = torch.cuda.get_device_properties(dev_index)
+        bus = "%08X:%02X:%02X.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        try:
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", bus, "--query-gpu=" + self.FIELDS, "--format=csv,noheader",
+                 "-lms", "100"], stdout=self.out, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1].split()[0]), float(parts[2].split()[0]),
+                                 parts[4], parts[5:9]))
+                except ValueError:
+                    continue
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3]) if v == "Active"})
+        load = [r[0] for r in rows if r[0] > 600] or [r[0] for r in rows]
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ accounting
+def expert_bytes(cfg):
+    """Bytes of one routed (and one shared) expert's stored weights."""
+    from expert_routing_grouped_layer_b200 import workloads as W
+    return (W.weight_bytes_per_matrix(cfg, cfg.moe_intermediate_size),
+            W.weight_bytes_per_matrix(cfg, cfg.shared_intermediate_size))
+
+
+def gate_up_bytes(cfg, active, T):
+    """Algorithmic bytes of one gate/up launch: the W1/W3 weights of every active
+    expert and of the shared experts (each read once), the expert input rows
+    (each read once) and the intermediate written once."""
+    routed, shared = expert_bytes(cfg)
+    frac = 2.0 / 3.0  # w13 holds 2 of the 3 H x I matrices
+    abytes = 2 if cfg.afmt == "bf16" else 1
+    N = T * cfg.num_experts_per_tok
+    S = cfg.n_shared_experts
+    return (active * routed + S * shared) * frac + (N + T) * cfg.hidden * abytes + \
+        (N + S * T) * cfg.moe_intermediate_size * abytes
+
+
+def layer_bytes(cfg, active, T):
+    """Algorithmic bytes of the whole layer: active experts' and shared experts'
+    weights, the router weight, x read once and the output written once."""
+    routed, shared = expert_bytes(cfg)
+    return active * routed + cfg.n_shared_experts * shared + \
+        cfg.n_routed_experts * cfg.hidden * 4 + 2 * T * cfg.hidden * 2
+
+
+def layer_flops(cfg, T):
+    N = T * cfg.num_experts_per_tok
+    return 2.0 * (N + T * cfg.n_shared_experts) * 3 * cfg.hidden * cfg.moe_intermediate_size
+
+
+def ncu_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current source of the kernel (else None)."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel)
+    if not e:
+        return None
+    src = os.path.join(ROOT, e["source"])
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return e["dram_bytes_per_launch"] if h == e["source_sha256_16"] else None
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, rank, world, dev):
+    import torch
+    import expert_routing_grouped_layer_b200 as moe
+    from expert_routing_grouped_layer_b200 import workloads as W
+
+    cfg = W.CONFIGS[args.workload]
+    if args.tokens:
+        cfg = cfg.replace(T=args.tokens)
+    if args.experts:
+        cfg = cfg.replace(n_routed_experts=args.experts)
+    T, k, E, H, I, S = (cfg.T, cfg.num_experts_per_tok, cfg.n_routed_experts, cfg.hidden,
+                        cfg.moe_intermediate_size, cfg.n_shared_experts)
+    inp = W.make_inputs(cfg, dev)
+    if rank > 0:  # replicas: same model, each rank its own tokens
+        inp["x"] = W.make_inputs(cfg.replace(seed=cfg.seed + 7919 * rank), dev)["x"]
+    wts = W.make_weights(cfg, dev)
+    torch.cuda.synchronize()
+
+    layer = moe.MoELayer(cfg, wts, inp["gate_w"], inp["gate_bias"], max_tokens=T, device=dev)
+    ccfg, cw = layer.ccfg, layer.cw
+    P = lambda which: layer.ws_ptr(T, which)
+    ws, wsb, st = layer.ws, layer.ws.numel(), layer.status
+    x = inp["x"]
+    out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+
+    def step(ev):
+        ev[0].record(stream)
+        moe.moe_gate_topk(ccfg, x, T, inp["gate_w"], inp["gate_bias"], P(moe.WS_TOPK_IDX),
+                          P(moe.WS_TOPK_W), ws, wsb, stream=sp)
+        ev[1].record(stream)
+        moe.moe_permute(ccfg, P(moe.WS_TOPK_IDX), T, P(moe.WS_OFFSETS), P(moe.WS_SORTED_PAIR),
+                        P(moe.WS_ROW_OF), st, ws, wsb, stream=sp)
+        ev[2].record(stream)
+        moe.moe_pack_expert_inputs(ccfg, x, T, P(moe.WS_SORTED_PAIR), P(moe.WS_XA),
+                                   P(moe.WS_XA_SCALE), stream=sp)
+        ev[3].record(stream)
+        moe.moe_expert_gate_up(ccfg, P(moe.WS_XA), P(moe.WS_XA_SCALE), T, P(moe.WS_OFFSETS), cw,
+                               P(moe.WS_H), P(moe.WS_H_SCALE), st, stream=sp)
+        ev[4].record(stream)
+        moe.moe_expert_down(ccfg, P(moe.WS_H), P(moe.WS_H_SCALE), T, P(moe.WS_OFFSETS), cw,
+                            P(moe.WS_Y), P(moe.WS_SHARED_Y), st, stream=sp)
+        ev[5].record(stream)
+        moe.moe_combine(ccfg, P(moe.WS_Y), P(moe.WS_SHARED_Y), P(moe.WS_ROW_OF), P(moe.WS_TOPK_W),
+                        T, out, stream=sp)
+        ev[6].record(stream)
+
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(7)]
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(mk())
+    torch.cuda.synchronize()
+    # the staged calls and moe_layer_forward must agree bit for bit
+    ref = layer.forward(x)
+    torch.cuda.synchronize()
+    assert torch.equal(ref.view(torch.int16), out.view(torch.int16)), "staged != layer forward"
+    assert st.item() == 0, "device status %d" % st.item()
+
+    events = [mk() for _ in range(args.steps)]
+    clocks = ClockSampler(dev.index if dev.index is not None else 0, enabled=not args.no_clocks)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t_wall = time.perf_counter()
+    for i in range(args.steps):
+        flush.zero_()  # L2 flush outside the timed events
+        step(events[i])
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - t_wall
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+
+    stage = [[events[i][j].elapsed_time(events[i][j + 1]) for i in range(args.steps)]
+             for j in range(6)]
+    step_ms = [sum(stage[j][i] for j in range(6)) for i in range(args.steps)]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    offsets = layer.intermediate(T, moe.WS_OFFSETS, torch.int32, (E + 1,)).cpu()
+    active = int((offsets[1:] - offsets[:-1] > 0).sum())
+
+    # end to end: host tokens in (pinned), layer through the public API, host result out
+    e2e = None
+    if not args.no_e2e:
+        xh = x.cpu().pin_memory()
+        oh = torch.empty(T, H, dtype=torch.bfloat16).pin_memory()
+        xd = torch.empty_like(x)
+        for _ in range(3):
+            xd.copy_(xh, non_blocking=True)
+            oh.copy_(layer.forward(xd), non_blocking=True)
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(1, min(args.steps, 100))
+        s0.record(stream)
+        for _ in range(n_e2e):
+            flush.zero_()
+            xd.copy_(xh, non_blocking=True)
+            oh.copy_(layer.forward(xd), non_blocking=True)
+        s1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = s0.elapsed_time(s1) / n_e2e
+        if world > 1:
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": world * T / (e2e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2,
+               "ms_per_step": e2e_ms, "includes_l2_flush": True}
+
+    peaks, peak_src = load_peaks()
+    ms = total_ms / args.steps
+    mean = lambda j: statistics.fmean(stage[j])
+    names = ["gate_topk", "permute", "pack_inputs", "gate_up", "down", "combine"]
+    stage_ms = {n: mean(j) for j, n in enumerate(names)}
+    gu_bytes = gate_up_bytes(cfg, active, T)
+    gu_ms = stage_ms["gate_up"]
+    hbm = peaks["hbm_gbs"]
+    achieved = gu_bytes / (gu_ms / 1e3) / 1e9
+    lb = layer_bytes(cfg, active, T)
+    line = {
+        "metric": METRIC,
+        "value": world * T / (ms / 1e3),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if cfg.wfmt == "bf16" else cfg.wfmt,
+        "data": "synthetic (seeded; x ~ N(0,1), router N(0,0.02), bias U[-0.1,0.1], "
+                "experts N(0,0.02)); random-init weights",
+        "config": {"workload": "%s: T=%d tokens, hidden %d, %d routed experts top-%d, "
+                               "intermediate %d, %d shared, %s weights, %s activations"
+                               % (cfg.name, T, H, E, k, I, S, cfg.wfmt, cfg.afmt),
+                   "T": T, "hidden": H, "experts": E, "top_k": k, "intermediate": I,
+                   "shared_experts": S, "active_experts": active,
+                   "parallelism": "replicas x%d" % world,
+                   "l2": "256 MiB write before every timed step, outside the timed events"},
+        "roofline": {"bound": "hbm", "kernel": "gate_up (grouped SwiGLU GEMM1)",
+                     "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                     "peak_source": peak_src, "traffic": ncu_traffic("gate_up"),
+                     "algorithmic_bytes_per_launch": gu_bytes},
+        "layer_roofline": {"bound": "hbm", "bytes": lb, "achieved_gbs": lb / (ms / 1e3) / 1e9,
+                           "frac": lb / (ms / 1e3) / 1e9 / hbm,
+                           "flops": layer_flops(cfg, T),
+                           "tflops": layer_flops(cfg, T) / (ms / 1e3) / 1e12},
+        "stage_ms": stage_ms,
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "wall_s_timed_loop": wall,
+        "clocks": clk,
+        "e2e": e2e,
+    }
+    return line, cfg, inp, wts
+
+
+# ------------------------------------------------------------------ oracle arm
+def oracle_timing(cfg, inp, wts, tokens_per_step, steps, seed=0):
+    """Time the float64 oracle (route + layer) on `steps` disjoint samples of
+    `tokens_per_step` tokens each; weights are fetched to host outside timing."""
+    import numpy as np
+    import oracle
+    from expert_routing_grouped_layer_b200 import workloads as W
+
+    rng = np.random.default_rng(seed)
+    x_all = W.bf16_codes(inp["x"])
+    wg = inp["gate_w"].cpu().numpy()
+    bias = inp["gate_bias"].cpu().numpy()
+    samples = [np.sort(rng.choice(cfg.T, tokens_per_step, replace=False)) for _ in range(steps)]
+    cache = {}
+
+    def get(e, shared=False):
+        key = (e, shared)
+        if key not in cache:
+            cache[key] = W.expert_slice(wts, e, shared=shared)
+        return cache[key]
+
+    times = []
+    for toks in samples:
+        # routing first (timed), then fetch any expert not yet on the host (untimed)
+        t0 = time.perf_counter()
+        r = oracle.route(cfg, x_all, wg, bias, tokens=toks.astype(np.int32))
+        t_route = time.perf_counter() - t0
+        for e in np.unique(r["idx"]):
+            get(int(e))
+        for s in range(cfg.n_shared_experts):
+            get(s, True)
+        t0 = time.perf_counter()
+        oracle.layer(cfg, x_all[toks], r["idx"], r["w"], lambda e: get(e),
+                     lambda s: get(s, True))
+        times.append(t_route + time.perf_counter() - t0)
+        if len(cache) > 64:  # bound host memory
+            cache.clear()
+    return times
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+def run_reference(args, dev):
+    import torch
+    from expert_routing_grouped_layer_b200 import workloads as W
+    cfg = W.CONFIGS[args.workload]
+    inp = W.make_inputs(cfg, dev)
+    wts = W.make_weights(cfg, dev)
+    torch.cuda.synchronize()
+    per_step = 1
+    oracle_timing(cfg, inp, wts, per_step, args.warmup, seed=1)
+    times = oracle_timing(cfg, inp, wts, per_step, args.steps, seed=2)
+    total = sum(times)
+    value = per_step * args.steps / total
+    sample = "%d token(s) per step, %d steps, disjoint seeded samples of the %d-token batch" % (
+        per_step, args.steps, cfg.T)
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded, same workload as the CUDA arm)",
+        "config": {"workload": cfg.name, "T": cfg.T, "hidden": cfg.hidden,
+                   "experts": cfg.n_routed_experts, "top_k": cfg.num_experts_per_tok},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    import torch
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        dev = torch.device("cuda", local)
+        torch.cuda.set_device(dev)
+        print(json.dumps(run_reference(args, dev)), flush=True)
+        return 0
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", device_id=dev,
+                                             timeout=datetime.timedelta(seconds=300))
+    line, cfg, inp, wts = run_ours(args, rank, world, dev)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tok = args.cpu_sample_tokens
+        times = oracle_timing(cfg, inp, wts, tok, 1, seed=3)
+        line["cpu_baseline"] = {"value": tok / times[0], "unit": UNIT, "cores": cpu_cores(),
+                                "kind": "oracle",
+                                "sample": "%d seeded tokens of the %d-token batch (route + layer, "
+                                          "float64), %.1f s" % (tok, cfg.T, times[0])}
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

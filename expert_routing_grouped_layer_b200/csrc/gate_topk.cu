@@ -1,0 +1,308 @@
+// gate_topk.cu -- router GEMM and warp-per-token selection.
+//
+// Router ("DeepSeek V3架构拆解：Kimi-K2-Thinking-NVFP4的MLA注意力与MoE路由实现原理",
+// 三.1 打分): logits = x . Wg^T with fp32 inputs and fp32 accumulation.
+// Selection (same page, 三.2 选专家 and 三.3 权重归一化 + 路由缩放; sqrtsoftplus
+// scoring and route_scale from "DeepSeek-V4-Pro 架构与代码概述", 架构):
+// score, bias, group-limited top-k, normalised and scaled weights.
+//
+// The router GEMM is split along H into `splits` partial sums so a decode batch
+// still fills the GPU; the selection kernel adds the partials in split order,
+// so the logits are deterministic.
+#include <cuda_bf16.h>
+
+#include <cfloat>
+#include <climits>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int RG_BM = 128;  // tokens per tile
+constexpr int RG_BN = 128;  // experts per tile
+constexpr int RG_BK = 16;
+constexpr int RG_PAD = 4;
+
+// part[split][t][e] = sum over this split's h of x[t][h] * wg[e][h]
+__global__ void __launch_bounds__(256) router_gemm_kernel(const __nv_bfloat16* __restrict__ x,
+                                                          const float* __restrict__ wg,
+                                                          float* __restrict__ part, int T, int E,
+                                                          int H, int ksteps_per_split) {
+    __shared__ __align__(16) float As[2][RG_BK][RG_BM + RG_PAD];
+    __shared__ __align__(16) float Bs[2][RG_BK][RG_BN + RG_PAD];
+
+    const int tid = threadIdx.x;
+    const int t0 = blockIdx.x * RG_BM;
+    const int e0 = blockIdx.y * RG_BN;
+    const int split = blockIdx.z;
+    const int nk = H / RG_BK;
+    const int kbeg = split * ksteps_per_split;
+    const int kend = min(nk, kbeg + ksteps_per_split);
+
+    // loader mapping: each thread moves 8 consecutive k of one row of A and of B
+    const int lrow = tid >> 1;       // 0..127
+    const int lcol = (tid & 1) * 8;  // 0 or 8
+    const bool a_ok = (t0 + lrow) < T;
+    const bool b_ok = (e0 + lrow) < E;
+    const __nv_bfloat16* a_src = x + (size_t)(t0 + lrow) * H + lcol;
+    const float* b_src = wg + (size_t)(e0 + lrow) * H + lcol;
+
+    const int ty = tid >> 4, tx = tid & 15;
+    float acc[8][8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+
+    uint4 ra;
+    float4 rb0, rb1;
+    auto gload = [&](int ks) {
+        const int koff = ks * RG_BK;
+        if (a_ok) ra = *reinterpret_cast<const uint4*>(a_src + koff);
+        else ra = make_uint4(0, 0, 0, 0);
+        if (b_ok) {
+            rb0 = *reinterpret_cast<const float4*>(b_src + koff);
+            rb1 = *reinterpret_cast<const float4*>(b_src + koff + 4);
+        } else {
+            rb0 = rb1 = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    };
+    auto sstore = [&](int buf) {
+        const __nv_bfloat16* av = reinterpret_cast<const __nv_bfloat16*>(&ra);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) As[buf][lcol + c][lrow] = __bfloat162float(av[c]);
+        Bs[buf][lcol + 0][lrow] = rb0.x;
+        Bs[buf][lcol + 1][lrow] = rb0.y;
+        Bs[buf][lcol + 2][lrow] = rb0.z;
+        Bs[buf][lcol + 3][lrow] = rb0.w;
+        Bs[buf][lcol + 4][lrow] = rb1.x;
+        Bs[buf][lcol + 5][lrow] = rb1.y;
+        Bs[buf][lcol + 6][lrow] = rb1.z;
+        Bs[buf][lcol + 7][lrow] = rb1.w;
+    };
+
+    if (kbeg < kend) {
+        gload(kbeg);
+        sstore(0);
+    }
+    __syncthreads();
+    int buf = 0;
+    for (int ks = kbeg; ks < kend; ++ks) {
+        const bool more = ks + 1 < kend;
+        if (more) gload(ks + 1);
+#pragma unroll
+        for (int kk = 0; kk < RG_BK; ++kk) {
+            float a[8], b[8];
+            *reinterpret_cast<float4*>(&a[0]) = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 4]);
+            *reinterpret_cast<float4*>(&a[4]) =
+                *reinterpret_cast<const float4*>(&As[buf][kk][64 + ty * 4]);
+            *reinterpret_cast<float4*>(&b[0]) = *reinterpret_cast<const float4*>(&Bs[buf][kk][tx * 4]);
+            *reinterpret_cast<float4*>(&b[4]) =
+                *reinterpret_cast<const float4*>(&Bs[buf][kk][64 + tx * 4]);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        }
+        if (more) sstore(buf ^ 1);
+        __syncthreads();
+        buf ^= 1;
+    }
+
+    float* out = part + (size_t)split * T * E;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int t = t0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + (i - 4));
+        if (t >= T) continue;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int e = e0 + (j < 4 ? tx * 4 + j : 64 + tx * 4 + (j - 4));
+            if (e < E) out[(size_t)t * E + e] = acc[i][j];
+        }
+    }
+}
+
+__device__ __forceinline__ float score_of(float l, int score_fn) {
+    if (score_fn == MOE_SCORE_SIGMOID) return 1.0f / (1.0f + expf(-l));
+    return sqrtf(fmaxf(l, 0.0f) + log1pf(expf(-fabsf(l))));
+}
+
+// (value, index) order used everywhere: larger value first, then lower index.
+__device__ __forceinline__ bool better(float va, int ia, float vb, int ib) {
+    return va > vb || (va == vb && ia < ib);
+}
+
+struct TopkParams {
+    const float* part;
+    int splits;
+    const float* bias;
+    int T, E, k, n_group, topk_group, norm, score_fn;
+    float rsf;
+    int32_t* idx;
+    float* w;
+};
+
+// One warp per token. Lane l holds experts e = l + 32*j, j < MAXJ.
+template <int MAXJ>
+__global__ void __launch_bounds__(256) topk_kernel(TopkParams p) {
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= p.T) return;
+    const int E = p.E;
+
+    float sv[MAXJ], spv[MAXJ];
+    uint32_t avail = 0;
+#pragma unroll
+    for (int j = 0; j < MAXJ; ++j) {
+        const int e = lane + 32 * j;
+        sv[j] = 0.f;
+        spv[j] = -FLT_MAX;
+        if (e < E) {
+            float l = 0.f;
+            for (int s = 0; s < p.splits; ++s) l += p.part[((size_t)s * p.T + t) * E + e];
+            sv[j] = score_of(l, p.score_fn);
+            spv[j] = sv[j] + p.bias[e];
+            avail |= 1u << j;
+        }
+    }
+
+    if (p.n_group > 1) {
+        const int gsz = E / p.n_group;
+        float gs = -FLT_MAX;  // lane g < n_group holds group g's score
+        for (int g = 0; g < p.n_group; ++g) {
+            float b1 = -FLT_MAX, b2 = -FLT_MAX;
+#pragma unroll
+            for (int j = 0; j < MAXJ; ++j) {
+                const int e = lane + 32 * j;
+                if (((avail >> j) & 1u) && e / gsz == g) {
+                    const float v = spv[j];
+                    if (v > b1) { b2 = b1; b1 = v; }
+                    else if (v > b2) b2 = v;
+                }
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                const float o1 = __shfl_xor_sync(0xffffffffu, b1, off);
+                const float o2 = __shfl_xor_sync(0xffffffffu, b2, off);
+                const float hi = fmaxf(b1, o1), lo = fminf(b1, o1);
+                b2 = fmaxf(lo, fmaxf(b2, o2));
+                b1 = hi;
+            }
+            const float score = (gsz == 1) ? b1 : b1 + b2;
+            if (lane == g) gs = score;
+        }
+        uint32_t kept = 0;
+        for (int r = 0; r < p.topk_group; ++r) {
+            float bv = (lane < p.n_group && !((kept >> lane) & 1u)) ? gs : -FLT_MAX;
+            int bi = (lane < p.n_group && !((kept >> lane) & 1u)) ? lane : INT_MAX;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+                const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+                if (better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
+            }
+            kept |= 1u << bi;
+        }
+#pragma unroll
+        for (int j = 0; j < MAXJ; ++j) {
+            const int e = lane + 32 * j;
+            if (((avail >> j) & 1u) && !((kept >> (e / gsz)) & 1u)) avail &= ~(1u << j);
+        }
+    }
+
+    int my_idx = 0;
+    float my_w = 0.f;
+    for (int r = 0; r < p.k; ++r) {
+        float bv = -FLT_MAX, bs = 0.f;
+        int bi = INT_MAX;
+#pragma unroll
+        for (int j = 0; j < MAXJ; ++j) {
+            const int e = lane + 32 * j;
+            if (((avail >> j) & 1u) && better(spv[j], e, bv, bi)) {
+                bv = spv[j];
+                bi = e;
+                bs = sv[j];
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+            const float os = __shfl_xor_sync(0xffffffffu, bs, off);
+            if (better(ov, oi, bv, bi)) { bv = ov; bi = oi; bs = os; }
+        }
+        if (bi != INT_MAX && (bi & 31) == lane) avail &= ~(1u << (bi >> 5));
+        if (lane == r) {
+            my_idx = bi;
+            my_w = bs;
+        }
+    }
+
+    float sum = (lane < p.k) ? my_w : 0.f;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    if (p.norm) my_w = my_w / sum;
+    my_w *= p.rsf;
+    if (lane < p.k) {
+        p.idx[(size_t)t * p.k + lane] = my_idx;
+        p.w[(size_t)t * p.k + lane] = my_w;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_router_gemm(const void* x, const float* gate_w, float* part, int T, int E, int H,
+                               int splits, cudaStream_t st) {
+    if (T == 0) return cudaSuccess;
+    const int nk = H / RG_BK;
+    const int per = (nk + splits - 1) / splits;
+    dim3 grid((T + RG_BM - 1) / RG_BM, (E + RG_BN - 1) / RG_BN, splits);
+    router_gemm_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), gate_w, part, T,
+                                             E, H, per);
+    return cudaGetLastError();
+}
+
+int router_splits_for(int T, int E, int H) {
+    const int tiles = ((T + RG_BM - 1) / RG_BM) * ((E + RG_BN - 1) / RG_BN);
+    const int target = 2 * num_sms();
+    int s = (target + tiles - 1) / tiles;
+    const int max_s = (H / RG_BK) / 4;  // at least 4 k-steps per split
+    if (s > max_s) s = max_s;
+    if (s < 1) s = 1;
+    // every split must own at least one k-step after rounding
+    const int nk = H / RG_BK;
+    const int per = (nk + s - 1) / s;
+    s = (nk + per - 1) / per;
+    return s;
+}
+
+cudaError_t launch_topk(const moe_config* c, const float* part, int splits, const float* bias, int T,
+                        int32_t* idx, float* w, cudaStream_t st) {
+    if (T == 0) return cudaSuccess;
+    TopkParams p;
+    p.part = part;
+    p.splits = splits;
+    p.bias = bias;
+    p.T = T;
+    p.E = c->n_routed_experts;
+    p.k = c->num_experts_per_tok;
+    p.n_group = c->n_group;
+    p.topk_group = c->topk_group;
+    p.norm = c->norm_topk_prob;
+    p.score_fn = c->score_fn;
+    p.rsf = c->routed_scaling_factor;
+    p.idx = idx;
+    p.w = w;
+    const int warps = 8;
+    dim3 grid((T + warps - 1) / warps);
+    if (p.E <= 32) topk_kernel<1><<<grid, warps * 32, 0, st>>>(p);
+    else if (p.E <= 128) topk_kernel<4><<<grid, warps * 32, 0, st>>>(p);
+    else if (p.E <= 512) topk_kernel<16><<<grid, warps * 32, 0, st>>>(p);
+    else topk_kernel<32><<<grid, warps * 32, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

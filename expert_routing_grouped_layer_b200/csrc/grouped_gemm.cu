@@ -1,0 +1,407 @@
+// grouped_gemm.cu -- per-expert SwiGLU MLP on the tcgen05 tensor cores.
+//
+// "DeepSeek V3架构拆解：Kimi-K2-Thinking-NVFP4的MLA注意力与MoE路由实现原理", 三.4 推理执行:
+// after the argsort each expert multiplies its contiguous block of tokens by
+// its gate/up/down projections with SiLU; the shared experts see every token.
+// ("DeepSeek-V4-Pro 架构与代码概述", 文件说明: FFNSwiGLU is the standard SwiGLU.)
+//
+// Two launches per layer:
+//   GEMM1: for every expert block, G = X W1^T and U = X W3^T, a = SiLU(G) * U;
+//   GEMM2: Y = a W2^T.
+// Both run "weights as the M operand": an MMA tile is 128 weight rows (output
+// features) x up to 128 tokens (N, a multiple of 16), so a decode expert with
+// a handful of tokens still issues full-height MMAs and its weights stream at
+// HBM speed, and a prefill expert with ~170 tokens needs only two N tiles.
+//
+// Kernel structure (one persistent CTA per SM, 6 warps):
+//   warp 0   TMA producer: weight tiles (128 rows x 64 K, 128B-swizzled) and
+//            token tiles (16-row boxes) into a ring of shared-memory stages;
+//   warp 1   MMA issuer: tcgen05.mma kind::f16 (bf16 x bf16 -> fp32 in TMEM),
+//            tcgen05.commit frees each stage and publishes each accumulator;
+//   warps 2-5 epilogue: tcgen05.ld the accumulator (lane = weight row,
+//            column = token), SwiGLU (GEMM1), bf16 stores.
+// Accumulators are double-buffered in tensor memory so the epilogue of one
+// tile overlaps the main loop of the next. The tile list (expert, M tile,
+// N tile) is derived on the device from expert_offsets; there is no host sync.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int BM = 128;   // weight rows per tile (MMA M)
+constexpr int BN = 128;   // max tokens per tile (MMA N)
+constexpr int BK = 64;    // bf16 elements in one 128-byte swizzled row
+constexpr int B_BOX = 16; // token rows per TMA box
+constexpr int MAX_SEG = 1024 + 4;
+
+template <int GEMM>
+struct Tile {
+    static constexpr int NA = (GEMM == 1) ? 2 : 1;  // A tiles per stage (gate + up)
+    static constexpr int A_BYTES = BM * BK * 2;
+    static constexpr int B_BYTES = BN * BK * 2;
+    static constexpr int STAGE_BYTES = NA * A_BYTES + B_BYTES;
+    static constexpr int STAGES = (GEMM == 1) ? 4 : 6;
+    static constexpr int ACC_COLS = NA * BN;        // TMEM columns of one accumulator set
+    static constexpr int TMEM_COLS = 2 * ACC_COLS;  // double-buffered
+    static constexpr int BAR_BYTES = 8 * (2 * STAGES + 5) + 16;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + 4 * (MAX_SEG + 1);
+};
+
+struct KParams {
+    int nseg;  // E + S
+    int E, S, T, N;
+    int K;               // reduction length
+    int M;               // output features per matrix
+    int a_rows_per_mat;  // 2I (GEMM1) or H (GEMM2)
+    int a_up_offset;     // I (GEMM1): first up-projection row
+    int b_shared_base;   // first B row of the shared-expert rows
+    int b_shared_stride; // B-row step per shared expert
+    const int32_t* offsets;
+    __nv_bfloat16* out_routed;
+    __nv_bfloat16* out_shared;
+    int ld_out;
+    int32_t* status;
+};
+
+struct Unit {
+    int seg, mt, n_valid, a_row, b_row;
+    __nv_bfloat16* out;  // row of the first token, column 0
+};
+
+__device__ __forceinline__ int seg_rows(const KParams& p, int s) {
+    return s < p.E ? (p.offsets[s + 1] - p.offsets[s]) : p.T;
+}
+
+__device__ __forceinline__ Unit decode_unit(const KParams& p, const int* pref, int u) {
+    int lo = 0, hi = p.nseg - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (pref[mid] <= u) lo = mid; else hi = mid - 1;
+    }
+    Unit t;
+    t.seg = lo;
+    const int m = seg_rows(p, lo);
+    const int ntiles = (m + BN - 1) / BN;
+    const int local = u - pref[lo];
+    t.mt = local / ntiles;
+    const int nt = local - t.mt * ntiles;
+    t.n_valid = min(BN, m - nt * BN);
+    if (lo < p.E) {
+        t.a_row = lo * p.a_rows_per_mat + t.mt * BM;
+        const int r0 = p.offsets[lo] + nt * BN;
+        t.b_row = r0;
+        t.out = p.out_routed + (size_t)r0 * p.ld_out;
+    } else {
+        const int s = lo - p.E;
+        t.a_row = s * p.a_rows_per_mat + t.mt * BM;
+        t.b_row = p.b_shared_base + s * p.b_shared_stride + nt * BN;
+        t.out = p.out_shared + ((size_t)s * p.T + nt * BN) * p.ld_out;
+    }
+    return t;
+}
+
+template <int GEMM>
+__global__ void __launch_bounds__(192, 1)
+    grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA_routed,
+                             const __grid_constant__ CUtensorMap tmA_shared,
+                             const __grid_constant__ CUtensorMap tmB, const KParams p) {
+    using C = Tile<GEMM>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+    uint64_t* empty = full + C::STAGES;
+    uint64_t* tfull = empty + C::STAGES;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* mma_done = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* pref = reinterpret_cast<int*>(tmem_slot + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], 128);
+        }
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&tmA_routed);
+        tma_prefetch_desc(&tmA_shared);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    // tile schedule: pref[s] = first unit of segment s
+    const int MT = p.M / BM;
+    if (warp == 1) {
+        const int per = (p.nseg + 31) / 32;
+        const int s0 = lane * per;
+        const int s1 = min(p.nseg, s0 + per);
+        int sum = 0;
+        for (int s = s0; s < s1; ++s) sum += ((seg_rows(p, s) + BN - 1) / BN) * MT;
+        int incl = sum;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += o;
+        }
+        int run = incl - sum;
+        for (int s = s0; s < s1; ++s) {
+            pref[s] = run;
+            run += ((seg_rows(p, s) + BN - 1) / BN) * MT;
+        }
+        if (lane == 31) pref[p.nseg] = incl;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int total = pref[p.nseg];
+    const int KB = p.K / BK;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued = 0;
+            for (int u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x) {
+                const Unit t = decode_unit(p, pref, u);
+                const int n_mma = (t.n_valid + 15) & ~15;
+                const int nb = n_mma / B_BOX;
+                const uint32_t tx = C::NA * C::A_BYTES + nb * B_BOX * BK * 2;
+                const CUtensorMap* tmA = (t.seg < p.E) ? &tmA_routed : &tmA_shared;
+                bool ok = true;
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+                    uint8_t* st = smem + stage * C::STAGE_BYTES;
+                    mbar_arrive_expect_tx(&full[stage], tx);
+                    tma_load_2d(st, tmA, kb * BK, t.a_row, &full[stage]);
+                    if (GEMM == 1)
+                        tma_load_2d(st + C::A_BYTES, tmA, kb * BK, t.a_row + p.a_up_offset, &full[stage]);
+                    uint8_t* sb = st + C::NA * C::A_BYTES;
+                    for (int i = 0; i < nb; ++i)
+                        tma_load_2d(sb + i * B_BOX * BK * 2, &tmB, kb * BK, t.b_row + i * B_BOX,
+                                    &full[stage]);
+                    ++issued;
+                    if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+            }
+            if (*abort_flag) {
+                // let every copy this thread issued land before the CTA exits
+                int s = stage;
+                uint32_t ph = phase;
+                for (int i = 0; i < min(issued, C::STAGES); ++i) {
+                    if (--s < 0) { s = C::STAGES - 1; ph ^= 1; }
+                    volatile int no_abort = 0;
+                    mbar_wait(&full[s], ph, &no_abort);
+                }
+                status_or(p.status, MOE_DEV_TIMEOUT);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            for (int u = blockIdx.x; u < total; u += gridDim.x) {
+                const Unit t = decode_unit(p, pref, u);
+                const int n_mma = (t.n_valid + 15) & ~15;
+                const uint32_t idesc = idesc_bf16(BM, n_mma);
+                if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t d0 = tmem_base + acc * C::ACC_COLS;
+                bool ok = true;
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t st = smem_u32(smem + stage * C::STAGE_BYTES);
+                    const uint32_t sb = st + C::NA * C::A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        const uint32_t acc_flag = (kb | kk) != 0;
+                        const uint64_t bd = sdesc_kmajor_sw128(sb + kk * 32);
+                        mma_bf16(d0, sdesc_kmajor_sw128(st + kk * 32), bd, idesc, acc_flag);
+                        if (GEMM == 1)
+                            mma_bf16(d0 + BN, sdesc_kmajor_sw128(st + C::A_BYTES + kk * 32), bd, idesc,
+                                     acc_flag);
+                    }
+                    mma_commit(&empty[stage]);
+                    if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                mma_commit(&tfull[acc]);
+                if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+            }
+            // every MMA this thread issued has finished once mma_done flips
+            mma_commit(mma_done);
+            volatile int no_abort = 0;
+            mbar_wait(mma_done, 0, &no_abort);
+            if (*abort_flag) status_or(p.status, MOE_DEV_TIMEOUT);
+        }
+    } else {
+        const int q = warp & 3;  // TMEM lane quadrant this warp may access
+        const int row = q * 32 + lane;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int u = blockIdx.x; u < total; u += gridDim.x) {
+            const Unit t = decode_unit(p, pref, u);
+            if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) break;
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::ACC_COLS;
+            __nv_bfloat16* out = t.out + t.mt * BM + row;
+            for (int c0 = 0; c0 < t.n_valid; c0 += 16) {
+                uint32_t g[16];
+                tmem_ld16(taddr + c0, g);
+                if (GEMM == 1) {
+                    uint32_t uu[16];
+                    tmem_ld16(taddr + BN + c0, uu);
+                    tmem_ld_wait(g, uu);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        if (c0 + j < t.n_valid) {
+                            const float gv = __uint_as_float(g[j]);
+                            const float a = gv / (1.0f + __expf(-gv)) * __uint_as_float(uu[j]);
+                            out[(size_t)(c0 + j) * p.ld_out] = __float2bfloat16_rn(a);
+                        }
+                    }
+                } else {
+                    tmem_ld_wait(g);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        if (c0 + j < t.n_valid)
+                            out[(size_t)(c0 + j) * p.ld_out] = __float2bfloat16_rn(__uint_as_float(g[j]));
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&tempty[acc]);
+            if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+// 2-D row-major bf16 tensor [rows][cols], box = box_rows x 64 columns, 128B swizzle.
+bool make_tmap_bf16(CUtensorMap* tm, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int GEMM>
+cudaError_t launch_bf16(const GroupedGemmArgs& a, cudaStream_t st) {
+    using C = Tile<GEMM>;
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(grouped_gemm_bf16_kernel<GEMM>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+
+    const int E = a.E, S = a.S, T = a.T, N = a.N, H = a.H, I = a.I;
+    KParams p;
+    p.nseg = E + S;
+    p.E = E;
+    p.S = S;
+    p.T = T;
+    p.N = N;
+    p.offsets = a.offsets;
+    p.status = a.status;
+    CUtensorMap tmAr, tmAs, tmB;
+    uint64_t b_rows;
+    if (GEMM == 1) {
+        p.K = H;
+        p.M = I;
+        p.a_rows_per_mat = 2 * I;
+        p.a_up_offset = I;
+        p.b_shared_base = N;
+        p.b_shared_stride = 0;
+        p.ld_out = I;
+        b_rows = (uint64_t)N + T;
+    } else {
+        p.K = I;
+        p.M = H;
+        p.a_rows_per_mat = H;
+        p.a_up_offset = 0;
+        p.b_shared_base = N;
+        p.b_shared_stride = T;
+        p.ld_out = H;
+        b_rows = (uint64_t)N + (uint64_t)S * T;
+    }
+    p.out_routed = static_cast<__nv_bfloat16*>(a.out_routed);
+    p.out_shared = static_cast<__nv_bfloat16*>(a.out_shared);
+    if (!make_tmap_bf16(&tmAr, a.w_routed, (uint64_t)E * p.a_rows_per_mat, p.K, BM))
+        return cudaErrorInvalidValue;
+    if (!make_tmap_bf16(&tmAs, S > 0 ? a.w_shared : a.w_routed,
+                        (uint64_t)(S > 0 ? S : E) * p.a_rows_per_mat, p.K, BM))
+        return cudaErrorInvalidValue;
+    if (b_rows == 0) return cudaSuccess;
+    if (!make_tmap_bf16(&tmB, a.b_rows, b_rows, p.K, B_BOX)) return cudaErrorInvalidValue;
+
+    // upper bound on tiles: sum_e ceil(m_e/BN) <= N/BN + min(E, N), plus shared
+    const long MT = p.M / BM;
+    const long routed_tiles = (long)N / BN + std::min<long>(E, N);
+    const long shared_tiles = (long)S * ((T + BN - 1) / BN);
+    const long units_max = (routed_tiles + shared_tiles) * MT;
+    const int grid = (int)std::max<long>(1, std::min<long>(num_sms(), units_max));
+    grouped_gemm_bf16_kernel<GEMM><<<grid, 192, C::SMEM_BYTES, st>>>(tmAr, tmAs, tmB, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st) {
+    if (a.wfmt != MOE_W_BF16 || a.afmt != MOE_A_BF16) return cudaErrorNotSupported;
+    return a.gemm == 1 ? launch_bf16<1>(a, st) : launch_bf16<2>(a, st);
+}
+
+}  // namespace moe

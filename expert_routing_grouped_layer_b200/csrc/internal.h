@@ -1,0 +1,74 @@
+// internal.h -- launchers shared between the library's translation units
+// (C++ linkage, not part of the public ABI).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "moe.h"
+
+namespace moe {
+
+// Workspace carve-up shared by every entry point (offsets in bytes).
+struct WsLayout {
+    size_t router_part;   // fp32 [S][T][E] partial router sums
+    size_t topk_idx;      // int32 [T][k]
+    size_t topk_w;        // fp32 [T][k]
+    size_t offsets;       // int32 [E+1]
+    size_t sorted_pair;   // int32 [N]
+    size_t row_of;        // int32 [N]
+    size_t chunk_counts;  // int32 [n_chunks][E]
+    size_t xa;            // gathered expert input rows [(N+T)][H] (bf16 or e4m3)
+    size_t xa_scale;      // uint8 [(N+T)][H/blk]
+    size_t hbuf;          // intermediate [(N+S*T)][I] (bf16 or e4m3)
+    size_t h_scale;       // uint8 [(N+S*T)][I/blk]
+    size_t y;             // bf16 [N][H]
+    size_t shared_y;      // bf16 [S][T][H]
+    size_t total;
+    int router_splits;
+    int n_chunks;
+};
+
+bool config_valid(const moe_config* c);
+moe_status config_supported(const moe_config* c);
+WsLayout ws_layout(const moe_config* c, int T);
+int num_sms();
+
+// Kernel launchers (return a cudaError_t of the launch).
+cudaError_t launch_router_gemm(const void* x, const float* gate_w, float* part, int T, int E, int H,
+                               int splits, cudaStream_t st);
+cudaError_t launch_topk(const moe_config* c, const float* part, int splits, const float* bias, int T,
+                        int32_t* idx, float* w, cudaStream_t st);
+cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int n_chunks, int32_t* chunk,
+                           int32_t* offsets, int32_t* sorted_pair, int32_t* row_of,
+                           int32_t* status, cudaStream_t st);
+cudaError_t launch_pack_rows(int afmt, const void* x, int H, const int32_t* sorted_pair, int N,
+                             int k, int T, int n_rows, void* out, uint8_t* out_scale,
+                             cudaStream_t st);
+cudaError_t launch_combine(const void* y, const void* shared_y, int S, const int32_t* row_of,
+                           const float* w, int T, int k, int H, void* out, cudaStream_t st);
+
+struct GroupedGemmArgs {
+    // problem
+    int gemm;           // 1: gate/up + SwiGLU, 2: down projection
+    int E, S, T, N, k;  // experts, shared experts, tokens, pairs, top-k
+    int H, I;
+    int wfmt, afmt;
+    const int32_t* offsets;  // [E+1]
+    // operands
+    const void* w_routed;  // w13 or w2
+    const void* w_routed_scale;
+    const void* w_shared;  // sh_w13 or sh_w2
+    const void* w_shared_scale;
+    const void* b_rows;  // gemm1: xa [(N+T)][H]; gemm2: hbuf [(N+S*T)][I]
+    const uint8_t* b_scale;
+    void* out_routed;  // gemm1: hbuf rows [0,N); gemm2: y
+    void* out_shared;  // gemm1: hbuf rows [N, N+S*T); gemm2: shared_y
+    uint8_t* out_routed_scale;
+    uint8_t* out_shared_scale;
+    int32_t* status;
+};
+cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st);
+
+}  // namespace moe

@@ -1,0 +1,196 @@
+// pack_combine.cu -- activation gather/quantisation in front of the expert
+// GEMMs, and the weighted combine behind them.
+//
+// Gather + quantise: each expert row r of the GEMM input is token
+// sorted_pair[r] / k of x (rows past N are the tokens in order, for the shared
+// experts). Quantisation follows the activation format:
+//  * FP8_E4M3_POW2_B128 ("DeepSeek-V4-Pro 架构与代码概述", 文件说明, kernel.py
+//    act_quant_kernel: FP8 per 128-element block, power-of-two scale): scale
+//    2^e with e the smallest integer such that amax <= 448 * 2^e;
+//  * MXFP8 ("开源巨头开放2.8T MoE权重:架构创新与本地部署实践指南", 存储与量化策略,
+//    MXFP8 activations; OCP MX rule): 2^(floor(log2 amax) - 8) per 32 elements;
+// both clamp the exponent to [-127, 127], write it as an E8M0 code, and round
+// the elements x / scale to E4M3 with round-to-nearest-even and saturation.
+//
+// Combine ("DeepSeek V3架构拆解：Kimi-K2-Thinking-NVFP4的MLA注意力与MoE路由实现原理",
+// 三.4: put the rows back in order, multiply by the top-k weights and sum; plus
+// the shared experts): one CTA per token, 16-byte vector loads of every row it
+// needs, fp32 sums in slot order, one bf16 rounding.
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace moe {
+
+namespace {
+
+// Token feeding expert row r; -1 when the row holds no valid pair (a row past
+// the valid pairs when some topk_idx entries were out of range).
+__device__ __forceinline__ int token_of_row(int r, const int32_t* sorted_pair, int N, int k, int T) {
+    const int t = r < N ? sorted_pair[r] / k : r - N;
+    return (t >= 0 && t < T) ? t : -1;
+}
+
+__global__ void __launch_bounds__(256) pack_bf16_kernel(const uint4* __restrict__ x, int H8,
+                                                        const int32_t* __restrict__ sorted_pair,
+                                                        int N, int k, int T, int n_rows,
+                                                        uint4* __restrict__ out) {
+    const int lane = threadIdx.x & 31;
+    const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (r >= n_rows) return;
+    const int t = token_of_row(r, sorted_pair, N, k, T);
+    uint4* dst = out + (size_t)r * H8;
+    if (t < 0) {
+        for (int v = lane; v < H8; v += 32) dst[v] = make_uint4(0, 0, 0, 0);
+        return;
+    }
+    const uint4* src = x + (size_t)t * H8;
+    for (int v = lane; v < H8; v += 32) dst[v] = src[v];
+}
+
+// exponent of the power-of-two scale: smallest e with a <= 448 * 2^e
+__device__ __forceinline__ int pow2_scale_exp(float a) {
+    if (a == 0.0f) return 0;
+    int adj = 0;
+    uint32_t b = __float_as_uint(a);
+    if ((b >> 23) == 0) {  // subnormal: scale up exactly first
+        b = __float_as_uint(a * 0x1p64f);
+        adj = -64;
+    }
+    const int E = (int)(b >> 23) - 127;
+    const uint32_t mant = b & 0x7FFFFFu;
+    // a = m * 2^E, m in [1,2); 448 = 1.75 * 2^8: a <= 448 * 2^e  <=>  e >= E - 8 (+1 if m > 1.75)
+    return E - 8 + (mant > 0x600000u ? 1 : 0) + adj;
+}
+
+// OCP MX shared exponent for E4M3 elements: floor(log2 a) - 8, clamped
+__device__ __forceinline__ int mx_scale_exp(float a) {
+    const uint32_t b = __float_as_uint(a);
+    const int f = (int)(b >> 23);
+    if (f == 0) return -127;  // zero or subnormal: floor(log2 a) - 8 < -127
+    return max(f - 127 - 8, -127);
+}
+
+// One warp per row; 4 elements per lane per step (a 128-element block for the
+// power-of-two format, four 32-element blocks for MX).
+template <int AFMT>
+__global__ void __launch_bounds__(256) pack_fp8_kernel(const __nv_bfloat16* __restrict__ x, int H,
+                                                       const int32_t* __restrict__ sorted_pair,
+                                                       int N, int k, int T, int n_rows,
+                                                       uint8_t* __restrict__ out,
+                                                       uint8_t* __restrict__ out_scale) {
+    constexpr int BLK = (AFMT == MOE_A_FP8_E4M3_POW2_B128) ? 128 : 32;
+    const int lane = threadIdx.x & 31;
+    const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (r >= n_rows) return;
+    const int t = token_of_row(r, sorted_pair, N, k, T);
+    const __nv_bfloat16* src = x + (size_t)(t < 0 ? 0 : t) * H;
+    uint8_t* dst = out + (size_t)r * H;
+    uint8_t* dsc = out_scale + (size_t)r * (H / BLK);
+    for (int c0 = 0; c0 < H; c0 += 128) {
+        uint2 raw = make_uint2(0, 0);
+        if (t >= 0) raw = *reinterpret_cast<const uint2*>(src + c0 + lane * 4);
+        const __nv_bfloat162* pr = reinterpret_cast<const __nv_bfloat162*>(&raw);
+        const float2 f01 = __bfloat1622float2(pr[0]);
+        const float2 f23 = __bfloat1622float2(pr[1]);
+        float amax = fmaxf(fmaxf(fabsf(f01.x), fabsf(f01.y)), fmaxf(fabsf(f23.x), fabsf(f23.y)));
+        constexpr int LANES = BLK / 4;  // lanes sharing one scale
+#pragma unroll
+        for (int off = LANES / 2; off > 0; off >>= 1)
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        int e = (AFMT == MOE_A_FP8_E4M3_POW2_B128) ? pow2_scale_exp(amax) : mx_scale_exp(amax);
+        e = min(max(e, -127), 127);
+        const float inv = __uint_as_float((uint32_t)(127 - e) << 23);  // 2^-e, e in [-127, 126]
+        const __nv_fp8x2_storage_t q01 =
+            __nv_cvt_float2_to_fp8x2(make_float2(f01.x * inv, f01.y * inv), __NV_SATFINITE, __NV_E4M3);
+        const __nv_fp8x2_storage_t q23 =
+            __nv_cvt_float2_to_fp8x2(make_float2(f23.x * inv, f23.y * inv), __NV_SATFINITE, __NV_E4M3);
+        const uint32_t packed = (uint32_t)q01 | ((uint32_t)q23 << 16);
+        *reinterpret_cast<uint32_t*>(dst + c0 + lane * 4) = packed;
+        if ((lane % LANES) == 0) dsc[(c0 + lane * 4) / BLK] = (uint8_t)(e + 127);
+    }
+}
+
+__global__ void __launch_bounds__(128) combine_kernel(const __nv_bfloat16* __restrict__ y,
+                                                      const __nv_bfloat16* __restrict__ shared_y,
+                                                      int S, const int32_t* __restrict__ row_of,
+                                                      const float* __restrict__ w, int T, int k,
+                                                      int H, __nv_bfloat16* __restrict__ out) {
+    __shared__ int32_t rows[32];
+    __shared__ float wts[32];
+    const int t = blockIdx.x;
+    if (threadIdx.x < k) {
+        rows[threadIdx.x] = row_of[(size_t)t * k + threadIdx.x];
+        wts[threadIdx.x] = w[(size_t)t * k + threadIdx.x];
+    }
+    __syncthreads();
+    const int H8 = H / 8;
+    for (int v = threadIdx.x; v < H8; v += blockDim.x) {
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+        for (int j = 0; j < k; ++j) {
+            const int r = rows[j];
+            if (r < 0) continue;
+            const float wj = wts[j];
+            const uint4 u = *reinterpret_cast<const uint4*>(y + (size_t)r * H + (size_t)v * 8);
+            const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 f = __bfloat1622float2(b[i]);
+                acc[2 * i] = fmaf(wj, f.x, acc[2 * i]);
+                acc[2 * i + 1] = fmaf(wj, f.y, acc[2 * i + 1]);
+            }
+        }
+        for (int s = 0; s < S; ++s) {
+            const uint4 u =
+                *reinterpret_cast<const uint4*>(shared_y + ((size_t)s * T + t) * H + (size_t)v * 8);
+            const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 f = __bfloat1622float2(b[i]);
+                acc[2 * i] += f.x;
+                acc[2 * i + 1] += f.y;
+            }
+        }
+        uint4 o;
+        __nv_bfloat162* ob = reinterpret_cast<__nv_bfloat162*>(&o);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) ob[i] = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+        *reinterpret_cast<uint4*>(out + (size_t)t * H + (size_t)v * 8) = o;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_pack_rows(int afmt, const void* x, int H, const int32_t* sorted_pair, int N,
+                             int k, int T, int n_rows, void* out, uint8_t* out_scale,
+                             cudaStream_t st) {
+    if (n_rows == 0) return cudaSuccess;
+    dim3 grid((n_rows + 7) / 8);
+    if (afmt == MOE_A_BF16)
+        pack_bf16_kernel<<<grid, 256, 0, st>>>(static_cast<const uint4*>(x), H / 8, sorted_pair, N,
+                                               k, T, n_rows, static_cast<uint4*>(out));
+    else if (afmt == MOE_A_FP8_E4M3_POW2_B128)
+        pack_fp8_kernel<MOE_A_FP8_E4M3_POW2_B128><<<grid, 256, 0, st>>>(
+            static_cast<const __nv_bfloat16*>(x), H, sorted_pair, N, k, T, n_rows,
+            static_cast<uint8_t*>(out), out_scale);
+    else
+        pack_fp8_kernel<MOE_A_MXFP8><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), H,
+                                                           sorted_pair, N, k, T, n_rows,
+                                                           static_cast<uint8_t*>(out), out_scale);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const void* y, const void* shared_y, int S, const int32_t* row_of,
+                           const float* w, int T, int k, int H, void* out, cudaStream_t st) {
+    if (T == 0) return cudaSuccess;
+    combine_kernel<<<T, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(y),
+                                      static_cast<const __nv_bfloat16*>(shared_y), S, row_of, w, T,
+                                      k, H, static_cast<__nv_bfloat16*>(out));
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,157 @@
+// permute.cu -- dispatch permutation ("DeepSeek V3架构拆解：Kimi-K2-Thinking-NVFP4的MLA注意力与
+// MoE路由实现原理", 三.4 推理执行: count each expert's tokens, argsort the tokens by
+// expert id into contiguous blocks).
+//
+// Deterministic stable counting sort of the N = T*k (token, slot) pairs by
+// expert id, in three launches without atomics on the output order:
+//   1. count:   per chunk of PERM_CHUNK pairs, a per-expert histogram;
+//   2. scan:    expert totals -> expert_offsets, and each chunk's starting row
+//               per expert (exclusive prefix over chunks);
+//   3. scatter: inside a chunk each warp owns a contiguous slice; warp bases
+//               come from per-warp histograms, and inside a warp the rank of a
+//               pair among equal experts is the count of lower lanes matching
+//               it (__match_any_sync), so pairs keep ascending order.
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int PERM_WARPS = 8;
+constexpr int PERM_PER_WARP = 512;
+constexpr int PERM_CHUNK = PERM_WARPS * PERM_PER_WARP;
+constexpr int PERM_MAX_E = 1024;
+
+__global__ void __launch_bounds__(256) perm_count_kernel(const int32_t* __restrict__ idx, long N,
+                                                         int E, int32_t* __restrict__ chunk,
+                                                         int32_t* status) {
+    __shared__ int32_t cnt[PERM_MAX_E];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+    __syncthreads();
+    const long base = (long)blockIdx.x * PERM_CHUNK;
+    bool bad = false;
+    for (int i = threadIdx.x; i < PERM_CHUNK; i += blockDim.x) {
+        const long p = base + i;
+        if (p >= N) break;
+        const int e = idx[p];
+        if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
+        else bad = true;
+    }
+    if (bad) status_or(status, MOE_DEV_BAD_EXPERT);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) chunk[(size_t)blockIdx.x * E + e] = cnt[e];
+}
+
+// Single CTA of 1024 threads; thread e owns expert e.
+__global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t* __restrict__ chunk, int n_chunks,
+                                                         int E, int32_t* __restrict__ offsets) {
+    __shared__ int32_t warp_sums[32];
+    const int e = threadIdx.x;
+    int total = 0;
+    if (e < E)
+        for (int c = 0; c < n_chunks; ++c) total += chunk[(size_t)c * E + e];
+    // block exclusive scan of totals over experts
+    const int lane = e & 31, wid = e >> 5;
+    int v = total;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += o;
+    }
+    if (lane == 31) warp_sums[wid] = v;
+    __syncthreads();
+    if (wid == 0) {
+        int s = warp_sums[lane];
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, s, off);
+            if (lane >= off) s += o;
+        }
+        warp_sums[lane] = s;  // inclusive over warps
+    }
+    __syncthreads();
+    const int excl = v - total + (wid > 0 ? warp_sums[wid - 1] : 0);
+    if (e < E) {
+        offsets[e] = excl;
+        int run = excl;
+        for (int c = 0; c < n_chunks; ++c) {
+            const int n = chunk[(size_t)c * E + e];
+            chunk[(size_t)c * E + e] = run;
+            run += n;
+        }
+    }
+    if (e == E - 1) offsets[E] = excl + total;
+}
+
+__global__ void __launch_bounds__(PERM_WARPS * 32) perm_scatter_kernel(
+    const int32_t* __restrict__ idx, long N, int E, const int32_t* __restrict__ chunk,
+    int32_t* __restrict__ sorted_pair, int32_t* __restrict__ row_of) {
+    __shared__ int32_t wbase[PERM_WARPS][PERM_MAX_E];
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    for (int i = threadIdx.x; i < PERM_WARPS * E; i += blockDim.x) wbase[i / E][i % E] = 0;
+    __syncthreads();
+    const long wstart = (long)blockIdx.x * PERM_CHUNK + (long)w * PERM_PER_WARP;
+    // phase 1: per-warp histogram (leader of each equal-expert lane set adds its size)
+    for (int it = 0; it < PERM_PER_WARP; it += 32) {
+        const long p = wstart + it + lane;
+        const bool valid = p < N;
+        const int e = valid ? idx[p] : -1;
+        const bool ok = valid && e >= 0 && e < E;
+        const unsigned act = __ballot_sync(0xffffffffu, ok);
+        if (ok) {
+            const unsigned m = __match_any_sync(act, e);
+            if ((__ffs(m) - 1) == lane) wbase[w][e] += __popc(m);
+        }
+        __syncwarp();
+    }
+    __syncthreads();
+    // phase 2: warp bases = chunk base + counts of lower warps
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int run = chunk[(size_t)blockIdx.x * E + e];
+        for (int ww = 0; ww < PERM_WARPS; ++ww) {
+            const int n = wbase[ww][e];
+            wbase[ww][e] = run;
+            run += n;
+        }
+    }
+    __syncthreads();
+    // phase 3: stable placement
+    const unsigned lt = (1u << lane) - 1u;
+    for (int it = 0; it < PERM_PER_WARP; it += 32) {
+        const long p = wstart + it + lane;
+        const bool valid = p < N;
+        const int e = valid ? idx[p] : -1;
+        const bool ok = valid && e >= 0 && e < E;
+        const unsigned act = __ballot_sync(0xffffffffu, ok);
+        if (ok) {
+            const unsigned m = __match_any_sync(act, e);
+            const int pos = wbase[w][e] + __popc(m & lt);
+            sorted_pair[pos] = (int32_t)p;
+            row_of[p] = pos;
+            __syncwarp(act);
+            if ((__ffs(m) - 1) == lane) wbase[w][e] += __popc(m);
+        } else if (valid) {
+            row_of[p] = -1;
+        }
+        __syncwarp();
+    }
+}
+
+}  // namespace
+
+int permute_chunks(long N) { return (int)((N + PERM_CHUNK - 1) / PERM_CHUNK); }
+
+cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int n_chunks, int32_t* chunk,
+                           int32_t* offsets, int32_t* sorted_pair, int32_t* row_of,
+                           int32_t* status, cudaStream_t st) {
+    const long N = (long)T * k;
+    if (n_chunks > 0) perm_count_kernel<<<n_chunks, 256, 0, st>>>(idx, N, E, chunk, status);
+    perm_scan_kernel<<<1, 1024, 0, st>>>(chunk, n_chunks, E, offsets);
+    if (n_chunks > 0)
+        perm_scatter_kernel<<<n_chunks, PERM_WARPS * 32, 0, st>>>(idx, N, E, chunk, sorted_pair,
+                                                                   row_of);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,87 @@
+"""Shared helpers of the parity tests: run the CUDA path through the C ABI,
+run the oracle on the same seeded bytes, and compare them by the rules the
+layer fixes (exact routing except oracle-reported near-ties, exact
+permutation, float tolerances)."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import expert_routing_grouped_layer_b200 as moe
+import oracle
+from expert_routing_grouped_layer_b200 import workloads as W
+
+WEIGHT_REL_TOL = 1e-5  # top-k weights: fp32 against float64
+LAYER_TOL = {"bf16": 1e-2, "fp8_e4m3_pow2_b128": 2e-2, "mxfp8": 2e-2}  # rel-L2 of the output
+
+
+def gpu_forward(cfg, inp, wts, T=None):
+    """Run moe_layer_forward; return host copies of the output and intermediates."""
+    T = cfg.T if T is None else T
+    dev = inp["x"].device
+    layer = moe.MoELayer(cfg, wts, inp["gate_w"], inp["gate_bias"], max_tokens=T, device=dev)
+    x = inp["x"][:T].contiguous()
+    out = layer.forward(x)
+    torch.cuda.synchronize()
+    k, E = cfg.num_experts_per_tok, cfg.n_routed_experts
+    res = {
+        "out": out.float().cpu().numpy().astype(np.float64),
+        "idx": layer.intermediate(T, 0, torch.int32, (T, k)).cpu().numpy(),
+        "w": layer.intermediate(T, 1, torch.float32, (T, k)).cpu().numpy(),
+        "offsets": layer.intermediate(T, 2, torch.int32, (E + 1,)).cpu().numpy(),
+        "sorted_pair": layer.intermediate(T, 3, torch.int32, (T * k,)).cpu().numpy(),
+        "row_of": layer.intermediate(T, 4, torch.int32, (T * k,)).cpu().numpy(),
+        "status": int(layer.status.item()),
+    }
+    del layer
+    return res
+
+
+def oracle_route(cfg, inp, tokens=None, T=None):
+    T = cfg.T if T is None else T
+    x = W.bf16_codes(inp["x"][:T])
+    return oracle.route(cfg, x, inp["gate_w"].cpu().numpy(), inp["gate_bias"].cpu().numpy(),
+                        tokens=tokens)
+
+
+def compare_routing(cfg, g, r, tokens):
+    """Expert sets equal and weights within tolerance for every token the oracle
+    does not report as a near-tie. Returns the number of near-tie tokens."""
+    n_tie = 0
+    for i, t in enumerate(tokens):
+        if r["near_tie"][i]:
+            n_tie += 1
+            continue
+        gi, oi = g["idx"][t], r["idx"][i]
+        assert set(gi.tolist()) == set(oi.tolist()), "token %d: gpu %s oracle %s" % (t, gi, oi)
+        gw = dict(zip(gi.tolist(), g["w"][t].tolist()))
+        for e, w in zip(oi.tolist(), r["w"][i].tolist()):
+            assert abs(gw[e] - w) <= WEIGHT_REL_TOL * abs(w), "token %d expert %d" % (t, e)
+    return n_tie
+
+
+def check_permutation_properties(cfg, g, T=None):
+    """The GPU permutation is the stable expert-major sort of the GPU's own
+    topk_idx: this fixes it uniquely, so checking these properties checks it
+    exactly at any size."""
+    T = cfg.T if T is None else T
+    k, E = cfg.num_experts_per_tok, cfg.n_routed_experts
+    flat = g["idx"].reshape(-1).astype(np.int64)
+    N = T * k
+    assert g["offsets"][0] == 0 and g["offsets"][E] == N
+    assert np.array_equal(np.diff(g["offsets"]), np.bincount(flat, minlength=E))
+    sp = g["sorted_pair"].astype(np.int64)
+    assert np.array_equal(np.sort(sp), np.arange(N))
+    assert np.array_equal(g["row_of"][sp], np.arange(N))
+    assert np.array_equal(sp, np.argsort(flat, kind="stable"))
+
+
+def oracle_layer_rows(cfg, inp, wts, idx, w, tokens):
+    """Oracle output for the listed tokens with the oracle's own routing."""
+    x = W.bf16_codes(inp["x"][torch.as_tensor(tokens, dtype=torch.long, device=inp["x"].device)])
+    return oracle.layer(cfg, x, idx, w, lambda e: W.expert_slice(wts, e),
+                        lambda s: W.expert_slice(wts, s, shared=True))
+
+
+def rel_l2(a, b):
+    return float(np.linalg.norm(a - b) / np.linalg.norm(b))
