@@ -30,7 +30,10 @@ AFMT = {"bf16": 0, "fp8_e4m3_pow2_b128": 1, "mxfp8": 2}
 EXPORTS = ("moe_workspace_bytes", "moe_gate_topk", "moe_permute", "moe_quantize_activations",
            "moe_pack_expert_inputs", "moe_expert_gate_up", "moe_expert_down",
            "moe_grouped_swiglu", "moe_combine", "moe_layer_forward", "moe_workspace_offset",
-           "moe_status_string")
+           "moe_status_string", "moe_permute_noalloc")
+
+# capacity (int32 counts) of the static scratch behind moe_permute_noalloc
+MOE_PERMUTE_NOALLOC_MAX_COUNTS = 262144
 
 # moe_workspace_offset selectors
 WS_TOPK_IDX, WS_TOPK_W, WS_OFFSETS, WS_SORTED_PAIR, WS_ROW_OF, WS_Y, WS_SHARED_Y, WS_XA, \
@@ -87,6 +90,8 @@ def lib() -> ctypes.CDLL:
             l.moe_gate_topk.argtypes = [CP, _P, _I32, _P, _P, _P, _P, _P, _SZ, _P]
             l.moe_permute.restype = ctypes.c_int
             l.moe_permute.argtypes = [CP, _P, _I32, _P, _P, _P, _P, _P, _SZ, _P]
+            l.moe_permute_noalloc.restype = ctypes.c_int
+            l.moe_permute_noalloc.argtypes = [CP, _P, _I32, _P, _P, _P, _P, _P]
             l.moe_quantize_activations.restype = ctypes.c_int
             l.moe_quantize_activations.argtypes = [CP, _P, _I32, _P, _P, _P]
             l.moe_pack_expert_inputs.restype = ctypes.c_int
@@ -178,6 +183,17 @@ def moe_permute(cfg, topk_idx, T, expert_offsets, sorted_pair, row_of, dev_statu
     _check(lib().moe_permute(ctypes.byref(_cfg(cfg)), _ptr(topk_idx), int(T), _ptr(expert_offsets),
                              _ptr(sorted_pair), _ptr(row_of), _ptr(dev_status), _ptr(ws), ws_bytes,
                              _stream(stream)), "moe_permute")
+
+
+def moe_permute_noalloc(cfg, topk_idx, T, expert_offsets, sorted_pair, row_of, dev_status,
+                        stream=None):
+    """moe_permute without a workspace, for callers that may not allocate device
+    memory: the library's own fixed 1 MiB device array holds the scratch.
+    Raises MoEError (workspace too small) when ceil(T*k/4096) * n_routed_experts
+    exceeds MOE_PERMUTE_NOALLOC_MAX_COUNTS. Concurrent calls race on that array."""
+    _check(lib().moe_permute_noalloc(ctypes.byref(_cfg(cfg)), _ptr(topk_idx), int(T),
+                                     _ptr(expert_offsets), _ptr(sorted_pair), _ptr(row_of),
+                                     _ptr(dev_status), _stream(stream)), "moe_permute_noalloc")
 
 
 def moe_quantize_activations(cfg, x, T, xq, xq_scale, stream=None):

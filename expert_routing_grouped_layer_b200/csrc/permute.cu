@@ -11,6 +11,8 @@
 //               come from per-warp histograms, and inside a warp the rank of a
 //               pair among equal experts is the count of lower lanes matching
 //               it (__match_any_sync), so pairs keep ascending order.
+#include <mutex>
+
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -155,3 +157,48 @@ cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int n_chunks
 }
 
 }  // namespace moe
+
+// ------------------------------------------------------------------------
+// moe_permute_noalloc: the same three launches, with the per-chunk counts in a
+// file-scope device array instead of a caller workspace, for callers that may
+// not allocate device memory (see include/moe.h). Host code must not pass the
+// array's name to a kernel: on the host that name is only a stand-in, so the
+// device address is looked up once per device with cudaGetSymbolAddress.
+static __device__ __align__(256) int32_t g_permute_noalloc_counts[MOE_PERMUTE_NOALLOC_MAX_COUNTS];
+
+// Device address of the array on the current device (looked up on first use).
+static int32_t* permute_noalloc_scratch() {
+    static std::mutex mu;
+    static int32_t* addr[64] = {nullptr};
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (addr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_permute_noalloc_counts) != cudaSuccess) return nullptr;
+        addr[dev] = static_cast<int32_t*>(p);
+    }
+    return addr[dev];
+}
+
+extern "C" moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* topk_idx,
+                                          int32_t T, int32_t* expert_offsets,
+                                          int32_t* sorted_pair, int32_t* row_of,
+                                          int32_t* dev_status, void* stream) {
+    using namespace moe;
+    if (!config_valid(cfg) || T < 0) return MOE_ERR_INVALID_ARG;
+    if (!expert_offsets) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!topk_idx || !sorted_pair || !row_of)) return MOE_ERR_INVALID_ARG;
+    const long N = (long)T * cfg->num_experts_per_tok;
+    if (N > 0x7fffffffL) return MOE_ERR_INVALID_ARG;
+    const int n_chunks = permute_chunks(N);
+    if ((long)n_chunks * cfg->n_routed_experts > MOE_PERMUTE_NOALLOC_MAX_COUNTS)
+        return MOE_ERR_WORKSPACE;
+    int32_t* counts = permute_noalloc_scratch();
+    if (!counts) return MOE_ERR_CUDA;
+    const cudaError_t e = launch_permute(topk_idx, T, cfg->num_experts_per_tok,
+                                         cfg->n_routed_experts, n_chunks, counts, expert_offsets,
+                                         sorted_pair, row_of, dev_status,
+                                         static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}

@@ -144,6 +144,29 @@ moe_status moe_permute(const moe_config *cfg, const int32_t *topk_idx, int32_t T
                        int32_t *expert_offsets, int32_t *sorted_pair, int32_t *row_of,
                        int32_t *dev_status, void *ws, size_t ws_bytes, void *stream);
 
+/* Permutation for callers that cannot allocate device memory.
+ * No counterpart on the source pages: this is a packaging variant of
+ * moe_permute for callers that are not allowed to allocate -- for example a
+ * plugin running inside a host runtime that owns every device allocation, or a
+ * latency-critical serving loop that may not enter the allocator (cudaMalloc
+ * can synchronise the device). Such callers have no workspace to pass.
+ *
+ * Same arguments, results and device-status behaviour as moe_permute, minus
+ * the workspace: its per-chunk expert counts live in one file-scope device
+ * array of MOE_PERMUTE_NOALLOC_MAX_COUNTS int32 (1 MiB), which every GPU that
+ * loads the library holds until the process exits. Limit: ceil(T*k / 4096) *
+ * n_routed_experts <= MOE_PERMUTE_NOALLOC_MAX_COUNTS, else MOE_ERR_WORKSPACE
+ * and nothing is launched. The call allocates and frees nothing.
+ * The first call on each device looks up the array's device address (with that
+ * device current); make that first call before any stream capture. All calls
+ * share the one array, so calls that overlap on the GPU (other streams, other
+ * threads) race and must be serialised by the caller. Each call writes every
+ * count it later reads, so nothing left from an earlier call is used. */
+#define MOE_PERMUTE_NOALLOC_MAX_COUNTS 262144
+moe_status moe_permute_noalloc(const moe_config *cfg, const int32_t *topk_idx, int32_t T,
+                               int32_t *expert_offsets, int32_t *sorted_pair, int32_t *row_of,
+                               int32_t *dev_status, void *stream);
+
 /* Activation quantisation of the layer input in the config's afmt ([V4]
  * act_quant_kernel; [MX] MXFP8), rows in token order. x bf16 [T][H] -> xq
  * uint8 E4M3 [T][H] and xq_scale uint8 E8M0 codes [T][H/block] (block 128 for
