@@ -34,13 +34,13 @@ UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "k2_decode_bf16"
 L2_FLUSH_BYTES = 256 << 20  # > 2x the 126 MB L2
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNELS_PER_STEP = 9  # router gemm, top-k, 3 permute, gather, gate/up, down, combine
+KERNELS_PER_STEP = 10  # router gemm + split reduce, top-k, 3 permute, gather, gate/up, down, combine
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
@@ -50,7 +50,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
-    ap.add_argument("--cpu-sample-tokens", type=int, default=24)
+    ap.add_argument("--cpu-sample-tokens", type=int, default=128)
     return ap.parse_args()
 
 
@@ -429,7 +429,7 @@ def main():
                                              timeout=datetime.timedelta(seconds=300))
     line, cfg, inp, wts = run_ours(args, rank, world, dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tok = args.cpu_sample_tokens
+        tok = min(args.cpu_sample_tokens, cfg.T)
         times = oracle_timing(cfg, inp, wts, tok, 1, seed=3)
         line["cpu_baseline"] = {"value": tok / times[0], "unit": UNIT, "cores": cpu_cores(),
                                 "kind": "oracle",

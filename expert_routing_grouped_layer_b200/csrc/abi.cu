@@ -51,7 +51,8 @@ bool config_valid(const moe_config* c) {
 moe_status config_supported(const moe_config* c) {
     if (c->n_shared_experts > 0 && c->shared_intermediate_size != c->moe_intermediate_size)
         return MOE_ERR_UNSUPPORTED;
-    if (c->wfmt == MOE_W_BF16 && c->afmt == MOE_A_BF16) return MOE_OK;
+    if (c->afmt == MOE_A_BF16 && (c->wfmt == MOE_W_BF16 || c->wfmt == MOE_W_FP8_E4M3_B128x128))
+        return MOE_OK;
     return MOE_ERR_UNSUPPORTED;
 }
 

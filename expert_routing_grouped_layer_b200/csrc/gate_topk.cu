@@ -7,8 +7,8 @@
 // score, bias, group-limited top-k, normalised and scaled weights.
 //
 // The router GEMM is split along H into `splits` partial sums so a decode batch
-// still fills the GPU; the selection kernel adds the partials in split order,
-// so the logits are deterministic.
+// still fills the GPU; a reduction kernel adds the partials of each logit in
+// split order, so the logits are deterministic.
 #include <cuda_bf16.h>
 
 #include <cfloat>
@@ -123,6 +123,17 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(const __nv_bfloat16* _
             if (e < E) out[(size_t)t * E + e] = acc[i][j];
         }
     }
+}
+
+// logits = sum over splits of the partial sums, added in split order; written
+// over split 0 so the selection kernel reads one slab.
+__global__ void __launch_bounds__(256) router_reduce_kernel(float* __restrict__ part, long n,
+                                                            int splits) {
+    const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    float l = 0.f;
+    for (int s = 0; s < splits; ++s) l += part[(size_t)s * n + i];
+    part[i] = l;
 }
 
 __device__ __forceinline__ float score_of(float l, int score_fn) {
@@ -262,12 +273,16 @@ cudaError_t launch_router_gemm(const void* x, const float* gate_w, float* part, 
     dim3 grid((T + RG_BM - 1) / RG_BM, (E + RG_BN - 1) / RG_BN, splits);
     router_gemm_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), gate_w, part, T,
                                              E, H, per);
+    if (splits > 1) {
+        const long n = (long)T * E;
+        router_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(part, n, splits);
+    }
     return cudaGetLastError();
 }
 
 int router_splits_for(int T, int E, int H) {
     const int tiles = ((T + RG_BM - 1) / RG_BM) * ((E + RG_BN - 1) / RG_BN);
-    const int target = 2 * num_sms();
+    const int target = num_sms();  // one wave: the kernel fits one CTA per SM
     int s = (target + tiles - 1) / tiles;
     const int max_s = (H / RG_BK) / 4;  // at least 4 k-steps per split
     if (s > max_s) s = max_s;
@@ -284,7 +299,7 @@ cudaError_t launch_topk(const moe_config* c, const float* part, int splits, cons
     if (T == 0) return cudaSuccess;
     TopkParams p;
     p.part = part;
-    p.splits = splits;
+    p.splits = 1;  // launch_router_gemm left the summed logits in split 0
     p.bias = bias;
     p.T = T;
     p.E = c->n_routed_experts;
