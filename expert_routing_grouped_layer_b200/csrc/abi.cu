@@ -53,6 +53,12 @@ moe_status config_supported(const moe_config* c) {
         return MOE_ERR_UNSUPPORTED;
     if (c->afmt == MOE_A_BF16 && (c->wfmt == MOE_W_BF16 || c->wfmt == MOE_W_FP8_E4M3_B128x128))
         return MOE_OK;
+    // block-scaled tensor cores: E2M1 weights x E4M3 activations; the scale tiles
+    // move by TMA in rows of 16 scales, so H and I must be multiples of 512
+    if ((c->wfmt == MOE_W_FP4_E2M1_UE8M0_B32 || c->wfmt == MOE_W_MXFP4) &&
+        (c->afmt == MOE_A_FP8_E4M3_POW2_B128 || c->afmt == MOE_A_MXFP8) && c->hidden % 512 == 0 &&
+        c->moe_intermediate_size % 512 == 0)
+        return MOE_OK;
     return MOE_ERR_UNSUPPORTED;
 }
 
@@ -64,7 +70,6 @@ WsLayout ws_layout(const moe_config* c, int T) {
     const size_t I = c->moe_intermediate_size, S = c->n_shared_experts;
     const size_t N = (size_t)T * k;
     const size_t act_bytes = (c->afmt == MOE_A_BF16) ? 2 : 1;
-    const size_t blk = (c->afmt == MOE_A_MXFP8) ? 32 : 128;
     L.router_splits = T > 0 ? router_splits_for(T, (int)E, (int)H) : 1;
     L.n_chunks = permute_chunks((long)N);
     size_t off = 0;
@@ -81,9 +86,9 @@ WsLayout ws_layout(const moe_config* c, int T) {
     L.row_of = take(N * 4);
     L.chunk_counts = take((size_t)L.n_chunks * E * 4);
     L.xa = take((N + T) * H * act_bytes);
-    L.xa_scale = take(act_bytes == 1 ? (N + T) * (H / blk) : 0);
+    L.xa_scale = take(act_bytes == 1 ? (N + T) * (H / 32) : 0);
     L.hbuf = take((N + S * T) * I * act_bytes);
-    L.h_scale = take(act_bytes == 1 ? (N + S * T) * (I / blk) : 0);
+    L.h_scale = take(act_bytes == 1 ? (N + S * T) * (I / 32) : 0);
     L.y = take(N * H * 2);
     L.shared_y = take(S * T * H * 2);
     L.total = off;
@@ -182,7 +187,7 @@ moe_status moe_quantize_activations(const moe_config* cfg, const void* x, int32_
     if (!x || !xq || !xq_scale || !aligned16(x) || !aligned16(xq)) return MOE_ERR_INVALID_ARG;
     return cuda_status(launch_pack_rows(cfg->afmt, x, cfg->hidden, nullptr, 0,
                                         cfg->num_experts_per_tok, T, T, xq,
-                                        static_cast<uint8_t*>(xq_scale), as_stream(stream)));
+                                        static_cast<uint8_t*>(xq_scale), 0, as_stream(stream)));
 }
 
 static bool weights_ok(const moe_config* cfg, const moe_weights* w, bool gate_up) {
@@ -222,7 +227,7 @@ moe_status moe_pack_expert_inputs(const moe_config* cfg, const void* x, int32_t 
     if (cfg->afmt != MOE_A_BF16 && !xa_scale) return MOE_ERR_INVALID_ARG;
     const int k = cfg->num_experts_per_tok, N = T * k;
     return cuda_status(launch_pack_rows(cfg->afmt, x, cfg->hidden, sorted_pair, N, k, T, N + T, xa,
-                                        static_cast<uint8_t*>(xa_scale), as_stream(stream)));
+                                        static_cast<uint8_t*>(xa_scale), 1, as_stream(stream)));
 }
 
 moe_status moe_expert_gate_up(const moe_config* cfg, const void* xa, const void* xa_scale,
@@ -238,7 +243,6 @@ moe_status moe_expert_gate_up(const moe_config* cfg, const void* xa, const void*
     if (!weights_ok(cfg, w, true)) return MOE_ERR_INVALID_ARG;
     GroupedGemmArgs a = gemm_args(cfg, T, expert_offsets, dev_status);
     const size_t hrow = (size_t)a.I * (q ? 1 : 2);
-    const size_t blk = (cfg->afmt == MOE_A_MXFP8) ? 32 : 128;
     a.gemm = 1;
     a.w_routed = w->w13;
     a.w_routed_scale = w->w13_scale;
@@ -249,7 +253,7 @@ moe_status moe_expert_gate_up(const moe_config* cfg, const void* xa, const void*
     a.out_routed = h;
     a.out_shared = static_cast<char*>(h) + (size_t)a.N * hrow;
     a.out_routed_scale = static_cast<uint8_t*>(h_scale);
-    a.out_shared_scale = q ? static_cast<uint8_t*>(h_scale) + (size_t)a.N * (a.I / blk) : nullptr;
+    a.out_shared_scale = q ? static_cast<uint8_t*>(h_scale) + (size_t)a.N * (a.I / 32) : nullptr;
     return cuda_status(launch_grouped_gemm(a, as_stream(stream)));
 }
 

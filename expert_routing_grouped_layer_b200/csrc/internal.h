@@ -20,9 +20,9 @@ struct WsLayout {
     size_t row_of;        // int32 [N]
     size_t chunk_counts;  // int32 [n_chunks][E]
     size_t xa;            // gathered expert input rows [(N+T)][H] (bf16 or e4m3)
-    size_t xa_scale;      // uint8 [(N+T)][H/blk]
+    size_t xa_scale;      // uint8 E8M0 [(N+T)][H/32]
     size_t hbuf;          // intermediate [(N+S*T)][I] (bf16 or e4m3)
-    size_t h_scale;       // uint8 [(N+S*T)][I/blk]
+    size_t h_scale;       // uint8 E8M0 [(N+S*T)][I/32]
     size_t y;             // bf16 [N][H]
     size_t shared_y;      // bf16 [S][T][H]
     size_t total;
@@ -44,7 +44,7 @@ cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int n_chunks
                            int32_t* offsets, int32_t* sorted_pair, int32_t* row_of,
                            int32_t* status, cudaStream_t st);
 cudaError_t launch_pack_rows(int afmt, const void* x, int H, const int32_t* sorted_pair, int N,
-                             int k, int T, int n_rows, void* out, uint8_t* out_scale,
+                             int k, int T, int n_rows, void* out, uint8_t* out_scale, int per32,
                              cudaStream_t st);
 cudaError_t launch_combine(const void* y, const void* shared_y, int S, const int32_t* row_of,
                            const float* w, int T, int k, int H, void* out, cudaStream_t st);

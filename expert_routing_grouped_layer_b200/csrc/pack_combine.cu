@@ -75,20 +75,24 @@ __device__ __forceinline__ int mx_scale_exp(float a) {
 
 // One warp per row; 4 elements per lane per step (a 128-element block for the
 // power-of-two format, four 32-element blocks for MX).
+// per32: write one scale code per 32 elements (a 128-element block's code is
+// repeated over its four 32-element sub-blocks), the layout the block-scaled
+// tensor-core GEMM reads; otherwise one code per block.
 template <int AFMT>
 __global__ void __launch_bounds__(256) pack_fp8_kernel(const __nv_bfloat16* __restrict__ x, int H,
                                                        const int32_t* __restrict__ sorted_pair,
                                                        int N, int k, int T, int n_rows,
                                                        uint8_t* __restrict__ out,
-                                                       uint8_t* __restrict__ out_scale) {
+                                                       uint8_t* __restrict__ out_scale, int per32) {
     constexpr int BLK = (AFMT == MOE_A_FP8_E4M3_POW2_B128) ? 128 : 32;
+    const int SBLK = per32 ? 32 : BLK;  // elements per stored scale
     const int lane = threadIdx.x & 31;
     const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
     if (r >= n_rows) return;
     const int t = token_of_row(r, sorted_pair, N, k, T);
     const __nv_bfloat16* src = x + (size_t)(t < 0 ? 0 : t) * H;
     uint8_t* dst = out + (size_t)r * H;
-    uint8_t* dsc = out_scale + (size_t)r * (H / BLK);
+    uint8_t* dsc = out_scale + (size_t)r * (H / SBLK);
     for (int c0 = 0; c0 < H; c0 += 128) {
         uint2 raw = make_uint2(0, 0);
         if (t >= 0) raw = *reinterpret_cast<const uint2*>(src + c0 + lane * 4);
@@ -109,7 +113,7 @@ __global__ void __launch_bounds__(256) pack_fp8_kernel(const __nv_bfloat16* __re
             __nv_cvt_float2_to_fp8x2(make_float2(f23.x * inv, f23.y * inv), __NV_SATFINITE, __NV_E4M3);
         const uint32_t packed = (uint32_t)q01 | ((uint32_t)q23 << 16);
         *reinterpret_cast<uint32_t*>(dst + c0 + lane * 4) = packed;
-        if ((lane % LANES) == 0) dsc[(c0 + lane * 4) / BLK] = (uint8_t)(e + 127);
+        if ((lane % (SBLK / 4)) == 0) dsc[(c0 + lane * 4) / SBLK] = (uint8_t)(e + 127);
     }
 }
 
@@ -166,7 +170,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const __nv_bfloat16* __res
 }  // namespace
 
 cudaError_t launch_pack_rows(int afmt, const void* x, int H, const int32_t* sorted_pair, int N,
-                             int k, int T, int n_rows, void* out, uint8_t* out_scale,
+                             int k, int T, int n_rows, void* out, uint8_t* out_scale, int per32,
                              cudaStream_t st) {
     if (n_rows == 0) return cudaSuccess;
     dim3 grid((n_rows + 7) / 8);
@@ -176,11 +180,12 @@ cudaError_t launch_pack_rows(int afmt, const void* x, int H, const int32_t* sort
     else if (afmt == MOE_A_FP8_E4M3_POW2_B128)
         pack_fp8_kernel<MOE_A_FP8_E4M3_POW2_B128><<<grid, 256, 0, st>>>(
             static_cast<const __nv_bfloat16*>(x), H, sorted_pair, N, k, T, n_rows,
-            static_cast<uint8_t*>(out), out_scale);
+            static_cast<uint8_t*>(out), out_scale, per32);
     else
         pack_fp8_kernel<MOE_A_MXFP8><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), H,
                                                            sorted_pair, N, k, T, n_rows,
-                                                           static_cast<uint8_t*>(out), out_scale);
+                                                           static_cast<uint8_t*>(out), out_scale,
+                                                           per32);
     return cudaGetLastError();
 }
 

@@ -179,7 +179,8 @@ moe_status moe_quantize_activations(const moe_config *cfg, const void *x, int32_
  * moe_permute. Row r < N of xa holds token sorted_pair[r] / k of x, rows N..N+T-1
  * hold the tokens in order (the shared experts' input). xa is bf16 [N+T][H]
  * for BF16 activations, else uint8 E4M3 [N+T][H] with xa_scale uint8 E8M0
- * [N+T][H/block] (xa_scale unused for BF16). */
+ * [N+T][H/32]: one code per 32 elements, the power-of-two format's per-128 code
+ * repeated over its four 32-element sub-blocks (xa_scale unused for BF16). */
 moe_status moe_pack_expert_inputs(const moe_config *cfg, const void *x, int32_t T,
                                   const int32_t *sorted_pair, void *xa, void *xa_scale,
                                   void *stream);
@@ -190,7 +191,9 @@ moe_status moe_pack_expert_inputs(const moe_config *cfg, const void *x, int32_t 
  *   a = SiLU(W1 xa[r]) * (W3 xa[r])   (fp32 accumulation on the tensor cores)
  * written to h as bf16 (BF16 activations) or E4M3 + E8M0 block scales along I
  * (quantised activations). h is [N + S*T][I]: rows 0..N-1 follow xa, rows
- * N + s*T + t belong to shared expert s and token t; h_scale [N + S*T][I/block].
+ * N + s*T + t belong to shared expert s and token t; h_scale [N + S*T][I/32]
+ * (one E8M0 code per 32 features, per-128 codes repeated as for xa_scale).
+ * E2M1 / MXFP4 weights need E4M3 activations and H, I multiples of 512.
  * A pipeline wait past its time limit sets MOE_DEV_TIMEOUT. */
 moe_status moe_expert_gate_up(const moe_config *cfg, const void *xa, const void *xa_scale,
                               int32_t T, const int32_t *expert_offsets, const moe_weights *w,

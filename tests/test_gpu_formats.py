@@ -65,3 +65,86 @@ def test_fp8_weights_group_limited_prefill_full_size():
     m = counts.mean()
     # the workload's balanced recipe: every expert within 20% of the mean load
     assert counts.min() >= 0.8 * m and counts.max() <= 1.2 * m
+
+
+# ----------------------------------------------------------- activation quantisers
+def _x_with_edge_cases(T, H, seed):
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    x = torch.randn(T, H, generator=g, device="cuda") * torch.exp2(
+        torch.randint(-20, 20, (T, 1), generator=g, device="cuda").float())
+    x[0, :128] = 0.0  # an all-zero block
+    x[1, :32] = 448.0 * 2.0 ** 3  # exact power-of-two edge
+    x[2, 5] = 3.0e38  # near the top of the bf16 range
+    x[3, :64] = 1.0e-39  # subnormal block
+    return x.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("afmt,blk", [("fp8_e4m3_pow2_b128", 128), ("mxfp8", 32)])
+def test_quantize_activations_bit_exact(afmt, blk):
+    cfg = W.CONFIGS["tiny_bf16"].replace(hidden=1024, afmt=afmt, wfmt="mxfp4")
+    T, H = 40, cfg.hidden
+    x = _x_with_edge_cases(T, H, 3)
+    xq = torch.empty(T, H, dtype=torch.uint8, device="cuda")
+    xs = torch.empty(T, H // blk, dtype=torch.uint8, device="cuda")
+    moe.moe_quantize_activations(cfg, x, T, xq, xs)
+    torch.cuda.synchronize()
+    _, q_ref, s_ref = oracle.expert_input(afmt, W.bf16_codes(x))
+    assert np.array_equal(xs.cpu().numpy(), s_ref)
+    assert np.array_equal(xq.cpu().numpy(), q_ref)
+
+
+@pytest.mark.parametrize("afmt,blk", [("fp8_e4m3_pow2_b128", 128), ("mxfp8", 32)])
+def test_pack_expert_inputs_gathers_and_repeats_scales(afmt, blk):
+    cfg = W.CONFIGS["tiny_bf16"].replace(hidden=1024, afmt=afmt, wfmt="mxfp4")
+    T, k, H = 24, cfg.num_experts_per_tok, cfg.hidden
+    N = T * k
+    x = _x_with_edge_cases(T, H, 4)
+    g = torch.Generator(device="cuda").manual_seed(5)
+    sp = torch.randperm(N, generator=g, device="cuda").to(torch.int32)
+    xa = torch.empty(N + T, H, dtype=torch.uint8, device="cuda")
+    xs = torch.empty(N + T, H // 32, dtype=torch.uint8, device="cuda")
+    moe.moe_pack_expert_inputs(cfg, x, T, sp, xa, xs)
+    torch.cuda.synchronize()
+    _, q_ref, s_ref = oracle.expert_input(afmt, W.bf16_codes(x))
+    tok = np.concatenate([sp.cpu().numpy() // k, np.arange(T)])
+    assert np.array_equal(xa.cpu().numpy(), q_ref[tok])
+    assert np.array_equal(xs.cpu().numpy(), np.repeat(s_ref[tok], blk // 32, axis=1))
+
+
+# ----------------------------------------------------------- block-scaled layers
+FP4_TINY = W.CONFIGS["tiny_bf16"].replace(
+    hidden=512, moe_intermediate_size=512, shared_intermediate_size=512,
+    wfmt="fp4_e2m1_ue8m0_b32", afmt="fp8_e4m3_pow2_b128", score_fn="sqrtsoftplus",
+    routed_scaling_factor=2.5)
+MX_TINY = W.CONFIGS["tiny_bf16"].replace(
+    hidden=512, moe_intermediate_size=512, shared_intermediate_size=512, wfmt="mxfp4",
+    afmt="mxfp8", n_shared_experts=2)
+
+
+@pytest.mark.parametrize("cfg", [FP4_TINY, MX_TINY], ids=["fp4_pow2", "mx"])
+def test_block_scaled_tiny(cfg):
+    _layer_check(cfg)
+
+
+@pytest.mark.parametrize("cfg", [FP4_TINY, MX_TINY], ids=["fp4_pow2", "mx"])
+def test_block_scaled_several_tiles_ragged(cfg):
+    # ~260 rows per expert: several 64- and 128-token tiles with ragged ends,
+    # H = 1024 -> 8 down-projection tiles and 8 K stages of the gate/up GEMM
+    _layer_check(cfg.replace(T=700, hidden=1024, n_routed_experts=8, num_experts_per_tok=3))
+
+
+@pytest.mark.parametrize("T", [1, 13])
+def test_block_scaled_few_tokens(T):
+    _layer_check(MX_TINY, T=T)
+
+
+def test_v4_fp4_full_size():
+    cfg = W.CONFIGS["v4_fp4"]
+    _layer_check(cfg, sample=8, seed=2)
+
+
+def test_mx896_full_size_zipf():
+    cfg = W.CONFIGS["mx896"]
+    g, _ = _layer_check(cfg, sample=6, seed=3)
+    counts = np.diff(g["offsets"])
+    assert counts.max() > 10 * counts.mean()  # hot experts take >10x the mean
