@@ -152,7 +152,7 @@ def layer_flops(cfg, T):
     return 2.0 * (N + T * cfg.n_shared_experts) * 3 * cfg.hidden * cfg.moe_intermediate_size
 
 
-def ncu_traffic(kernel: str):
+def ncu_traffic(kernel: str, workload: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
     the current source of the kernel (else None)."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
@@ -161,11 +161,30 @@ def ncu_traffic(kernel: str):
     with open(p) as f:
         d = json.load(f)
     e = d.get(kernel)
-    if not e:
+    if not e or e.get("workload") != workload:
         return None
-    src = os.path.join(ROOT, e["source"])
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    return e["dram_bytes_per_launch"] if h == e["source_sha256_16"] else None
+    h = hashlib.sha256()
+    for src in e["sources"]:
+        with open(os.path.join(ROOT, src), "rb") as f:
+            h.update(f.read())
+    return e["dram_bytes_per_launch"] if h.hexdigest()[:16] == e["source_sha256_16"] else None
+
+
+# ------------------------------------------------------------------ ranks
+def max_over_ranks(value: float, device) -> float:
+    """Max of a per-rank timing over all ranks (identity on a single process)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_seed(seed: int, rank: int) -> int:
+    """Token seed of a replica: rank 0 runs the workload's own batch."""
+    return seed if rank == 0 else seed + 7919 * rank
 
 
 # ------------------------------------------------------------------ our arm
@@ -183,7 +202,7 @@ def run_ours(args, rank, world, dev):
                         cfg.moe_intermediate_size, cfg.n_shared_experts)
     inp = W.make_inputs(cfg, dev)
     if rank > 0:  # replicas: same model, each rank its own tokens
-        inp["x"] = W.make_inputs(cfg.replace(seed=cfg.seed + 7919 * rank), dev)["x"]
+        inp["x"] = W.make_inputs(cfg.replace(seed=replica_seed(cfg.seed, rank)), dev)["x"]
     wts = W.make_weights(cfg, dev)
     torch.cuda.synchronize()
 
@@ -247,11 +266,7 @@ def run_ours(args, rank, world, dev):
     stage = [[events[i][j].elapsed_time(events[i][j + 1]) for i in range(args.steps)]
              for j in range(6)]
     step_ms = [sum(stage[j][i] for j in range(6)) for i in range(args.steps)]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dev)
     offsets = layer.intermediate(T, moe.WS_OFFSETS, torch.int32, (E + 1,)).cpu()
     active = int((offsets[1:] - offsets[:-1] > 0).sum())
 
@@ -276,11 +291,7 @@ def run_ours(args, rank, world, dev):
             oh.copy_(layer.forward(xd), non_blocking=True)
         s1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = s0.elapsed_time(s1) / n_e2e
-        if world > 1:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(s0.elapsed_time(s1) / n_e2e, dev)
         e2e = {"value": world * T / (e2e_ms / 1e3), "unit": UNIT,
                "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2,
                "ms_per_step": e2e_ms, "includes_l2_flush": True}
@@ -318,7 +329,8 @@ def run_ours(args, rank, world, dev):
                    "l2": "256 MiB write before every timed step, outside the timed events"},
         "roofline": {"bound": "hbm", "kernel": "gate_up (grouped SwiGLU GEMM1)",
                      "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                     "peak_source": peak_src, "traffic": ncu_traffic("gate_up"),
+                     "peak_source": peak_src, "traffic": ncu_traffic("gate_up", args.workload)
+                     if not (args.tokens or args.experts) else None,
                      "algorithmic_bytes_per_launch": gu_bytes},
         "layer_roofline": {"bound": "hbm", "bytes": lb, "achieved_gbs": lb / (ms / 1e3) / 1e9,
                            "frac": lb / (ms / 1e3) / 1e9 / hbm,

@@ -1,0 +1,286 @@
+// gemm_fp8w.cu -- per-expert SwiGLU MLP with FP8 (E4M3, 128x128 block-scaled)
+// weights and bf16 activations on the tcgen05 tensor cores. The expert
+// structure, tile schedule and epilogue are those of gemm_bf16.cu.
+#include "gemm_common.cuh"
+
+namespace moe {
+namespace gemm {
+namespace {
+
+// ---------------------------------------------------------------- FP8 weights
+// E4M3 weights with one fp32 scale per 128x128 block ("DeepSeek-V4-Pro 架构与代码概述",
+// 文件说明: Linear with block-scaled FP8 weights; block 128x128). The activations
+// stay bf16, so the tensor-core operands are bf16: a converter warpgroup turns
+// each TMA-staged E4M3 weight tile (64-byte swizzled rows) into bf16 values
+// times the tile's block scale, written straight into the 128B-swizzled
+// K-major layout tcgen05.mma reads. With BK = 64 inside a 128-wide scale block
+// and M tiles aligned to the 128-row blocks, one scalar scale covers a tile.
+// E4M3 -> bf16 is exact; the product with the fp32 scale is rounded once to
+// bf16 (relative error <= 2^-9 per weight).
+constexpr int CVT_WARPS = 8;
+constexpr int CVT_THREADS = CVT_WARPS * 32;
+constexpr int F8_THREADS = 64 + 128 + CVT_THREADS;
+
+template <int GEMM>
+struct TileF8 {
+    static constexpr int NA = (GEMM == 1) ? 2 : 1;
+    static constexpr int A8_BYTES = BM * BK;      // e4m3 staging tile
+    static constexpr int A_BYTES = BM * BK * 2;   // bf16 MMA tile
+    static constexpr int B_BYTES = BN * BK * 2;
+    static constexpr int CVT_OFF = 0;                       // NA bf16 A tiles
+    static constexpr int B_OFF = NA * A_BYTES;              // token tile
+    static constexpr int A8_OFF = B_OFF + B_BYTES;          // NA e4m3 tiles
+    static constexpr int STAGE_BYTES = A8_OFF + NA * A8_BYTES;
+    static constexpr int STAGES = (GEMM == 1) ? 3 : 5;
+    static constexpr int ACC_COLS = NA * BN;
+    static constexpr int TMEM_COLS = 2 * ACC_COLS;
+    static constexpr int BAR_BYTES = 8 * (4 * STAGES + 5) + 16;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + 4 * (MAX_SEG + 1);
+};
+
+// 16 E4M3 values -> 16 bf16 values of (value * scale), in element order.
+__device__ __forceinline__ void e4m3x16_to_bf16_scaled(uint4 v, float scale, uint4& lo, uint4& hi) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const __nv_fp8x2_storage_t pair = (__nv_fp8x2_storage_t)((w[i] >> (16 * h)) & 0xFFFFu);
+            const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+            const __nv_bfloat162 b = __floats2bfloat162_rn(f.x * scale, f.y * scale);
+            o[2 * i + h] = *reinterpret_cast<const uint32_t*>(&b);
+        }
+    }
+    lo = make_uint4(o[0], o[1], o[2], o[3]);
+    hi = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+template <int GEMM>
+__global__ void __launch_bounds__(F8_THREADS, 1)
+    grouped_gemm_fp8w_kernel(const __grid_constant__ CUtensorMap tmA_routed,
+                             const __grid_constant__ CUtensorMap tmA_shared,
+                             const __grid_constant__ CUtensorMap tmB, const KParams p,
+                             const float* __restrict__ scale_routed,
+                             const float* __restrict__ scale_shared) {
+    using C = TileF8<GEMM>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t* raw_full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+    uint64_t* raw_empty = raw_full + C::STAGES;
+    uint64_t* cvt_full = raw_empty + C::STAGES;
+    uint64_t* cvt_empty = cvt_full + C::STAGES;
+    uint64_t* tfull = cvt_empty + C::STAGES;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* mma_done = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* pref = reinterpret_cast<int*>(tmem_slot + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&raw_full[s], 1);
+            mbar_init(&raw_empty[s], 1 + CVT_THREADS);  // MMA commit + every converter thread
+            mbar_init(&cvt_full[s], CVT_THREADS);
+            mbar_init(&cvt_empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], 128);
+        }
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&tmA_routed);
+        tma_prefetch_desc(&tmA_shared);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    const int MT = p.M / BM;
+    if (warp == 1) build_schedule(p, pref, MT, lane);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int total = pref[p.nseg];
+    const int KB = p.K / BK;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued = 0;
+            for (int u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x) {
+                const Unit t = decode_unit(p, pref, u);
+                const int n_mma = (t.n_valid + 15) & ~15;
+                const int nb = n_mma / B_BOX;
+                const uint32_t tx = C::NA * C::A8_BYTES + nb * B_BOX * BK * 2;
+                const CUtensorMap* tmA = (t.seg < p.E) ? &tmA_routed : &tmA_shared;
+                bool ok = true;
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(&raw_empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+                    uint8_t* st = smem + stage * C::STAGE_BYTES;
+                    mbar_arrive_expect_tx(&raw_full[stage], tx);
+                    tma_load_2d(st + C::A8_OFF, tmA, kb * BK, t.a_row, &raw_full[stage]);
+                    if (GEMM == 1)
+                        tma_load_2d(st + C::A8_OFF + C::A8_BYTES, tmA, kb * BK,
+                                    t.a_row + p.a_up_offset, &raw_full[stage]);
+                    for (int i = 0; i < nb; ++i)
+                        tma_load_2d(st + C::B_OFF + i * B_BOX * BK * 2, &tmB, kb * BK,
+                                    t.b_row + i * B_BOX, &raw_full[stage]);
+                    ++issued;
+                    if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+            }
+            if (*abort_flag) {
+                int s = stage;
+                uint32_t ph = phase;
+                for (int i = 0; i < min(issued, C::STAGES); ++i) {
+                    if (--s < 0) { s = C::STAGES - 1; ph ^= 1; }
+                    volatile int no_abort = 0;
+                    mbar_wait(&raw_full[s], ph, &no_abort);
+                }
+                status_or(p.status, MOE_DEV_TIMEOUT);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            for (int u = blockIdx.x; u < total; u += gridDim.x) {
+                const Unit t = decode_unit(p, pref, u);
+                const int n_mma = (t.n_valid + 15) & ~15;
+                const uint32_t idesc = idesc_bf16(BM, n_mma);
+                if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t d0 = tmem_base + acc * C::ACC_COLS;
+                bool ok = true;
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(&raw_full[stage], phase, abort_flag) ||
+                        !mbar_wait(&cvt_full[stage], phase, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t st = smem_u32(smem + stage * C::STAGE_BYTES);
+                    const uint32_t sb = st + C::B_OFF;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        const uint32_t acc_flag = (kb | kk) != 0;
+                        const uint64_t bd = sdesc_kmajor_sw128(sb + kk * 32);
+                        mma_bf16(d0, sdesc_kmajor_sw128(st + C::CVT_OFF + kk * 32), bd, idesc, acc_flag);
+                        if (GEMM == 1)
+                            mma_bf16(d0 + BN, sdesc_kmajor_sw128(st + C::CVT_OFF + C::A_BYTES + kk * 32),
+                                     bd, idesc, acc_flag);
+                    }
+                    mma_commit(&raw_empty[stage]);
+                    mma_commit(&cvt_empty[stage]);
+                    if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                mma_commit(&tfull[acc]);
+                if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+            }
+            mma_commit(mma_done);
+            volatile int no_abort = 0;
+            mbar_wait(mma_done, 0, &no_abort);
+            if (*abort_flag) status_or(p.status, MOE_DEV_TIMEOUT);
+        }
+    } else if (warp < 6) {
+        epilogue_loop<GEMM, C::ACC_COLS>(p, pref, total, tmem_base, tfull, tempty, abort_flag,
+                                         warp, lane);
+    } else {
+        // converters: e4m3 staging tile -> scaled bf16 MMA tile
+        const int ct = threadIdx.x - 192;
+        const int KS = p.K / 128;  // scale blocks along K
+        const int RS = p.a_rows_per_mat / 128;
+        int stage = 0;
+        uint32_t phase = 0;
+        for (int u = blockIdx.x; u < total; u += gridDim.x) {
+            const Unit t = decode_unit(p, pref, u);
+            const bool routed = t.seg < p.E;
+            const int mat = routed ? t.seg : t.seg - p.E;
+            const float* sbase = (routed ? scale_routed : scale_shared) + (size_t)mat * RS * KS;
+            const float* s_gate = sbase + (size_t)(t.mt) * KS;
+            const float* s_up = sbase + (size_t)(p.a_up_offset / 128 + t.mt) * KS;
+            bool ok = true;
+            for (int kb = 0; kb < KB; ++kb) {
+                if (!mbar_wait(&raw_full[stage], phase, abort_flag) ||
+                    !mbar_wait(&cvt_empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+                uint8_t* st = smem + stage * C::STAGE_BYTES;
+                const float sc[2] = {s_gate[kb >> 1], GEMM == 1 ? s_up[kb >> 1] : 0.f};
+#pragma unroll
+                for (int i = 0; i < C::NA * 512 / CVT_THREADS; ++i) {
+                    const int task = ct + i * CVT_THREADS;
+                    const int tile = task >> 9;
+                    const int r = task & 127;
+                    const int c = (task >> 7) & 3;
+                    const uint8_t* src = st + C::A8_OFF + tile * C::A8_BYTES + r * 64 +
+                                         ((c ^ ((r >> 1) & 3)) << 4);
+                    uint8_t* dst = st + C::CVT_OFF + tile * C::A_BYTES + r * 128;
+                    uint4 lo, hi;
+                    e4m3x16_to_bf16_scaled(*reinterpret_cast<const uint4*>(src), sc[tile], lo, hi);
+                    *reinterpret_cast<uint4*>(dst + (((2 * c) ^ (r & 7)) << 4)) = lo;
+                    *reinterpret_cast<uint4*>(dst + (((2 * c + 1) ^ (r & 7)) << 4)) = hi;
+                }
+                fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
+                mbar_arrive(&cvt_full[stage]);
+                mbar_arrive(&raw_empty[stage]);
+                if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+            }
+            if (!ok) break;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+
+}  // namespace
+
+template <int GEMM>
+cudaError_t launch_fp8w(const GroupedGemmArgs& a, cudaStream_t st) {
+    using C = TileF8<GEMM>;
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(grouped_gemm_fp8w_kernel<GEMM>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    uint64_t b_rows;
+    const KParams p = make_params(a, GEMM, &b_rows);
+    CUtensorMap tmAr, tmAs, tmB;
+    const int S = a.S;
+    if (!make_tmap_u8_sw64(&tmAr, a.w_routed, (uint64_t)a.E * p.a_rows_per_mat, p.K, BM))
+        return cudaErrorInvalidValue;
+    if (!make_tmap_u8_sw64(&tmAs, S > 0 ? a.w_shared : a.w_routed,
+                           (uint64_t)(S > 0 ? S : a.E) * p.a_rows_per_mat, p.K, BM))
+        return cudaErrorInvalidValue;
+    if (b_rows == 0) return cudaSuccess;
+    if (!make_tmap_bf16(&tmB, a.b_rows, b_rows, p.K, B_BOX)) return cudaErrorInvalidValue;
+    grouped_gemm_fp8w_kernel<GEMM><<<grid_for(p), F8_THREADS, C::SMEM_BYTES, st>>>(
+        tmAr, tmAs, tmB, p, static_cast<const float*>(a.w_routed_scale),
+        static_cast<const float*>(S > 0 ? a.w_shared_scale : a.w_routed_scale));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_fp8w(const GroupedGemmArgs& a, cudaStream_t st) {
+    return a.gemm == 1 ? launch_fp8w<1>(a, st) : launch_fp8w<2>(a, st);
+}
+
+}  // namespace gemm
+}  // namespace moe
