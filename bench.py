@@ -34,7 +34,7 @@ UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "k2_decode_bf16"
 L2_FLUSH_BYTES = 256 << 20  # > 2x the 126 MB L2
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNELS_PER_STEP = 10  # router gemm + split reduce, top-k, 3 permute, gather, gate/up, down, combine
+KERNELS_PER_STEP = 11  # router split + gemm + reduce, top-k, 3 permute, gather, gate/up, down, combine
 
 
 def parse():
@@ -218,7 +218,7 @@ def run_ours(args, rank, world, dev):
     def step(ev):
         ev[0].record(stream)
         moe.moe_gate_topk(ccfg, x, T, inp["gate_w"], inp["gate_bias"], P(moe.WS_TOPK_IDX),
-                          P(moe.WS_TOPK_W), ws, wsb, stream=sp)
+                          P(moe.WS_TOPK_W), ws, st, wsb, stream=sp)
         ev[1].record(stream)
         moe.moe_permute(ccfg, P(moe.WS_TOPK_IDX), T, P(moe.WS_OFFSETS), P(moe.WS_SORTED_PAIR),
                         P(moe.WS_ROW_OF), st, ws, wsb, stream=sp)

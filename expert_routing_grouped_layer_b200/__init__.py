@@ -87,7 +87,7 @@ def lib() -> ctypes.CDLL:
             l.moe_status_string.restype = ctypes.c_char_p
             l.moe_status_string.argtypes = [ctypes.c_int]
             l.moe_gate_topk.restype = ctypes.c_int
-            l.moe_gate_topk.argtypes = [CP, _P, _I32, _P, _P, _P, _P, _P, _SZ, _P]
+            l.moe_gate_topk.argtypes = [CP, _P, _I32, _P, _P, _P, _P, _P, _P, _SZ, _P]
             l.moe_permute.restype = ctypes.c_int
             l.moe_permute.argtypes = [CP, _P, _I32, _P, _P, _P, _P, _P, _SZ, _P]
             l.moe_permute_noalloc.restype = ctypes.c_int
@@ -170,11 +170,12 @@ def moe_workspace_offset(cfg, T: int, which: int) -> int:
     return lib().moe_workspace_offset(ctypes.byref(_cfg(cfg)), int(T), int(which))
 
 
-def moe_gate_topk(cfg, x, T, gate_w, gate_bias, topk_idx, topk_w, ws, ws_bytes=None, stream=None):
+def moe_gate_topk(cfg, x, T, gate_w, gate_bias, topk_idx, topk_w, ws, dev_status=None,
+                  ws_bytes=None, stream=None):
     ws_bytes = ws.numel() * ws.element_size() if ws_bytes is None else ws_bytes
     _check(lib().moe_gate_topk(ctypes.byref(_cfg(cfg)), _ptr(x), int(T), _ptr(gate_w),
-                               _ptr(gate_bias), _ptr(topk_idx), _ptr(topk_w), _ptr(ws), ws_bytes,
-                               _stream(stream)), "moe_gate_topk")
+                               _ptr(gate_bias), _ptr(topk_idx), _ptr(topk_w), _ptr(dev_status),
+                               _ptr(ws), ws_bytes, _stream(stream)), "moe_gate_topk")
 
 
 def moe_permute(cfg, topk_idx, T, expert_offsets, sorted_pair, row_of, dev_status, ws,

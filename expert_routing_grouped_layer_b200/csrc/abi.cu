@@ -9,7 +9,6 @@
 
 namespace moe {
 
-int router_splits_for(int T, int E, int H);
 int permute_chunks(long N);
 
 int num_sms() {
@@ -70,7 +69,8 @@ WsLayout ws_layout(const moe_config* c, int T) {
     const size_t I = c->moe_intermediate_size, S = c->n_shared_experts;
     const size_t N = (size_t)T * k;
     const size_t act_bytes = (c->afmt == MOE_A_BF16) ? 2 : 1;
-    L.router_splits = T > 0 ? router_splits_for(T, (int)E, (int)H) : 1;
+    const RouterPlan rp = router_plan(T > 0 ? T : 1, (int)E, (int)H);
+    L.router_splits = rp.splits;
     L.n_chunks = permute_chunks((long)N);
     size_t off = 0;
     auto take = [&](size_t bytes) {
@@ -78,6 +78,7 @@ WsLayout ws_layout(const moe_config* c, int T) {
         off = align_up(off + bytes);
         return o;
     };
+    L.router_planes = take((size_t)3 * rp.Epad * H * 2);
     L.router_part = take((size_t)L.router_splits * T * E * 4);
     L.topk_idx = take(N * 4);
     L.topk_w = take(N * 4);
@@ -147,8 +148,8 @@ const char* moe_status_string(moe_status s) {
 }
 
 moe_status moe_gate_topk(const moe_config* cfg, const void* x, int32_t T, const float* gate_w,
-                         const float* gate_bias, int32_t* topk_idx, float* topk_w, void* ws,
-                         size_t ws_bytes, void* stream) {
+                         const float* gate_bias, int32_t* topk_idx, float* topk_w,
+                         int32_t* dev_status, void* ws, size_t ws_bytes, void* stream) {
     if (!config_valid(cfg) || T < 0) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
     if (!x || !gate_w || !gate_bias || !topk_idx || !topk_w || !ws) return MOE_ERR_INVALID_ARG;
@@ -156,11 +157,12 @@ moe_status moe_gate_topk(const moe_config* cfg, const void* x, int32_t T, const 
     const WsLayout L = ws_layout(cfg, T);
     if (ws_bytes < L.router_part + (size_t)L.router_splits * T * cfg->n_routed_experts * 4)
         return MOE_ERR_WORKSPACE;
-    float* part = reinterpret_cast<float*>(static_cast<char*>(ws) + L.router_part);
+    char* base = static_cast<char*>(ws);
+    float* part = reinterpret_cast<float*>(base + L.router_part);
     cudaStream_t st = as_stream(stream);
-    cudaError_t e = launch_router_gemm(x, gate_w, part, T, cfg->n_routed_experts, cfg->hidden,
-                                       L.router_splits, st);
-    if (e == cudaSuccess) e = launch_topk(cfg, part, L.router_splits, gate_bias, T, topk_idx, topk_w, st);
+    cudaError_t e = launch_router_tc(x, gate_w, base + L.router_planes, part, T,
+                                     cfg->n_routed_experts, cfg->hidden, dev_status, st);
+    if (e == cudaSuccess) e = launch_topk(cfg, part, 1, gate_bias, T, topk_idx, topk_w, st);
     return cuda_status(e);
 }
 
@@ -344,7 +346,8 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* x, int32_t T, co
     int32_t* ro = reinterpret_cast<int32_t*>(base + L.row_of);
     void* y = base + L.y;
     void* sy = base + L.shared_y;
-    moe_status s = moe_gate_topk(cfg, x, T, w->gate_w, w->gate_bias, idx, tw, ws, ws_bytes, stream);
+    moe_status s = moe_gate_topk(cfg, x, T, w->gate_w, w->gate_bias, idx, tw, dev_status, ws,
+                                 ws_bytes, stream);
     if (s == MOE_OK) s = moe_permute(cfg, idx, T, off, sp, ro, dev_status, ws, ws_bytes, stream);
     if (s == MOE_OK)
         s = moe_grouped_swiglu(cfg, x, T, sp, off, w, y, sy, ws, ws_bytes, dev_status, stream);

@@ -1,13 +1,10 @@
-// gate_topk.cu -- router GEMM and warp-per-token selection.
+// gate_topk.cu -- warp-per-token expert selection, and the reduction of the
+// router's split-K partial sums (the router GEMM itself is router_tc.cu).
 //
-// Router ("DeepSeek V3架构拆解：Kimi-K2-Thinking-NVFP4的MLA注意力与MoE路由实现原理",
-// 三.1 打分): logits = x . Wg^T with fp32 inputs and fp32 accumulation.
-// Selection (same page, 三.2 选专家 and 三.3 权重归一化 + 路由缩放; sqrtsoftplus
-// scoring and route_scale from "DeepSeek-V4-Pro 架构与代码概述", 架构):
-// score, bias, group-limited top-k, normalised and scaled weights.
-//
-// The router GEMM is split along H into `splits` partial sums so a decode batch
-// still fills the GPU; a reduction kernel adds the partials of each logit in
+// Selection ("DeepSeek V3架构拆解：Kimi-K2-Thinking-NVFP4的MLA注意力与MoE路由实现原理",
+// 三.2 选专家 and 三.3 权重归一化 + 路由缩放; sqrtsoftplus scoring and route_scale
+// from "DeepSeek-V4-Pro 架构与代码概述", 架构): score, bias, group-limited top-k,
+// normalised and scaled weights. The reduction adds each logit's partials in
 // split order, so the logits are deterministic.
 #include <cuda_bf16.h>
 
@@ -20,110 +17,6 @@
 namespace moe {
 
 namespace {
-
-constexpr int RG_BM = 128;  // tokens per tile
-constexpr int RG_BN = 128;  // experts per tile
-constexpr int RG_BK = 16;
-constexpr int RG_PAD = 4;
-
-// part[split][t][e] = sum over this split's h of x[t][h] * wg[e][h]
-__global__ void __launch_bounds__(256) router_gemm_kernel(const __nv_bfloat16* __restrict__ x,
-                                                          const float* __restrict__ wg,
-                                                          float* __restrict__ part, int T, int E,
-                                                          int H, int ksteps_per_split) {
-    __shared__ __align__(16) float As[2][RG_BK][RG_BM + RG_PAD];
-    __shared__ __align__(16) float Bs[2][RG_BK][RG_BN + RG_PAD];
-
-    const int tid = threadIdx.x;
-    const int t0 = blockIdx.x * RG_BM;
-    const int e0 = blockIdx.y * RG_BN;
-    const int split = blockIdx.z;
-    const int nk = H / RG_BK;
-    const int kbeg = split * ksteps_per_split;
-    const int kend = min(nk, kbeg + ksteps_per_split);
-
-    // loader mapping: each thread moves 8 consecutive k of one row of A and of B
-    const int lrow = tid >> 1;       // 0..127
-    const int lcol = (tid & 1) * 8;  // 0 or 8
-    const bool a_ok = (t0 + lrow) < T;
-    const bool b_ok = (e0 + lrow) < E;
-    const __nv_bfloat16* a_src = x + (size_t)(t0 + lrow) * H + lcol;
-    const float* b_src = wg + (size_t)(e0 + lrow) * H + lcol;
-
-    const int ty = tid >> 4, tx = tid & 15;
-    float acc[8][8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-
-    uint4 ra;
-    float4 rb0, rb1;
-    auto gload = [&](int ks) {
-        const int koff = ks * RG_BK;
-        if (a_ok) ra = *reinterpret_cast<const uint4*>(a_src + koff);
-        else ra = make_uint4(0, 0, 0, 0);
-        if (b_ok) {
-            rb0 = *reinterpret_cast<const float4*>(b_src + koff);
-            rb1 = *reinterpret_cast<const float4*>(b_src + koff + 4);
-        } else {
-            rb0 = rb1 = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-    };
-    auto sstore = [&](int buf) {
-        const __nv_bfloat16* av = reinterpret_cast<const __nv_bfloat16*>(&ra);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) As[buf][lcol + c][lrow] = __bfloat162float(av[c]);
-        Bs[buf][lcol + 0][lrow] = rb0.x;
-        Bs[buf][lcol + 1][lrow] = rb0.y;
-        Bs[buf][lcol + 2][lrow] = rb0.z;
-        Bs[buf][lcol + 3][lrow] = rb0.w;
-        Bs[buf][lcol + 4][lrow] = rb1.x;
-        Bs[buf][lcol + 5][lrow] = rb1.y;
-        Bs[buf][lcol + 6][lrow] = rb1.z;
-        Bs[buf][lcol + 7][lrow] = rb1.w;
-    };
-
-    if (kbeg < kend) {
-        gload(kbeg);
-        sstore(0);
-    }
-    __syncthreads();
-    int buf = 0;
-    for (int ks = kbeg; ks < kend; ++ks) {
-        const bool more = ks + 1 < kend;
-        if (more) gload(ks + 1);
-#pragma unroll
-        for (int kk = 0; kk < RG_BK; ++kk) {
-            float a[8], b[8];
-            *reinterpret_cast<float4*>(&a[0]) = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 4]);
-            *reinterpret_cast<float4*>(&a[4]) =
-                *reinterpret_cast<const float4*>(&As[buf][kk][64 + ty * 4]);
-            *reinterpret_cast<float4*>(&b[0]) = *reinterpret_cast<const float4*>(&Bs[buf][kk][tx * 4]);
-            *reinterpret_cast<float4*>(&b[4]) =
-                *reinterpret_cast<const float4*>(&Bs[buf][kk][64 + tx * 4]);
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-#pragma unroll
-                for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
-        }
-        if (more) sstore(buf ^ 1);
-        __syncthreads();
-        buf ^= 1;
-    }
-
-    float* out = part + (size_t)split * T * E;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int t = t0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + (i - 4));
-        if (t >= T) continue;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int e = e0 + (j < 4 ? tx * 4 + j : 64 + tx * 4 + (j - 4));
-            if (e < E) out[(size_t)t * E + e] = acc[i][j];
-        }
-    }
-}
 
 // logits = sum over splits of the partial sums, added in split order; written
 // over split 0 so the selection kernel reads one slab.
@@ -265,33 +158,9 @@ __global__ void __launch_bounds__(256) topk_kernel(TopkParams p) {
 
 }  // namespace
 
-cudaError_t launch_router_gemm(const void* x, const float* gate_w, float* part, int T, int E, int H,
-                               int splits, cudaStream_t st) {
-    if (T == 0) return cudaSuccess;
-    const int nk = H / RG_BK;
-    const int per = (nk + splits - 1) / splits;
-    dim3 grid((T + RG_BM - 1) / RG_BM, (E + RG_BN - 1) / RG_BN, splits);
-    router_gemm_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), gate_w, part, T,
-                                             E, H, per);
-    if (splits > 1) {
-        const long n = (long)T * E;
-        router_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(part, n, splits);
-    }
+cudaError_t launch_router_reduce(float* part, long n, int splits, cudaStream_t st) {
+    router_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(part, n, splits);
     return cudaGetLastError();
-}
-
-int router_splits_for(int T, int E, int H) {
-    const int tiles = ((T + RG_BM - 1) / RG_BM) * ((E + RG_BN - 1) / RG_BN);
-    const int target = num_sms();  // one wave: the kernel fits one CTA per SM
-    int s = (target + tiles - 1) / tiles;
-    const int max_s = (H / RG_BK) / 4;  // at least 4 k-steps per split
-    if (s > max_s) s = max_s;
-    if (s < 1) s = 1;
-    // every split must own at least one k-step after rounding
-    const int nk = H / RG_BK;
-    const int per = (nk + s - 1) / s;
-    s = (nk + per - 1) / per;
-    return s;
 }
 
 cudaError_t launch_topk(const moe_config* c, const float* part, int splits, const float* bias, int T,
@@ -299,7 +168,7 @@ cudaError_t launch_topk(const moe_config* c, const float* part, int splits, cons
     if (T == 0) return cudaSuccess;
     TopkParams p;
     p.part = part;
-    p.splits = 1;  // launch_router_gemm left the summed logits in split 0
+    p.splits = 1;  // the router left the summed logits in split 0
     p.bias = bias;
     p.T = T;
     p.E = c->n_routed_experts;

@@ -11,8 +11,16 @@
 namespace moe {
 
 // Workspace carve-up shared by every entry point (offsets in bytes).
+// Router GEMM plan: expert rows padded to 128, K split for small batches.
+struct RouterPlan {
+    int Epad;    // experts rounded up to 128
+    int splits;  // K splits (partial-sum slabs)
+    int kbps;    // 64-wide k-blocks per split
+};
+
 struct WsLayout {
-    size_t router_part;   // fp32 [S][T][E] partial router sums
+    size_t router_planes; // bf16 [3][Epad][H] hi/mid/lo planes of the router weight
+    size_t router_part;   // fp32 [splits][T][E] partial router sums
     size_t topk_idx;      // int32 [T][k]
     size_t topk_w;        // fp32 [T][k]
     size_t offsets;       // int32 [E+1]
@@ -36,8 +44,10 @@ WsLayout ws_layout(const moe_config* c, int T);
 int num_sms();
 
 // Kernel launchers (return a cudaError_t of the launch).
-cudaError_t launch_router_gemm(const void* x, const float* gate_w, float* part, int T, int E, int H,
-                               int splits, cudaStream_t st);
+RouterPlan router_plan(int T, int E, int H);
+cudaError_t launch_router_tc(const void* x, const float* gate_w, void* planes, float* part, int T,
+                             int E, int H, int32_t* status, cudaStream_t st);
+cudaError_t launch_router_reduce(float* part, long n, int splits, cudaStream_t st);
 cudaError_t launch_topk(const moe_config* c, const float* part, int splits, const float* bias, int T,
                         int32_t* idx, float* w, cudaStream_t st);
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int n_chunks, int32_t* chunk,

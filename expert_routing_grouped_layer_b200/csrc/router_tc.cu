@@ -1,0 +1,276 @@
+// router_tc.cu -- router logits on the tcgen05 tensor cores with fp32 accuracy.
+//
+// "DeepSeek V3架构拆解：Kimi-K2-Thinking-NVFP4的MLA注意力与MoE路由实现原理", 三.1 打分:
+// logits = x . Wg^T with an fp32 router weight and fp32 arithmetic. The bf16
+// input x is exact in bf16; the fp32 weight is split exactly enough into three
+// bf16 planes, Wg = hi + mid + lo (hi = bf16(Wg), mid = bf16(Wg - hi),
+// lo = bf16(Wg - hi - mid): 24 significand bits), and one GEMM accumulates
+// x.hi + x.mid + x.lo into the same fp32 tensor-memory accumulator. Every
+// product of two bf16 values is exact in fp32, so the result has fp32-class
+// error like a plain fp32 dot product, at tensor-core throughput.
+//
+// Layout: experts are the MMA M operand (128 per tile, the three planes of the
+// same 128 experts are three A tiles of one stage), tokens are N (<= 128).
+// Small batches split K across CTAs; partial sums go to part[split][T][E] and a
+// reduction kernel adds them in split order (deterministic).
+#include "gemm_common.cuh"
+
+namespace moe {
+namespace {
+
+using gemm::BK;
+using gemm::BM;
+using gemm::B_BOX;
+
+constexpr int RT_BN = 128;
+constexpr int RT_STAGES = 3;
+constexpr int RT_A_BYTES = BM * BK * 2;
+constexpr int RT_B_BYTES = RT_BN * BK * 2;
+constexpr int RT_STAGE_BYTES = 3 * RT_A_BYTES + RT_B_BYTES;
+constexpr int RT_TMEM_COLS = 2 * RT_BN;
+constexpr int RT_SMEM_BYTES = 1024 + RT_STAGES * RT_STAGE_BYTES + 8 * (2 * RT_STAGES + 5) + 16;
+
+struct RouterParams {
+    int T, E, Epad, H;
+    int mtiles, ntiles, ksplit, kbps;  // k-blocks of 64 per split
+    float* part;
+    int32_t* status;
+};
+
+struct RUnit {
+    int mt, ks, t0, n_valid, kb0, kb1;
+};
+
+__device__ __forceinline__ RUnit router_unit(const RouterParams& p, int u) {
+    RUnit r;
+    r.ks = u % p.ksplit;
+    const int tile = u / p.ksplit;
+    r.mt = tile % p.mtiles;
+    const int nt = tile / p.mtiles;
+    r.t0 = nt * RT_BN;
+    r.n_valid = min(RT_BN, p.T - r.t0);
+    r.kb0 = r.ks * p.kbps;
+    r.kb1 = min(p.H / BK, r.kb0 + p.kbps);
+    return r;
+}
+
+// hi / mid / lo bf16 planes of the fp32 router weight, rows padded to Epad with zeros.
+__global__ void __launch_bounds__(256) router_split_kernel(const float* __restrict__ wg,
+                                                           __nv_bfloat16* __restrict__ planes,
+                                                           int E, int Epad, int H) {
+    const long n = (long)Epad * H;
+    for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (long)gridDim.x * blockDim.x) {
+        const long e = i / H;
+        const float w = e < E ? wg[i] : 0.0f;
+        const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+        const float r1 = w - __bfloat162float(hi);
+        const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+        const float r2 = r1 - __bfloat162float(mid);
+        planes[i] = hi;
+        planes[n + i] = mid;
+        planes[2 * n + i] = __float2bfloat16_rn(r2);
+    }
+}
+
+__global__ void __launch_bounds__(192, 1)
+    router_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                     const RouterParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + RT_STAGES * RT_STAGE_BYTES);
+    uint64_t* empty = full + RT_STAGES;
+    uint64_t* tfull = empty + RT_STAGES;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* mma_done = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < RT_STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], 128);
+        }
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&tmW);
+        tma_prefetch_desc(&tmX);
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, RT_TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int total = p.mtiles * p.ntiles * p.ksplit;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued = 0;
+            for (int u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x) {
+                const RUnit r = router_unit(p, u);
+                const int nb = ((r.n_valid + 15) & ~15) / B_BOX;
+                const uint32_t tx = 3 * RT_A_BYTES + nb * B_BOX * BK * 2;
+                bool ok = true;
+                for (int kb = r.kb0; kb < r.kb1; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+                    uint8_t* st = smem + stage * RT_STAGE_BYTES;
+                    mbar_arrive_expect_tx(&full[stage], tx);
+                    for (int pl = 0; pl < 3; ++pl)
+                        tma_load_2d(st + pl * RT_A_BYTES, &tmW, kb * BK, pl * p.Epad + r.mt * BM,
+                                    &full[stage]);
+                    for (int i = 0; i < nb; ++i)
+                        tma_load_2d(st + 3 * RT_A_BYTES + i * B_BOX * BK * 2, &tmX, kb * BK,
+                                    r.t0 + i * B_BOX, &full[stage]);
+                    ++issued;
+                    if (++stage == RT_STAGES) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+            }
+            if (*abort_flag) {
+                int s = stage;
+                uint32_t ph = phase;
+                for (int i = 0; i < min(issued, RT_STAGES); ++i) {
+                    if (--s < 0) { s = RT_STAGES - 1; ph ^= 1; }
+                    volatile int no_abort = 0;
+                    mbar_wait(&full[s], ph, &no_abort);
+                }
+                status_or(p.status, MOE_DEV_TIMEOUT);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            for (int u = blockIdx.x; u < total; u += gridDim.x) {
+                const RUnit r = router_unit(p, u);
+                const uint32_t idesc = idesc_bf16(BM, (r.n_valid + 15) & ~15);
+                if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t d = tmem_base + acc * RT_BN;
+                bool ok = true;
+                for (int kb = r.kb0; kb < r.kb1; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t st = smem_u32(smem + stage * RT_STAGE_BYTES);
+                    const uint32_t sb = st + 3 * RT_A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        const uint64_t bd = sdesc_kmajor_sw128(sb + kk * 32);
+#pragma unroll
+                        for (int pl = 0; pl < 3; ++pl)
+                            mma_bf16(d, sdesc_kmajor_sw128(st + pl * RT_A_BYTES + kk * 32), bd, idesc,
+                                     (kb != r.kb0 || kk != 0 || pl != 0) ? 1u : 0u);
+                    }
+                    mma_commit(&empty[stage]);
+                    if (++stage == RT_STAGES) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                mma_commit(&tfull[acc]);
+                if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+            }
+            mma_commit(mma_done);
+            volatile int no_abort = 0;
+            mbar_wait(mma_done, 0, &no_abort);
+            if (*abort_flag) status_or(p.status, MOE_DEV_TIMEOUT);
+        }
+    } else {
+        const int q = warp & 3;
+        const int e = q * 32 + lane;  // expert within the M tile
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int u = blockIdx.x; u < total; u += gridDim.x) {
+            const RUnit r = router_unit(p, u);
+            if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) break;
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * RT_BN;
+            const int eg = r.mt * BM + e;
+            float* out = p.part + ((size_t)r.ks * p.T + r.t0) * p.E + eg;
+            for (int c0 = 0; c0 < r.n_valid; c0 += 16) {
+                uint32_t v[16];
+                tmem_ld16(taddr + c0, v);
+                tmem_ld_wait(v);
+                if (eg < p.E) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        if (c0 + j < r.n_valid) out[(size_t)(c0 + j) * p.E] = __uint_as_float(v[j]);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&tempty[acc]);
+            if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, RT_TMEM_COLS);
+    }
+}
+
+}  // namespace
+
+RouterPlan router_plan(int T, int E, int H) {
+    RouterPlan r;
+    r.Epad = (E + BM - 1) / BM * BM;
+    const int KB = H / BK;
+    const int base = (r.Epad / BM) * ((T + RT_BN - 1) / RT_BN);
+    int s = (num_sms() + base - 1) / base;
+    s = std::max(1, std::min(s, KB / 4));  // at least 4 k-blocks per split
+    r.kbps = (KB + s - 1) / s;
+    r.splits = (KB + r.kbps - 1) / r.kbps;  // no empty split
+    return r;
+}
+
+cudaError_t launch_router_tc(const void* x, const float* gate_w, void* planes, float* part, int T,
+                             int E, int H, int32_t* status, cudaStream_t st) {
+    if (T == 0) return cudaSuccess;
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        RT_SMEM_BYTES);
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    const RouterPlan plan = router_plan(T, E, H);
+    const long n = (long)plan.Epad * H;
+    router_split_kernel<<<(unsigned)std::min<long>((n + 255) / 256, 4L * num_sms()), 256, 0, st>>>(
+        gate_w, static_cast<__nv_bfloat16*>(planes), E, plan.Epad, H);
+    CUtensorMap tmW, tmX;
+    if (!gemm::make_tmap_bf16(&tmW, planes, 3ull * plan.Epad, H, BM) ||
+        !gemm::make_tmap_bf16(&tmX, x, (uint64_t)T, H, B_BOX))
+        return cudaErrorInvalidValue;
+    RouterParams p;
+    p.T = T;
+    p.E = E;
+    p.Epad = plan.Epad;
+    p.H = H;
+    p.mtiles = plan.Epad / BM;
+    p.ntiles = (T + RT_BN - 1) / RT_BN;
+    p.ksplit = plan.splits;
+    p.kbps = plan.kbps;
+    p.part = part;
+    p.status = status;
+    const int units = p.mtiles * p.ntiles * p.ksplit;
+    router_tc_kernel<<<std::min(units, num_sms()), 192, RT_SMEM_BYTES, st>>>(tmW, tmX, p);
+    cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess && plan.splits > 1) e = launch_router_reduce(part, (long)T * E, plan.splits, st);
+    return e;
+}
+
+}  // namespace moe

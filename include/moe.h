@@ -121,17 +121,19 @@ size_t moe_workspace_bytes(const moe_config *cfg, int32_t T);
 
 /* Router and selection ([V3] 三.1-三.3; [V4] 架构 for sqrtsoftplus / route_scale).
  *  x bf16 [T][H]; gate_w fp32 [E][H]; gate_bias fp32 [E].
- *  logits = x . gate_w^T accumulated in fp32; s = score(logits); s' = s + bias;
- *  with n_group > 1 the E experts form n_group contiguous groups scored by the
- *  sum of their two largest s' (a one-expert group by its s'), the topk_group
- *  best groups are kept, then the k largest s' among kept experts are chosen
- *  (ties to the lower index). topk_idx int32 [T][k] in s'-descending slot order;
- *  topk_w fp32 [T][k] = s (unbiased) of the chosen experts, divided by their sum
- *  when norm_topk_prob, times routed_scaling_factor.
- *  ws: workspace (>= moe_workspace_bytes) for partial router sums. */
+ *  logits = x . gate_w^T with fp32-class accuracy (on the tensor cores, with
+ *  gate_w split exactly into three bf16 planes and fp32 accumulation);
+ *  s = score(logits); s' = s + bias; with n_group > 1 the E experts form
+ *  n_group contiguous groups scored by the sum of their two largest s' (a
+ *  one-expert group by its s'), the topk_group best groups are kept, then the
+ *  k largest s' among kept experts are chosen (ties to the lower index).
+ *  topk_idx int32 [T][k] in s'-descending slot order; topk_w fp32 [T][k] = s
+ *  (unbiased) of the chosen experts, divided by their sum when norm_topk_prob,
+ *  times routed_scaling_factor. dev_status: MOE_DEV_TIMEOUT if a pipeline wait
+ *  ran out (may be NULL). ws: workspace (>= moe_workspace_bytes). */
 moe_status moe_gate_topk(const moe_config *cfg, const void *x, int32_t T, const float *gate_w,
-                         const float *gate_bias, int32_t *topk_idx, float *topk_w, void *ws,
-                         size_t ws_bytes, void *stream);
+                         const float *gate_bias, int32_t *topk_idx, float *topk_w,
+                         int32_t *dev_status, void *ws, size_t ws_bytes, void *stream);
 
 /* Dispatch permutation ([V3] 三.4: count tokens per expert, argsort by expert id).
  *  topk_idx int32 [T][k]. Pairs p = t*k + j are ordered by (expert, p)

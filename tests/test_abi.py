@@ -58,7 +58,7 @@ def test_invalid_configs_are_rejected(lib, bad):
     for k, v in bad.items():
         setattr(c, k, v)  # raw struct fields, as a C caller would pass them
     assert moe.moe_workspace_bytes(c, 64) == 0
-    st = lib.moe_gate_topk(ctypes.byref(c), 16, 64, 16, 16, 16, 16, 16, 1 << 30, None)
+    st = lib.moe_gate_topk(ctypes.byref(c), 16, 64, 16, 16, 16, 16, None, 16, 1 << 30, None)
     assert st == moe.MOE_ERR_INVALID_ARG
     st = lib.moe_layer_forward(ctypes.byref(c), 16, 64, ctypes.byref(moe.moe_weights()), 16, 16,
                                1 << 30, None, None)
@@ -69,12 +69,12 @@ def test_null_pointers_and_short_workspace_are_rejected(lib):
     c = cfg()
     need = moe.moe_workspace_bytes(c, 64)
     assert need > 0
-    assert lib.moe_gate_topk(ctypes.byref(c), None, 64, 256, 256, 256, 256, 256, need, None) == \
-        moe.MOE_ERR_INVALID_ARG
-    assert lib.moe_gate_topk(ctypes.byref(c), 256, 64, 256, 256, 256, 256, 256, 16, None) == \
-        moe.MOE_ERR_WORKSPACE
-    assert lib.moe_gate_topk(ctypes.byref(c), 8, 64, 256, 256, 256, 256, 256, need, None) == \
-        moe.MOE_ERR_INVALID_ARG  # misaligned x
+    assert lib.moe_gate_topk(ctypes.byref(c), None, 64, 256, 256, 256, 256, None, 256, need,
+                             None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_gate_topk(ctypes.byref(c), 256, 64, 256, 256, 256, 256, None, 256, 16,
+                             None) == moe.MOE_ERR_WORKSPACE
+    assert lib.moe_gate_topk(ctypes.byref(c), 8, 64, 256, 256, 256, 256, None, 256, need,
+                             None) == moe.MOE_ERR_INVALID_ARG  # misaligned x
     assert lib.moe_permute(ctypes.byref(c), 256, 64, None, 256, 256, 256, 256, need, None) == \
         moe.MOE_ERR_INVALID_ARG
     assert lib.moe_permute(ctypes.byref(c), 256, 64, 256, 256, 256, 256, 256, 0, None) == \
@@ -96,7 +96,8 @@ def test_null_pointers_and_short_workspace_are_rejected(lib):
 def test_zero_tokens_is_a_no_op(lib):
     c = cfg()
     w = moe.moe_weights()
-    assert lib.moe_gate_topk(ctypes.byref(c), None, 0, None, None, None, None, None, 0, None) == 0
+    assert lib.moe_gate_topk(ctypes.byref(c), None, 0, None, None, None, None, None, None, 0,
+                             None) == 0
     assert lib.moe_layer_forward(ctypes.byref(c), None, 0, ctypes.byref(w), None, None, 0, None,
                                  None) == 0
 

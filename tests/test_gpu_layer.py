@@ -136,7 +136,7 @@ def test_step_entry_points_match_layer():
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
     tw = torch.empty(T, k, dtype=torch.float32, device="cuda")
-    moe.moe_gate_topk(cfg, inp["x"], T, inp["gate_w"], inp["gate_bias"], idx, tw, ws)
+    moe.moe_gate_topk(cfg, inp["x"], T, inp["gate_w"], inp["gate_bias"], idx, tw, ws, st)
     off = torch.empty(E + 1, dtype=torch.int32, device="cuda")
     sp = torch.empty(T * k, dtype=torch.int32, device="cuda")
     ro = torch.empty(T * k, dtype=torch.int32, device="cuda")
