@@ -24,18 +24,21 @@ constexpr int F8_THREADS = 64 + 128 + CVT_THREADS;
 template <int GEMM>
 struct TileF8 {
     static constexpr int NA = (GEMM == 1) ? 2 : 1;
+    static constexpr int BNF = (GEMM == 1) ? 128 : 240;  // tokens per tile (TMEM: 2 x NA x BNF <= 512)
     static constexpr int A8_BYTES = BM * BK;      // e4m3 staging tile
     static constexpr int A_BYTES = BM * BK * 2;   // bf16 MMA tile
-    static constexpr int B_BYTES = BN * BK * 2;
+    static constexpr int B_BYTES = BNF * BK * 2;
     static constexpr int CVT_OFF = 0;                       // NA bf16 A tiles
     static constexpr int B_OFF = NA * A_BYTES;              // token tile
-    static constexpr int A8_OFF = B_OFF + B_BYTES;          // NA e4m3 tiles
-    static constexpr int STAGE_BYTES = A8_OFF + NA * A8_BYTES;
-    static constexpr int STAGES = (GEMM == 1) ? 3 : 5;
-    static constexpr int ACC_COLS = NA * BN;
-    static constexpr int TMEM_COLS = 2 * ACC_COLS;
+    static constexpr int A8_OFF = (B_OFF + B_BYTES + 1023) / 1024 * 1024;  // NA e4m3 tiles
+    static constexpr int STAGE_BYTES = (A8_OFF + NA * A8_BYTES + 1023) / 1024 * 1024;
+    static constexpr int STAGES = (GEMM == 1) ? 3 : 4;
+    static constexpr int ACC_COLS = NA * BNF;
+    static constexpr int TMEM_COLS = 512;
+    static_assert(2 * ACC_COLS <= TMEM_COLS, "tensor memory budget");
     static constexpr int BAR_BYTES = 8 * (4 * STAGES + 5) + 16;
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + 4 * (MAX_SEG + 1);
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
 // 16 E4M3 values -> 16 bf16 values of (value * scale), in element order.
@@ -178,7 +181,7 @@ __global__ void __launch_bounds__(F8_THREADS, 1)
                         const uint64_t bd = sdesc_kmajor_sw128(sb + kk * 32);
                         mma_bf16(d0, sdesc_kmajor_sw128(st + C::CVT_OFF + kk * 32), bd, idesc, acc_flag);
                         if (GEMM == 1)
-                            mma_bf16(d0 + BN, sdesc_kmajor_sw128(st + C::CVT_OFF + C::A_BYTES + kk * 32),
+                            mma_bf16(d0 + C::BNF, sdesc_kmajor_sw128(st + C::CVT_OFF + C::A_BYTES + kk * 32),
                                      bd, idesc, acc_flag);
                     }
                     mma_commit(&raw_empty[stage]);
@@ -262,7 +265,8 @@ cudaError_t launch_fp8w(const GroupedGemmArgs& a, cudaStream_t st) {
     });
     if (attr_err != cudaSuccess) return attr_err;
     uint64_t b_rows;
-    const KParams p = make_params(a, GEMM, &b_rows);
+    KParams p = make_params(a, GEMM, &b_rows);
+    p.bn = C::BNF;
     CUtensorMap tmAr, tmAs, tmB;
     const int S = a.S;
     if (!make_tmap_u8_sw64(&tmAr, a.w_routed, (uint64_t)a.E * p.a_rows_per_mat, p.K, BM))

@@ -29,22 +29,28 @@ constexpr int SF_TILE = 128 * 16; // scale tile: 128 rows x 16 k-blocks of 32
 template <int GEMM>
 struct TileMX {
     static constexpr int NA = (GEMM == 1) ? 2 : 1;
-    static constexpr int BNX = (GEMM == 1) ? 64 : 128;  // tokens per tile
-    static constexpr int A_BYTES = BM * MX_BK;          // one byte per E2M1 value in smem
+    // tokens per tile: the largest multiple of 16 whose double-buffered
+    // accumulators (x2 for gate + up) leave room for the scale columns
+    static constexpr int BNX = (GEMM == 1) ? 112 : 240;
+    static constexpr int SFB_ROWS = (BNX + 127) / 128 * 128;  // token rows of the scale tile
+    static constexpr int SFB_ATOMS = SFB_ROWS / 128;
+    static constexpr int A_BYTES = BM * MX_BK;                // one byte per E2M1 value in smem
     static constexpr int B_BYTES = BNX * MX_BK;
     static constexpr int A_OFF = 0;
     static constexpr int B_OFF = NA * A_BYTES;
     static constexpr int SFA_OFF = B_OFF + B_BYTES;
     static constexpr int SFB_OFF = SFA_OFF + NA * SF_TILE;
-    static constexpr int ATOM_OFF = SFB_OFF + SF_TILE;  // regrouped scales: A gate, [A up], B
-    static constexpr int STAGE_BYTES = ((ATOM_OFF + (NA + 1) * 512) + 1023) / 1024 * 1024;
-    static constexpr int STAGES = (GEMM == 1) ? 4 : 5;
+    static constexpr int ATOM_OFF = SFB_OFF + SFB_ROWS * 16;  // regrouped scales: A gate, [A up], B
+    static constexpr int STAGE_BYTES = ((ATOM_OFF + (NA + SFB_ATOMS) * 512) + 1023) / 1024 * 1024;
+    static constexpr int STAGES = 4;
     static constexpr int ACC_COLS = NA * BNX;
-    static constexpr int SF_COL = 2 * ACC_COLS;  // scale columns: A gate, A up, B (4 each)
+    static constexpr int SF_COL = 2 * ACC_COLS;  // scale columns: A gate, [A up], B atoms (4 each)
     static constexpr int TMEM_COLS = 512;
+    static_assert(SF_COL + 4 * (NA + SFB_ATOMS) <= TMEM_COLS, "tensor memory budget");
     static constexpr int BAR_BYTES = 8 * (3 * STAGES + 7) + 16;
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + 4 * (MAX_SEG + 1) +
                                       2 * 4 * 16 * 4;  // + cross-warp amax exchange
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -150,7 +156,7 @@ __global__ void __launch_bounds__(224, 1)
                 // a padded E2M1 tile occupies A_BYTES of shared memory but the copy
                 // counts its packed size (4 bits per value) toward the transaction
                 const uint32_t tx =
-                    C::NA * (C::A_BYTES / 2 + SF_TILE) + nb * B_BOX * MX_BK + SF_TILE;
+                    C::NA * (C::A_BYTES / 2 + SF_TILE) + nb * B_BOX * MX_BK + C::SFB_ROWS * 16;
                 const bool routed = t.seg < p.E;
                 const CUtensorMap* tmA = routed ? &tmA_routed : &tmA_shared;
                 const CUtensorMap* tmSFA = routed ? &tmSFA_routed : &tmSFA_shared;
@@ -196,7 +202,7 @@ __global__ void __launch_bounds__(224, 1)
             uint32_t acc_phase = 0;
             const uint32_t sfa_gate = tmem_base + C::SF_COL;
             const uint32_t sfa_up = tmem_base + C::SF_COL + 4;
-            const uint32_t sfb = tmem_base + C::SF_COL + 8;
+            const uint32_t sfb = tmem_base + C::SF_COL + 4 * C::NA;
             for (int u = blockIdx.x; u < total; u += gridDim.x) {
                 const Unit t = decode_unit(p, pref, u);
                 const int n_mma = (t.n_valid + 15) & ~15;
@@ -213,8 +219,10 @@ __global__ void __launch_bounds__(224, 1)
                     if (GEMM == 1)
                         tmem_cp_32x128b_x4(sfa_up,
                                            sdesc_kmajor_noswizzle_rows16(st + C::ATOM_OFF + 512));
-                    tmem_cp_32x128b_x4(sfb, sdesc_kmajor_noswizzle_rows16(st + C::ATOM_OFF +
-                                                                          C::NA * 512));
+#pragma unroll
+                    for (int a = 0; a < C::SFB_ATOMS; ++a)
+                        tmem_cp_32x128b_x4(sfb + 4 * a, sdesc_kmajor_noswizzle_rows16(
+                                                            st + C::ATOM_OFF + (C::NA + a) * 512));
 #pragma unroll
                     for (int kk = 0; kk < MX_BK / 32; ++kk) {
                         const uint32_t acc_flag = (kb | kk) != 0;
@@ -251,8 +259,10 @@ __global__ void __launch_bounds__(224, 1)
                 uint8_t* st = smem + stage * C::STAGE_BYTES;
                 const int j4 = (kb & 3) * 4;  // byte offset of this stage's k-blocks in a row
 #pragma unroll
-                for (int tile = 0; tile < C::NA + 1; ++tile) {
-                    const uint8_t* src = st + (tile < C::NA ? C::SFA_OFF + tile * SF_TILE : C::SFB_OFF);
+                for (int tile = 0; tile < C::NA + C::SFB_ATOMS; ++tile) {
+                    const uint8_t* src =
+                        st + (tile < C::NA ? C::SFA_OFF + tile * SF_TILE
+                                           : C::SFB_OFF + (tile - C::NA) * SF_TILE);
                     uint4 v;
                     v.x = *reinterpret_cast<const uint32_t*>(src + 16 * (lane + 0) + j4);
                     v.y = *reinterpret_cast<const uint32_t*>(src + 16 * (lane + 32) + j4);
@@ -387,7 +397,7 @@ cudaError_t launch_mx(const GroupedGemmArgs& a, cudaStream_t st) {
     if (!make_tmap_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.b_rows, b_rows, K, K, MX_BK, B_BOX,
                       CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_tmap_2d(&tmSFB, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.b_scale, b_rows, K / 32, K / 32, 16,
-                      128, CU_TENSOR_MAP_SWIZZLE_NONE))
+                      C::SFB_ROWS, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     grouped_gemm_mx_kernel<GEMM, AFMT><<<grid_for(p), 224, C::SMEM_BYTES, st>>>(
         tmA, tmAs, tmSFA, tmSFAs, tmB, tmSFB, p);
