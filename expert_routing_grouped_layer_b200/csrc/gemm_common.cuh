@@ -129,7 +129,7 @@ __device__ __forceinline__ void build_schedule(const KParams& p, int* pref, int 
 // Epilogue warps (4 of them, one per TMEM lane quadrant): per unit, wait for
 // the accumulator, read it 16 columns at a time (lane = output feature,
 // column = token), apply SwiGLU for GEMM1, store bf16, release the buffer.
-template <int GEMM, int ACC_COLS>
+template <int GEMM, int ACC_COLS, int ACCB = 2>
 __device__ __forceinline__ void epilogue_loop(const KParams& p, const int* pref, int total,
                                               uint32_t tmem_base, uint64_t* tfull,
                                               uint64_t* tempty, volatile int* abort_flag,
@@ -169,8 +169,13 @@ __device__ __forceinline__ void epilogue_loop(const KParams& p, const int* pref,
         }
         tc_fence_before();
         mbar_arrive(&tempty[acc]);
-        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+        if (++acc == ACCB) { acc = 0; acc_phase ^= 1; }
     }
+}
+
+// Pipeline depth that fits the shared-memory budget (at most `cap` stages).
+constexpr int stages_for(int stage_bytes, int fixed_bytes, int cap) {
+    return ((232448 - fixed_bytes) / stage_bytes) < cap ? ((232448 - fixed_bytes) / stage_bytes) : cap;
 }
 
 

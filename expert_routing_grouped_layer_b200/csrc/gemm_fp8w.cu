@@ -21,10 +21,13 @@ constexpr int CVT_WARPS = 8;
 constexpr int CVT_THREADS = CVT_WARPS * 32;
 constexpr int F8_THREADS = 64 + 128 + CVT_THREADS;
 
-template <int GEMM>
+// GEMM: 1 gate/up, 2 down. BNF_: tokens per tile. ACCB_: accumulator buffers in
+// tensor memory (2 overlaps a tile's epilogue with the next main loop).
+template <int GEMM, int BNF_, int ACCB_>
 struct TileF8 {
     static constexpr int NA = (GEMM == 1) ? 2 : 1;
-    static constexpr int BNF = (GEMM == 1) ? 128 : 240;  // tokens per tile (TMEM: 2 x NA x BNF <= 512)
+    static constexpr int BNF = BNF_;
+    static constexpr int ACCB = ACCB_;
     static constexpr int A8_BYTES = BM * BK;      // e4m3 staging tile
     static constexpr int A_BYTES = BM * BK * 2;   // bf16 MMA tile
     static constexpr int B_BYTES = BNF * BK * 2;
@@ -32,13 +35,14 @@ struct TileF8 {
     static constexpr int B_OFF = NA * A_BYTES;              // token tile
     static constexpr int A8_OFF = (B_OFF + B_BYTES + 1023) / 1024 * 1024;  // NA e4m3 tiles
     static constexpr int STAGE_BYTES = (A8_OFF + NA * A8_BYTES + 1023) / 1024 * 1024;
-    static constexpr int STAGES = (GEMM == 1) ? 3 : 4;
+    static constexpr int FIXED_BYTES = 1024 + 8 * (4 * 6 + 5) + 16 + 4 * (MAX_SEG + 1);
+    static constexpr int STAGES = stages_for(STAGE_BYTES, FIXED_BYTES, 6);
     static constexpr int ACC_COLS = NA * BNF;
     static constexpr int TMEM_COLS = 512;
-    static_assert(2 * ACC_COLS <= TMEM_COLS, "tensor memory budget");
+    static_assert(ACCB * ACC_COLS <= TMEM_COLS, "tensor memory budget");
     static constexpr int BAR_BYTES = 8 * (4 * STAGES + 5) + 16;
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + 4 * (MAX_SEG + 1);
-    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+    static_assert(STAGES >= 2 && SMEM_BYTES <= 232448, "shared memory budget");
 };
 
 // 16 E4M3 values -> 16 bf16 values of (value * scale), in element order.
@@ -60,14 +64,14 @@ __device__ __forceinline__ void e4m3x16_to_bf16_scaled(uint4 v, float scale, uin
     hi = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
-template <int GEMM>
+template <int GEMM, int BNF_, int ACCB_>
 __global__ void __launch_bounds__(F8_THREADS, 1)
     grouped_gemm_fp8w_kernel(const __grid_constant__ CUtensorMap tmA_routed,
                              const __grid_constant__ CUtensorMap tmA_shared,
                              const __grid_constant__ CUtensorMap tmB, const KParams p,
                              const float* __restrict__ scale_routed,
                              const float* __restrict__ scale_shared) {
-    using C = TileF8<GEMM>;
+    using C = TileF8<GEMM, BNF_, ACCB_>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -190,7 +194,7 @@ __global__ void __launch_bounds__(F8_THREADS, 1)
                 }
                 if (!ok) break;
                 mma_commit(&tfull[acc]);
-                if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+                if (++acc == C::ACCB) { acc = 0; acc_phase ^= 1; }
             }
             mma_commit(mma_done);
             volatile int no_abort = 0;
@@ -198,7 +202,7 @@ __global__ void __launch_bounds__(F8_THREADS, 1)
             if (*abort_flag) status_or(p.status, MOE_DEV_TIMEOUT);
         }
     } else if (warp < 6) {
-        epilogue_loop<GEMM, C::ACC_COLS>(p, pref, total, tmem_base, tfull, tempty, abort_flag,
+        epilogue_loop<GEMM, C::ACC_COLS, C::ACCB>(p, pref, total, tmem_base, tfull, tempty, abort_flag,
                                          warp, lane);
     } else {
         // converters: e4m3 staging tile -> scaled bf16 MMA tile
@@ -254,13 +258,13 @@ __global__ void __launch_bounds__(F8_THREADS, 1)
 
 }  // namespace
 
-template <int GEMM>
+template <int GEMM, int BNF_, int ACCB_>
 cudaError_t launch_fp8w(const GroupedGemmArgs& a, cudaStream_t st) {
-    using C = TileF8<GEMM>;
+    using C = TileF8<GEMM, BNF_, ACCB_>;
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(grouped_gemm_fp8w_kernel<GEMM>,
+        attr_err = cudaFuncSetAttribute(grouped_gemm_fp8w_kernel<GEMM, BNF_, ACCB_>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     });
     if (attr_err != cudaSuccess) return attr_err;
@@ -276,14 +280,19 @@ cudaError_t launch_fp8w(const GroupedGemmArgs& a, cudaStream_t st) {
         return cudaErrorInvalidValue;
     if (b_rows == 0) return cudaSuccess;
     if (!make_tmap_bf16(&tmB, a.b_rows, b_rows, p.K, B_BOX)) return cudaErrorInvalidValue;
-    grouped_gemm_fp8w_kernel<GEMM><<<grid_for(p), F8_THREADS, C::SMEM_BYTES, st>>>(
+    grouped_gemm_fp8w_kernel<GEMM, BNF_, ACCB_><<<grid_for(p), F8_THREADS, C::SMEM_BYTES, st>>>(
         tmAr, tmAs, tmB, p, static_cast<const float*>(a.w_routed_scale),
         static_cast<const float*>(S > 0 ? a.w_shared_scale : a.w_routed_scale));
     return cudaGetLastError();
 }
 
 cudaError_t launch_gemm_fp8w(const GroupedGemmArgs& a, cudaStream_t st) {
-    return a.gemm == 1 ? launch_fp8w<1>(a, st) : launch_fp8w<2>(a, st);
+    // many tokens per expert: wide token tiles (each weight tile converted once
+    // per expert); few tokens per expert: narrower double-buffered tiles
+    const bool wide = a.N >= 128L * a.E;
+    if (a.gemm == 1)
+        return wide ? launch_fp8w<1, 240, 1>(a, st) : launch_fp8w<1, 128, 2>(a, st);
+    return wide ? launch_fp8w<2, 240, 2>(a, st) : launch_fp8w<2, 128, 2>(a, st);
 }
 
 }  // namespace gemm
