@@ -28,9 +28,16 @@ constexpr int SF_TILE = 128 * 16; // scale tile: 128 rows x 16 k-blocks of 32
 
 // GEMM: 1 gate/up, 2 down. BNX_: tokens per tile. ACCB: accumulator buffers
 // in tensor memory (2 overlaps a tile's epilogue with the next tile's main
-// loop; 1 lets gate/up use 240-token tiles).
+// loop; 1 lets gate/up use 240-token tiles). Warps: 0 TMA, 1 MMA, then EG
+// groups of 4 epilogue warps (one per TMEM lane quadrant), then the scale
+// warp. Single-buffered gate/up tiles take two epilogue groups, since there
+// the quantising epilogue is not overlapped with the next tile's main loop.
 template <int GEMM, int BNX_, int ACCB_>
 struct TileMX {
+    static constexpr int EG = (GEMM == 1 && ACCB_ == 1) ? 2 : 1;
+    static constexpr int THREADS = 64 + 128 * EG + 32;
+    static constexpr int SCALE_WARP = 2 + 4 * EG;
+    static constexpr int RED_BYTES = EG * 2 * 4 * 16 * 4;  // [group][parity][warp][16 columns]
     static constexpr int NA = (GEMM == 1) ? 2 : 1;
     static constexpr int BNX = BNX_;
     static constexpr int ACCB = ACCB_;
@@ -44,23 +51,23 @@ struct TileMX {
     static constexpr int SFB_OFF = SFA_OFF + NA * SF_TILE;
     static constexpr int ATOM_OFF = SFB_OFF + SFB_ROWS * 16;  // regrouped scales: A gate, [A up], B
     static constexpr int STAGE_BYTES = ((ATOM_OFF + (NA + SFB_ATOMS) * 512) + 1023) / 1024 * 1024;
-    static constexpr int FIXED_BYTES = 1024 + 8 * (3 * 6 + 7) + 16 + 4 * (MAX_SEG + 1) + 2 * 4 * 16 * 4;
+    static constexpr int FIXED_BYTES = 1024 + 8 * (3 * 6 + 5 + 2 * EG) + 16 + 4 * (MAX_SEG + 1) + RED_BYTES;
     static constexpr int STAGES = stages_for(STAGE_BYTES, FIXED_BYTES, 6);
     static constexpr int ACC_COLS = NA * BNX;
     static constexpr int SF_COL = ACCB * ACC_COLS;  // scale columns: A gate, [A up], B atoms (4 each)
     static constexpr int TMEM_COLS = 512;
     static_assert(SF_COL % 4 == 0, "scale columns start on a multiple of 4");
     static_assert(SF_COL + 4 * (NA + SFB_ATOMS) <= TMEM_COLS, "tensor memory budget");
-    static constexpr int BAR_BYTES = 8 * (3 * STAGES + 7) + 16;
+    static constexpr int BAR_BYTES = 8 * (3 * STAGES + 5 + 2 * EG) + 16;
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + 4 * (MAX_SEG + 1) +
-                                      2 * 4 * 16 * 4;  // + cross-warp amax exchange
+                                      RED_BYTES;  // + cross-warp amax exchange
     static_assert(STAGES >= 2 && SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
-    return v;
+// Max over the warp of non-negative floats: their bit patterns order like the
+// values, so one integer max reduction does it.
+__device__ __forceinline__ float warp_max_nonneg(float v) {
+    return __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(v)));
 }
 
 // exponent of the power-of-two scale: smallest e with a <= 448 * 2^e (a >= 0)
@@ -87,7 +94,7 @@ __device__ __forceinline__ uint8_t e4m3_sat(float v) {
 }
 
 template <int GEMM, int AFMT, int BNX_, int ACCB_>
-__global__ void __launch_bounds__(224, 1)
+__global__ void __launch_bounds__(TileMX<GEMM, BNX_, ACCB_>::THREADS, 1)
     grouped_gemm_mx_kernel(const __grid_constant__ CUtensorMap tmA_routed,
                            const __grid_constant__ CUtensorMap tmA_shared,
                            const __grid_constant__ CUtensorMap tmSFA_routed,
@@ -104,11 +111,11 @@ __global__ void __launch_bounds__(224, 1)
     uint64_t* tfull = sf_ready + C::STAGES;
     uint64_t* tempty = tfull + 2;
     uint64_t* mma_done = tempty + 2;
-    uint64_t* red_bar = mma_done + 1;  // [2]: the 4 epilogue warps' amax exchange
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red_bar + 2);
+    uint64_t* red_bar = mma_done + 1;  // [group][parity]: the amax exchange of a group's 4 warps
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red_bar + 2 * C::EG);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* pref = reinterpret_cast<int*>(tmem_slot + 4);
-    float* red = reinterpret_cast<float*>(pref + MAX_SEG + 1);  // [2][4 warps][16 columns]
+    float* red = reinterpret_cast<float*>(pref + MAX_SEG + 1);  // [group][parity][4 warps][16]
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -121,11 +128,10 @@ __global__ void __launch_bounds__(224, 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull[a], 1);
-            mbar_init(&tempty[a], 128);
+            mbar_init(&tempty[a], 128 * C::EG);
         }
         mbar_init(mma_done, 1);
-        mbar_init(&red_bar[0], 4);
-        mbar_init(&red_bar[1], 4);
+        for (int i = 0; i < 2 * C::EG; ++i) mbar_init(&red_bar[i], 4);
         *abort_flag = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tmA_routed);
@@ -251,7 +257,7 @@ __global__ void __launch_bounds__(224, 1)
             mbar_wait(mma_done, 0, &no_abort);
             if (*abort_flag) status_or(p.status, MOE_DEV_TIMEOUT);
         }
-    } else if (warp == 6) {
+    } else if (warp == C::SCALE_WARP) {
         // scale warp: regroup this stage's 4 k-blocks of every 128 x 16-byte scale
         // tile into the tcgen05.cp 32x128b order (lane m0 gathers rows m0 + 32*m1)
         int stage = 0;
@@ -285,12 +291,16 @@ __global__ void __launch_bounds__(224, 1)
         epilogue_loop<2, C::ACC_COLS, C::ACCB>(p, pref, total, tmem_base, tfull, tempty, abort_flag,
                                                warp, lane);
     } else {
-        // GEMM1 epilogue: SwiGLU, then E4M3 + E8M0 block quantisation along I
+        // GEMM1 epilogue: SwiGLU, then E4M3 + E8M0 block quantisation along I.
+        // Group grp takes the 16-column chunks grp, grp + EG, ...
         const int q = warp & 3;
+        const int grp = (warp - 2) >> 2;
         const int row = q * 32 + lane;
+        float* red_g = red + grp * 128;
+        uint64_t* red_bar_g = red_bar + 2 * grp;
         int acc = 0;
         uint32_t acc_phase = 0;
-        int chunk = 0;
+        int chunk = 0;  // chunks this group has processed (amax exchange parity)
         bool ok = true;
         for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
             const Unit t = decode_unit(p, pref, u);
@@ -301,7 +311,7 @@ __global__ void __launch_bounds__(224, 1)
             uint8_t* out = t.out + feat;
             uint8_t* sc = t.sc + (t.mt * BM + q * 32) / 32;
             const int ld_sc = p.ld_out / 32;
-            for (int c0 = 0; c0 < t.n_valid; c0 += 16, ++chunk) {
+            for (int c0 = 16 * grp; c0 < t.n_valid; c0 += 16 * C::EG, ++chunk) {
                 uint32_t g[16], uu[16];
                 tmem_ld16(taddr + c0, g);
                 tmem_ld16(taddr + C::BNX + c0, uu);
@@ -310,25 +320,25 @@ __global__ void __launch_bounds__(224, 1)
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
                     const float gv = __uint_as_float(g[j]);
-                    a[j] = gv / (1.0f + __expf(-gv)) * __uint_as_float(uu[j]);
-                    wmax[j] = warp_max(fabsf(a[j]));
+                    a[j] = __fdividef(gv, 1.0f + __expf(-gv)) * __uint_as_float(uu[j]);
+                    wmax[j] = warp_max_nonneg(fabsf(a[j]));
                 }
                 int e[16];
                 if (AFMT == MOE_A_MXFP8) {
 #pragma unroll
                     for (int j = 0; j < 16; ++j) e[j] = mx_exp(wmax[j]);
                 } else {
-                    // block of 128 features = the 4 epilogue warps: exchange warp maxima
+                    // block of 128 features = the group's 4 warps: exchange warp maxima
                     const int par = chunk & 1;
-                    float* r = red + par * 64;
+                    float* r = red_g + par * 64;
                     if (lane < 16) {
 #pragma unroll
                         for (int j = 0; j < 16; ++j)
                             if (j == lane) r[q * 16 + j] = wmax[j];
                     }
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&red_bar[par]);
-                    if (!mbar_wait(&red_bar[par], (chunk >> 1) & 1, abort_flag)) { ok = false; break; }
+                    if (lane == 0) mbar_arrive(&red_bar_g[par]);
+                    if (!mbar_wait(&red_bar_g[par], (chunk >> 1) & 1, abort_flag)) { ok = false; break; }
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         const float m = fmaxf(fmaxf(r[j], r[16 + j]), fmaxf(r[32 + j], r[48 + j]));
@@ -403,19 +413,20 @@ cudaError_t launch_mx(const GroupedGemmArgs& a, cudaStream_t st) {
         !make_tmap_2d(&tmSFB, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.b_scale, b_rows, K / 32, K / 32, 16,
                       C::SFB_ROWS, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    grouped_gemm_mx_kernel<GEMM, AFMT, BNX_, ACCB_><<<grid_for(p), 224, C::SMEM_BYTES, st>>>(
+    grouped_gemm_mx_kernel<GEMM, AFMT, BNX_, ACCB_><<<grid_for(p), C::THREADS, C::SMEM_BYTES, st>>>(
         tmA, tmAs, tmSFA, tmSFAs, tmB, tmSFB, p);
     return cudaGetLastError();
 }
 
 template <int AFMT>
 cudaError_t launch_mx_tiles(const GroupedGemmArgs& a, cudaStream_t st) {
-    // gate/up: 112-token tiles with double-buffered accumulators, so the
-    // quantising epilogue overlaps the next tile (measured faster than 240-token
-    // single-buffered tiles on the 896-expert layer). Down projection: wide
-    // 240-token tiles when experts average many tokens, else 128 with a deeper ring.
-    if (a.gemm == 1) return launch_mx<1, AFMT, 112, 2>(a, st);
+    // When experts average many tokens: 240-token tiles (gate/up single-buffered
+    // with two epilogue groups, down double-buffered). Otherwise gate/up takes
+    // 112-token tiles with double-buffered accumulators, so the quantising
+    // epilogue overlaps the next tile, and down 128-token tiles with a deeper ring.
     const bool wide = a.N >= 128L * a.E;
+    if (a.gemm == 1)
+        return wide ? launch_mx<1, AFMT, 240, 1>(a, st) : launch_mx<1, AFMT, 112, 2>(a, st);
     return wide ? launch_mx<2, AFMT, 240, 2>(a, st) : launch_mx<2, AFMT, 128, 2>(a, st);
 }
 
