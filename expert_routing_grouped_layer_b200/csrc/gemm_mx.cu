@@ -16,11 +16,14 @@ namespace {
 // tcgen05.mma kind::mxf8f6f4 applies both scales inside the MMA, so the FP4
 // weights are never dequantised in software: TMA expands each packed row of
 // 128 E2M1 values to the one-byte-per-value layout the MMA reads
-// (16U4_ALIGN16B). Scales travel by TMA as 128 rows x 16 bytes (16 k-blocks);
-// a scale warp regroups the 4 k-blocks of the current stage into the 512-byte
-// order tcgen05.cp.32x128b.warpx4 expects (row m = m0 + 32*m1 at byte
-// 16*m0 + 4*m1 + kb), which puts row m's scales in lane m mod 32 of every lane
-// quadrant, column m / 32, one k-block per byte.
+// (16U4_ALIGN16B). Scales travel by TMA as 128 rows x 16 bytes (16 k-blocks).
+// The MMA reads row m's scale (m = m0 + 32*m1) from TMEM lane m0 of every
+// lane quadrant, column m1, one k-block per byte. A scale warp regroups the 4
+// k-blocks of the current stage into that order (row m at byte
+// 16*m0 + 4*m1 + kb of a 512-byte atom), in place over the staged scale
+// tiles, and two operands' atoms share one 128-lane x 256-bit copy (each atom
+// repeated for the 4 lane quadrants), so a stage issues half as many
+// tensor-memory copies as operands.
 // GEMM1's epilogue quantises the SwiGLU output per 32 (MXFP8) or per 128
 // (power of two) along I, exactly as the activation quantiser does.
 constexpr int MX_BK = 128;        // K elements per stage (one 128-byte smem row)
@@ -43,26 +46,33 @@ struct TileMX {
     static constexpr int ACCB = ACCB_;
     static constexpr int SFB_ROWS = (BNX + 127) / 128 * 128;  // token rows of the scale tile
     static constexpr int SFB_ATOMS = SFB_ROWS / 128;
+    static constexpr int NOPS = NA + SFB_ATOMS;  // scale operands: A gate, [A up], B rows 0-127, [128-255]
+    static constexpr int NPAIR = NOPS / 2;       // operand pairs copied by one 128x256b copy
     static constexpr int A_BYTES = BM * MX_BK;                // one byte per E2M1 value in smem
     static constexpr int B_BYTES = BNX * MX_BK;
     static constexpr int A_OFF = 0;
     static constexpr int B_OFF = NA * A_BYTES;
-    static constexpr int SFA_OFF = B_OFF + B_BYTES;
-    static constexpr int SFB_OFF = SFA_OFF + NA * SF_TILE;
-    static constexpr int ATOM_OFF = SFB_OFF + SFB_ROWS * 16;  // regrouped scales: A gate, [A up], B
-    static constexpr int STAGE_BYTES = ((ATOM_OFF + (NA + SFB_ATOMS) * 512) + 1023) / 1024 * 1024;
+    static constexpr int SF_OFF = B_OFF + B_BYTES;  // staged scale tiles, operand i at SF_OFF + i*SF_TILE
+    static constexpr int SFB_OFF = SF_OFF + NA * SF_TILE;
+    static constexpr int STAGE_BYTES = (SF_OFF + NOPS * SF_TILE + 1023) / 1024 * 1024;
     static constexpr int FIXED_BYTES = 1024 + 8 * (3 * 6 + 5 + 2 * EG) + 16 + 4 * (MAX_SEG + 1) + RED_BYTES;
     static constexpr int STAGES = stages_for(STAGE_BYTES, FIXED_BYTES, 6);
     static constexpr int ACC_COLS = NA * BNX;
-    static constexpr int SF_COL = ACCB * ACC_COLS;  // scale columns: A gate, [A up], B atoms (4 each)
+    static constexpr int SF_COL = ACCB * ACC_COLS;  // scale columns: operand i at SF_COL + 4*i
     static constexpr int TMEM_COLS = 512;
-    static_assert(SF_COL % 4 == 0, "scale columns start on a multiple of 4");
-    static_assert(SF_COL + 4 * (NA + SFB_ATOMS) <= TMEM_COLS, "tensor memory budget");
+    static_assert(SF_COL % 8 == 0, "256-bit scale copies start on a multiple of 8 columns");
+    static_assert(SF_COL + 4 * NOPS <= TMEM_COLS, "tensor memory budget");
     static constexpr int BAR_BYTES = 8 * (3 * STAGES + 5 + 2 * EG) + 16;
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + 4 * (MAX_SEG + 1) +
                                       RED_BYTES;  // + cross-warp amax exchange
     static_assert(STAGES >= 2 && SMEM_BYTES <= 232448, "shared memory budget");
 };
+
+// 128 lanes x 256 bits from shared memory (two 16-byte halves 2048 bytes apart,
+// rows 16 bytes apart) to 8 TMEM columns.
+__device__ __forceinline__ void tmem_cp_128x256b(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
 
 // Max over the warp of non-negative floats: their bit patterns order like the
 // values, so one integer max reduction does it.
@@ -177,11 +187,11 @@ __global__ void __launch_bounds__(TileMX<GEMM, BNX_, ACCB_>::THREADS, 1)
                     const int sfx = (kb >> 2) * 16;  // 16-k-block group holding this stage
                     mbar_arrive_expect_tx(&full[stage], tx);
                     tma_load_2d(st + C::A_OFF, tmA, kb * MX_BK, t.a_row, &full[stage]);
-                    tma_load_2d(st + C::SFA_OFF, tmSFA, sfx, t.a_row, &full[stage]);
+                    tma_load_2d(st + C::SF_OFF, tmSFA, sfx, t.a_row, &full[stage]);
                     if (GEMM == 1) {
                         tma_load_2d(st + C::A_OFF + C::A_BYTES, tmA, kb * MX_BK,
                                     t.a_row + p.a_up_offset, &full[stage]);
-                        tma_load_2d(st + C::SFA_OFF + SF_TILE, tmSFA, sfx, t.a_row + p.a_up_offset,
+                        tma_load_2d(st + C::SF_OFF + SF_TILE, tmSFA, sfx, t.a_row + p.a_up_offset,
                                     &full[stage]);
                     }
                     for (int i = 0; i < nb; ++i)
@@ -225,14 +235,13 @@ __global__ void __launch_bounds__(TileMX<GEMM, BNX_, ACCB_>::THREADS, 1)
                         !mbar_wait(&sf_ready[stage], phase, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t st = smem_u32(smem + stage * C::STAGE_BYTES);
-                    tmem_cp_32x128b_x4(sfa_gate, sdesc_kmajor_noswizzle_rows16(st + C::ATOM_OFF));
-                    if (GEMM == 1)
-                        tmem_cp_32x128b_x4(sfa_up,
-                                           sdesc_kmajor_noswizzle_rows16(st + C::ATOM_OFF + 512));
 #pragma unroll
-                    for (int a = 0; a < C::SFB_ATOMS; ++a)
-                        tmem_cp_32x128b_x4(sfb + 4 * a, sdesc_kmajor_noswizzle_rows16(
-                                                            st + C::ATOM_OFF + (C::NA + a) * 512));
+                    for (int pr = 0; pr < C::NPAIR; ++pr)
+                        tmem_cp_128x256b(sfa_gate + 8 * pr,
+                                         sdesc_kmajor_noswizzle_rows16(st + C::SF_OFF + pr * 2 * SF_TILE));
+                    if (C::NOPS & 1)
+                        tmem_cp_32x128b_x4(sfa_gate + 8 * C::NPAIR, sdesc_kmajor_noswizzle_rows16(
+                                                                     st + C::SF_OFF + 2 * C::NPAIR * SF_TILE));
 #pragma unroll
                     for (int kk = 0; kk < MX_BK / 32; ++kk) {
                         const uint32_t acc_flag = (kb | kk) != 0;
@@ -258,28 +267,38 @@ __global__ void __launch_bounds__(TileMX<GEMM, BNX_, ACCB_>::THREADS, 1)
             if (*abort_flag) status_or(p.status, MOE_DEV_TIMEOUT);
         }
     } else if (warp == C::SCALE_WARP) {
-        // scale warp: regroup this stage's 4 k-blocks of every 128 x 16-byte scale
-        // tile into the tcgen05.cp 32x128b order (lane m0 gathers rows m0 + 32*m1)
+        // scale warp: regroup this stage's 4 k-blocks of every staged 128 x 16-byte
+        // scale tile (lane m0 gathers rows m0 + 32*m1), in place. Operand pair pr
+        // becomes a 128-row x 32-byte copy source: operand 2pr in the first 16-byte
+        // half, 2pr+1 in the second (2048 bytes on), each atom written for rows
+        // m0, m0+32, m0+64, m0+96. An odd last operand stays one 512-byte atom.
         int stage = 0;
         uint32_t phase = 0;
         for (int u = blockIdx.x; u < total; u += gridDim.x) {
             bool ok = true;
             for (int kb = 0; kb < KB; ++kb) {
                 if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
-                uint8_t* st = smem + stage * C::STAGE_BYTES;
+                uint8_t* sf = smem + stage * C::STAGE_BYTES + C::SF_OFF;
                 const int j4 = (kb & 3) * 4;  // byte offset of this stage's k-blocks in a row
+                uint4 v[C::NOPS];
 #pragma unroll
-                for (int tile = 0; tile < C::NA + C::SFB_ATOMS; ++tile) {
-                    const uint8_t* src =
-                        st + (tile < C::NA ? C::SFA_OFF + tile * SF_TILE
-                                           : C::SFB_OFF + (tile - C::NA) * SF_TILE);
-                    uint4 v;
-                    v.x = *reinterpret_cast<const uint32_t*>(src + 16 * (lane + 0) + j4);
-                    v.y = *reinterpret_cast<const uint32_t*>(src + 16 * (lane + 32) + j4);
-                    v.z = *reinterpret_cast<const uint32_t*>(src + 16 * (lane + 64) + j4);
-                    v.w = *reinterpret_cast<const uint32_t*>(src + 16 * (lane + 96) + j4);
-                    *reinterpret_cast<uint4*>(st + C::ATOM_OFF + tile * 512 + 16 * lane) = v;
+                for (int i = 0; i < C::NOPS; ++i) {
+                    const uint8_t* src = sf + i * SF_TILE;
+                    v[i].x = *reinterpret_cast<const uint32_t*>(src + 16 * (lane + 0) + j4);
+                    v[i].y = *reinterpret_cast<const uint32_t*>(src + 16 * (lane + 32) + j4);
+                    v[i].z = *reinterpret_cast<const uint32_t*>(src + 16 * (lane + 64) + j4);
+                    v[i].w = *reinterpret_cast<const uint32_t*>(src + 16 * (lane + 96) + j4);
                 }
+                __syncwarp();  // every lane has read the staged tiles before they are overwritten
+#pragma unroll
+                for (int i = 0; i < 2 * C::NPAIR; ++i) {
+                    uint8_t* dst = sf + (i >> 1) * 2 * SF_TILE + (i & 1) * SF_TILE;
+#pragma unroll
+                    for (int r = 0; r < 4; ++r)
+                        *reinterpret_cast<uint4*>(dst + 16 * (lane + 32 * r)) = v[i];
+                }
+                if (C::NOPS & 1)
+                    *reinterpret_cast<uint4*>(sf + 2 * C::NPAIR * SF_TILE + 16 * lane) = v[C::NOPS - 1];
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sf_ready[stage]);
