@@ -173,6 +173,35 @@ __device__ __forceinline__ void epilogue_loop(const KParams& p, const int* pref,
     }
 }
 
+// Token rows of the B operand are fetched with tensor maps whose boxes are
+// 16, 32, 64 and 128 rows high: a tile of n rows (n a multiple of 16, below
+// 256) takes one copy per set bit of n / 16, largest first, so every copy
+// starts on a 16-row (2 KB for 128-byte rows) boundary of the swizzled tile.
+// One TMA instruction per 16 rows kept the single producer thread busy for
+// longer than the tensor cores needed per stage.
+constexpr int B_HEIGHTS = 4;
+struct BMaps {
+    CUtensorMap m[B_HEIGHTS];  // m[i]: box of 16 << i rows
+};
+
+__device__ __forceinline__ void prefetch_bmaps(const BMaps& bm) {
+#pragma unroll
+    for (int i = 0; i < B_HEIGHTS; ++i) tma_prefetch_desc(&bm.m[i]);
+}
+
+__device__ __forceinline__ void load_b_rows(uint8_t* dst, const BMaps& bm, int x, int row, int n,
+                                            int row_bytes, uint64_t* bar) {
+    const int blocks = n >> 4;
+    int off = 0;
+#pragma unroll
+    for (int i = B_HEIGHTS - 1; i >= 0; --i) {
+        if ((blocks >> i) & 1) {
+            tma_load_2d(dst + off * row_bytes, &bm.m[i], x, row + off, bar);
+            off += 16 << i;
+        }
+    }
+}
+
 // Pipeline depth that fits the shared-memory budget (at most `cap` stages).
 constexpr int stages_for(int stage_bytes, int fixed_bytes, int cap) {
     return ((232448 - fixed_bytes) / stage_bytes) < cap ? ((232448 - fixed_bytes) / stage_bytes) : cap;
@@ -221,6 +250,25 @@ inline bool make_tmap_u8_sw64(CUtensorMap* tm, const void* ptr, uint64_t rows, u
                      box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+// The four B maps of one row-major tensor [rows][cols] of esize-byte elements,
+// box = box_x elements x (16 << i) rows, 128-byte swizzle.
+inline bool make_bmaps(BMaps* bm, CUtensorMapDataType dtype, int esize, const void* ptr,
+                       uint64_t rows, uint64_t cols, uint32_t box_x) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    for (int i = 0; i < B_HEIGHTS; ++i) {
+        cuuint64_t dims[2] = {cols, rows};
+        cuuint64_t strides[1] = {cols * (uint64_t)esize};
+        cuuint32_t box[2] = {box_x, (cuuint32_t)(16 << i)};
+        cuuint32_t estr[2] = {1, 1};
+        CUresult r = enc(&bm->m[i], dtype, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return false;
+    }
+    return true;
 }
 
 // Problem geometry shared by every variant of the two GEMMs.

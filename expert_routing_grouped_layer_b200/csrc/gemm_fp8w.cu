@@ -68,7 +68,7 @@ template <int GEMM, int BNF_, int ACCB_>
 __global__ void __launch_bounds__(F8_THREADS, 1)
     grouped_gemm_fp8w_kernel(const __grid_constant__ CUtensorMap tmA_routed,
                              const __grid_constant__ CUtensorMap tmA_shared,
-                             const __grid_constant__ CUtensorMap tmB, const KParams p,
+                             const __grid_constant__ BMaps tmB, const KParams p,
                              const float* __restrict__ scale_routed,
                              const float* __restrict__ scale_shared) {
     using C = TileF8<GEMM, BNF_, ACCB_>;
@@ -105,7 +105,7 @@ __global__ void __launch_bounds__(F8_THREADS, 1)
         fence_barrier_init();
         tma_prefetch_desc(&tmA_routed);
         tma_prefetch_desc(&tmA_shared);
-        tma_prefetch_desc(&tmB);
+        prefetch_bmaps(tmB);
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -140,9 +140,8 @@ __global__ void __launch_bounds__(F8_THREADS, 1)
                     if (GEMM == 1)
                         tma_load_2d(st + C::A8_OFF + C::A8_BYTES, tmA, kb * BK,
                                     t.a_row + p.a_up_offset, &raw_full[stage]);
-                    for (int i = 0; i < nb; ++i)
-                        tma_load_2d(st + C::B_OFF + i * B_BOX * BK * 2, &tmB, kb * BK,
-                                    t.b_row + i * B_BOX, &raw_full[stage]);
+                    load_b_rows(st + C::B_OFF, tmB, kb * BK, t.b_row, n_mma, BK * 2,
+                                &raw_full[stage]);
                     ++issued;
                     if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
                 }
@@ -271,7 +270,8 @@ cudaError_t launch_fp8w(const GroupedGemmArgs& a, cudaStream_t st) {
     uint64_t b_rows;
     KParams p = make_params(a, GEMM, &b_rows);
     p.bn = C::BNF;
-    CUtensorMap tmAr, tmAs, tmB;
+    CUtensorMap tmAr, tmAs;
+    BMaps tmB;
     const int S = a.S;
     if (!make_tmap_u8_sw64(&tmAr, a.w_routed, (uint64_t)a.E * p.a_rows_per_mat, p.K, BM))
         return cudaErrorInvalidValue;
@@ -279,7 +279,8 @@ cudaError_t launch_fp8w(const GroupedGemmArgs& a, cudaStream_t st) {
                            (uint64_t)(S > 0 ? S : a.E) * p.a_rows_per_mat, p.K, BM))
         return cudaErrorInvalidValue;
     if (b_rows == 0) return cudaSuccess;
-    if (!make_tmap_bf16(&tmB, a.b_rows, b_rows, p.K, B_BOX)) return cudaErrorInvalidValue;
+    if (!make_bmaps(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.b_rows, b_rows, p.K, BK))
+        return cudaErrorInvalidValue;
     grouped_gemm_fp8w_kernel<GEMM, BNF_, ACCB_><<<grid_for(p), F8_THREADS, C::SMEM_BYTES, st>>>(
         tmAr, tmAs, tmB, p, static_cast<const float*>(a.w_routed_scale),
         static_cast<const float*>(S > 0 ? a.w_shared_scale : a.w_routed_scale));

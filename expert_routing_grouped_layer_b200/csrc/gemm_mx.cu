@@ -109,7 +109,7 @@ __global__ void __launch_bounds__(TileMX<GEMM, BNX_, ACCB_>::THREADS, 1)
                            const __grid_constant__ CUtensorMap tmA_shared,
                            const __grid_constant__ CUtensorMap tmSFA_routed,
                            const __grid_constant__ CUtensorMap tmSFA_shared,
-                           const __grid_constant__ CUtensorMap tmB,
+                           const __grid_constant__ BMaps tmB,
                            const __grid_constant__ CUtensorMap tmSFB, const KParams p) {
     using C = TileMX<GEMM, BNX_, ACCB_>;
     extern __shared__ uint8_t smem_raw[];
@@ -148,7 +148,7 @@ __global__ void __launch_bounds__(TileMX<GEMM, BNX_, ACCB_>::THREADS, 1)
         tma_prefetch_desc(&tmA_shared);
         tma_prefetch_desc(&tmSFA_routed);
         tma_prefetch_desc(&tmSFA_shared);
-        tma_prefetch_desc(&tmB);
+        prefetch_bmaps(tmB);
         tma_prefetch_desc(&tmSFB);
     }
     if (warp == 0) {
@@ -194,9 +194,7 @@ __global__ void __launch_bounds__(TileMX<GEMM, BNX_, ACCB_>::THREADS, 1)
                         tma_load_2d(st + C::SF_OFF + SF_TILE, tmSFA, sfx, t.a_row + p.a_up_offset,
                                     &full[stage]);
                     }
-                    for (int i = 0; i < nb; ++i)
-                        tma_load_2d(st + C::B_OFF + i * B_BOX * MX_BK, &tmB, kb * MX_BK,
-                                    t.b_row + i * B_BOX, &full[stage]);
+                    load_b_rows(st + C::B_OFF, tmB, kb * MX_BK, t.b_row, n_mma, MX_BK, &full[stage]);
                     tma_load_2d(st + C::SFB_OFF, &tmSFB, sfx, t.b_row, &full[stage]);
                     ++issued;
                     if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
@@ -416,7 +414,8 @@ cudaError_t launch_mx(const GroupedGemmArgs& a, cudaStream_t st) {
     const void* wAs = S > 0 ? a.w_shared : a.w_routed;
     const void* sA = a.w_routed_scale;
     const void* sAs = S > 0 ? a.w_shared_scale : a.w_routed_scale;
-    CUtensorMap tmA, tmAs, tmSFA, tmSFAs, tmB, tmSFB;
+    CUtensorMap tmA, tmAs, tmSFA, tmSFAs, tmSFB;
+    BMaps tmB;
     if (!make_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, wA, rowsA, K, K / 2, MX_BK, BM,
                       CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_tmap_2d(&tmAs, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, wAs, rowsAs, K, K / 2, MX_BK, BM,
@@ -427,8 +426,7 @@ cudaError_t launch_mx(const GroupedGemmArgs& a, cudaStream_t st) {
                       CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     if (b_rows == 0) return cudaSuccess;
-    if (!make_tmap_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.b_rows, b_rows, K, K, MX_BK, B_BOX,
-                      CU_TENSOR_MAP_SWIZZLE_128B) ||
+    if (!make_bmaps(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.b_rows, b_rows, K, MX_BK) ||
         !make_tmap_2d(&tmSFB, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.b_scale, b_rows, K / 32, K / 32, 16,
                       C::SFB_ROWS, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
