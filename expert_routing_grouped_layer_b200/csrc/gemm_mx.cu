@@ -52,19 +52,32 @@ struct TileMX {
     static constexpr int B_BYTES = BNX * MX_BK;
     static constexpr int A_OFF = 0;
     static constexpr int B_OFF = NA * A_BYTES;
-    static constexpr int SF_OFF = B_OFF + B_BYTES;  // staged scale tiles, operand i at SF_OFF + i*SF_TILE
-    static constexpr int SFB_OFF = SF_OFF + NA * SF_TILE;
-    static constexpr int STAGE_BYTES = (SF_OFF + NOPS * SF_TILE + 1023) / 1024 * 1024;
-    static constexpr int FIXED_BYTES = 1024 + 8 * (3 * 6 + 5 + 2 * EG) + 16 + 4 * (MAX_SEG + 1) + RED_BYTES;
-    static constexpr int STAGES = stages_for(STAGE_BYTES, FIXED_BYTES, 6);
+    static constexpr int SF_OFF = B_OFF + B_BYTES;  // regrouped scale atoms of the stage
+    static constexpr int RAW_BYTES = NOPS * SF_TILE;  // staged scale tiles, operand i at i*SF_TILE
+    static constexpr int ATOM_BYTES = NPAIR * 2 * SF_TILE + (NOPS & 1) * 512;
+    // A scale box covers 16 k-blocks, four stages. Normally the boxes go to a
+    // two-slot ring, loaded once per four stages, and the scale warp writes the
+    // atoms into the stage. Where that ring would cost a pipeline stage (wide
+    // gate/up tiles), each stage loads the boxes itself and the atoms overwrite
+    // them in place.
+    static constexpr int FIXED_BYTES =
+        1024 + 8 * (3 * 6 + 9 + 2 * EG) + 16 + 4 * (MAX_SEG + 1) + RED_BYTES;
+    static constexpr int STAGE_RING = (SF_OFF + ATOM_BYTES + 1023) / 1024 * 1024;
+    static constexpr int STAGES_RING = stages_for(STAGE_RING, FIXED_BYTES + 2 * RAW_BYTES, 6);
+    static constexpr int STAGE_INPLACE = (SF_OFF + RAW_BYTES + 1023) / 1024 * 1024;
+    static constexpr int STAGES_INPLACE = stages_for(STAGE_INPLACE, FIXED_BYTES, 6);
+    static constexpr bool SF_RING = STAGES_RING >= 4 || STAGES_RING >= STAGES_INPLACE;
+    static constexpr int STAGE_BYTES = SF_RING ? STAGE_RING : STAGE_INPLACE;
+    static constexpr int STAGES = SF_RING ? STAGES_RING : STAGES_INPLACE;
+    static constexpr int RING_BYTES = SF_RING ? 2 * RAW_BYTES : 0;
     static constexpr int ACC_COLS = NA * BNX;
     static constexpr int SF_COL = ACCB * ACC_COLS;  // scale columns: operand i at SF_COL + 4*i
     static constexpr int TMEM_COLS = 512;
     static_assert(SF_COL % 8 == 0, "256-bit scale copies start on a multiple of 8 columns");
     static_assert(SF_COL + 4 * NOPS <= TMEM_COLS, "tensor memory budget");
-    static constexpr int BAR_BYTES = 8 * (3 * STAGES + 5 + 2 * EG) + 16;
-    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + 4 * (MAX_SEG + 1) +
-                                      RED_BYTES;  // + cross-warp amax exchange
+    static constexpr int BAR_BYTES = 8 * (3 * STAGES + 9 + 2 * EG) + 16;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + RING_BYTES + BAR_BYTES +
+                                      4 * (MAX_SEG + 1) + RED_BYTES;  // + cross-warp amax exchange
     static_assert(STAGES >= 2 && SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -115,13 +128,16 @@ __global__ void __launch_bounds__(TileMX<GEMM, BNX_, ACCB_>::THREADS, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+    uint8_t* sf_ring = smem + C::STAGES * C::STAGE_BYTES;  // [2][RAW_BYTES] (ring variant)
+    uint64_t* full = reinterpret_cast<uint64_t*>(sf_ring + C::RING_BYTES);
     uint64_t* empty = full + C::STAGES;
     uint64_t* sf_ready = empty + C::STAGES;  // scales regrouped for the stage
     uint64_t* tfull = sf_ready + C::STAGES;
     uint64_t* tempty = tfull + 2;
     uint64_t* mma_done = tempty + 2;
-    uint64_t* red_bar = mma_done + 1;  // [group][parity]: the amax exchange of a group's 4 warps
+    uint64_t* sf_full = mma_done + 1;  // [2] scale ring slots
+    uint64_t* sf_empty = sf_full + 2;  // [2]
+    uint64_t* red_bar = sf_empty + 2;  // [group][parity]: the amax exchange of a group's 4 warps
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red_bar + 2 * C::EG);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* pref = reinterpret_cast<int*>(tmem_slot + 4);
@@ -141,6 +157,10 @@ __global__ void __launch_bounds__(TileMX<GEMM, BNX_, ACCB_>::THREADS, 1)
             mbar_init(&tempty[a], 128 * C::EG);
         }
         mbar_init(mma_done, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sf_full[i], 1);
+            mbar_init(&sf_empty[i], 1);
+        }
         for (int i = 0; i < 2 * C::EG; ++i) mbar_init(&red_bar[i], 4);
         *abort_flag = 0;
         fence_barrier_init();
@@ -169,45 +189,67 @@ __global__ void __launch_bounds__(TileMX<GEMM, BNX_, ACCB_>::THREADS, 1)
             int stage = 0;
             uint32_t phase = 0;
             int issued = 0;
+            int sfs = 0, sf_issued = 0;  // scale ring slot and loads issued into the ring
+            uint32_t sf_phase = 0;
             for (int u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x) {
                 const Unit t = decode_unit(p, pref, u);
                 const int n_mma = (t.n_valid + 15) & ~15;
-                const int nb = n_mma / B_BOX;
                 // a padded E2M1 tile occupies A_BYTES of shared memory but the copy
                 // counts its packed size (4 bits per value) toward the transaction
-                const uint32_t tx =
-                    C::NA * (C::A_BYTES / 2 + SF_TILE) + nb * B_BOX * MX_BK + C::SFB_ROWS * 16;
+                const uint32_t tx = C::NA * (C::A_BYTES / 2) + n_mma * MX_BK +
+                                    (C::SF_RING ? 0 : C::RAW_BYTES);
                 const bool routed = t.seg < p.E;
                 const CUtensorMap* tmA = routed ? &tmA_routed : &tmA_shared;
                 const CUtensorMap* tmSFA = routed ? &tmSFA_routed : &tmSFA_shared;
                 bool ok = true;
                 for (int kb = 0; kb < KB; ++kb) {
+                    const int sfx = (kb >> 2) * 16;  // 16-k-block group holding this stage
+                    if (C::SF_RING && (kb & 3) == 0) {
+                        if (!mbar_wait(&sf_empty[sfs], sf_phase ^ 1, abort_flag)) { ok = false; break; }
+                        uint8_t* sl = sf_ring + sfs * C::RAW_BYTES;
+                        mbar_arrive_expect_tx(&sf_full[sfs], C::RAW_BYTES);
+                        tma_load_2d(sl, tmSFA, sfx, t.a_row, &sf_full[sfs]);
+                        if (GEMM == 1)
+                            tma_load_2d(sl + SF_TILE, tmSFA, sfx, t.a_row + p.a_up_offset, &sf_full[sfs]);
+                        tma_load_2d(sl + C::NA * SF_TILE, &tmSFB, sfx, t.b_row, &sf_full[sfs]);
+                        ++sf_issued;
+                        if (++sfs == 2) { sfs = 0; sf_phase ^= 1; }
+                    }
                     if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
                     uint8_t* st = smem + stage * C::STAGE_BYTES;
-                    const int sfx = (kb >> 2) * 16;  // 16-k-block group holding this stage
                     mbar_arrive_expect_tx(&full[stage], tx);
                     tma_load_2d(st + C::A_OFF, tmA, kb * MX_BK, t.a_row, &full[stage]);
-                    tma_load_2d(st + C::SF_OFF, tmSFA, sfx, t.a_row, &full[stage]);
-                    if (GEMM == 1) {
+                    if (GEMM == 1)
                         tma_load_2d(st + C::A_OFF + C::A_BYTES, tmA, kb * MX_BK,
                                     t.a_row + p.a_up_offset, &full[stage]);
-                        tma_load_2d(st + C::SF_OFF + SF_TILE, tmSFA, sfx, t.a_row + p.a_up_offset,
+                    load_b_rows(st + C::B_OFF, tmB, kb * MX_BK, t.b_row, n_mma, MX_BK, &full[stage]);
+                    if (!C::SF_RING) {
+                        tma_load_2d(st + C::SF_OFF, tmSFA, sfx, t.a_row, &full[stage]);
+                        if (GEMM == 1)
+                            tma_load_2d(st + C::SF_OFF + SF_TILE, tmSFA, sfx, t.a_row + p.a_up_offset,
+                                        &full[stage]);
+                        tma_load_2d(st + C::SF_OFF + C::NA * SF_TILE, &tmSFB, sfx, t.b_row,
                                     &full[stage]);
                     }
-                    load_b_rows(st + C::B_OFF, tmB, kb * MX_BK, t.b_row, n_mma, MX_BK, &full[stage]);
-                    tma_load_2d(st + C::SFB_OFF, &tmSFB, sfx, t.b_row, &full[stage]);
                     ++issued;
                     if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
                 }
                 if (!ok) break;
             }
             if (*abort_flag) {
+                // wait (bounded) for this thread's copies still in flight
+                volatile int no_abort = 0;
                 int s = stage;
                 uint32_t ph = phase;
                 for (int i = 0; i < min(issued, C::STAGES); ++i) {
                     if (--s < 0) { s = C::STAGES - 1; ph ^= 1; }
-                    volatile int no_abort = 0;
                     mbar_wait(&full[s], ph, &no_abort);
+                }
+                s = sfs;
+                ph = sf_phase;
+                for (int i = 0; i < min(sf_issued, 2); ++i) {
+                    if (--s < 0) { s = 1; ph ^= 1; }
+                    mbar_wait(&sf_full[s], ph, &no_abort);
                 }
                 status_or(p.status, MOE_DEV_TIMEOUT);
             }
@@ -266,37 +308,50 @@ __global__ void __launch_bounds__(TileMX<GEMM, BNX_, ACCB_>::THREADS, 1)
         }
     } else if (warp == C::SCALE_WARP) {
         // scale warp: regroup this stage's 4 k-blocks of every staged 128 x 16-byte
-        // scale tile (lane m0 gathers rows m0 + 32*m1), in place. Operand pair pr
-        // becomes a 128-row x 32-byte copy source: operand 2pr in the first 16-byte
-        // half, 2pr+1 in the second (2048 bytes on), each atom written for rows
-        // m0, m0+32, m0+64, m0+96. An odd last operand stays one 512-byte atom.
+        // scale tile (lane m0 gathers rows m0 + 32*m1) into the stage's atoms.
+        // Operand pair pr becomes a 128-row x 32-byte copy source: operand 2pr in
+        // the first 16-byte half, 2pr+1 in the second (2048 bytes on), each atom
+        // written for rows m0, m0+32, m0+64, m0+96. An odd last operand stays one
+        // 512-byte atom. A ring slot serves four stages, then is released.
         int stage = 0;
         uint32_t phase = 0;
+        int sfs = 0;
+        uint32_t sf_phase = 0;
         for (int u = blockIdx.x; u < total; u += gridDim.x) {
             bool ok = true;
             for (int kb = 0; kb < KB; ++kb) {
+                if (C::SF_RING && (kb & 3) == 0 && !mbar_wait(&sf_full[sfs], sf_phase, abort_flag)) {
+                    ok = false;
+                    break;
+                }
                 if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
-                uint8_t* sf = smem + stage * C::STAGE_BYTES + C::SF_OFF;
+                uint8_t* atoms = smem + stage * C::STAGE_BYTES + C::SF_OFF;
+                const uint8_t* raw = C::SF_RING ? sf_ring + sfs * C::RAW_BYTES : atoms;
                 const int j4 = (kb & 3) * 4;  // byte offset of this stage's k-blocks in a row
                 uint4 v[C::NOPS];
 #pragma unroll
                 for (int i = 0; i < C::NOPS; ++i) {
-                    const uint8_t* src = sf + i * SF_TILE;
+                    const uint8_t* src = raw + i * SF_TILE;
                     v[i].x = *reinterpret_cast<const uint32_t*>(src + 16 * (lane + 0) + j4);
                     v[i].y = *reinterpret_cast<const uint32_t*>(src + 16 * (lane + 32) + j4);
                     v[i].z = *reinterpret_cast<const uint32_t*>(src + 16 * (lane + 64) + j4);
                     v[i].w = *reinterpret_cast<const uint32_t*>(src + 16 * (lane + 96) + j4);
                 }
-                __syncwarp();  // every lane has read the staged tiles before they are overwritten
+                __syncwarp();  // in place: every lane has read the tiles before they are overwritten
+                if (C::SF_RING && (kb & 3) == 3) {
+                    if (lane == 0) mbar_arrive(&sf_empty[sfs]);
+                    if (++sfs == 2) { sfs = 0; sf_phase ^= 1; }
+                }
 #pragma unroll
                 for (int i = 0; i < 2 * C::NPAIR; ++i) {
-                    uint8_t* dst = sf + (i >> 1) * 2 * SF_TILE + (i & 1) * SF_TILE;
+                    uint8_t* dst = atoms + (i >> 1) * 2 * SF_TILE + (i & 1) * SF_TILE;
 #pragma unroll
                     for (int r = 0; r < 4; ++r)
                         *reinterpret_cast<uint4*>(dst + 16 * (lane + 32 * r)) = v[i];
                 }
                 if (C::NOPS & 1)
-                    *reinterpret_cast<uint4*>(sf + 2 * C::NPAIR * SF_TILE + 16 * lane) = v[C::NOPS - 1];
+                    *reinterpret_cast<uint4*>(atoms + 2 * C::NPAIR * SF_TILE + 16 * lane) =
+                        v[C::NOPS - 1];
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sf_ready[stage]);
