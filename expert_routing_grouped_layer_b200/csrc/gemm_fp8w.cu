@@ -19,11 +19,17 @@ namespace {
 // bf16 (relative error <= 2^-9 per weight).
 constexpr int CVT_WARPS = 8;
 constexpr int CVT_THREADS = CVT_WARPS * 32;
-constexpr int F8_THREADS = 64 + 128 + CVT_THREADS;
+constexpr int B_WARP = 6 + CVT_WARPS;  // token-tile loader, after the converters
+constexpr int F8_THREADS = 64 + 128 + CVT_THREADS + 32;
+static_assert(512 % CVT_THREADS == 0, "converter tasks: whole tiles per round");
 
 // GEMM: 1 gate/up, 2 down. BNF_: tokens per tile. ACCB_: accumulator buffers in
 // tensor memory (2 overlaps a tile's epilogue with the next main loop).
-template <int GEMM, int BNF_, int ACCB_>
+// Two rings: the raw ring holds the TMA-staged e4m3 weight tiles and is freed
+// as soon as the converters have read a slot, so it can run many stages ahead
+// of the tensor cores; the MMA ring holds the converted bf16 weight tiles and
+// the token tile, freed by the MMA commit.
+template <int GEMM, int BNF_, int ACCB_, int MST_>
 struct TileF8 {
     static constexpr int NA = (GEMM == 1) ? 2 : 1;
     static constexpr int BNF = BNF_;
@@ -33,16 +39,19 @@ struct TileF8 {
     static constexpr int B_BYTES = BNF * BK * 2;
     static constexpr int CVT_OFF = 0;                       // NA bf16 A tiles
     static constexpr int B_OFF = NA * A_BYTES;              // token tile
-    static constexpr int A8_OFF = (B_OFF + B_BYTES + 1023) / 1024 * 1024;  // NA e4m3 tiles
-    static constexpr int STAGE_BYTES = (A8_OFF + NA * A8_BYTES + 1023) / 1024 * 1024;
-    static constexpr int FIXED_BYTES = 1024 + 8 * (4 * 6 + 5) + 16 + 4 * (MAX_SEG + 1);
-    static constexpr int STAGES = stages_for(STAGE_BYTES, FIXED_BYTES, 6);
+    static constexpr int MSLOT_BYTES = (B_OFF + B_BYTES + 1023) / 1024 * 1024;
+    static constexpr int RSLOT_BYTES = NA * A8_BYTES;       // NA e4m3 tiles
+    static constexpr int MSTAGES = MST_;
+    static constexpr int FIXED_BYTES = 1024 + 8 * (2 * 8 + 3 * MSTAGES + 5) + 16 + 4 * (MAX_SEG + 1);
+    static constexpr int RSTAGES_FIT = (232448 - FIXED_BYTES - MSTAGES * MSLOT_BYTES) / RSLOT_BYTES;
+    static constexpr int RSTAGES = RSTAGES_FIT < 8 ? RSTAGES_FIT : 8;
     static constexpr int ACC_COLS = NA * BNF;
     static constexpr int TMEM_COLS = 512;
     static_assert(ACCB * ACC_COLS <= TMEM_COLS, "tensor memory budget");
-    static constexpr int BAR_BYTES = 8 * (4 * STAGES + 5) + 16;
-    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + 4 * (MAX_SEG + 1);
-    static_assert(STAGES >= 2 && SMEM_BYTES <= 232448, "shared memory budget");
+    static constexpr int RING_BYTES = MSTAGES * MSLOT_BYTES + RSTAGES * RSLOT_BYTES;
+    static constexpr int BAR_BYTES = 8 * (2 * RSTAGES + 3 * MSTAGES + 5) + 16;
+    static constexpr int SMEM_BYTES = 1024 + RING_BYTES + BAR_BYTES + 4 * (MAX_SEG + 1);
+    static_assert(RSTAGES >= 2 && SMEM_BYTES <= 232448, "shared memory budget");
 };
 
 // 16 E4M3 values -> 16 bf16 values of (value * scale), in element order.
@@ -64,22 +73,25 @@ __device__ __forceinline__ void e4m3x16_to_bf16_scaled(uint4 v, float scale, uin
     hi = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
-template <int GEMM, int BNF_, int ACCB_>
+template <int GEMM, int BNF_, int ACCB_, int MST_>
 __global__ void __launch_bounds__(F8_THREADS, 1)
     grouped_gemm_fp8w_kernel(const __grid_constant__ CUtensorMap tmA_routed,
                              const __grid_constant__ CUtensorMap tmA_shared,
                              const __grid_constant__ BMaps tmB, const KParams p,
                              const float* __restrict__ scale_routed,
                              const float* __restrict__ scale_shared) {
-    using C = TileF8<GEMM, BNF_, ACCB_>;
+    using C = TileF8<GEMM, BNF_, ACCB_, MST_>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint64_t* raw_full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
-    uint64_t* raw_empty = raw_full + C::STAGES;
-    uint64_t* cvt_full = raw_empty + C::STAGES;
-    uint64_t* cvt_empty = cvt_full + C::STAGES;
-    uint64_t* tfull = cvt_empty + C::STAGES;
+    uint8_t* mring = smem;                                    // [MSTAGES][MSLOT_BYTES]
+    uint8_t* rring = smem + C::MSTAGES * C::MSLOT_BYTES;      // [RSTAGES][RSLOT_BYTES]
+    uint64_t* raw_full = reinterpret_cast<uint64_t*>(smem + C::RING_BYTES);
+    uint64_t* raw_empty = raw_full + C::RSTAGES;
+    uint64_t* b_full = raw_empty + C::RSTAGES;   // token tile landed in the MMA slot
+    uint64_t* cvt_full = b_full + C::MSTAGES;    // weight tiles converted into the MMA slot
+    uint64_t* m_empty = cvt_full + C::MSTAGES;   // MMA slot consumed
+    uint64_t* tfull = m_empty + C::MSTAGES;
     uint64_t* tempty = tfull + 2;
     uint64_t* mma_done = tempty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
@@ -90,11 +102,14 @@ __global__ void __launch_bounds__(F8_THREADS, 1)
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < C::STAGES; ++s) {
+        for (int s = 0; s < C::RSTAGES; ++s) {
             mbar_init(&raw_full[s], 1);
-            mbar_init(&raw_empty[s], 1 + CVT_THREADS);  // MMA commit + every converter thread
+            mbar_init(&raw_empty[s], CVT_THREADS);
+        }
+        for (int s = 0; s < C::MSTAGES; ++s) {
+            mbar_init(&b_full[s], 1);
             mbar_init(&cvt_full[s], CVT_THREADS);
-            mbar_init(&cvt_empty[s], 1);
+            mbar_init(&m_empty[s], 1);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull[a], 1);
@@ -121,37 +136,33 @@ __global__ void __launch_bounds__(F8_THREADS, 1)
     const int KB = p.K / BK;
 
     if (warp == 0) {
+        // producer: e4m3 weight tiles into the raw ring
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
             int issued = 0;
             for (int u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x) {
                 const Unit t = decode_unit(p, pref, u);
-                const int n_mma = (t.n_valid + 15) & ~15;
-                const int nb = n_mma / B_BOX;
-                const uint32_t tx = C::NA * C::A8_BYTES + nb * B_BOX * BK * 2;
                 const CUtensorMap* tmA = (t.seg < p.E) ? &tmA_routed : &tmA_shared;
                 bool ok = true;
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!mbar_wait(&raw_empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
-                    uint8_t* st = smem + stage * C::STAGE_BYTES;
-                    mbar_arrive_expect_tx(&raw_full[stage], tx);
-                    tma_load_2d(st + C::A8_OFF, tmA, kb * BK, t.a_row, &raw_full[stage]);
+                    uint8_t* rs = rring + stage * C::RSLOT_BYTES;
+                    mbar_arrive_expect_tx(&raw_full[stage], C::RSLOT_BYTES);
+                    tma_load_2d(rs, tmA, kb * BK, t.a_row, &raw_full[stage]);
                     if (GEMM == 1)
-                        tma_load_2d(st + C::A8_OFF + C::A8_BYTES, tmA, kb * BK,
-                                    t.a_row + p.a_up_offset, &raw_full[stage]);
-                    load_b_rows(st + C::B_OFF, tmB, kb * BK, t.b_row, n_mma, BK * 2,
-                                &raw_full[stage]);
+                        tma_load_2d(rs + C::A8_BYTES, tmA, kb * BK, t.a_row + p.a_up_offset,
+                                    &raw_full[stage]);
                     ++issued;
-                    if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+                    if (++stage == C::RSTAGES) { stage = 0; phase ^= 1; }
                 }
                 if (!ok) break;
             }
             if (*abort_flag) {
                 int s = stage;
                 uint32_t ph = phase;
-                for (int i = 0; i < min(issued, C::STAGES); ++i) {
-                    if (--s < 0) { s = C::STAGES - 1; ph ^= 1; }
+                for (int i = 0; i < min(issued, C::RSTAGES); ++i) {
+                    if (--s < 0) { s = C::RSTAGES - 1; ph ^= 1; }
                     volatile int no_abort = 0;
                     mbar_wait(&raw_full[s], ph, &no_abort);
                 }
@@ -173,10 +184,10 @@ __global__ void __launch_bounds__(F8_THREADS, 1)
                 const uint32_t d0 = tmem_base + acc * C::ACC_COLS;
                 bool ok = true;
                 for (int kb = 0; kb < KB; ++kb) {
-                    if (!mbar_wait(&raw_full[stage], phase, abort_flag) ||
+                    if (!mbar_wait(&b_full[stage], phase, abort_flag) ||
                         !mbar_wait(&cvt_full[stage], phase, abort_flag)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t st = smem_u32(smem + stage * C::STAGE_BYTES);
+                    const uint32_t st = smem_u32(mring + stage * C::MSLOT_BYTES);
                     const uint32_t sb = st + C::B_OFF;
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
@@ -187,9 +198,8 @@ __global__ void __launch_bounds__(F8_THREADS, 1)
                             mma_bf16(d0 + C::BNF, sdesc_kmajor_sw128(st + C::CVT_OFF + C::A_BYTES + kk * 32),
                                      bd, idesc, acc_flag);
                     }
-                    mma_commit(&raw_empty[stage]);
-                    mma_commit(&cvt_empty[stage]);
-                    if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+                    mma_commit(&m_empty[stage]);
+                    if (++stage == C::MSTAGES) { stage = 0; phase ^= 1; }
                 }
                 if (!ok) break;
                 mma_commit(&tfull[acc]);
@@ -200,18 +210,49 @@ __global__ void __launch_bounds__(F8_THREADS, 1)
             mbar_wait(mma_done, 0, &no_abort);
             if (*abort_flag) status_or(p.status, MOE_DEV_TIMEOUT);
         }
+    } else if (warp == B_WARP) {
+        // token-tile loader: fills each MMA slot's token tile as soon as it is free
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued = 0;
+            for (int u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x) {
+                const Unit t = decode_unit(p, pref, u);
+                const int n_mma = (t.n_valid + 15) & ~15;
+                bool ok = true;
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(&m_empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&b_full[stage], (uint32_t)(n_mma * BK * 2));
+                    load_b_rows(mring + stage * C::MSLOT_BYTES + C::B_OFF, tmB, kb * BK, t.b_row, n_mma,
+                                BK * 2, &b_full[stage]);
+                    ++issued;
+                    if (++stage == C::MSTAGES) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+            }
+            if (*abort_flag) {
+                int s = stage;
+                uint32_t ph = phase;
+                for (int i = 0; i < min(issued, C::MSTAGES); ++i) {
+                    if (--s < 0) { s = C::MSTAGES - 1; ph ^= 1; }
+                    volatile int no_abort = 0;
+                    mbar_wait(&b_full[s], ph, &no_abort);
+                }
+            }
+        }
     } else if (warp < 6) {
         epilogue_loop<GEMM, C::ACC_COLS, C::ACCB>(p, pref, total, tmem_base, tfull, tempty, abort_flag,
                                          warp, lane);
     } else {
-        // converters: e4m3 staging tile -> scaled bf16 MMA tile
+        // converters: e4m3 raw slot -> scaled bf16 tiles of the MMA slot
         const int ct = threadIdx.x - 192;
         const int KS = p.K / 128;  // scale blocks along K
         const int RS = p.a_rows_per_mat / 128;
-        int stage = 0;
-        uint32_t phase = 0;
+        int rstage = 0, mstage = 0;
+        uint32_t rphase = 0, mphase = 0;
         for (int u = blockIdx.x; u < total; u += gridDim.x) {
             const Unit t = decode_unit(p, pref, u);
+            const int n_mma = (t.n_valid + 15) & ~15;
             const bool routed = t.seg < p.E;
             const int mat = routed ? t.seg : t.seg - p.E;
             const float* sbase = (routed ? scale_routed : scale_shared) + (size_t)mat * RS * KS;
@@ -219,28 +260,29 @@ __global__ void __launch_bounds__(F8_THREADS, 1)
             const float* s_up = sbase + (size_t)(p.a_up_offset / 128 + t.mt) * KS;
             bool ok = true;
             for (int kb = 0; kb < KB; ++kb) {
-                if (!mbar_wait(&raw_full[stage], phase, abort_flag) ||
-                    !mbar_wait(&cvt_empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
-                uint8_t* st = smem + stage * C::STAGE_BYTES;
+                if (!mbar_wait(&m_empty[mstage], mphase ^ 1, abort_flag)) { ok = false; break; }
+                if (!mbar_wait(&raw_full[rstage], rphase, abort_flag)) { ok = false; break; }
+                uint8_t* ms = mring + mstage * C::MSLOT_BYTES;
+                const uint8_t* rs = rring + rstage * C::RSLOT_BYTES;
                 const float sc[2] = {s_gate[kb >> 1], GEMM == 1 ? s_up[kb >> 1] : 0.f};
 #pragma unroll
                 for (int i = 0; i < C::NA * 512 / CVT_THREADS; ++i) {
                     const int task = ct + i * CVT_THREADS;
-                    const int tile = task >> 9;
+                    const int tile = (i * CVT_THREADS) >> 9;  // 512 tasks per tile, ct < CVT_THREADS
                     const int r = task & 127;
                     const int c = (task >> 7) & 3;
-                    const uint8_t* src = st + C::A8_OFF + tile * C::A8_BYTES + r * 64 +
-                                         ((c ^ ((r >> 1) & 3)) << 4);
-                    uint8_t* dst = st + C::CVT_OFF + tile * C::A_BYTES + r * 128;
+                    const uint8_t* src = rs + tile * C::A8_BYTES + r * 64 + ((c ^ ((r >> 1) & 3)) << 4);
+                    uint8_t* dst = ms + C::CVT_OFF + tile * C::A_BYTES + r * 128;
                     uint4 lo, hi;
                     e4m3x16_to_bf16_scaled(*reinterpret_cast<const uint4*>(src), sc[tile], lo, hi);
                     *reinterpret_cast<uint4*>(dst + (((2 * c) ^ (r & 7)) << 4)) = lo;
                     *reinterpret_cast<uint4*>(dst + (((2 * c + 1) ^ (r & 7)) << 4)) = hi;
                 }
+                mbar_arrive(&raw_empty[rstage]);
                 fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
-                mbar_arrive(&cvt_full[stage]);
-                mbar_arrive(&raw_empty[stage]);
-                if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+                mbar_arrive(&cvt_full[mstage]);
+                if (++rstage == C::RSTAGES) { rstage = 0; rphase ^= 1; }
+                if (++mstage == C::MSTAGES) { mstage = 0; mphase ^= 1; }
             }
             if (!ok) break;
         }
@@ -257,13 +299,13 @@ __global__ void __launch_bounds__(F8_THREADS, 1)
 
 }  // namespace
 
-template <int GEMM, int BNF_, int ACCB_>
+template <int GEMM, int BNF_, int ACCB_, int MST_>
 cudaError_t launch_fp8w(const GroupedGemmArgs& a, cudaStream_t st) {
-    using C = TileF8<GEMM, BNF_, ACCB_>;
+    using C = TileF8<GEMM, BNF_, ACCB_, MST_>;
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(grouped_gemm_fp8w_kernel<GEMM, BNF_, ACCB_>,
+        attr_err = cudaFuncSetAttribute(grouped_gemm_fp8w_kernel<GEMM, BNF_, ACCB_, MST_>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     });
     if (attr_err != cudaSuccess) return attr_err;
@@ -281,7 +323,7 @@ cudaError_t launch_fp8w(const GroupedGemmArgs& a, cudaStream_t st) {
     if (b_rows == 0) return cudaSuccess;
     if (!make_bmaps(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.b_rows, b_rows, p.K, BK))
         return cudaErrorInvalidValue;
-    grouped_gemm_fp8w_kernel<GEMM, BNF_, ACCB_><<<grid_for(p), F8_THREADS, C::SMEM_BYTES, st>>>(
+    grouped_gemm_fp8w_kernel<GEMM, BNF_, ACCB_, MST_><<<grid_for(p), F8_THREADS, C::SMEM_BYTES, st>>>(
         tmAr, tmAs, tmB, p, static_cast<const float*>(a.w_routed_scale),
         static_cast<const float*>(S > 0 ? a.w_shared_scale : a.w_routed_scale));
     return cudaGetLastError();
@@ -289,11 +331,13 @@ cudaError_t launch_fp8w(const GroupedGemmArgs& a, cudaStream_t st) {
 
 cudaError_t launch_gemm_fp8w(const GroupedGemmArgs& a, cudaStream_t st) {
     // many tokens per expert: wide token tiles (each weight tile converted once
-    // per expert); few tokens per expert: narrower double-buffered tiles
+    // per expert); few tokens per expert: narrower double-buffered tiles. The
+    // last argument is the MMA-ring depth; the raw ring takes the rest of
+    // shared memory (up to 8 slots).
     const bool wide = a.N >= 128L * a.E;
     if (a.gemm == 1)
-        return wide ? launch_fp8w<1, 240, 1>(a, st) : launch_fp8w<1, 128, 2>(a, st);
-    return wide ? launch_fp8w<2, 240, 2>(a, st) : launch_fp8w<2, 128, 2>(a, st);
+        return wide ? launch_fp8w<1, 240, 1, 2>(a, st) : launch_fp8w<1, 128, 2, 3>(a, st);
+    return wide ? launch_fp8w<2, 240, 2, 3>(a, st) : launch_fp8w<2, 128, 2, 3>(a, st);
 }
 
 }  // namespace gemm
