@@ -258,13 +258,26 @@ __global__ void __launch_bounds__(F8_THREADS, 1)
             const float* sbase = (routed ? scale_routed : scale_shared) + (size_t)mat * RS * KS;
             const float* s_gate = sbase + (size_t)(t.mt) * KS;
             const float* s_up = sbase + (size_t)(p.a_up_offset / 128 + t.mt) * KS;
+            // the scales of K block j serve stages 2j and 2j+1; the next block's are
+            // loaded two stages ahead so the load never stalls a conversion
+            float g_cur = s_gate[0], u_cur = GEMM == 1 ? s_up[0] : 0.f;
+            float g_nxt = KS > 1 ? s_gate[1] : 0.f, u_nxt = (GEMM == 1 && KS > 1) ? s_up[1] : 0.f;
             bool ok = true;
             for (int kb = 0; kb < KB; ++kb) {
+                if (kb > 0 && (kb & 1) == 0) {
+                    g_cur = g_nxt;
+                    u_cur = u_nxt;
+                    const int nj = (kb >> 1) + 1;
+                    if (nj < KS) {
+                        g_nxt = s_gate[nj];
+                        if (GEMM == 1) u_nxt = s_up[nj];
+                    }
+                }
                 if (!mbar_wait(&m_empty[mstage], mphase ^ 1, abort_flag)) { ok = false; break; }
                 if (!mbar_wait(&raw_full[rstage], rphase, abort_flag)) { ok = false; break; }
                 uint8_t* ms = mring + mstage * C::MSLOT_BYTES;
                 const uint8_t* rs = rring + rstage * C::RSLOT_BYTES;
-                const float sc[2] = {s_gate[kb >> 1], GEMM == 1 ? s_up[kb >> 1] : 0.f};
+                const float sc[2] = {g_cur, u_cur};
 #pragma unroll
                 for (int i = 0; i < C::NA * 512 / CVT_THREADS; ++i) {
                     const int task = ct + i * CVT_THREADS;
