@@ -252,7 +252,6 @@ __global__ void __launch_bounds__(F8_THREADS, 1)
         uint32_t rphase = 0, mphase = 0;
         for (int u = blockIdx.x; u < total; u += gridDim.x) {
             const Unit t = decode_unit(p, pref, u);
-            const int n_mma = (t.n_valid + 15) & ~15;
             const bool routed = t.seg < p.E;
             const int mat = routed ? t.seg : t.seg - p.E;
             const float* sbase = (routed ? scale_routed : scale_shared) + (size_t)mat * RS * KS;

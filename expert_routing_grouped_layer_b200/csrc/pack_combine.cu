@@ -3,7 +3,9 @@
 //
 // Gather + quantise: each expert row r of the GEMM input is token
 // sorted_pair[r] / k of x (rows past N are the tokens in order, for the shared
-// experts). Quantisation follows the activation format:
+// experts). When those shared-expert rows exist, they are quantised first and
+// the routed rows are byte copies of them, so every token is quantised once.
+// Quantisation follows the activation format:
 //  * FP8_E4M3_POW2_B128 ("DeepSeek-V4-Pro 架构与代码概述", 文件说明, kernel.py
 //    act_quant_kernel: FP8 per 128-element block, power-of-two scale): scale
 //    2^e with e the smallest integer such that amax <= 448 * 2^e;
@@ -33,21 +35,46 @@ __device__ __forceinline__ int token_of_row(int r, const int32_t* sorted_pair, i
     return (t >= 0 && t < T) ? t : -1;
 }
 
-__global__ void __launch_bounds__(256) pack_bf16_kernel(const uint4* __restrict__ x, int H8,
-                                                        const int32_t* __restrict__ sorted_pair,
-                                                        int N, int k, int T, int n_rows,
-                                                        uint4* __restrict__ out) {
+__device__ __forceinline__ void st_stream16(uint4* p, uint4 v) {
+    asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
+                 "r"(v.w)
+                 : "memory");
+}
+
+// Row gather: expert row r (< n_rows) becomes row src_row0 + token_of_row(r) of
+// src, row16 16-byte vectors (and, when ssrc is set, the same for srow16-vector
+// scale rows); a row without a valid pair is zero-filled. One warp per row,
+// four loads in flight per lane, streaming stores (the rows are read once, by
+// the GEMM, after the whole gather).
+__global__ void __launch_bounds__(256) gather_rows_kernel(
+    const uint4* __restrict__ src, int src_row0, int row16, const uint4* __restrict__ ssrc,
+    int srow16, const int32_t* __restrict__ sorted_pair, int N, int k, int T, int n_rows,
+    uint4* __restrict__ dst, uint4* __restrict__ sdst) {
     const int lane = threadIdx.x & 31;
     const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
     if (r >= n_rows) return;
     const int t = token_of_row(r, sorted_pair, N, k, T);
-    uint4* dst = out + (size_t)r * H8;
+    uint4* d = dst + (size_t)r * row16;
     if (t < 0) {
-        for (int v = lane; v < H8; v += 32) dst[v] = make_uint4(0, 0, 0, 0);
+        for (int v = lane; v < row16; v += 32) d[v] = make_uint4(0, 0, 0, 0);
+        if (ssrc)
+            for (int v = lane; v < srow16; v += 32) sdst[(size_t)r * srow16 + v] = make_uint4(0, 0, 0, 0);
         return;
     }
-    const uint4* src = x + (size_t)t * H8;
-    for (int v = lane; v < H8; v += 32) dst[v] = src[v];
+    const uint4* s = src + (size_t)(src_row0 + t) * row16;
+    int v = lane;
+    for (; v + 96 < row16; v += 128) {
+        const uint4 a0 = s[v], a1 = s[v + 32], a2 = s[v + 64], a3 = s[v + 96];
+        st_stream16(d + v, a0);
+        st_stream16(d + v + 32, a1);
+        st_stream16(d + v + 64, a2);
+        st_stream16(d + v + 96, a3);
+    }
+    for (; v < row16; v += 32) st_stream16(d + v, s[v]);
+    if (ssrc) {
+        const uint4* ss = ssrc + (size_t)(src_row0 + t) * srow16;
+        for (int w = lane; w < srow16; w += 32) st_stream16(sdst + (size_t)r * srow16 + w, ss[w]);
+    }
 }
 
 // exponent of the power-of-two scale: smallest e with a <= 448 * 2^e
@@ -83,11 +110,12 @@ __global__ void __launch_bounds__(256) pack_fp8_kernel(const __nv_bfloat16* __re
                                                        const int32_t* __restrict__ sorted_pair,
                                                        int N, int k, int T, int n_rows,
                                                        uint8_t* __restrict__ out,
-                                                       uint8_t* __restrict__ out_scale, int per32) {
+                                                       uint8_t* __restrict__ out_scale, int per32,
+                                                       int row0) {
     constexpr int BLK = (AFMT == MOE_A_FP8_E4M3_POW2_B128) ? 128 : 32;
     const int SBLK = per32 ? 32 : BLK;  // elements per stored scale
     const int lane = threadIdx.x & 31;
-    const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int r = row0 + blockIdx.x * 8 + (threadIdx.x >> 5);
     if (r >= n_rows) return;
     const int t = token_of_row(r, sorted_pair, N, k, T);
     const __nv_bfloat16* src = x + (size_t)(t < 0 ? 0 : t) * H;
@@ -173,19 +201,40 @@ cudaError_t launch_pack_rows(int afmt, const void* x, int H, const int32_t* sort
                              int k, int T, int n_rows, void* out, uint8_t* out_scale, int per32,
                              cudaStream_t st) {
     if (n_rows == 0) return cudaSuccess;
-    dim3 grid((n_rows + 7) / 8);
-    if (afmt == MOE_A_BF16)
-        pack_bf16_kernel<<<grid, 256, 0, st>>>(static_cast<const uint4*>(x), H / 8, sorted_pair, N,
-                                               k, T, n_rows, static_cast<uint4*>(out));
-    else if (afmt == MOE_A_FP8_E4M3_POW2_B128)
+    if (afmt == MOE_A_BF16) {
+        gather_rows_kernel<<<(n_rows + 7) / 8, 256, 0, st>>>(
+            static_cast<const uint4*>(x), 0, H / 8, nullptr, 0, sorted_pair, N, k, T, n_rows,
+            static_cast<uint4*>(out), nullptr);
+        return cudaGetLastError();
+    }
+    const int blk = (afmt == MOE_A_FP8_E4M3_POW2_B128) ? 128 : 32;
+    const int sbytes = H / (per32 ? 32 : blk);  // scale bytes per row
+    // With shared-expert rows (rows N..N+T-1 are the tokens in order), quantise
+    // those T rows once and gather the routed rows from them; otherwise each
+    // routed row is quantised where it is gathered.
+    const bool two_pass = n_rows == N + T && T > 0 && H % 16 == 0 && sbytes % 16 == 0 &&
+                          reinterpret_cast<uintptr_t>(out) % 16 == 0 &&
+                          reinterpret_cast<uintptr_t>(out_scale) % 16 == 0;
+    const int row0 = two_pass ? N : 0;
+    const int q_rows = n_rows - row0;
+    dim3 grid((q_rows + 7) / 8);
+    if (afmt == MOE_A_FP8_E4M3_POW2_B128)
         pack_fp8_kernel<MOE_A_FP8_E4M3_POW2_B128><<<grid, 256, 0, st>>>(
             static_cast<const __nv_bfloat16*>(x), H, sorted_pair, N, k, T, n_rows,
-            static_cast<uint8_t*>(out), out_scale, per32);
+            static_cast<uint8_t*>(out), out_scale, per32, row0);
     else
         pack_fp8_kernel<MOE_A_MXFP8><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), H,
                                                            sorted_pair, N, k, T, n_rows,
                                                            static_cast<uint8_t*>(out), out_scale,
-                                                           per32);
+                                                           per32, row0);
+    if (two_pass && N > 0) {
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        gather_rows_kernel<<<(N + 7) / 8, 256, 0, st>>>(
+            static_cast<const uint4*>(out), N, H / 16, reinterpret_cast<const uint4*>(out_scale),
+            sbytes / 16, sorted_pair, N, k, T, N, static_cast<uint4*>(out),
+            reinterpret_cast<uint4*>(out_scale));
+    }
     return cudaGetLastError();
 }
 
