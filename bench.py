@@ -34,7 +34,22 @@ UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "k2_decode_bf16"
 L2_FLUSH_BYTES = 256 << 20  # > 2x the 126 MB L2
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNELS_PER_STEP = 11  # router split + gemm + reduce, top-k, 3 permute, gather, gate/up, down, combine
+
+
+def launches_per_step(cfg, T, n_sms):
+    """Kernels one layer step launches: router plane split, router GEMM, its
+    split-K reduction when K is split, top-k, 3 permutation kernels, the input
+    pack (quantise + gather for quantised activations with shared experts),
+    gate/up, down, combine. Mirrors the library's router split rule."""
+    E, H = cfg.n_routed_experts, cfg.hidden
+    epad = (E + 127) // 128 * 128
+    kb = H // 64
+    base = (epad // 128) * ((T + 127) // 128)
+    s = max(1, min((n_sms + base - 1) // base, kb // 4))
+    kbps = (kb + s - 1) // s
+    splits = (kb + kbps - 1) // kbps
+    two_pass = cfg.afmt != "bf16" and cfg.n_shared_experts > 0
+    return 2 + (1 if splits > 1 else 0) + 1 + 3 + (2 if two_pass else 1) + 3
 
 
 def parse():
@@ -337,7 +352,7 @@ def run_ours(args, rank, world, dev):
                            "flops": layer_flops(cfg, T),
                            "tflops": layer_flops(cfg, T) / (ms / 1e3) / 1e12},
         "stage_ms": stage_ms,
-        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "gpu_launches": launches_per_step(cfg, T, torch.cuda.get_device_properties(dev).multi_processor_count) * args.steps,
         "wall_s_timed_loop": wall,
         "clocks": clk,
         "e2e": e2e,

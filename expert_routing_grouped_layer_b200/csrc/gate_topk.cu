@@ -40,8 +40,7 @@ __device__ __forceinline__ bool better(float va, int ia, float vb, int ib) {
 }
 
 struct TopkParams {
-    const float* part;
-    int splits;
+    const float* part;  // summed logits [T][E]
     const float* bias;
     int T, E, k, n_group, topk_group, norm, score_fn;
     float rsf;
@@ -57,18 +56,17 @@ __global__ void __launch_bounds__(256) topk_kernel(TopkParams p) {
     if (t >= p.T) return;
     const int E = p.E;
 
-    float sv[MAXJ], spv[MAXJ];
+    // only the biased scores stay in registers; a selected expert's score is
+    // recomputed from its logit at the end (same arithmetic, same value)
+    const float* logit = p.part + (size_t)t * E;  // the router left the summed logits in split 0
+    float spv[MAXJ];
     uint32_t avail = 0;
 #pragma unroll
     for (int j = 0; j < MAXJ; ++j) {
         const int e = lane + 32 * j;
-        sv[j] = 0.f;
         spv[j] = -FLT_MAX;
         if (e < E) {
-            float l = 0.f;
-            for (int s = 0; s < p.splits; ++s) l += p.part[((size_t)s * p.T + t) * E + e];
-            sv[j] = score_of(l, p.score_fn);
-            spv[j] = sv[j] + p.bias[e];
+            spv[j] = score_of(logit[e], p.score_fn) + p.bias[e];
             avail |= 1u << j;
         }
     }
@@ -117,33 +115,47 @@ __global__ void __launch_bounds__(256) topk_kernel(TopkParams p) {
         }
     }
 
-    int my_idx = 0;
-    float my_w = 0.f;
-    for (int r = 0; r < p.k; ++r) {
-        float bv = -FLT_MAX, bs = 0.f;
-        int bi = INT_MAX;
+    // Each lane caches its two best available experts (same order as better());
+    // a round is one warp argmax over the lanes' heads, the winning lane pops
+    // its head and rescans its experts only when its cache runs empty.
+    float v1, v2;
+    int i1, i2;
+    auto refill = [&]() {
+        v1 = v2 = -FLT_MAX;
+        i1 = i2 = INT_MAX;
 #pragma unroll
         for (int j = 0; j < MAXJ; ++j) {
             const int e = lane + 32 * j;
-            if (((avail >> j) & 1u) && better(spv[j], e, bv, bi)) {
-                bv = spv[j];
-                bi = e;
-                bs = sv[j];
+            if ((avail >> j) & 1u) {
+                if (better(spv[j], e, v1, i1)) {
+                    v2 = v1; i2 = i1;
+                    v1 = spv[j]; i1 = e;
+                } else if (better(spv[j], e, v2, i2)) {
+                    v2 = spv[j]; i2 = e;
+                }
             }
         }
+    };
+    refill();
+    int my_idx = 0;
+    for (int r = 0; r < p.k; ++r) {
+        float bv = v1;
+        int bi = i1;
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) {
             const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
             const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-            const float os = __shfl_xor_sync(0xffffffffu, bs, off);
-            if (better(ov, oi, bv, bi)) { bv = ov; bi = oi; bs = os; }
+            if (better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
         }
-        if (bi != INT_MAX && (bi & 31) == lane) avail &= ~(1u << (bi >> 5));
-        if (lane == r) {
-            my_idx = bi;
-            my_w = bs;
+        if (lane == r) my_idx = bi;
+        if (bi != INT_MAX && (bi & 31) == lane) {
+            avail &= ~(1u << (bi >> 5));
+            v1 = v2; i1 = i2;
+            v2 = -FLT_MAX; i2 = INT_MAX;
+            if (i1 == INT_MAX) refill();
         }
     }
+    float my_w = (lane < p.k && my_idx >= 0 && my_idx < E) ? score_of(logit[my_idx], p.score_fn) : 0.f;
 
     float sum = (lane < p.k) ? my_w : 0.f;
 #pragma unroll
@@ -168,7 +180,6 @@ cudaError_t launch_topk(const moe_config* c, const float* part, int splits, cons
     if (T == 0) return cudaSuccess;
     TopkParams p;
     p.part = part;
-    p.splits = 1;  // the router left the summed logits in split 0
     p.bias = bias;
     p.T = T;
     p.E = c->n_routed_experts;

@@ -20,7 +20,7 @@ namespace {
 
 using gemm::BK;
 using gemm::BM;
-using gemm::B_BOX;
+using gemm::BMaps;
 
 constexpr int RT_BN = 128;
 constexpr int RT_STAGES = 3;
@@ -54,6 +54,16 @@ __device__ __forceinline__ RUnit router_unit(const RouterParams& p, int u) {
     return r;
 }
 
+// One 3-D box: the same 128 x 64 tile of the three weight planes, planes outermost.
+__device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* tmap, int32_t x, int32_t y,
+                                            int32_t z, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+        : "memory");
+}
+
 // hi / mid / lo bf16 planes of the fp32 router weight, rows padded to Epad with zeros.
 __global__ void __launch_bounds__(256) router_split_kernel(const float* __restrict__ wg,
                                                            __nv_bfloat16* __restrict__ planes,
@@ -74,7 +84,7 @@ __global__ void __launch_bounds__(256) router_split_kernel(const float* __restri
 }
 
 __global__ void __launch_bounds__(192, 1)
-    router_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+    router_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ BMaps tmX,
                      const RouterParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -102,7 +112,7 @@ __global__ void __launch_bounds__(192, 1)
         *abort_flag = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tmW);
-        tma_prefetch_desc(&tmX);
+        gemm::prefetch_bmaps(tmX);
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, RT_TMEM_COLS);
@@ -121,19 +131,16 @@ __global__ void __launch_bounds__(192, 1)
             int issued = 0;
             for (int u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x) {
                 const RUnit r = router_unit(p, u);
-                const int nb = ((r.n_valid + 15) & ~15) / B_BOX;
-                const uint32_t tx = 3 * RT_A_BYTES + nb * B_BOX * BK * 2;
+                const int n16 = (r.n_valid + 15) & ~15;
+                const uint32_t tx = 3 * RT_A_BYTES + n16 * BK * 2;
                 bool ok = true;
                 for (int kb = r.kb0; kb < r.kb1; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
                     uint8_t* st = smem + stage * RT_STAGE_BYTES;
                     mbar_arrive_expect_tx(&full[stage], tx);
-                    for (int pl = 0; pl < 3; ++pl)
-                        tma_load_2d(st + pl * RT_A_BYTES, &tmW, kb * BK, pl * p.Epad + r.mt * BM,
-                                    &full[stage]);
-                    for (int i = 0; i < nb; ++i)
-                        tma_load_2d(st + 3 * RT_A_BYTES + i * B_BOX * BK * 2, &tmX, kb * BK,
-                                    r.t0 + i * B_BOX, &full[stage]);
+                    tma_load_3d(st, &tmW, kb * BK, r.mt * BM, 0, &full[stage]);
+                    gemm::load_b_rows(st + 3 * RT_A_BYTES, tmX, kb * BK, r.t0, n16, BK * 2,
+                                      &full[stage]);
                     ++issued;
                     if (++stage == RT_STAGES) { stage = 0; phase ^= 1; }
                 }
@@ -225,6 +232,20 @@ __global__ void __launch_bounds__(192, 1)
 
 }  // namespace
 
+// The three planes [3][Epad][H] as a 3-D tensor: box 64 columns x 128 rows x 3
+// planes, 128-byte swizzle, so one copy fills the three A tiles of a stage.
+static bool make_tmap_planes(CUtensorMap* tm, const void* planes, uint64_t Epad, uint64_t H) {
+    auto enc = gemm::get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {H, Epad, 3};
+    cuuint64_t strides[2] = {H * 2, Epad * H * 2};
+    cuuint32_t box[3] = {(cuuint32_t)BK, (cuuint32_t)BM, 3};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(planes), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 RouterPlan router_plan(int T, int E, int H) {
     RouterPlan r;
     r.Epad = (E + BM - 1) / BM * BM;
@@ -251,9 +272,10 @@ cudaError_t launch_router_tc(const void* x, const float* gate_w, void* planes, f
     const long n = (long)plan.Epad * H;
     router_split_kernel<<<(unsigned)std::min<long>((n + 255) / 256, 4L * num_sms()), 256, 0, st>>>(
         gate_w, static_cast<__nv_bfloat16*>(planes), E, plan.Epad, H);
-    CUtensorMap tmW, tmX;
-    if (!gemm::make_tmap_bf16(&tmW, planes, 3ull * plan.Epad, H, BM) ||
-        !gemm::make_tmap_bf16(&tmX, x, (uint64_t)T, H, B_BOX))
+    CUtensorMap tmW;
+    BMaps tmX;
+    if (!make_tmap_planes(&tmW, planes, plan.Epad, H) ||
+        !gemm::make_bmaps(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, (uint64_t)T, H, BK))
         return cudaErrorInvalidValue;
     RouterParams p;
     p.T = T;
