@@ -87,7 +87,7 @@ WsLayout ws_layout(const moe_config* c, int T) {
     L.row_of = take(N * 4);
     L.chunk_counts = take((size_t)L.n_chunks * E * 4);
     L.xa = take((N + T) * H * act_bytes);
-    L.xa_scale = take(act_bytes == 1 ? (N + T) * (H / 32) : 0);
+    L.xa_scale = take(act_bytes == 1 ? (N + T) * (H / 32) : (f16_gate_up(c) ? (N + T) : 0));
     L.hbuf = take((N + S * T) * I * act_bytes);
     L.h_scale = take(act_bytes == 1 ? (N + S * T) * (I / 32) : 0);
     L.y = take(N * H * 2);
@@ -226,8 +226,11 @@ moe_status moe_pack_expert_inputs(const moe_config* cfg, const void* x, int32_t 
     if (!config_valid(cfg) || T < 0) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
     if (!x || !sorted_pair || !xa || !aligned16(x) || !aligned16(xa)) return MOE_ERR_INVALID_ARG;
-    if (cfg->afmt != MOE_A_BF16 && !xa_scale) return MOE_ERR_INVALID_ARG;
+    if ((cfg->afmt != MOE_A_BF16 || f16_gate_up(cfg)) && !xa_scale) return MOE_ERR_INVALID_ARG;
     const int k = cfg->num_experts_per_tok, N = T * k;
+    if (f16_gate_up(cfg))
+        return cuda_status(launch_pack_f16_rows(x, cfg->hidden, sorted_pair, N, k, T, N + T, xa,
+                                                static_cast<int8_t*>(xa_scale), as_stream(stream)));
     return cuda_status(launch_pack_rows(cfg->afmt, x, cfg->hidden, sorted_pair, N, k, T, N + T, xa,
                                         static_cast<uint8_t*>(xa_scale), 1, as_stream(stream)));
 }
@@ -242,6 +245,7 @@ moe_status moe_expert_gate_up(const moe_config* cfg, const void* xa, const void*
     const bool q = cfg->afmt != MOE_A_BF16;
     if (!xa || !expert_offsets || !h || !aligned16(xa) || !aligned16(h)) return MOE_ERR_INVALID_ARG;
     if (q && (!xa_scale || !h_scale)) return MOE_ERR_INVALID_ARG;
+    if (f16_gate_up(cfg) && !xa_scale) return MOE_ERR_INVALID_ARG;
     if (!weights_ok(cfg, w, true)) return MOE_ERR_INVALID_ARG;
     GroupedGemmArgs a = gemm_args(cfg, T, expert_offsets, dev_status);
     const size_t hrow = (size_t)a.I * (q ? 1 : 2);

@@ -1,6 +1,8 @@
 // gemm_fp8w.cu -- per-expert SwiGLU MLP with FP8 (E4M3, 128x128 block-scaled)
 // weights and bf16 activations on the tcgen05 tensor cores. The expert
-// structure, tile schedule and epilogue are those of gemm_bf16.cu.
+// structure and tile schedule are those of gemm_bf16.cu.
+#include <cuda_fp16.h>
+
 #include "gemm_common.cuh"
 
 namespace moe {
@@ -9,14 +11,18 @@ namespace {
 
 // ---------------------------------------------------------------- FP8 weights
 // E4M3 weights with one fp32 scale per 128x128 block ("DeepSeek-V4-Pro 架构与代码概述",
-// 文件说明: Linear with block-scaled FP8 weights; block 128x128). The activations
-// stay bf16, so the tensor-core operands are bf16: a converter warpgroup turns
-// each TMA-staged E4M3 weight tile (64-byte swizzled rows) into bf16 values
+// 文件说明: Linear with block-scaled FP8 weights; block 128x128). There is no
+// tensor-core instruction for E4M3 times bf16, so a converter warpgroup turns
+// each TMA-staged E4M3 weight tile (64-byte swizzled rows) into 16-bit values
 // times the tile's block scale, written straight into the 128B-swizzled
 // K-major layout tcgen05.mma reads. With BK = 64 inside a 128-wide scale block
 // and M tiles aligned to the 128-row blocks, one scalar scale covers a tile.
-// E4M3 -> bf16 is exact; the product with the fp32 scale is rounded once to
-// bf16 (relative error <= 2^-9 per weight).
+//  * gate/up: f16 operands (see the f16 path below): one cvt and one f16x2
+//    multiply per two weights; token rows come in as f16 with a power-of-two
+//    row scale.
+//  * down: bf16 operands, since its input h is the bf16 SwiGLU output; E4M3 ->
+//    bf16 is exact and the product with the fp32 scale is rounded once to bf16
+//    (relative error <= 2^-9 per weight).
 constexpr int CVT_WARPS = 8;
 constexpr int CVT_THREADS = CVT_WARPS * 32;
 constexpr int B_WARP = 6 + CVT_WARPS;  // token-tile loader, after the converters
@@ -73,13 +79,115 @@ __device__ __forceinline__ void e4m3x16_to_bf16_scaled(uint4 v, float scale, uin
     hi = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
+// ---- f16 path of the gate/up GEMM. The tensor-core operands are f16: token
+// rows arrive as x * 2^-e (exact, see pack_f16_kernel) and each weight tile is
+// E4M3 (exact in f16) times m = s * 2^-E rounded to f16, where s is the tile's
+// 128x128 block scale and 2^E the largest power of two not above the largest
+// block scale of the 128 rows' K range (|m| < 2; weight products round once in
+// f16, <= 2^-11 relative, plus <= 2^-12 for m). The epilogue multiplies the
+// accumulator by 2^E * 2^e exactly. Conversion is one cvt and one f16x2
+// multiply per two weights.
+
+// Exponent E of a 128-row tile: max over its KS block scales of floor(log2 s),
+// kept in [-126, 126]. Every lane of the warp returns the same value.
+__device__ __forceinline__ int tile_exp(const float* __restrict__ srow, int KS, int lane) {
+    int e = -126;
+    for (int j = lane; j < KS; j += 32) {
+        const float sj = srow[j];
+        if (sj > 0.f) e = max(e, ilogbf(sj));
+    }
+    e = __reduce_max_sync(0xffffffffu, e);
+    return min(e, 126);
+}
+
+__device__ __forceinline__ float pow2f(int e) {  // 2^e for e in [-126, 127]
+    return __uint_as_float((uint32_t)(127 + e) << 23);
+}
+
+// 16 E4M3 values times the f16 pair (m, m) -> 16 f16 values, in element order.
+__device__ __forceinline__ void e4m3x16_to_f16_scaled(uint4 v, __half2 m2, uint4& lo, uint4& hi) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const __nv_fp8x2_storage_t pair = (__nv_fp8x2_storage_t)((w[i] >> (16 * h)) & 0xFFFFu);
+            const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+            const __half2 p = __hmul2(*reinterpret_cast<const __half2*>(&hr), m2);
+            o[2 * i + h] = *reinterpret_cast<const uint32_t*>(&p);
+        }
+    }
+    lo = make_uint4(o[0], o[1], o[2], o[3]);
+    hi = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+// Instruction descriptor, kind::f16 with f16 A and B (format 0), fp32 accumulate.
+__host__ __device__ __forceinline__ uint32_t idesc_f16(uint32_t M, uint32_t N) {
+    return (1u << 4) | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+
+// Gate/up epilogue of the f16 path: per unit, wait for the accumulator, read it
+// 16 token columns at a time (lane = output feature), restore 2^E (gate and up
+// tiles) and 2^e (token row), apply SwiGLU, store bf16, release the buffer.
+template <int ACC_COLS, int ACCB>
+__device__ __forceinline__ void epilogue_f16_gate_up(const KParams& p, const int* pref, int total,
+                                                     uint32_t tmem_base, uint64_t* tfull,
+                                                     uint64_t* tempty, volatile int* abort_flag,
+                                                     int warp, int lane,
+                                                     const float* __restrict__ scale_routed,
+                                                     const float* __restrict__ scale_shared,
+                                                     const int8_t* __restrict__ row_exp) {
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const int KS = p.K / 128;
+    const int RS = p.a_rows_per_mat / 128;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int u = blockIdx.x; u < total; u += gridDim.x) {
+        const Unit t = decode_unit(p, pref, u);
+        const bool routed = t.seg < p.E;
+        const int mat = routed ? t.seg : t.seg - p.E;
+        const float* sbase = (routed ? scale_routed : scale_shared) + (size_t)mat * RS * KS;
+        const float fg = pow2f(tile_exp(sbase + (size_t)t.mt * KS, KS, lane));
+        const float fu = pow2f(tile_exp(sbase + (size_t)(p.a_up_offset / 128 + t.mt) * KS, KS, lane));
+        if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * ACC_COLS;
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(t.out) + t.mt * BM + row;
+        for (int c0 = 0; c0 < t.n_valid; c0 += 16) {
+            uint32_t g[16], uu[16];
+            tmem_ld16(taddr + c0, g);
+            tmem_ld16(taddr + ACC_COLS / 2 + c0, uu);
+            // 2^e of this lane's token column (e in [-127, 114]; 2^-127 is subnormal)
+            const int ex_l = (lane < 16 && c0 + lane < t.n_valid) ? row_exp[t.b_row + c0 + lane] : 0;
+            const float fe_l = ex_l >= -126 ? pow2f(ex_l) : __uint_as_float(0x00400000u);
+            tmem_ld_wait(g, uu);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const float fe = __shfl_sync(0xffffffffu, fe_l, j);
+                if (c0 + j < t.n_valid) {
+                    const float gv = __uint_as_float(g[j]) * fg * fe;  // exact power-of-two factors
+                    const float uv = __uint_as_float(uu[j]) * fu * fe;
+                    const float a = gv / (1.0f + __expf(-gv)) * uv;
+                    out[(size_t)(c0 + j) * p.ld_out] = __float2bfloat16_rn(a);
+                }
+            }
+        }
+        tc_fence_before();
+        mbar_arrive(&tempty[acc]);
+        if (++acc == ACCB) { acc = 0; acc_phase ^= 1; }
+    }
+}
+
 template <int GEMM, int BNF_, int ACCB_, int MST_>
 __global__ void __launch_bounds__(F8_THREADS, 1)
     grouped_gemm_fp8w_kernel(const __grid_constant__ CUtensorMap tmA_routed,
                              const __grid_constant__ CUtensorMap tmA_shared,
                              const __grid_constant__ BMaps tmB, const KParams p,
                              const float* __restrict__ scale_routed,
-                             const float* __restrict__ scale_shared) {
+                             const float* __restrict__ scale_shared,
+                             const int8_t* __restrict__ row_exp) {
     using C = TileF8<GEMM, BNF_, ACCB_, MST_>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -178,7 +286,7 @@ __global__ void __launch_bounds__(F8_THREADS, 1)
             for (int u = blockIdx.x; u < total; u += gridDim.x) {
                 const Unit t = decode_unit(p, pref, u);
                 const int n_mma = (t.n_valid + 15) & ~15;
-                const uint32_t idesc = idesc_bf16(BM, n_mma);
+                const uint32_t idesc = GEMM == 1 ? idesc_f16(BM, n_mma) : idesc_bf16(BM, n_mma);
                 if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag)) break;
                 tc_fence_after();
                 const uint32_t d0 = tmem_base + acc * C::ACC_COLS;
@@ -241,8 +349,13 @@ __global__ void __launch_bounds__(F8_THREADS, 1)
             }
         }
     } else if (warp < 6) {
-        epilogue_loop<GEMM, C::ACC_COLS, C::ACCB>(p, pref, total, tmem_base, tfull, tempty, abort_flag,
-                                         warp, lane);
+        if (GEMM == 1)
+            epilogue_f16_gate_up<C::ACC_COLS, C::ACCB>(p, pref, total, tmem_base, tfull, tempty,
+                                                       abort_flag, warp, lane, scale_routed,
+                                                       scale_shared, row_exp);
+        else
+            epilogue_loop<2, C::ACC_COLS, C::ACCB>(p, pref, total, tmem_base, tfull, tempty,
+                                                   abort_flag, warp, lane);
     } else {
         // converters: e4m3 raw slot -> scaled bf16 tiles of the MMA slot
         const int ct = threadIdx.x - 192;
@@ -257,6 +370,9 @@ __global__ void __launch_bounds__(F8_THREADS, 1)
             const float* sbase = (routed ? scale_routed : scale_shared) + (size_t)mat * RS * KS;
             const float* s_gate = sbase + (size_t)(t.mt) * KS;
             const float* s_up = sbase + (size_t)(p.a_up_offset / 128 + t.mt) * KS;
+            // gate/up (f16 path): block scales relative to the tile's power of two
+            const float inv_g = GEMM == 1 ? pow2f(-tile_exp(s_gate, KS, lane)) : 1.f;
+            const float inv_u = GEMM == 1 ? pow2f(-tile_exp(s_up, KS, lane)) : 1.f;
             // the scales of K block j serve stages 2j and 2j+1; the next block's are
             // loaded two stages ahead so the load never stalls a conversion
             float g_cur = s_gate[0], u_cur = GEMM == 1 ? s_up[0] : 0.f;
@@ -277,6 +393,7 @@ __global__ void __launch_bounds__(F8_THREADS, 1)
                 uint8_t* ms = mring + mstage * C::MSLOT_BYTES;
                 const uint8_t* rs = rring + rstage * C::RSLOT_BYTES;
                 const float sc[2] = {g_cur, u_cur};
+                const __half2 m2[2] = {__float2half2_rn(g_cur * inv_g), __float2half2_rn(u_cur * inv_u)};
 #pragma unroll
                 for (int i = 0; i < C::NA * 512 / CVT_THREADS; ++i) {
                     const int task = ct + i * CVT_THREADS;
@@ -286,7 +403,10 @@ __global__ void __launch_bounds__(F8_THREADS, 1)
                     const uint8_t* src = rs + tile * C::A8_BYTES + r * 64 + ((c ^ ((r >> 1) & 3)) << 4);
                     uint8_t* dst = ms + C::CVT_OFF + tile * C::A_BYTES + r * 128;
                     uint4 lo, hi;
-                    e4m3x16_to_bf16_scaled(*reinterpret_cast<const uint4*>(src), sc[tile], lo, hi);
+                    if (GEMM == 1)
+                        e4m3x16_to_f16_scaled(*reinterpret_cast<const uint4*>(src), m2[tile], lo, hi);
+                    else
+                        e4m3x16_to_bf16_scaled(*reinterpret_cast<const uint4*>(src), sc[tile], lo, hi);
                     *reinterpret_cast<uint4*>(dst + (((2 * c) ^ (r & 7)) << 4)) = lo;
                     *reinterpret_cast<uint4*>(dst + (((2 * c + 1) ^ (r & 7)) << 4)) = hi;
                 }
@@ -333,11 +453,14 @@ cudaError_t launch_fp8w(const GroupedGemmArgs& a, cudaStream_t st) {
                            (uint64_t)(S > 0 ? S : a.E) * p.a_rows_per_mat, p.K, BM))
         return cudaErrorInvalidValue;
     if (b_rows == 0) return cudaSuccess;
-    if (!make_bmaps(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.b_rows, b_rows, p.K, BK))
+    // gate/up reads f16 token rows (x * 2^-e), down reads the bf16 SwiGLU output
+    if (!make_bmaps(&tmB, GEMM == 1 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                    2, a.b_rows, b_rows, p.K, BK))
         return cudaErrorInvalidValue;
     grouped_gemm_fp8w_kernel<GEMM, BNF_, ACCB_, MST_><<<grid_for(p), F8_THREADS, C::SMEM_BYTES, st>>>(
         tmAr, tmAs, tmB, p, static_cast<const float*>(a.w_routed_scale),
-        static_cast<const float*>(S > 0 ? a.w_shared_scale : a.w_routed_scale));
+        static_cast<const float*>(S > 0 ? a.w_shared_scale : a.w_routed_scale),
+        reinterpret_cast<const int8_t*>(a.b_scale));
     return cudaGetLastError();
 }
 
@@ -348,7 +471,7 @@ cudaError_t launch_gemm_fp8w(const GroupedGemmArgs& a, cudaStream_t st) {
     // shared memory (up to 8 slots).
     const bool wide = a.N >= 128L * a.E;
     if (a.gemm == 1)
-        return wide ? launch_fp8w<1, 240, 1, 2>(a, st) : launch_fp8w<1, 128, 2, 3>(a, st);
+        return wide ? launch_fp8w<1, 240, 1, 3>(a, st) : launch_fp8w<1, 128, 2, 3>(a, st);
     return wide ? launch_fp8w<2, 240, 2, 3>(a, st) : launch_fp8w<2, 128, 2, 3>(a, st);
 }
 

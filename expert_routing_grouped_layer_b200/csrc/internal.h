@@ -56,6 +56,13 @@ cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int n_chunks
 cudaError_t launch_pack_rows(int afmt, const void* x, int H, const int32_t* sorted_pair, int N,
                              int k, int T, int n_rows, void* out, uint8_t* out_scale, int per32,
                              cudaStream_t st);
+// f16 expert input rows with per-row power-of-two exponents (FP8-weight layers)
+cudaError_t launch_pack_f16_rows(const void* x, int H, const int32_t* sorted_pair, int N, int k,
+                                 int T, int n_rows, void* out, int8_t* xs, cudaStream_t st);
+// true when the gate/up GEMM runs on f16 operands (FP8 weights, bf16 activations)
+inline bool f16_gate_up(const moe_config* c) {
+    return c->wfmt == MOE_W_FP8_E4M3_B128x128 && c->afmt == MOE_A_BF16;
+}
 cudaError_t launch_combine(const void* y, const void* shared_y, int S, const int32_t* row_of,
                            const float* w, int T, int k, int H, void* out, cudaStream_t st);
 

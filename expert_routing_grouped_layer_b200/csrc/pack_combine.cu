@@ -19,6 +19,7 @@
 // the shared experts): one CTA per token, 16-byte vector loads of every row it
 // needs, fp32 sums in slot order, one bf16 rounding.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
 #include "internal.h"
@@ -43,13 +44,15 @@ __device__ __forceinline__ void st_stream16(uint4* p, uint4 v) {
 
 // Row gather: expert row r (< n_rows) becomes row src_row0 + token_of_row(r) of
 // src, row16 16-byte vectors (and, when ssrc is set, the same for srow16-vector
-// scale rows); a row without a valid pair is zero-filled. One warp per row,
+// scale rows; when esrc is set, one exponent byte per row); a row without a
+// valid pair is zero-filled. One warp per row,
 // four loads in flight per lane, streaming stores (the rows are read once, by
 // the GEMM, after the whole gather).
 __global__ void __launch_bounds__(256) gather_rows_kernel(
     const uint4* __restrict__ src, int src_row0, int row16, const uint4* __restrict__ ssrc,
     int srow16, const int32_t* __restrict__ sorted_pair, int N, int k, int T, int n_rows,
-    uint4* __restrict__ dst, uint4* __restrict__ sdst) {
+    uint4* __restrict__ dst, uint4* __restrict__ sdst, const int8_t* __restrict__ esrc,
+    int8_t* __restrict__ edst) {
     const int lane = threadIdx.x & 31;
     const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
     if (r >= n_rows) return;
@@ -59,8 +62,10 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(
         for (int v = lane; v < row16; v += 32) d[v] = make_uint4(0, 0, 0, 0);
         if (ssrc)
             for (int v = lane; v < srow16; v += 32) sdst[(size_t)r * srow16 + v] = make_uint4(0, 0, 0, 0);
+        if (esrc && lane == 0) edst[r] = 0;
         return;
     }
+    if (esrc && lane == 0) edst[r] = esrc[src_row0 + t];
     const uint4* s = src + (size_t)(src_row0 + t) * row16;
     int v = lane;
     for (; v + 96 < row16; v += 128) {
@@ -145,6 +150,59 @@ __global__ void __launch_bounds__(256) pack_fp8_kernel(const __nv_bfloat16* __re
     }
 }
 
+// f16 rows with a power-of-two row scale, the input of the f16 tensor-core path
+// of the FP8-weight gate/up GEMM: row r holds x[t] * 2^-e_r and xs[r] = e_r,
+// with e_r chosen so the row's largest magnitude lies in [2^13, 2^14). A bf16
+// value has an 8-bit significand, so it is exact in f16 wherever the scaled
+// value is at least 2^-17 (every element within 2^-30 of the row's largest);
+// only smaller ones round, by at most 2^-25 of 2^e_r. One warp per row, rows
+// from row0; two passes over the row (amax, then conversion).
+__global__ void __launch_bounds__(256) pack_f16_kernel(const uint4* __restrict__ x, int H8,
+                                                       const int32_t* __restrict__ sorted_pair,
+                                                       int N, int k, int T, int n_rows, int row0,
+                                                       uint4* __restrict__ out,
+                                                       int8_t* __restrict__ xs) {
+    const int lane = threadIdx.x & 31;
+    const int r = row0 + blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (r >= n_rows) return;
+    const int t = token_of_row(r, sorted_pair, N, k, T);
+    uint4* dst = out + (size_t)r * H8;
+    if (t < 0) {
+        for (int v = lane; v < H8; v += 32) dst[v] = make_uint4(0, 0, 0, 0);
+        if (lane == 0) xs[r] = 0;
+        return;
+    }
+    const uint4* src = x + (size_t)t * H8;
+    // bf16 magnitudes order like their bit patterns (sign bit cleared)
+    uint32_t m = 0;
+    for (int v = lane; v < H8; v += 32) {
+        const uint4 u = src[v];
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) m = max(m, max(w[i] & 0x7FFFu, (w[i] >> 16) & 0x7FFFu));
+    }
+    m = __reduce_max_sync(0xffffffffu, m);
+    int e = 0;
+    if (m != 0) {
+        const int E = ilogbf(__uint_as_float(m << 16));  // floor(log2(amax)), exact
+        e = min(max(E - 13, -127), 114);
+    }
+    const float sc = __uint_as_float((uint32_t)(127 - e) << 23);  // 2^-e, a normal float
+    for (int v = lane; v < H8; v += 32) {
+        const uint4 u = src[v];
+        const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&u);
+        uint4 o;
+        __half2* h = reinterpret_cast<__half2*>(&o);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(b[i]);
+            h[i] = __floats2half2_rn(f.x * sc, f.y * sc);
+        }
+        st_stream16(dst + v, o);
+    }
+    if (lane == 0) xs[r] = (int8_t)e;
+}
+
 __global__ void __launch_bounds__(128) combine_kernel(const __nv_bfloat16* __restrict__ y,
                                                       const __nv_bfloat16* __restrict__ shared_y,
                                                       int S, const int32_t* __restrict__ row_of,
@@ -204,7 +262,7 @@ cudaError_t launch_pack_rows(int afmt, const void* x, int H, const int32_t* sort
     if (afmt == MOE_A_BF16) {
         gather_rows_kernel<<<(n_rows + 7) / 8, 256, 0, st>>>(
             static_cast<const uint4*>(x), 0, H / 8, nullptr, 0, sorted_pair, N, k, T, n_rows,
-            static_cast<uint4*>(out), nullptr);
+            static_cast<uint4*>(out), nullptr, nullptr, nullptr);
         return cudaGetLastError();
     }
     const int blk = (afmt == MOE_A_FP8_E4M3_POW2_B128) ? 128 : 32;
@@ -233,7 +291,26 @@ cudaError_t launch_pack_rows(int afmt, const void* x, int H, const int32_t* sort
         gather_rows_kernel<<<(N + 7) / 8, 256, 0, st>>>(
             static_cast<const uint4*>(out), N, H / 16, reinterpret_cast<const uint4*>(out_scale),
             sbytes / 16, sorted_pair, N, k, T, N, static_cast<uint4*>(out),
-            reinterpret_cast<uint4*>(out_scale));
+            reinterpret_cast<uint4*>(out_scale), nullptr, nullptr);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_pack_f16_rows(const void* x, int H, const int32_t* sorted_pair, int N, int k,
+                                 int T, int n_rows, void* out, int8_t* xs, cudaStream_t st) {
+    if (n_rows == 0) return cudaSuccess;
+    // with shared-expert rows, convert the T token rows once and gather the rest
+    const bool two_pass = n_rows == N + T && T > 0;
+    const int row0 = two_pass ? N : 0;
+    pack_f16_kernel<<<(n_rows - row0 + 7) / 8, 256, 0, st>>>(static_cast<const uint4*>(x), H / 8,
+                                                            sorted_pair, N, k, T, n_rows, row0,
+                                                            static_cast<uint4*>(out), xs);
+    if (two_pass && N > 0) {
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        gather_rows_kernel<<<(N + 7) / 8, 256, 0, st>>>(
+            static_cast<const uint4*>(out), N, H / 8, nullptr, 0, sorted_pair, N, k, T, N,
+            static_cast<uint4*>(out), nullptr, xs, xs);
     }
     return cudaGetLastError();
 }

@@ -180,9 +180,14 @@ moe_status moe_quantize_activations(const moe_config *cfg, const void *x, int32_
  * per [V4] act_quant_kernel / [MX] MXFP8). x bf16 [T][H]; sorted_pair from
  * moe_permute. Row r < N of xa holds token sorted_pair[r] / k of x, rows N..N+T-1
  * hold the tokens in order (the shared experts' input). xa is bf16 [N+T][H]
- * for BF16 activations, else uint8 E4M3 [N+T][H] with xa_scale uint8 E8M0
+ * for BF16 activations with BF16 weights; with FP8 weights (BF16 activations) xa
+ * is f16 [N+T][H] holding the row times 2^-e and xa_scale int8 [N+T] holds e
+ * (the row's largest magnitude scaled into [2^13, 2^14); exact for every
+ * element within 2^-30 of it), the input of the f16 tensor-core gate/up GEMM;
+ * for quantised activations xa is uint8 E4M3 [N+T][H] with xa_scale uint8 E8M0
  * [N+T][H/32]: one code per 32 elements, the power-of-two format's per-128 code
- * repeated over its four 32-element sub-blocks (xa_scale unused for BF16). */
+ * repeated over its four 32-element sub-blocks (xa_scale unused for BF16
+ * activations with BF16 weights). */
 moe_status moe_pack_expert_inputs(const moe_config *cfg, const void *x, int32_t T,
                                   const int32_t *sorted_pair, void *xa, void *xa_scale,
                                   void *stream);
@@ -195,6 +200,7 @@ moe_status moe_pack_expert_inputs(const moe_config *cfg, const void *x, int32_t 
  * (quantised activations). h is [N + S*T][I]: rows 0..N-1 follow xa, rows
  * N + s*T + t belong to shared expert s and token t; h_scale [N + S*T][I/32]
  * (one E8M0 code per 32 features, per-128 codes repeated as for xa_scale).
+ * xa / xa_scale as written by moe_pack_expert_inputs for the same config.
  * E2M1 / MXFP4 weights need E4M3 activations and H, I multiples of 512.
  * A pipeline wait past its time limit sets MOE_DEV_TIMEOUT. */
 moe_status moe_expert_gate_up(const moe_config *cfg, const void *xa, const void *xa_scale,

@@ -148,3 +148,49 @@ def test_mx896_full_size_zipf():
     g, _ = _layer_check(cfg, sample=6, seed=3)
     counts = np.diff(g["offsets"])
     assert counts.max() > 10 * counts.mean()  # hot experts take >10x the mean
+
+
+def test_fp8_weights_extreme_row_magnitudes():
+    """FP8 weights run gate/up on f16 operands, each token row scaled by its own
+    power of two: rows from 2^-30 to 2^30 times the usual magnitude (far outside
+    f16's range unscaled) and a row whose elements span 2^30 must still match the
+    oracle row by row. Routing comes from the unscaled inputs and is passed to
+    both sides, so only the expert computation sees the extreme rows."""
+    cfg = FP8_TINY.replace(T=96, hidden=512, moe_intermediate_size=256,
+                           shared_intermediate_size=256, n_routed_experts=8,
+                           num_experts_per_tok=3, n_shared_experts=2)
+    T, H, k = cfg.T, cfg.hidden, cfg.num_experts_per_tok
+    dev = torch.device("cuda")
+    inp = W.make_inputs(cfg, dev)
+    wts = W.make_weights(cfg, dev)
+    r = oracle_route(cfg, inp, T=T)
+    g = torch.Generator(device="cpu").manual_seed(11)
+    row_exp = torch.tensor([-30, -17, -8, 0, 9, 16, 30], dtype=torch.float64)[
+        torch.randint(0, 7, (T,), generator=g)]
+    xs = inp["x"].double().cpu() * torch.exp2(row_exp)[:, None]
+    xs[5] = inp["x"][5].double().cpu() * torch.exp2(
+        torch.randint(-20, 11, (H,), generator=g).double())  # one row spanning 2^30
+    x_big = xs.to(torch.bfloat16).to(dev)
+    layer = moe.MoELayer(cfg, wts, inp["gate_w"], inp["gate_bias"], max_tokens=T, device=dev)
+    P = lambda which: layer.ws_ptr(T, which)
+    st, ws, ccfg, cw = layer.status, layer.ws, layer.ccfg, layer.cw
+    idx = torch.as_tensor(r["idx"], dtype=torch.int32, device=dev).contiguous()
+    w = torch.as_tensor(r["w"], dtype=torch.float32, device=dev).contiguous()
+    out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    moe.moe_permute(ccfg, idx, T, P(moe.WS_OFFSETS), P(moe.WS_SORTED_PAIR), P(moe.WS_ROW_OF), st,
+                    ws, ws.numel())
+    moe.moe_pack_expert_inputs(ccfg, x_big, T, P(moe.WS_SORTED_PAIR), P(moe.WS_XA),
+                               P(moe.WS_XA_SCALE))
+    moe.moe_expert_gate_up(ccfg, P(moe.WS_XA), P(moe.WS_XA_SCALE), T, P(moe.WS_OFFSETS), cw,
+                           P(moe.WS_H), P(moe.WS_H_SCALE), st)
+    moe.moe_expert_down(ccfg, P(moe.WS_H), P(moe.WS_H_SCALE), T, P(moe.WS_OFFSETS), cw,
+                        P(moe.WS_Y), P(moe.WS_SHARED_Y), st)
+    moe.moe_combine(ccfg, P(moe.WS_Y), P(moe.WS_SHARED_Y), P(moe.WS_ROW_OF), w, T, out)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    want = oracle.layer(cfg, W.bf16_codes(x_big), r["idx"], r["w"],
+                        lambda e: W.expert_slice(wts, e), lambda s: W.expert_slice(wts, s, shared=True))
+    got = out.double().cpu().numpy()
+    assert np.isfinite(got).all()
+    err = np.linalg.norm(got - want, axis=1) / np.maximum(np.linalg.norm(want, axis=1), 1e-300)
+    assert err.max() <= LAYER_TOL["bf16"], (err.max(), int(err.argmax()))
