@@ -26,7 +26,7 @@ namespace {
 constexpr int CVT_WARPS = 8;
 constexpr int CVT_THREADS = CVT_WARPS * 32;
 constexpr int B_WARP = 6 + CVT_WARPS;  // token-tile loader, after the converters
-constexpr int F8_THREADS = 64 + 128 + CVT_THREADS + 32;
+constexpr int EPI2_WARP = B_WARP + 1;  // second epilogue group (gate/up), after the loader
 static_assert(512 % CVT_THREADS == 0, "converter tasks: whole tiles per round");
 
 // GEMM: 1 gate/up, 2 down. BNF_: tokens per tile. ACCB_: accumulator buffers in
@@ -37,6 +37,10 @@ static_assert(512 % CVT_THREADS == 0, "converter tasks: whole tiles per round");
 // the token tile, freed by the MMA commit.
 template <int GEMM, int BNF_, int ACCB_, int MST_>
 struct TileF8 {
+    // gate/up (f16 path, ~86 registers) affords a second group of 4 epilogue
+    // warps, which halves the drain of its single accumulator buffer
+    static constexpr int EG = (GEMM == 1) ? 2 : 1;
+    static constexpr int THREADS = 64 + 128 + CVT_THREADS + 32 + 128 * (EG - 1);
     static constexpr int NA = (GEMM == 1) ? 2 : 1;
     static constexpr int BNF = BNF_;
     static constexpr int ACCB = ACCB_;
@@ -128,13 +132,14 @@ __host__ __device__ __forceinline__ uint32_t idesc_f16(uint32_t M, uint32_t N) {
 }
 
 // Gate/up epilogue of the f16 path: per unit, wait for the accumulator, read it
-// 16 token columns at a time (lane = output feature), restore 2^E (gate and up
-// tiles) and 2^e (token row), apply SwiGLU, store bf16, release the buffer.
-template <int ACC_COLS, int ACCB>
+// 16 token columns at a time (lane = output feature; group g of GROUPS takes
+// chunks g, g + GROUPS, ...), restore 2^E (gate and up tiles) and 2^e (token
+// row), apply SwiGLU, store bf16, release the buffer (128 * GROUPS arrivals).
+template <int ACC_COLS, int ACCB, int GROUPS>
 __device__ __forceinline__ void epilogue_f16_gate_up(const KParams& p, const int* pref, int total,
                                                      uint32_t tmem_base, uint64_t* tfull,
                                                      uint64_t* tempty, volatile int* abort_flag,
-                                                     int warp, int lane,
+                                                     int warp, int lane, int group,
                                                      const float* __restrict__ scale_routed,
                                                      const float* __restrict__ scale_shared,
                                                      const int8_t* __restrict__ row_exp) {
@@ -155,7 +160,7 @@ __device__ __forceinline__ void epilogue_f16_gate_up(const KParams& p, const int
         tc_fence_after();
         const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * ACC_COLS;
         __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(t.out) + t.mt * BM + row;
-        for (int c0 = 0; c0 < t.n_valid; c0 += 16) {
+        for (int c0 = 16 * group; c0 < t.n_valid; c0 += 16 * GROUPS) {
             uint32_t g[16], uu[16];
             tmem_ld16(taddr + c0, g);
             tmem_ld16(taddr + ACC_COLS / 2 + c0, uu);
@@ -181,7 +186,7 @@ __device__ __forceinline__ void epilogue_f16_gate_up(const KParams& p, const int
 }
 
 template <int GEMM, int BNF_, int ACCB_, int MST_>
-__global__ void __launch_bounds__(F8_THREADS, 1)
+__global__ void __launch_bounds__(TileF8<GEMM, BNF_, ACCB_, MST_>::THREADS, 1)
     grouped_gemm_fp8w_kernel(const __grid_constant__ CUtensorMap tmA_routed,
                              const __grid_constant__ CUtensorMap tmA_shared,
                              const __grid_constant__ BMaps tmB, const KParams p,
@@ -221,7 +226,7 @@ __global__ void __launch_bounds__(F8_THREADS, 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull[a], 1);
-            mbar_init(&tempty[a], 128);
+            mbar_init(&tempty[a], 128 * C::EG);
         }
         mbar_init(mma_done, 1);
         *abort_flag = 0;
@@ -348,11 +353,11 @@ __global__ void __launch_bounds__(F8_THREADS, 1)
                 }
             }
         }
-    } else if (warp < 6) {
+    } else if (warp < 6 || warp >= EPI2_WARP) {
         if (GEMM == 1)
-            epilogue_f16_gate_up<C::ACC_COLS, C::ACCB>(p, pref, total, tmem_base, tfull, tempty,
-                                                       abort_flag, warp, lane, scale_routed,
-                                                       scale_shared, row_exp);
+            epilogue_f16_gate_up<C::ACC_COLS, C::ACCB, C::EG>(
+                p, pref, total, tmem_base, tfull, tempty, abort_flag, warp, lane,
+                warp < 6 ? 0 : 1, scale_routed, scale_shared, row_exp);
         else
             epilogue_loop<2, C::ACC_COLS, C::ACCB>(p, pref, total, tmem_base, tfull, tempty,
                                                    abort_flag, warp, lane);
@@ -457,7 +462,7 @@ cudaError_t launch_fp8w(const GroupedGemmArgs& a, cudaStream_t st) {
     if (!make_bmaps(&tmB, GEMM == 1 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
                     2, a.b_rows, b_rows, p.K, BK))
         return cudaErrorInvalidValue;
-    grouped_gemm_fp8w_kernel<GEMM, BNF_, ACCB_, MST_><<<grid_for(p), F8_THREADS, C::SMEM_BYTES, st>>>(
+    grouped_gemm_fp8w_kernel<GEMM, BNF_, ACCB_, MST_><<<grid_for(p), C::THREADS, C::SMEM_BYTES, st>>>(
         tmAr, tmAs, tmB, p, static_cast<const float*>(a.w_routed_scale),
         static_cast<const float*>(S > 0 ? a.w_shared_scale : a.w_routed_scale),
         reinterpret_cast<const int8_t*>(a.b_scale));
