@@ -33,11 +33,12 @@ constexpr int SF_TILE = 128 * 16; // scale tile: 128 rows x 16 k-blocks of 32
 // in tensor memory (2 overlaps a tile's epilogue with the next tile's main
 // loop; 1 lets gate/up use 240-token tiles). Warps: 0 TMA, 1 MMA, then EG
 // groups of 4 epilogue warps (one per TMEM lane quadrant), then the scale
-// warp. Single-buffered gate/up tiles take two epilogue groups, since there
-// the quantising epilogue is not overlapped with the next tile's main loop.
+// warp. Single-buffered gate/up tiles take three epilogue groups (measured
+// faster than two), since there the quantising epilogue is not overlapped
+// with the next tile's main loop.
 template <int GEMM, int BNX_, int ACCB_>
 struct TileMX {
-    static constexpr int EG = (GEMM == 1 && ACCB_ == 1) ? 2 : 1;
+    static constexpr int EG = (GEMM == 1 && ACCB_ == 1) ? 3 : 1;
     static constexpr int THREADS = 64 + 128 * EG + 32;
     static constexpr int SCALE_WARP = 2 + 4 * EG;
     static constexpr int RED_BYTES = EG * 2 * 4 * 16 * 4;  // [group][parity][warp][16 columns]
