@@ -203,7 +203,9 @@ __global__ void __launch_bounds__(256) pack_f16_kernel(const uint4* __restrict__
     if (lane == 0) xs[r] = (int8_t)e;
 }
 
-__global__ void __launch_bounds__(128) combine_kernel(const __nv_bfloat16* __restrict__ y,
+// Large batches: one CTA per token, threads striding over the row's 16-byte
+// columns, the k expert rows and S shared rows of a column summed in order.
+__global__ void __launch_bounds__(128) combine_token_kernel(const __nv_bfloat16* __restrict__ y,
                                                       const __nv_bfloat16* __restrict__ shared_y,
                                                       int S, const int32_t* __restrict__ row_of,
                                                       const float* __restrict__ w, int T, int k,
@@ -251,6 +253,76 @@ __global__ void __launch_bounds__(128) combine_kernel(const __nv_bfloat16* __res
         for (int i = 0; i < 4; ++i) ob[i] = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
         *reinterpret_cast<uint4*>(out + (size_t)t * H + (size_t)v * 8) = o;
     }
+}
+
+// Small batches: one CTA per (token, block of 128 16-byte columns): thread v loads column v of all of
+// the token's k expert rows and S shared rows first (up to 32 + 4 loads in
+// flight), then sums them in slot order, then shared order, in fp32, and
+// rounds once to bf16. MAXR >= k + S rows are held per thread (k <= 32, S <= 4).
+template <int MAXR>
+__global__ void __launch_bounds__(128) combine_kernel(const __nv_bfloat16* __restrict__ y,
+                                                      const __nv_bfloat16* __restrict__ shared_y,
+                                                      int S, const int32_t* __restrict__ row_of,
+                                                      const float* __restrict__ w, int T, int k,
+                                                      int H, __nv_bfloat16* __restrict__ out) {
+    __shared__ int32_t rows[32];
+    __shared__ float wts[32];
+    // column blocks of one token are consecutive CTAs, so each token's rows are
+    // read front to back in time
+    const int H8 = H / 8;
+    const int nblk = (H8 + 127) / 128;
+    const int t = blockIdx.x / nblk;
+    if (threadIdx.x < k) {
+        rows[threadIdx.x] = row_of[(size_t)t * k + threadIdx.x];
+        wts[threadIdx.x] = w[(size_t)t * k + threadIdx.x];
+    }
+    __syncthreads();
+    const int v = (blockIdx.x % nblk) * blockDim.x + threadIdx.x;
+    if (v >= H8) return;
+    const int nr = k + S;
+    uint4 u[MAXR];
+#pragma unroll
+    for (int j = 0; j < MAXR; ++j) {
+        if (j < nr) {
+            const uint4* src = nullptr;
+            if (j < k) {
+                if (rows[j] >= 0) src = reinterpret_cast<const uint4*>(y + (size_t)rows[j] * H) + v;
+            } else {
+                src = reinterpret_cast<const uint4*>(shared_y + ((size_t)(j - k) * T + t) * H) + v;
+            }
+            u[j] = src ? *src : make_uint4(0, 0, 0, 0);
+        }
+    }
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll
+    for (int j = 0; j < MAXR; ++j) {
+        if (j < k) {
+            if (rows[j] < 0) continue;
+            const float wj = wts[j];
+            const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&u[j]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 f = __bfloat1622float2(b[i]);
+                acc[2 * i] = fmaf(wj, f.x, acc[2 * i]);
+                acc[2 * i + 1] = fmaf(wj, f.y, acc[2 * i + 1]);
+            }
+        } else if (j < nr) {
+            const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&u[j]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 f = __bfloat1622float2(b[i]);
+                acc[2 * i] += f.x;
+                acc[2 * i + 1] += f.y;
+            }
+        }
+    }
+    uint4 o;
+    __nv_bfloat162* ob = reinterpret_cast<__nv_bfloat162*>(&o);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) ob[i] = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+    *reinterpret_cast<uint4*>(out + (size_t)t * H + (size_t)v * 8) = o;
 }
 
 }  // namespace
@@ -318,9 +390,22 @@ cudaError_t launch_pack_f16_rows(const void* x, int H, const int32_t* sorted_pai
 cudaError_t launch_combine(const void* y, const void* shared_y, int S, const int32_t* row_of,
                            const float* w, int T, int k, int H, void* out, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
-    combine_kernel<<<T, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(y),
-                                      static_cast<const __nv_bfloat16*>(shared_y), S, row_of, w, T,
-                                      k, H, static_cast<__nv_bfloat16*>(out));
+    const unsigned grid = (unsigned)T * (unsigned)((H / 8 + 127) / 128);
+    const auto* yy = static_cast<const __nv_bfloat16*>(y);
+    const auto* sy = static_cast<const __nv_bfloat16*>(shared_y);
+    auto* o = static_cast<__nv_bfloat16*>(out);
+    // enough tokens to fill the GPU with one CTA each (the column-split CTAs
+    // are latency-bound: measured slower at 16384 tokens, faster at 128)
+    if (T >= 8 * num_sms()) {
+        combine_token_kernel<<<T, 128, 0, st>>>(yy, sy, S, row_of, w, T, k, H, o);
+        return cudaGetLastError();
+    }
+    if (k + S <= 12)
+        combine_kernel<12><<<grid, 128, 0, st>>>(yy, sy, S, row_of, w, T, k, H, o);
+    else if (k + S <= 20)
+        combine_kernel<20><<<grid, 128, 0, st>>>(yy, sy, S, row_of, w, T, k, H, o);
+    else
+        combine_kernel<36><<<grid, 128, 0, st>>>(yy, sy, S, row_of, w, T, k, H, o);
     return cudaGetLastError();
 }
 

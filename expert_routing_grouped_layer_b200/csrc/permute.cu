@@ -3,7 +3,8 @@
 // expert id into contiguous blocks).
 //
 // Deterministic stable counting sort of the N = T*k (token, slot) pairs by
-// expert id, in three launches without atomics on the output order:
+// expert id, in three launches without atomics on the output order (one
+// launch doing all three steps when the pairs fit one chunk):
 //   1. count:   per chunk of PERM_CHUNK pairs, a per-expert histogram;
 //   2. scan:    expert totals -> expert_offsets, and each chunk's starting row
 //               per expert (exclusive prefix over chunks);
@@ -140,6 +141,88 @@ __global__ void __launch_bounds__(PERM_WARPS * 32) perm_scatter_kernel(
     }
 }
 
+// All pairs in one chunk (N <= PERM_CHUNK): count, scan and scatter in one CTA,
+// the same per-warp histograms and in-warp ranks as the three launches, so the
+// order is the same.
+__global__ void __launch_bounds__(PERM_WARPS * 32) perm_single_kernel(
+    const int32_t* __restrict__ idx, long N, int E, int32_t* __restrict__ offsets,
+    int32_t* __restrict__ sorted_pair, int32_t* __restrict__ row_of, int32_t* status) {
+    __shared__ int32_t wbase[PERM_WARPS][PERM_MAX_E];
+    __shared__ int32_t excl[PERM_MAX_E];
+    __shared__ int32_t part[PERM_WARPS * 32];
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    for (int i = tid; i < PERM_WARPS * E; i += blockDim.x) wbase[i / E][i % E] = 0;
+    __syncthreads();
+    const long wstart = (long)w * PERM_PER_WARP;
+    bool bad = false;
+    for (int it = 0; it < PERM_PER_WARP; it += 32) {
+        const long p = wstart + it + lane;
+        const bool valid = p < N;
+        const int e = valid ? idx[p] : -1;
+        const bool ok = valid && e >= 0 && e < E;
+        bad |= valid && !ok;
+        const unsigned act = __ballot_sync(0xffffffffu, ok);
+        if (ok) {
+            const unsigned m = __match_any_sync(act, e);
+            if ((__ffs(m) - 1) == lane) wbase[w][e] += __popc(m);
+        }
+        __syncwarp();
+    }
+    if (bad) status_or(status, MOE_DEV_BAD_EXPERT);
+    __syncthreads();
+    // exclusive scan of the expert totals: thread tid owns experts [tid*per, (tid+1)*per)
+    const int per = (E + blockDim.x - 1) / blockDim.x;
+    int mine = 0;
+    for (int e = tid * per; e < min(E, (tid + 1) * per); ++e) {
+        int tot = 0;
+        for (int ww = 0; ww < PERM_WARPS; ++ww) tot += wbase[ww][e];
+        excl[e] = tot;
+        mine += tot;
+    }
+    int v = mine;  // inclusive scan over threads
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += o;
+    }
+    part[tid] = v;
+    __syncthreads();
+    int base = v - mine;
+    for (int ww = 0; ww < w; ++ww) base += part[ww * 32 + 31];
+    for (int e = tid * per; e < min(E, (tid + 1) * per); ++e) {
+        const int tot = excl[e];
+        offsets[e] = base;
+        int run = base;
+        for (int ww = 0; ww < PERM_WARPS; ++ww) {
+            const int n = wbase[ww][e];
+            wbase[ww][e] = run;
+            run += n;
+        }
+        base += tot;
+    }
+    if (tid == blockDim.x - 1) offsets[E] = base;
+    __syncthreads();
+    const unsigned lt = (1u << lane) - 1u;
+    for (int it = 0; it < PERM_PER_WARP; it += 32) {
+        const long p = wstart + it + lane;
+        const bool valid = p < N;
+        const int e = valid ? idx[p] : -1;
+        const bool ok = valid && e >= 0 && e < E;
+        const unsigned act = __ballot_sync(0xffffffffu, ok);
+        if (ok) {
+            const unsigned m = __match_any_sync(act, e);
+            const int pos = wbase[w][e] + __popc(m & lt);
+            sorted_pair[pos] = (int32_t)p;
+            row_of[p] = pos;
+            __syncwarp(act);
+            if ((__ffs(m) - 1) == lane) wbase[w][e] += __popc(m);
+        } else if (valid) {
+            row_of[p] = -1;
+        }
+        __syncwarp();
+    }
+}
+
 }  // namespace
 
 int permute_chunks(long N) { return (int)((N + PERM_CHUNK - 1) / PERM_CHUNK); }
@@ -148,11 +231,14 @@ cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int n_chunks
                            int32_t* offsets, int32_t* sorted_pair, int32_t* row_of,
                            int32_t* status, cudaStream_t st) {
     const long N = (long)T * k;
-    if (n_chunks > 0) perm_count_kernel<<<n_chunks, 256, 0, st>>>(idx, N, E, chunk, status);
+    if (n_chunks <= 1) {
+        perm_single_kernel<<<1, PERM_WARPS * 32, 0, st>>>(idx, N, E, offsets, sorted_pair, row_of,
+                                                          status);
+        return cudaGetLastError();
+    }
+    perm_count_kernel<<<n_chunks, 256, 0, st>>>(idx, N, E, chunk, status);
     perm_scan_kernel<<<1, 1024, 0, st>>>(chunk, n_chunks, E, offsets);
-    if (n_chunks > 0)
-        perm_scatter_kernel<<<n_chunks, PERM_WARPS * 32, 0, st>>>(idx, N, E, chunk, sorted_pair,
-                                                                   row_of);
+    perm_scatter_kernel<<<n_chunks, PERM_WARPS * 32, 0, st>>>(idx, N, E, chunk, sorted_pair, row_of);
     return cudaGetLastError();
 }
 
