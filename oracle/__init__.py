@@ -34,7 +34,7 @@ _lib = None
 
 W_FMT = {"bf16": 0, "fp8_e4m3_b128x128": 1, "fp4_e2m1_ue8m0_b32": 2, "mxfp4": 3}
 A_FMT = {"bf16": 0, "fp8_e4m3_pow2_b128": 1, "mxfp8": 2}
-SCORE = {"sigmoid": 0, "sqrtsoftplus": 1}
+SCORE = {"sigmoid": 0, "sqrtsoftplus": 1, "softmax": 2}
 NEAR_TIE_REL = 1e-6  # relative score gap under which a selection counts as a near-tie
 
 _P = ctypes.c_void_p
@@ -86,7 +86,7 @@ def lib() -> ctypes.CDLL:
             l.or_expert_input.restype = _I
             l.or_expert_input.argtypes = [_I, _P, _I, _I, _P, _P, _P]
             l.or_expert_rows.restype = _I
-            l.or_expert_rows.argtypes = [_I, _I, _P, _P, _P, _P, _I, _I, _I, _P, _I, _P]
+            l.or_expert_rows.argtypes = [_I, _I, _P, _P, _P, _P, _I, _I, _I, _P, _I, _D, _P]
             l.or_combine.restype = None
             l.or_combine.argtypes = [_I, _I, _I, _I, _P, _P, _P, _P]
             _lib = l
@@ -255,8 +255,10 @@ def expert_input(afmt: str, x_rows_u16):
     return xin, q, sc
 
 
-def expert_rows(wfmt: str, afmt: str, w13, w13s, w2, w2s, e: int, I: int, H: int, xin):
-    """SwiGLU of matrix e of the given weight tensors on rows xin[n, H] -> y[n, H]."""
+def expert_rows(wfmt: str, afmt: str, w13, w13s, w2, w2s, e: int, I: int, H: int, xin,
+                limit: float = 0.0):
+    """SwiGLU of matrix e of the given weight tensors on rows xin[n, H] -> y[n, H];
+    limit > 0 clamps the gate from above and the up projection to +-limit."""
     xin = _c(xin, np.float64)
     n = xin.shape[0]
     y = np.zeros((n, H), np.float64)
@@ -265,7 +267,7 @@ def expert_rows(wfmt: str, afmt: str, w13, w13s, w2, w2s, e: int, I: int, H: int
     w13s = None if w13s is None else np.ascontiguousarray(w13s)
     w2s = None if w2s is None else np.ascontiguousarray(w2s)
     rc = lib().or_expert_rows(W_FMT[wfmt], A_FMT[afmt], _ptr(w13), _ptr(w13s), _ptr(w2), _ptr(w2s),
-                              e, I, H, _ptr(xin), n, _ptr(y))
+                              e, I, H, _ptr(xin), n, float(limit), _ptr(y))
     if rc != 0:
         raise ValueError("bad expert arguments")
     return y
@@ -295,13 +297,14 @@ def layer(cfg, x_rows_u16, idx, w, get_expert, get_shared):
     idx = np.asarray(idx)
     n, k = idx.shape
     xin, _, _ = expert_input(cfg.afmt, x_rows_u16)
+    lim = float(getattr(cfg, "swiglu_limit", 0.0))
     y = np.zeros((n, k, H), np.float64)
     for e in np.unique(idx):
         rows, slots = np.nonzero(idx == e)
         w13, w13s, w2, w2s = get_expert(int(e))
-        y[rows, slots] = expert_rows(cfg.wfmt, cfg.afmt, w13, w13s, w2, w2s, 0, I, H, xin[rows])
+        y[rows, slots] = expert_rows(cfg.wfmt, cfg.afmt, w13, w13s, w2, w2s, 0, I, H, xin[rows], lim)
     ys = np.zeros((cfg.n_shared_experts, n, H), np.float64)
     for s in range(cfg.n_shared_experts):
         w13, w13s, w2, w2s = get_shared(s)
-        ys[s] = expert_rows(cfg.wfmt, cfg.afmt, w13, w13s, w2, w2s, 0, Ish, H, xin)
+        ys[s] = expert_rows(cfg.wfmt, cfg.afmt, w13, w13s, w2, w2s, 0, Ish, H, xin, lim)
     return combine(w, y, ys)

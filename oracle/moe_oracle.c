@@ -48,6 +48,7 @@
 /* scoring */
 #define OR_SCORE_SIGMOID 0
 #define OR_SCORE_SQRTSOFTPLUS 1
+#define OR_SCORE_SOFTMAX 2
 
 #define OR_OK 0
 #define OR_ERR_ARG 1
@@ -209,8 +210,25 @@ enum { C_H, C_E, C_K, C_NG, C_TG, C_I, C_NS, C_ISH, C_NORM, C_SCORE, C_WFMT, C_A
  * form max(l,0) + log1p(exp(-|l|)). */
 double or_score(double l, int score_fn) {
     if (score_fn == OR_SCORE_SIGMOID) return 1.0 / (1.0 + exp(-l));
+    if (score_fn == OR_SCORE_SOFTMAX) return NAN; /* depends on all of a token's logits */
     double sp = (l > 0 ? l : 0.0) + log1p(exp(-fabs(l)));
     return sqrt(sp);
+}
+
+/* [V3] 三.1 contrasts the independent sigmoid scores with softmax ("此消彼长":
+ * one expert's gain is the others' loss). READING: softmax scoring is the usual
+ * softmax over the token's E router logits, s_e = exp(l_e - m) / sum_e' exp(l_e' - m)
+ * with m = max_e l_e (the shift changes nothing mathematically and keeps exp
+ * finite); bias, group selection, top-k and weights then proceed as for the
+ * other scores. */
+static void softmax_scores(const double *l, int E, double *s) {
+    double m = -INFINITY, z = 0.0;
+    for (int e = 0; e < E; e++) m = fmax(m, l[e]);
+    for (int e = 0; e < E; e++) {
+        s[e] = exp(l[e] - m);
+        z += s[e];
+    }
+    for (int e = 0; e < E; e++) s[e] /= z;
 }
 
 /* "a comes before b": larger value first, equal values by lower index
@@ -257,9 +275,10 @@ int or_route_token(const int *icfg, double rsf, const uint16_t *xrow, const floa
         double l = 0.0;
         for (int h = 0; h < H; h++) l += or_bf16_value(xrow[h]) * (double)wg[(size_t)e * H + h];
         if (logits_out) logits_out[e] = l;
-        s[e] = or_score(l, icfg[C_SCORE]);
-        sp[e] = s[e] + (double)bias[e];
+        s[e] = (icfg[C_SCORE] == OR_SCORE_SOFTMAX) ? l : or_score(l, icfg[C_SCORE]);
     }
+    if (icfg[C_SCORE] == OR_SCORE_SOFTMAX) softmax_scores(s, E, s);
+    for (int e = 0; e < E; e++) sp[e] = s[e] + (double)bias[e];
 
     /* group selection */
     int gsz = E / NG;
@@ -409,6 +428,8 @@ int or_expert_input(int afmt, const uint16_t *x, int n, int H, double *xin, uint
 /* One expert's SwiGLU MLP on n input rows ([V3] 三.4: each expert is the
  * gate/up/down MLP with SiLU; [V4] 文件说明 model.py FFNSwiGLU):
  *   g_i = sum_h W13[e][i][h] * xin_h,   u_i = sum_h W13[e][I+i][h] * xin_h,
+ *   with limit > 0 ([V4] 架构: FFNSwiGLU with an optional swiglu_limit cut-off;
+ *   READING: g_i = min(g_i, limit), u_i = clamp(u_i, -limit, limit)),
  *   a_i = SiLU(g_i) * u_i = g_i / (1 + exp(-g_i)) * u_i,
  *   a   -> block quantised along I when activations are quantised (READING:
  *          the second GEMM consumes the intermediate in the layer's activation
@@ -416,7 +437,8 @@ int or_expert_input(int afmt, const uint16_t *x, int n, int H, double *xin, uint
  *   y_n = sum_i W2[e][n][i] * a_i.
  * w13 / w2 point at the whole [n_mat][..] tensors; e selects the matrix. */
 int or_expert_rows(int wfmt, int afmt, const void *w13, const void *w13s, const void *w2,
-                   const void *w2s, int e, int I, int H, const double *xin, int n, double *y) {
+                   const void *w2s, int e, int I, int H, const double *xin, int n, double limit,
+                   double *y) {
     int blk = (afmt == OR_A_FP8_POW2_128) ? 128 : (afmt == OR_A_MXFP8) ? 32 : 0;
     if (blk && I % blk) return OR_ERR_ARG;
     double *a = (double *)malloc(sizeof(double) * (size_t)I * (n > 0 ? n : 1));
@@ -429,6 +451,10 @@ int or_expert_rows(int wfmt, int afmt, const void *w13, const void *w13s, const 
             for (int h = 0; h < H; h++) {
                 g += w_at(wfmt, w13, w13s, 2 * I, H, e, i, h) * xr[h];
                 u += w_at(wfmt, w13, w13s, 2 * I, H, e, I + i, h) * xr[h];
+            }
+            if (limit > 0.0) {
+                g = fmin(g, limit);
+                u = fmax(fmin(u, limit), -limit);
             }
             ar[i] = g / (1.0 + exp(-g)) * u;
         }

@@ -199,3 +199,32 @@ def test_layer_zero_shared_and_weighted_sum():
         want = sum(w[t, j] * oracle.expert_rows("bf16", "bf16", w13, None, w2, None, int(idx[t, j]),
                                                 I, H, xin[t:t + 1])[0] for j in range(3))
         assert np.allclose(out[t], want, rtol=1e-12, atol=1e-15)
+
+
+def test_swiglu_limit_closed_forms():
+    """One-hot input rows make g and u equal to chosen weight columns, so the
+    clamped SwiGLU has closed forms: min(g, L) for the gate, clamp(u, -L, L) for
+    the up projection; a limit above every |g|, |u| changes nothing."""
+    H, I, L = 8, 4, 0.5
+    g = np.array([2.0, -3.0, 0.25, -0.5], np.float32)
+    u = np.array([1.0, -2.0, 0.125, 4.0], np.float32)
+    w13 = np.zeros((1, 2 * I, H), np.float32)
+    w13[0, :I, 0] = g
+    w13[0, I:, 0] = u
+    w2 = np.zeros((1, H, I), np.float32)
+    w2[0, np.arange(I), np.arange(I)] = 1.0  # y_i = a_i for i < I
+    x = np.zeros((1, H))
+    x[0, 0] = 1.0
+
+    def silu(z):
+        return z / (1.0 + math.exp(-z))
+
+    y = oracle.expert_rows("bf16", "bf16", bf16(w13), None, bf16(w2), None, 0, I, H, x, limit=L)
+    want = [silu(min(float(gi), L)) * max(min(float(ui), L), -L) for gi, ui in zip(g, u)]
+    assert np.allclose(y[0, :I], want, rtol=1e-15, atol=0)
+    y_off = oracle.expert_rows("bf16", "bf16", bf16(w13), None, bf16(w2), None, 0, I, H, x)
+    y_big = oracle.expert_rows("bf16", "bf16", bf16(w13), None, bf16(w2), None, 0, I, H, x,
+                               limit=10.0)
+    assert np.array_equal(y_off, y_big)
+    assert np.allclose(y_off[0, :I], [silu(float(gi)) * float(ui) for gi, ui in zip(g, u)],
+                       rtol=1e-15)

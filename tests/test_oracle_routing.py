@@ -231,3 +231,61 @@ def test_route_many_tokens_equals_per_token():
         assert np.array_equal(r["w"][t], one["w"])
     # each token picks k distinct experts
     assert all(len(set(row)) == k for row in r["idx"].tolist())
+
+
+# ----------------------------------------------------------------- softmax scoring
+def test_softmax_equal_logits_give_uniform_scores():
+    """All logits equal: every expert scores 1/E; ties go to the lower indices,
+    and the unnormalised weights are rsf/E each."""
+    E, k = 16, 4
+    c = cfg(E, k, norm=False, rsf=1.5, score="softmax")
+    x, wg = onehot_router(np.full(E, 0.75, np.float32))
+    r = oracle.route_token(c, x, wg, np.zeros(E, np.float32))
+    assert list(r["idx"]) == [0, 1, 2, 3]
+    assert np.allclose(r["w"], 1.5 / E, rtol=1e-15)
+
+
+def test_softmax_scores_sum_to_one_and_follow_exp_ratios():
+    """k = E without normalisation returns every probability: they sum to rsf,
+    and any two are in the ratio exp(l_i - l_j) (the property that defines
+    softmax); adding a constant to all logits changes nothing."""
+    rng = np.random.default_rng(11)
+    E = 32
+    c = cfg(E, E, norm=False, rsf=2.0, score="softmax")
+    # on a 2^-10 grid, so adding 40 below is exact in float32
+    logits = (np.round(rng.standard_normal(E) * 3 * 1024) / 1024).astype(np.float32)
+    x, wg = onehot_router(logits)
+    r = oracle.route_token(c, x, wg, np.zeros(E, np.float32))
+    w = r["w"] / 2.0
+    assert abs(w.sum() - 1.0) < 1e-14
+    l = logits.astype(np.float64)[r["idx"]]
+    for i in range(E):
+        assert math.isclose(w[i] / w[0], math.exp(l[i] - l[0]), rel_tol=1e-12)
+    x2, wg2 = onehot_router(logits + np.float32(40.0))  # large shift: exp would overflow unshifted
+    r2 = oracle.route_token(c, x2, wg2, np.zeros(E, np.float32))
+    assert np.array_equal(r["idx"], r2["idx"]) and np.allclose(r["w"], r2["w"], rtol=1e-12)
+
+
+@pytest.mark.parametrize("ng,tg", [(1, 1), (4, 2)])
+def test_softmax_selection_is_brute_force_topk_of_biased_scores(ng, tg):
+    """Selection on softmax + bias matches exhaustive search over expert subsets
+    of the kept groups (softmax is monotone in the logit, but the bias is added
+    to the probability, so the order can differ from the logits' order)."""
+    rng = np.random.default_rng(12 + ng)
+    E, k = 8, 3
+    c = cfg(E, k, ng=ng, tg=tg, score="softmax")
+    logits = rng.standard_normal(E).astype(np.float32)
+    bias = rng.uniform(-0.2, 0.2, E).astype(np.float32)
+    x, wg = onehot_router(logits)
+    r = oracle.route_token(c, x, wg, bias)
+    l = logits.astype(np.float64)
+    p = np.exp(l - l.max())
+    p /= p.sum()
+    sp = p + bias
+    gsz = E // ng
+    gs = [sum(sorted(sp[g * gsz:(g + 1) * gsz])[-2:]) for g in range(ng)]
+    kept = sorted(range(ng), key=lambda g: -gs[g])[:tg] if ng > 1 else [0]
+    cand = [e for e in range(E) if e // gsz in kept]
+    best = max(itertools.combinations(cand, k), key=lambda sub: sum(sp[e] for e in sub))
+    assert sorted(r["idx"]) == sorted(best)
+    assert np.allclose(r["w"], p[r["idx"]] / p[r["idx"]].sum() * c.routed_scaling_factor, rtol=1e-12)
