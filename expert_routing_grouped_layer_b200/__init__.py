@@ -22,7 +22,7 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUD
 MOE_DEV_BAD_EXPERT = 1
 MOE_DEV_TIMEOUT = 2
 
-SCORE_FN = {"sigmoid": 0, "sqrtsoftplus": 1}
+SCORE_FN = {"sigmoid": 0, "sqrtsoftplus": 1, "softmax": 2}
 WFMT = {"bf16": 0, "fp8_e4m3_b128x128": 1, "fp4_e2m1_ue8m0_b32": 2, "mxfp4": 3}
 AFMT = {"bf16": 0, "fp8_e4m3_pow2_b128": 1, "mxfp8": 2}
 
@@ -52,7 +52,8 @@ class moe_config(ctypes.Structure):
                 ("topk_group", ctypes.c_int32), ("moe_intermediate_size", ctypes.c_int32),
                 ("n_shared_experts", ctypes.c_int32), ("shared_intermediate_size", ctypes.c_int32),
                 ("norm_topk_prob", ctypes.c_int32), ("routed_scaling_factor", ctypes.c_float),
-                ("score_fn", ctypes.c_int32), ("wfmt", ctypes.c_int32), ("afmt", ctypes.c_int32)]
+                ("score_fn", ctypes.c_int32), ("wfmt", ctypes.c_int32), ("afmt", ctypes.c_int32),
+                ("swiglu_limit", ctypes.c_float)]
 
 
 class moe_weights(ctypes.Structure):
@@ -146,7 +147,7 @@ def make_config(cfg) -> moe_config:
                       cfg.topk_group, cfg.moe_intermediate_size, cfg.n_shared_experts,
                       cfg.shared_intermediate_size, int(bool(cfg.norm_topk_prob)),
                       float(cfg.routed_scaling_factor), SCORE_FN[cfg.score_fn], WFMT[cfg.wfmt],
-                      AFMT[cfg.afmt])
+                      AFMT[cfg.afmt], float(getattr(cfg, "swiglu_limit", 0.0)))
 
 
 def make_weights(w: dict, gate_w=None, gate_bias=None) -> moe_weights:

@@ -5,6 +5,8 @@
 #include <algorithm>
 #include <mutex>
 
+#include <cmath>
+
 #include "internal.h"
 
 namespace moe {
@@ -40,7 +42,10 @@ bool config_valid(const moe_config* c) {
         return false;
     if (c->norm_topk_prob != 0 && c->norm_topk_prob != 1) return false;
     if (!(c->routed_scaling_factor > 0.0f)) return false;
-    if (c->score_fn != MOE_SCORE_SIGMOID && c->score_fn != MOE_SCORE_SQRTSOFTPLUS) return false;
+    if (c->score_fn != MOE_SCORE_SIGMOID && c->score_fn != MOE_SCORE_SQRTSOFTPLUS &&
+        c->score_fn != MOE_SCORE_SOFTMAX)
+        return false;
+    if (!(c->swiglu_limit >= 0.0f) || isinf(c->swiglu_limit)) return false;
     if (c->wfmt < MOE_W_BF16 || c->wfmt > MOE_W_MXFP4) return false;
     if (c->afmt < MOE_A_BF16 || c->afmt > MOE_A_MXFP8) return false;
     return true;
@@ -217,6 +222,7 @@ static GroupedGemmArgs gemm_args(const moe_config* cfg, int T, const int32_t* of
     a.afmt = cfg->afmt;
     a.offsets = offsets;
     a.status = dev_status;
+    a.swiglu_limit = cfg->swiglu_limit;
     return a;
 }
 

@@ -3,7 +3,8 @@
 //
 // Selection ("DeepSeek V3架构拆解：Kimi-K2-Thinking-NVFP4的MLA注意力与MoE路由实现原理",
 // 三.2 选专家 and 三.3 权重归一化 + 路由缩放; sqrtsoftplus scoring and route_scale
-// from "DeepSeek-V4-Pro 架构与代码概述", 架构): score, bias, group-limited top-k,
+// from "DeepSeek-V4-Pro 架构与代码概述", 架构; softmax, the alternative 三.1
+// contrasts with sigmoid, over a token's logits): score, bias, group-limited top-k,
 // normalised and scaled weights. The reduction adds each logit's partials in
 // split order, so the logits are deterministic.
 #include <cuda_bf16.h>
@@ -66,9 +67,35 @@ __global__ void __launch_bounds__(256) topk_kernel(TopkParams p) {
         const int e = lane + 32 * j;
         spv[j] = -FLT_MAX;
         if (e < E) {
-            spv[j] = score_of(logit[e], p.score_fn) + p.bias[e];
+            spv[j] = logit[e];
             avail |= 1u << j;
         }
+    }
+    // softmax: s_e = exp(l_e - m) / Z over the token's E logits; m and Z come from
+    // xor-butterfly reductions, which leave the same value in every lane
+    float m = 0.f, z = 1.f;
+    if (p.score_fn == MOE_SCORE_SOFTMAX) {
+        float lm = -FLT_MAX;
+#pragma unroll
+        for (int j = 0; j < MAXJ; ++j) lm = fmaxf(lm, spv[j]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) lm = fmaxf(lm, __shfl_xor_sync(0xffffffffu, lm, off));
+        m = lm;
+        float zs = 0.f;
+#pragma unroll
+        for (int j = 0; j < MAXJ; ++j)
+            if ((avail >> j) & 1u) zs += expf(spv[j] - m);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, off);
+        z = zs;
+    }
+    auto score = [&](float l) {
+        return p.score_fn == MOE_SCORE_SOFTMAX ? expf(l - m) / z : score_of(l, p.score_fn);
+    };
+#pragma unroll
+    for (int j = 0; j < MAXJ; ++j) {
+        const int e = lane + 32 * j;
+        if ((avail >> j) & 1u) spv[j] = score(spv[j]) + p.bias[e];
     }
 
     if (p.n_group > 1) {
@@ -155,7 +182,7 @@ __global__ void __launch_bounds__(256) topk_kernel(TopkParams p) {
             if (i1 == INT_MAX) refill();
         }
     }
-    float my_w = (lane < p.k && my_idx >= 0 && my_idx < E) ? score_of(logit[my_idx], p.score_fn) : 0.f;
+    float my_w = (lane < p.k && my_idx >= 0 && my_idx < E) ? score(logit[my_idx]) : 0.f;
 
     float sum = (lane < p.k) ? my_w : 0.f;
 #pragma unroll

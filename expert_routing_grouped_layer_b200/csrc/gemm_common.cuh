@@ -56,7 +56,17 @@ struct KParams {
     uint8_t* sc_routed;   // per-32 E8M0 scales of quantised outputs (or null)
     uint8_t* sc_shared;
     int32_t* status;
+    float swiglu_limit;   // gate/up: 0 = off, else clamp g from above and u to +-limit
 };
+
+// SwiGLU with the optional limit: SiLU(min(g, L)) * clamp(u, -L, L) for L > 0.
+__device__ __forceinline__ float swiglu(float g, float u, float limit) {
+    if (limit > 0.0f) {
+        g = fminf(g, limit);
+        u = fminf(fmaxf(u, -limit), limit);
+    }
+    return g / (1.0f + __expf(-g)) * u;
+}
 
 struct Unit {
     int seg, mt, n_valid, a_row, b_row;
@@ -154,8 +164,8 @@ __device__ __forceinline__ void epilogue_loop(const KParams& p, const int* pref,
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
                     if (c0 + j < t.n_valid) {
-                        const float gv = __uint_as_float(g[j]);
-                        const float a = gv / (1.0f + __expf(-gv)) * __uint_as_float(uu[j]);
+                        const float a =
+                            swiglu(__uint_as_float(g[j]), __uint_as_float(uu[j]), p.swiglu_limit);
                         out[(size_t)(c0 + j) * p.ld_out] = __float2bfloat16_rn(a);
                     }
                 }
@@ -281,6 +291,7 @@ inline KParams make_params(const GroupedGemmArgs& a, int GEMM, uint64_t* b_rows)
     p.N = a.N;
     p.offsets = a.offsets;
     p.status = a.status;
+    p.swiglu_limit = a.swiglu_limit;
     if (GEMM == 1) {
         p.K = a.H;
         p.M = a.I;

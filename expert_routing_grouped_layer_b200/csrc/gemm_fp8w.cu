@@ -174,7 +174,7 @@ __device__ __forceinline__ void epilogue_f16_gate_up(const KParams& p, const int
                 if (c0 + j < t.n_valid) {
                     const float gv = __uint_as_float(g[j]) * fg * fe;  // exact power-of-two factors
                     const float uv = __uint_as_float(uu[j]) * fu * fe;
-                    const float a = gv / (1.0f + __expf(-gv)) * uv;
+                    const float a = swiglu(gv, uv, p.swiglu_limit);
                     out[(size_t)(c0 + j) * p.ld_out] = __float2bfloat16_rn(a);
                 }
             }

@@ -392,8 +392,12 @@ __global__ void __launch_bounds__(TileMX<GEMM, BNX_, ACCB_>::THREADS, 1)
                 float a[16], wmax[16];
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
-                    const float gv = __uint_as_float(g[j]);
-                    a[j] = __fdividef(gv, 1.0f + __expf(-gv)) * __uint_as_float(uu[j]);
+                    float gv = __uint_as_float(g[j]), uv = __uint_as_float(uu[j]);
+                    if (p.swiglu_limit > 0.0f) {  // optional limit: min(g, L), clamp(u, -L, L)
+                        gv = fminf(gv, p.swiglu_limit);
+                        uv = fminf(fmaxf(uv, -p.swiglu_limit), p.swiglu_limit);
+                    }
+                    a[j] = __fdividef(gv, 1.0f + __expf(-gv)) * uv;
                     wmax[j] = warp_max_nonneg(fabsf(a[j]));
                 }
                 int e[16];

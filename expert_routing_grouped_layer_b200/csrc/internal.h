@@ -85,6 +85,7 @@ struct GroupedGemmArgs {
     uint8_t* out_routed_scale;
     uint8_t* out_shared_scale;
     int32_t* status;
+    float swiglu_limit;  // gemm1: 0 = off, else SiLU(min(g, L)) * clamp(u, -L, L)
 };
 cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st);
 

@@ -48,12 +48,13 @@ class MoEConfig:
     shared_intermediate_size: int
     norm_topk_prob: bool
     routed_scaling_factor: float
-    score_fn: str  # "sigmoid" | "sqrtsoftplus"
+    score_fn: str  # "sigmoid" | "sqrtsoftplus" | "softmax"
     wfmt: str  # "bf16" | "fp8_e4m3_b128x128" | "fp4_e2m1_ue8m0_b32" | "mxfp4"
     afmt: str  # "bf16" | "fp8_e4m3_pow2_b128" | "mxfp8"
     routing: str  # input recipe: "bias_uniform" | "balanced" | "zipf"
     seed: int
     description: str = ""
+    swiglu_limit: float = 0.0  # 0: plain SwiGLU; L > 0: SiLU(min(g, L)) * clamp(u, -L, L)
 
     def replace(self, **kw) -> "MoEConfig":
         return dataclasses.replace(self, **kw)

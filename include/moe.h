@@ -59,6 +59,9 @@ typedef enum {
 /* scoring function ([V3] 三.1 sigmoid; [V4] 架构 sqrtsoftplus = sqrt(softplus)) */
 #define MOE_SCORE_SIGMOID 0
 #define MOE_SCORE_SQRTSOFTPLUS 1
+/* softmax over a token's E logits (the alternative [V3] 三.1 contrasts with
+ * sigmoid): s_e = exp(l_e - m) / sum_e' exp(l_e' - m), m = max_e l_e */
+#define MOE_SCORE_SOFTMAX 2
 
 /* expert weight formats (routed and shared experts use the same one)
  *  BF16:              bf16 codes.
@@ -101,6 +104,9 @@ typedef struct {
     int32_t score_fn;                 /* MOE_SCORE_*                            */
     int32_t wfmt;                     /* MOE_W_*                                */
     int32_t afmt;                     /* MOE_A_*                                */
+    /* [V4] 架构 FFNSwiGLU's optional swiglu_limit: 0 = off; L > 0 computes
+     * SiLU(min(g, L)) * clamp(u, -L, L) in every expert (finite, >= 0) */
+    float swiglu_limit;
 } moe_config;
 
 /* Device pointers to the layer's parameters.
@@ -123,7 +129,8 @@ size_t moe_workspace_bytes(const moe_config *cfg, int32_t T);
  *  x bf16 [T][H]; gate_w fp32 [E][H]; gate_bias fp32 [E].
  *  logits = x . gate_w^T with fp32-class accuracy (on the tensor cores, with
  *  gate_w split exactly into three bf16 planes and fp32 accumulation);
- *  s = score(logits); s' = s + bias; with n_group > 1 the E experts form
+ *  s = score(logits) (sigmoid / sqrtsoftplus per logit, or softmax over the
+ *  token's logits); s' = s + bias; with n_group > 1 the E experts form
  *  n_group contiguous groups scored by the sum of their two largest s' (a
  *  one-expert group by its s'), the topk_group best groups are kept, then the
  *  k largest s' among kept experts are chosen (ties to the lower index).

@@ -35,7 +35,8 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_struct_layouts_match_header():
-    assert ctypes.sizeof(moe.moe_config) == 13 * 4
+    assert ctypes.sizeof(moe.moe_config) == 14 * 4
+    assert moe.moe_config.swiglu_limit.offset == 13 * 4  # appended after afmt
     assert ctypes.sizeof(moe.moe_weights) == 10 * 8
 
 
@@ -48,8 +49,9 @@ BAD = [dict(hidden=100), dict(hidden=0), dict(n_routed_experts=0), dict(n_routed
        dict(n_group=3), dict(n_group=64, n_routed_experts=64), dict(topk_group=0),
        dict(n_group=4, topk_group=5), dict(n_group=8, topk_group=1, num_experts_per_tok=4),
        dict(moe_intermediate_size=100), dict(n_shared_experts=-1), dict(n_shared_experts=5),
-       dict(norm_topk_prob=2), dict(routed_scaling_factor=0.0), dict(score_fn=7), dict(wfmt=9),
-       dict(afmt=-1)]
+       dict(norm_topk_prob=2), dict(routed_scaling_factor=0.0), dict(score_fn=7), dict(score_fn=3),
+       dict(wfmt=9), dict(afmt=-1), dict(swiglu_limit=-1.0), dict(swiglu_limit=float("inf")),
+       dict(swiglu_limit=float("nan"))]
 
 
 @pytest.mark.parametrize("bad", BAD)

@@ -194,3 +194,11 @@ def test_fp8_weights_extreme_row_magnitudes():
     assert np.isfinite(got).all()
     err = np.linalg.norm(got - want, axis=1) / np.maximum(np.linalg.norm(want, axis=1), 1e-300)
     assert err.max() <= LAYER_TOL["bf16"], (err.max(), int(err.argmax()))
+
+
+@pytest.mark.parametrize("name", ["bf16", "fp8w", "fp4", "mx"])
+def test_swiglu_limit_every_format(name):
+    """swiglu_limit = 0.25, below the typical |g| and |u| of these inputs, so the
+    clamp changes many features: the layer still matches the oracle."""
+    base = {"bf16": W.CONFIGS["tiny_bf16"], "fp8w": FP8_TINY, "fp4": FP4_TINY, "mx": MX_TINY}[name]
+    _layer_check(base.replace(swiglu_limit=0.25))

@@ -171,3 +171,29 @@ def test_bad_expert_id_sets_status_and_is_skipped():
     ro = ro.cpu().numpy()
     assert ro[3 * k + 1] == -1 and ro[5 * k] == -1
     assert off.cpu().numpy()[E] == T * k - 2
+
+
+@pytest.mark.parametrize("ng,tg,norm", [(1, 1, True), (4, 2, True), (1, 1, False)])
+def test_tiny_softmax_scoring(ng, tg, norm):
+    """Softmax over each token's logits instead of sigmoid: routing (sets, slot
+    order, weights to 1e-5) and the layer output against the oracle."""
+    cfg = W.CONFIGS["tiny_bf16"].replace(score_fn="softmax", n_group=ng, topk_group=tg,
+                                         norm_topk_prob=norm)
+    inp, wts = _data(cfg)
+    g, r, _ = _full_check(cfg, inp, wts)
+    ok = ~r["near_tie"]
+    assert np.array_equal(g["idx"][ok], r["idx"][ok])
+    assert (np.abs(g["w"][ok] - r["w"][ok]) <= 1e-5 * np.abs(r["w"][ok])).all()
+
+
+@pytest.mark.parametrize("E,k", [(384, 8), (896, 16)])
+def test_softmax_scoring_wide_expert_counts(E, k):
+    """Softmax across 384 and 896 experts (12 and 28 scores per lane)."""
+    cfg = W.CONFIGS["k2_decode_bf16"].replace(score_fn="softmax", T=64, hidden=512,
+                                              moe_intermediate_size=256,
+                                              shared_intermediate_size=256, n_routed_experts=E,
+                                              num_experts_per_tok=k)
+    inp, wts = _data(cfg)
+    g, r, _ = _full_check(cfg, inp, wts)
+    ok = ~r["near_tie"]
+    assert (np.abs(g["w"][ok] - r["w"][ok]) <= 1e-5 * np.abs(r["w"][ok])).all()
