@@ -65,6 +65,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--clock-log", default=None,
+                    help="keep the raw nvidia-smi samples here (%%d = device index)")
     ap.add_argument("--cpu-sample-tokens", type=int, default=128)
     return ap.parse_args()
 
@@ -86,15 +88,21 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, dev_index: int, enabled: bool = True):
+    def __init__(self, dev_index: int, enabled: bool = True, log_path=None):
+        """log_path: where the raw samples go (kept); default a temporary file."""
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", "clocks_rank%d.csv" % dev_index)
+        self.keep = log_path is not None
+        if log_path is None:
+            import tempfile
+            fd, log_path = tempfile.mkstemp(prefix="moe_clocks_%d_" % dev_index, suffix=".csv")
+            os.close(fd)
+        self.path = log_path
         if not enabled:
             return
         import torch
         p = torch.cuda.get_device_properties(dev_index)
         bus = "%08X:%02X:%02X.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
-        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        os.makedirs(os.path.dirname(os.path.abspath(self.path)), exist_ok=True)
         try:
             self.out = open(self.path, "w")
             self.proc = subprocess.Popen(
@@ -124,6 +132,8 @@ class ClockSampler:
                                  parts[4], parts[5:9]))
                 except ValueError:
                     continue
+        if not self.keep:
+            os.remove(self.path)
         if not rows:
             return None
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
@@ -264,7 +274,9 @@ def run_ours(args, rank, world, dev):
     assert st.item() == 0, "device status %d" % st.item()
 
     events = [mk() for _ in range(args.steps)]
-    clocks = ClockSampler(dev.index if dev.index is not None else 0, enabled=not args.no_clocks)
+    di = dev.index if dev.index is not None else 0
+    clocks = ClockSampler(di, enabled=not args.no_clocks,
+                          log_path=args.clock_log % di if args.clock_log else None)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
