@@ -309,19 +309,22 @@ def run_ours(args, rank, world, dev):
         torch.cuda.synchronize()
         if world > 1:
             torch.distributed.barrier()
-        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        # each step: L2 flushed first (outside the timed events), then the
+        # pinned-host copy in, the layer, and the copy of the result back out
         n_e2e = max(1, min(args.steps, 100))
-        s0.record(stream)
-        for _ in range(n_e2e):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n_e2e)]
+        for e0, e1 in evs:
             flush.zero_()
+            e0.record(stream)
             xd.copy_(xh, non_blocking=True)
             oh.copy_(layer.forward(xd), non_blocking=True)
-        s1.record(stream)
+            e1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = max_over_ranks(s0.elapsed_time(s1) / n_e2e, dev)
+        e2e_ms = max_over_ranks(statistics.fmean(e0.elapsed_time(e1) for e0, e1 in evs), dev)
         e2e = {"value": world * T / (e2e_ms / 1e3), "unit": UNIT,
                "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2,
-               "ms_per_step": e2e_ms, "includes_l2_flush": True}
+               "ms_per_step": e2e_ms, "includes_l2_flush": False}
 
     peaks, peak_src = load_peaks()
     ms = total_ms / args.steps
