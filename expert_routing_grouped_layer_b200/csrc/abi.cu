@@ -167,7 +167,7 @@ moe_status moe_gate_topk(const moe_config* cfg, const void* x, int32_t T, const 
     cudaStream_t st = as_stream(stream);
     cudaError_t e = launch_router_tc(x, gate_w, base + L.router_planes, part, T,
                                      cfg->n_routed_experts, cfg->hidden, dev_status, st);
-    if (e == cudaSuccess) e = launch_topk(cfg, part, 1, gate_bias, T, topk_idx, topk_w, st);
+    if (e == cudaSuccess) e = launch_topk(cfg, part, gate_bias, T, topk_idx, topk_w, st);
     return cuda_status(e);
 }
 

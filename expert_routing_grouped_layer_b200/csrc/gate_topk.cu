@@ -202,7 +202,7 @@ cudaError_t launch_router_reduce(float* part, long n, int splits, cudaStream_t s
     return cudaGetLastError();
 }
 
-cudaError_t launch_topk(const moe_config* c, const float* part, int splits, const float* bias, int T,
+cudaError_t launch_topk(const moe_config* c, const float* part, const float* bias, int T,
                         int32_t* idx, float* w, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
     TopkParams p;

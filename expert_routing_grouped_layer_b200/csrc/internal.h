@@ -48,7 +48,7 @@ RouterPlan router_plan(int T, int E, int H);
 cudaError_t launch_router_tc(const void* x, const float* gate_w, void* planes, float* part, int T,
                              int E, int H, int32_t* status, cudaStream_t st);
 cudaError_t launch_router_reduce(float* part, long n, int splits, cudaStream_t st);
-cudaError_t launch_topk(const moe_config* c, const float* part, int splits, const float* bias, int T,
+cudaError_t launch_topk(const moe_config* c, const float* part, const float* bias, int T,
                         int32_t* idx, float* w, cudaStream_t st);
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int n_chunks, int32_t* chunk,
                            int32_t* offsets, int32_t* sorted_pair, int32_t* row_of,

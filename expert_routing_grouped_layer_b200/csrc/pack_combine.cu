@@ -48,11 +48,12 @@ __device__ __forceinline__ void st_stream16(uint4* p, uint4 v) {
 // valid pair is zero-filled. One warp per row,
 // four loads in flight per lane, streaming stores (the rows are read once, by
 // the GEMM, after the whole gather).
+// src and dst may be one buffer (routed rows gathered from its token rows), so
+// they carry no __restrict__: the rows read and the rows written never overlap.
 __global__ void __launch_bounds__(256) gather_rows_kernel(
-    const uint4* __restrict__ src, int src_row0, int row16, const uint4* __restrict__ ssrc,
-    int srow16, const int32_t* __restrict__ sorted_pair, int N, int k, int T, int n_rows,
-    uint4* __restrict__ dst, uint4* __restrict__ sdst, const int8_t* __restrict__ esrc,
-    int8_t* __restrict__ edst) {
+    const uint4* src, int src_row0, int row16, const uint4* ssrc, int srow16,
+    const int32_t* __restrict__ sorted_pair, int N, int k, int T, int n_rows, uint4* dst,
+    uint4* sdst, const int8_t* esrc, int8_t* edst) {
     const int lane = threadIdx.x & 31;
     const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
     if (r >= n_rows) return;
