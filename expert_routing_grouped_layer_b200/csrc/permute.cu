@@ -143,24 +143,32 @@ __global__ void __launch_bounds__(PERM_WARPS * 32) perm_scatter_kernel(
 
 // All pairs in one chunk (N <= PERM_CHUNK): count, scan and scatter in one CTA,
 // the same per-warp histograms and in-warp ranks as the three launches, so the
-// order is the same.
+// order is the same. Each lane loads its PERM_PER_WARP / 32 expert ids once, up
+// front (independent loads), and both passes run on the registers.
 __global__ void __launch_bounds__(PERM_WARPS * 32) perm_single_kernel(
     const int32_t* __restrict__ idx, long N, int E, int32_t* __restrict__ offsets,
     int32_t* __restrict__ sorted_pair, int32_t* __restrict__ row_of, int32_t* status) {
+    constexpr int PER_LANE = PERM_PER_WARP / 32;
     __shared__ int32_t wbase[PERM_WARPS][PERM_MAX_E];
     __shared__ int32_t excl[PERM_MAX_E];
     __shared__ int32_t part[PERM_WARPS * 32];
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const long wstart = (long)w * PERM_PER_WARP;
+    int ev[PER_LANE];  // expert id of pair wstart + 32*i + lane, or -1 past N
+#pragma unroll
+    for (int i = 0; i < PER_LANE; ++i) {
+        const long p = wstart + 32 * i + lane;
+        ev[i] = p < N ? idx[p] : -1;
+    }
     for (int i = tid; i < PERM_WARPS * E; i += blockDim.x) wbase[i / E][i % E] = 0;
     __syncthreads();
-    const long wstart = (long)w * PERM_PER_WARP;
     bool bad = false;
-    for (int it = 0; it < PERM_PER_WARP; it += 32) {
-        const long p = wstart + it + lane;
-        const bool valid = p < N;
-        const int e = valid ? idx[p] : -1;
-        const bool ok = valid && e >= 0 && e < E;
-        bad |= valid && !ok;
+#pragma unroll
+    for (int i = 0; i < PER_LANE; ++i) {
+        const long p = wstart + 32 * i + lane;
+        const int e = ev[i];
+        const bool ok = p < N && e >= 0 && e < E;
+        bad |= p < N && !ok;
         const unsigned act = __ballot_sync(0xffffffffu, ok);
         if (ok) {
             const unsigned m = __match_any_sync(act, e);
@@ -203,10 +211,11 @@ __global__ void __launch_bounds__(PERM_WARPS * 32) perm_single_kernel(
     if (tid == blockDim.x - 1) offsets[E] = base;
     __syncthreads();
     const unsigned lt = (1u << lane) - 1u;
-    for (int it = 0; it < PERM_PER_WARP; it += 32) {
-        const long p = wstart + it + lane;
+#pragma unroll
+    for (int i = 0; i < PER_LANE; ++i) {
+        const long p = wstart + 32 * i + lane;
+        const int e = ev[i];
         const bool valid = p < N;
-        const int e = valid ? idx[p] : -1;
         const bool ok = valid && e >= 0 && e < E;
         const unsigned act = __ballot_sync(0xffffffffu, ok);
         if (ok) {
