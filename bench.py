@@ -172,6 +172,12 @@ def layer_bytes(cfg, active, T):
         cfg.n_routed_experts * cfg.hidden * 4 + 2 * T * cfg.hidden * 2
 
 
+def expert_weight_bytes(cfg, active):
+    """Stored weight bytes of the active routed experts and the shared experts."""
+    routed, shared = expert_bytes(cfg)
+    return active * routed + cfg.n_shared_experts * shared
+
+
 def layer_flops(cfg, T):
     N = T * cfg.num_experts_per_tok
     return 2.0 * (N + T * cfg.n_shared_experts) * 3 * cfg.hidden * cfg.moe_intermediate_size
@@ -336,6 +342,7 @@ def run_ours(args, rank, world, dev):
     hbm = peaks["hbm_gbs"]
     achieved = gu_bytes / (gu_ms / 1e3) / 1e9
     lb = layer_bytes(cfg, active, T)
+    ewb = expert_weight_bytes(cfg, active)
     line = {
         "metric": METRIC,
         "value": world * T / (ms / 1e3),
@@ -364,6 +371,10 @@ def run_ours(args, rank, world, dev):
                      "algorithmic_bytes_per_launch": gu_bytes},
         "layer_roofline": {"bound": "hbm", "bytes": lb, "achieved_gbs": lb / (ms / 1e3) / 1e9,
                            "frac": lb / (ms / 1e3) / 1e9 / hbm,
+                           # the activated and shared experts' weights alone (no router
+                           # weight, no activations)
+                           "expert_weight_bytes": ewb,
+                           "expert_weight_frac": ewb / (ms / 1e3) / 1e9 / hbm,
                            "flops": layer_flops(cfg, T),
                            "tflops": layer_flops(cfg, T) / (ms / 1e3) / 1e12},
         "stage_ms": stage_ms,
