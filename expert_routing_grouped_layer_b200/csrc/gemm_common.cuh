@@ -44,7 +44,8 @@ struct KParams {
     int K;               // reduction length
     int M;               // output features per matrix
     int a_rows_per_mat;  // 2I (GEMM1) or H (GEMM2)
-    int a_up_offset;     // I (GEMM1): first up-projection row
+    int a_up_offset;     // row offset of a unit's second weight tile (GEMM1: I, the up projection)
+    int tile_rows;       // weight rows (output features) per tile unit
     int b_shared_base;   // first B row of the shared-expert rows
     int b_shared_stride; // B-row step per shared expert
     int bn;              // tokens per tile (MMA N upper bound)
@@ -96,14 +97,14 @@ __device__ __forceinline__ Unit decode_unit(const KParams& p, const int* pref, i
     size_t r0;
     uint8_t *out, *sc;
     if (lo < p.E) {
-        t.a_row = lo * p.a_rows_per_mat + t.mt * BM;
+        t.a_row = lo * p.a_rows_per_mat + t.mt * p.tile_rows;
         r0 = (size_t)p.offsets[lo] + nt * p.bn;
         t.b_row = (int)r0;
         out = p.out_routed;
         sc = p.sc_routed;
     } else {
         const int s = lo - p.E;
-        t.a_row = s * p.a_rows_per_mat + t.mt * BM;
+        t.a_row = s * p.a_rows_per_mat + t.mt * p.tile_rows;
         t.b_row = p.b_shared_base + s * p.b_shared_stride + nt * p.bn;
         r0 = (size_t)s * p.T + nt * p.bn;
         out = p.out_shared;
@@ -312,6 +313,7 @@ inline KParams make_params(const GroupedGemmArgs& a, int GEMM, uint64_t* b_rows)
         *b_rows = (uint64_t)a.N + (uint64_t)a.S * a.T;
     }
     p.bn = BN;
+    p.tile_rows = BM;
     p.out_routed = static_cast<uint8_t*>(a.out_routed);
     p.out_shared = static_cast<uint8_t*>(a.out_shared);
     p.out_esize = 2;
@@ -321,7 +323,7 @@ inline KParams make_params(const GroupedGemmArgs& a, int GEMM, uint64_t* b_rows)
 
 inline int grid_for(const KParams& p) {
     // upper bound on tiles: sum_e ceil(m_e/BN) <= N/BN + min(E, N), plus shared
-    const long MT = p.M / BM;
+    const long MT = p.M / p.tile_rows;
     const long routed_tiles = (long)p.N / p.bn + std::min<long>(p.E, p.N);
     const long shared_tiles = (long)p.S * ((p.T + p.bn - 1) / p.bn);
     const long units_max = (routed_tiles + shared_tiles) * MT;

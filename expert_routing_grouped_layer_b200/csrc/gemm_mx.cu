@@ -16,77 +16,76 @@ namespace {
 // tcgen05.mma kind::mxf8f6f4 applies both scales inside the MMA, so the FP4
 // weights are never dequantised in software: TMA expands each packed row of
 // 128 E2M1 values to the one-byte-per-value layout the MMA reads
-// (16U4_ALIGN16B). Scales travel by TMA as 128 rows x 16 bytes (16 k-blocks).
-// The MMA reads row m's scale (m = m0 + 32*m1) from TMEM lane m0 of every
-// lane quadrant, column m1, one k-block per byte. A scale warp regroups the 4
-// k-blocks of the current stage into that order (row m at byte
-// 16*m0 + 4*m1 + kb of a 512-byte atom), in place over the staged scale
-// tiles, and two operands' atoms share one 128-lane x 256-bit copy (each atom
-// repeated for the 4 lane quadrants), so a stage issues half as many
-// tensor-memory copies as operands.
+// (16U4_ALIGN16B). Scales travel by TMA as 128 rows x 32 bytes (32 k-blocks)
+// into a two-slot ring. The MMA reads row m's scale (m = m0 + 32*m1) from
+// TMEM lane m0 of every lane quadrant, column m1, one k-block per byte. Four
+// scale warps, one per lane quadrant, store each stage's 4 k-blocks in that
+// order (tcgen05.st) into a ring of TMEM column sets: a tcgen05.cp issued by
+// the MMA thread costs the tensor pipe about as much as two small MMAs, a
+// store from another warp next to nothing.
+// The TMA unit keeps a bounded number of row requests in flight, and a row
+// fetched from HBM holds its slot for the whole DRAM latency whatever its
+// width: the scale boxes are therefore 32 bytes (eight stages) wide, so that
+// the narrow scale rows take as few of those slots as the ring allows.
+// A unit's NA weight tiles (gate and up for GEMM1; two consecutive 128-row
+// blocks of the down projection when NA = 2) share its token tile, and each
+// has its own MMA-issuing thread and accumulator: one thread issuing small
+// block-scaled MMAs with per-stage commits sustains ~72 cycles per MMA, two
+// threads ~48 at 64 tokens and the full rate from 112 tokens.
 // GEMM1's epilogue quantises the SwiGLU output per 32 (MXFP8) or per 128
 // (power of two) along I, exactly as the activation quantiser does.
 constexpr int MX_BK = 128;        // K elements per stage (one 128-byte smem row)
-constexpr int SF_TILE = 128 * 16; // scale tile: 128 rows x 16 k-blocks of 32
+constexpr int SF_KB = 32;         // k-blocks of 32 per scale box row (8 stages)
+constexpr int SF_STAGES = SF_KB / 4;
+constexpr int SF_TILE = 128 * SF_KB;  // scale tile: 128 rows x 32 k-blocks
 
-// GEMM: 1 gate/up, 2 down. BNX_: tokens per tile. ACCB: accumulator buffers
-// in tensor memory (2 overlaps a tile's epilogue with the next tile's main
-// loop; 1 lets gate/up use 240-token tiles). Warps: 0 TMA, 1 MMA, then EG
-// groups of 4 epilogue warps (one per TMEM lane quadrant), then the scale
-// warp. Single-buffered gate/up tiles take three epilogue groups (measured
-// faster than two), since there the quantising epilogue is not overlapped
-// with the next tile's main loop.
-template <int GEMM, int BNX_, int ACCB_>
+// GEMM: 1 gate/up, 2 down. NA: weight tiles per unit (= MMA threads). BNX_:
+// tokens per tile. ACCB: accumulator buffers in tensor memory (2 overlaps a
+// tile's epilogue with the next tile's main loop; 1 lets gate/up use
+// 224-token tiles). Warps: 0 TMA, 1 MMA (tile 0), then EG groups of 4
+// epilogue warps (one per TMEM lane quadrant), then the 4 scale warps, then
+// the MMA warp of tile 1. Single-buffered gate/up tiles take three epilogue
+// groups, since there the quantising epilogue is not overlapped with the
+// next tile's main loop.
+template <int GEMM, int NA_, int BNX_, int ACCB_>
 struct TileMX {
-    static constexpr int EG = (GEMM == 1 && ACCB_ == 1) ? 3 : 1;
-    static constexpr int THREADS = 64 + 128 * EG + 32;
-    static constexpr int SCALE_WARP = 2 + 4 * EG;
+    static constexpr int NA = NA_;
+    // epilogue groups: single-buffered gate/up 3; wide double-buffered down 2
+    static constexpr int EG = (GEMM == 1 && ACCB_ == 1) ? 3 : (GEMM == 2 && BNX_ > 128) ? 2 : 1;
+    static constexpr int SCALE_WARP = 2 + 4 * EG;     // first of the 4 scale warps
+    static constexpr int MMA2_WARP = SCALE_WARP + 4;  // MMA thread of tile 1 (NA == 2)
+    static constexpr int THREADS = 32 * (MMA2_WARP + (NA == 2 ? 1 : 0));
     static constexpr int RED_BYTES = EG * 2 * 4 * 16 * 4;  // [group][parity][warp][16 columns]
-    static constexpr int NA = (GEMM == 1) ? 2 : 1;
+    static constexpr int EPI_BYTES = GEMM == 2 ? EG * 2 * 16 * BM * 2 + 128 : 0;  // down: [group][2][16][128] bf16
     static constexpr int BNX = BNX_;
     static constexpr int ACCB = ACCB_;
     static constexpr int SFB_ROWS = (BNX + 127) / 128 * 128;  // token rows of the scale tile
     static constexpr int SFB_ATOMS = SFB_ROWS / 128;
-    static constexpr int NOPS = NA + SFB_ATOMS;  // scale operands: A gate, [A up], B rows 0-127, [128-255]
-    static constexpr int NPAIR = NOPS / 2;       // operand pairs copied by one 128x256b copy
-    static constexpr int A_BYTES = BM * MX_BK;                // one byte per E2M1 value in smem
+    static constexpr int NOPS = NA + SFB_ATOMS;  // scale operands: A tiles, B rows 0-127, [128-255]
+    static constexpr int A_BYTES = BM * MX_BK;   // one byte per E2M1 value in smem
     static constexpr int B_BYTES = BNX * MX_BK;
     static constexpr int A_OFF = 0;
     static constexpr int B_OFF = NA * A_BYTES;
-    static constexpr int SF_OFF = B_OFF + B_BYTES;  // regrouped scale atoms of the stage
-    static constexpr int RAW_BYTES = NOPS * SF_TILE;  // staged scale tiles, operand i at i*SF_TILE
-    static constexpr int ATOM_BYTES = NPAIR * 2 * SF_TILE + (NOPS & 1) * 512;
-    // A scale box covers 16 k-blocks, four stages. Normally the boxes go to a
-    // two-slot ring, loaded once per four stages, and the scale warp writes the
-    // atoms into the stage. Where that ring would cost a pipeline stage (wide
-    // gate/up tiles), each stage loads the boxes itself and the atoms overwrite
-    // them in place.
+    static constexpr int RAW_BYTES = NOPS * SF_TILE;  // one scale ring slot: operand i at i*SF_TILE
+    static constexpr int RING_BYTES = 2 * RAW_BYTES;
     static constexpr int FIXED_BYTES =
-        1024 + 8 * (3 * 6 + 9 + 2 * EG) + 16 + 4 * (MAX_SEG + 1) + RED_BYTES;
-    static constexpr int STAGE_RING = (SF_OFF + ATOM_BYTES + 1023) / 1024 * 1024;
-    static constexpr int STAGES_RING = stages_for(STAGE_RING, FIXED_BYTES + 2 * RAW_BYTES, 6);
-    static constexpr int STAGE_INPLACE = (SF_OFF + RAW_BYTES + 1023) / 1024 * 1024;
-    static constexpr int STAGES_INPLACE = stages_for(STAGE_INPLACE, FIXED_BYTES, 6);
-    static constexpr bool SF_RING = STAGES_RING >= 4 || STAGES_RING >= STAGES_INPLACE;
-    static constexpr int STAGE_BYTES = SF_RING ? STAGE_RING : STAGE_INPLACE;
-    static constexpr int STAGES = SF_RING ? STAGES_RING : STAGES_INPLACE;
-    static constexpr int RING_BYTES = SF_RING ? 2 * RAW_BYTES : 0;
+        1024 + 8 * (3 * 6 + 9 + 4 * EG) + 16 + 4 * (MAX_SEG + 1) + RED_BYTES + EPI_BYTES;
+    static constexpr int STAGE_BYTES = (B_OFF + B_BYTES + 1023) / 1024 * 1024;
+    static constexpr int STAGES = stages_for(STAGE_BYTES, FIXED_BYTES + RING_BYTES, 6);
     static constexpr int ACC_COLS = NA * BNX;
-    static constexpr int SF_COL = ACCB * ACC_COLS;  // scale columns: operand i at SF_COL + 4*i
     static constexpr int TMEM_COLS = 512;
-    static_assert(SF_COL % 8 == 0, "256-bit scale copies start on a multiple of 8 columns");
-    static_assert(SF_COL + 4 * NOPS <= TMEM_COLS, "tensor memory budget");
-    static constexpr int BAR_BYTES = 8 * (3 * STAGES + 9 + 2 * EG) + 16;
+    static constexpr int SF_COL = ACCB * ACC_COLS;  // scale sets: set s, operand i at SF_COL + s*SET_COLS + 4*i
+    static constexpr int SET_COLS = 4 * NOPS;
+    static constexpr int NSETS_FIT = (TMEM_COLS - SF_COL) / SET_COLS;
+    static constexpr int NSETS = NSETS_FIT < STAGES ? NSETS_FIT : STAGES;
+    static_assert(NSETS >= 2, "tensor memory budget: two scale sets");
+    static constexpr int BAR_BYTES = 8 * (3 * STAGES + 9 + 4 * EG) + 16;
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + RING_BYTES + BAR_BYTES +
-                                      4 * (MAX_SEG + 1) + RED_BYTES;  // + cross-warp amax exchange
+                                      4 * (MAX_SEG + 1) + RED_BYTES + EPI_BYTES;
     static_assert(STAGES >= 2 && SMEM_BYTES <= 232448, "shared memory budget");
+    static_assert(NA == 1 || NA == 2, "one or two weight tiles per unit");
+    static_assert(GEMM == 2 || NA == 2, "gate/up units hold both projections");
 };
-
-// 128 lanes x 256 bits from shared memory (two 16-byte halves 2048 bytes apart,
-// rows 16 bytes apart) to 8 TMEM columns.
-__device__ __forceinline__ void tmem_cp_128x256b(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
 
 // Max over the warp of non-negative floats: their bit patterns order like the
 // values, so one integer max reduction does it.
@@ -117,32 +116,45 @@ __device__ __forceinline__ uint8_t e4m3_sat(float v) {
     return (uint8_t)(__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3));
 }
 
-template <int GEMM, int AFMT, int BNX_, int ACCB_>
-__global__ void __launch_bounds__(TileMX<GEMM, BNX_, ACCB_>::THREADS, 1)
+// Wait by lane 0 only, the outcome shared with the warp.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int lane) {
+    int ok = 1;
+    if (lane == 0) ok = mbar_wait(bar, parity, abort) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok != 0;
+}
+
+
+template <int GEMM, int AFMT, int NA_, int BNX_, int ACCB_>
+__global__ void __launch_bounds__(TileMX<GEMM, NA_, BNX_, ACCB_>::THREADS, 1)
     grouped_gemm_mx_kernel(const __grid_constant__ CUtensorMap tmA_routed,
                            const __grid_constant__ CUtensorMap tmA_shared,
                            const __grid_constant__ CUtensorMap tmSFA_routed,
                            const __grid_constant__ CUtensorMap tmSFA_shared,
                            const __grid_constant__ BMaps tmB,
                            const __grid_constant__ CUtensorMap tmSFB, const KParams p) {
-    using C = TileMX<GEMM, BNX_, ACCB_>;
+    using C = TileMX<GEMM, NA_, BNX_, ACCB_>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint8_t* sf_ring = smem + C::STAGES * C::STAGE_BYTES;  // [2][RAW_BYTES] (ring variant)
+    uint8_t* sf_ring = smem + C::STAGES * C::STAGE_BYTES;  // [2][RAW_BYTES]
     uint64_t* full = reinterpret_cast<uint64_t*>(sf_ring + C::RING_BYTES);
     uint64_t* empty = full + C::STAGES;
-    uint64_t* sf_ready = empty + C::STAGES;  // scales regrouped for the stage
+    uint64_t* sf_ready = empty + C::STAGES;  // the stage's scales are in their TMEM set
     uint64_t* tfull = sf_ready + C::STAGES;
     uint64_t* tempty = tfull + 2;
     uint64_t* mma_done = tempty + 2;
     uint64_t* sf_full = mma_done + 1;  // [2] scale ring slots
-    uint64_t* sf_empty = sf_full + 2;  // [2]
+    uint64_t* sf_empty = sf_full + 2;  // [2] released by the 4 scale warps
     uint64_t* red_bar = sf_empty + 2;  // [group][parity]: the amax exchange of a group's 4 warps
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red_bar + 2 * C::EG);
+    uint64_t* ep_bar = red_bar + 2 * C::EG;  // [group][parity]: the down epilogue's staged chunk
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ep_bar + 2 * C::EG);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* pref = reinterpret_cast<int*>(tmem_slot + 4);
     float* red = reinterpret_cast<float*>(pref + MAX_SEG + 1);  // [group][parity][4 warps][16]
+    __nv_bfloat16* ep_buf = reinterpret_cast<__nv_bfloat16*>(  // [group][2][16][128], 128-byte aligned
+        (reinterpret_cast<uintptr_t>(red + C::RED_BYTES / 4) + 127) & ~static_cast<uintptr_t>(127));
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -150,19 +162,20 @@ __global__ void __launch_bounds__(TileMX<GEMM, BNX_, ACCB_>::THREADS, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
-            mbar_init(&sf_ready[s], 1);
+            mbar_init(&empty[s], C::NA);  // one commit per MMA thread
+            mbar_init(&sf_ready[s], 4);   // one arrival per scale warp
         }
         for (int a = 0; a < 2; ++a) {
-            mbar_init(&tfull[a], 1);
+            mbar_init(&tfull[a], C::NA);
             mbar_init(&tempty[a], 128 * C::EG);
         }
-        mbar_init(mma_done, 1);
+        mbar_init(mma_done, C::NA);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sf_full[i], 1);
-            mbar_init(&sf_empty[i], 1);
+            mbar_init(&sf_empty[i], 4);
         }
         for (int i = 0; i < 2 * C::EG; ++i) mbar_init(&red_bar[i], 4);
+        for (int i = 0; i < 2 * C::EG; ++i) mbar_init(&ep_bar[i], 4);
         *abort_flag = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tmA_routed);
@@ -176,7 +189,7 @@ __global__ void __launch_bounds__(TileMX<GEMM, BNX_, ACCB_>::THREADS, 1)
         tmem_alloc(tmem_slot, C::TMEM_COLS);
         tmem_relinquish();
     }
-    const int MT = p.M / BM;
+    const int MT = p.M / p.tile_rows;
     if (warp == 1) build_schedule(p, pref, MT, lane);
     tc_fence_before();
     __syncthreads();
@@ -197,21 +210,21 @@ __global__ void __launch_bounds__(TileMX<GEMM, BNX_, ACCB_>::THREADS, 1)
                 const int n_mma = (t.n_valid + 15) & ~15;
                 // a padded E2M1 tile occupies A_BYTES of shared memory but the copy
                 // counts its packed size (4 bits per value) toward the transaction
-                const uint32_t tx = C::NA * (C::A_BYTES / 2) + n_mma * MX_BK +
-                                    (C::SF_RING ? 0 : C::RAW_BYTES);
+                const uint32_t tx = C::NA * (C::A_BYTES / 2) + n_mma * MX_BK;
                 const bool routed = t.seg < p.E;
                 const CUtensorMap* tmA = routed ? &tmA_routed : &tmA_shared;
                 const CUtensorMap* tmSFA = routed ? &tmSFA_routed : &tmSFA_shared;
                 bool ok = true;
                 for (int kb = 0; kb < KB; ++kb) {
-                    const int sfx = (kb >> 2) * 16;  // 16-k-block group holding this stage
-                    if (C::SF_RING && (kb & 3) == 0) {
+                    if (kb % SF_STAGES == 0) {  // the scales of this stage and the next seven
                         if (!mbar_wait(&sf_empty[sfs], sf_phase ^ 1, abort_flag)) { ok = false; break; }
                         uint8_t* sl = sf_ring + sfs * C::RAW_BYTES;
+                        const int sfx = kb * 4;  // first k-block of the box
                         mbar_arrive_expect_tx(&sf_full[sfs], C::RAW_BYTES);
-                        tma_load_2d(sl, tmSFA, sfx, t.a_row, &sf_full[sfs]);
-                        if (GEMM == 1)
-                            tma_load_2d(sl + SF_TILE, tmSFA, sfx, t.a_row + p.a_up_offset, &sf_full[sfs]);
+#pragma unroll
+                        for (int j = 0; j < C::NA; ++j)
+                            tma_load_2d(sl + j * SF_TILE, tmSFA, sfx, t.a_row + j * p.a_up_offset,
+                                        &sf_full[sfs]);
                         tma_load_2d(sl + C::NA * SF_TILE, &tmSFB, sfx, t.b_row, &sf_full[sfs]);
                         ++sf_issued;
                         if (++sfs == 2) { sfs = 0; sf_phase ^= 1; }
@@ -219,19 +232,11 @@ __global__ void __launch_bounds__(TileMX<GEMM, BNX_, ACCB_>::THREADS, 1)
                     if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
                     uint8_t* st = smem + stage * C::STAGE_BYTES;
                     mbar_arrive_expect_tx(&full[stage], tx);
-                    tma_load_2d(st + C::A_OFF, tmA, kb * MX_BK, t.a_row, &full[stage]);
-                    if (GEMM == 1)
-                        tma_load_2d(st + C::A_OFF + C::A_BYTES, tmA, kb * MX_BK,
-                                    t.a_row + p.a_up_offset, &full[stage]);
+#pragma unroll
+                    for (int j = 0; j < C::NA; ++j)
+                        tma_load_2d(st + C::A_OFF + j * C::A_BYTES, tmA, kb * MX_BK,
+                                    t.a_row + j * p.a_up_offset, &full[stage]);
                     load_b_rows(st + C::B_OFF, tmB, kb * MX_BK, t.b_row, n_mma, MX_BK, &full[stage]);
-                    if (!C::SF_RING) {
-                        tma_load_2d(st + C::SF_OFF, tmSFA, sfx, t.a_row, &full[stage]);
-                        if (GEMM == 1)
-                            tma_load_2d(st + C::SF_OFF + SF_TILE, tmSFA, sfx, t.a_row + p.a_up_offset,
-                                        &full[stage]);
-                        tma_load_2d(st + C::SF_OFF + C::NA * SF_TILE, &tmSFB, sfx, t.b_row,
-                                    &full[stage]);
-                    }
                     ++issued;
                     if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
                 }
@@ -255,48 +260,42 @@ __global__ void __launch_bounds__(TileMX<GEMM, BNX_, ACCB_>::THREADS, 1)
                 status_or(p.status, MOE_DEV_TIMEOUT);
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == 1 || (C::NA == 2 && warp == C::MMA2_WARP)) {
+        // MMA thread of weight tile w: its own accumulator, the shared token tile
         if (lane == 0) {
+            const int w = (warp == 1) ? 0 : 1;
             int stage = 0;
             uint32_t phase = 0;
+            int set = 0;  // TMEM scale set of the stage
             int acc = 0;
             uint32_t acc_phase = 0;
-            const uint32_t sfa_gate = tmem_base + C::SF_COL;
-            const uint32_t sfa_up = tmem_base + C::SF_COL + 4;
-            const uint32_t sfb = tmem_base + C::SF_COL + 4 * C::NA;
             for (int u = blockIdx.x; u < total; u += gridDim.x) {
                 const Unit t = decode_unit(p, pref, u);
                 const int n_mma = (t.n_valid + 15) & ~15;
                 if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag)) break;
                 tc_fence_after();
-                const uint32_t d0 = tmem_base + acc * C::ACC_COLS;
+                const uint32_t d0 = tmem_base + acc * C::ACC_COLS + w * C::BNX;
                 bool ok = true;
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!mbar_wait(&full[stage], phase, abort_flag) ||
                         !mbar_wait(&sf_ready[stage], phase, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t st = smem_u32(smem + stage * C::STAGE_BYTES);
-#pragma unroll
-                    for (int pr = 0; pr < C::NPAIR; ++pr)
-                        tmem_cp_128x256b(sfa_gate + 8 * pr,
-                                         sdesc_kmajor_noswizzle_rows16(st + C::SF_OFF + pr * 2 * SF_TILE));
-                    if (C::NOPS & 1)
-                        tmem_cp_32x128b_x4(sfa_gate + 8 * C::NPAIR, sdesc_kmajor_noswizzle_rows16(
-                                                                     st + C::SF_OFF + 2 * C::NPAIR * SF_TILE));
+                    const uint32_t sfs = tmem_base + C::SF_COL + set * C::SET_COLS;
+                    const uint32_t sfa = sfs + 4 * w;
+                    const uint32_t sfb = sfs + 4 * C::NA;
 #pragma unroll
                     for (int kk = 0; kk < MX_BK / 32; ++kk) {
                         const uint32_t acc_flag = (kb | kk) != 0;
                         const uint32_t idesc = idesc_mx_e2m1_e4m3(BM, n_mma, kk, kk);
                         const uint32_t sub = (uint32_t)kk << 30;  // k-block byte in each column
-                        const uint64_t bd = sdesc_kmajor_sw128(st + C::B_OFF + kk * 32);
-                        mma_mx(d0, sdesc_kmajor_sw128(st + C::A_OFF + kk * 32), bd, idesc,
-                               sfa_gate | sub, sfb | sub, acc_flag);
-                        if (GEMM == 1)
-                            mma_mx(d0 + C::BNX, sdesc_kmajor_sw128(st + C::A_OFF + C::A_BYTES + kk * 32),
-                                   bd, idesc, sfa_up | sub, sfb | sub, acc_flag);
+                        mma_mx(d0, sdesc_kmajor_sw128(st + C::A_OFF + w * C::A_BYTES + kk * 32),
+                               sdesc_kmajor_sw128(st + C::B_OFF + kk * 32), idesc, sfa | sub,
+                               sfb | sub, acc_flag);
                     }
                     mma_commit(&empty[stage]);
                     if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+                    if (++set == C::NSETS) set = 0;
                 }
                 if (!ok) break;
                 mma_commit(&tfull[acc]);
@@ -307,62 +306,113 @@ __global__ void __launch_bounds__(TileMX<GEMM, BNX_, ACCB_>::THREADS, 1)
             mbar_wait(mma_done, 0, &no_abort);
             if (*abort_flag) status_or(p.status, MOE_DEV_TIMEOUT);
         }
-    } else if (warp == C::SCALE_WARP) {
-        // scale warp: regroup this stage's 4 k-blocks of every staged 128 x 16-byte
-        // scale tile (lane m0 gathers rows m0 + 32*m1) into the stage's atoms.
-        // Operand pair pr becomes a 128-row x 32-byte copy source: operand 2pr in
-        // the first 16-byte half, 2pr+1 in the second (2048 bytes on), each atom
-        // written for rows m0, m0+32, m0+64, m0+96. An odd last operand stays one
-        // 512-byte atom. A ring slot serves four stages, then is released.
+    } else if (warp >= C::SCALE_WARP && warp < C::SCALE_WARP + 4) {
+        // scale warps. Per stage, lane m0 of quadrant q gathers for every operand
+        // the stage's 4 k-block bytes of rows m0, m0+32, m0+64, m0+96 from the
+        // ring slot and stores them to columns 0..3 of the operand in the
+        // stage's TMEM set. A set is rewritten only after the MMAs that read it
+        // completed (the empty barrier of the stage that last used it). A ring
+        // slot serves eight stages (fewer at the end of a unit), then is released.
+        const uint32_t lane_cols = tmem_base + ((uint32_t)((warp & 3) * 32) << 16) + C::SF_COL;
         int stage = 0;
-        uint32_t phase = 0;
+        int set = 0;
+        int g = 0;  // stages processed
         int sfs = 0;
         uint32_t sf_phase = 0;
-        for (int u = blockIdx.x; u < total; u += gridDim.x) {
-            bool ok = true;
+        bool ok = true;
+        for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
             for (int kb = 0; kb < KB; ++kb) {
-                if (C::SF_RING && (kb & 3) == 0 && !mbar_wait(&sf_full[sfs], sf_phase, abort_flag)) {
+                if (kb % SF_STAGES == 0 && !warp_wait(&sf_full[sfs], sf_phase, abort_flag, lane)) {
                     ok = false;
                     break;
                 }
-                if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
-                uint8_t* atoms = smem + stage * C::STAGE_BYTES + C::SF_OFF;
-                const uint8_t* raw = C::SF_RING ? sf_ring + sfs * C::RAW_BYTES : atoms;
-                const int j4 = (kb & 3) * 4;  // byte offset of this stage's k-blocks in a row
+                if (g >= C::NSETS) {
+                    const int gp = g - C::NSETS;
+                    if (!warp_wait(&empty[gp % C::STAGES], (uint32_t)(gp / C::STAGES) & 1u, abort_flag, lane)) {
+                        ok = false;
+                        break;
+                    }
+                }
+                const uint8_t* raw = sf_ring + sfs * C::RAW_BYTES;
+                const int j4 = (kb % SF_STAGES) * 4;  // byte offset of this stage's k-blocks in a row
                 uint4 v[C::NOPS];
 #pragma unroll
                 for (int i = 0; i < C::NOPS; ++i) {
                     const uint8_t* src = raw + i * SF_TILE;
-                    v[i].x = *reinterpret_cast<const uint32_t*>(src + 16 * (lane + 0) + j4);
-                    v[i].y = *reinterpret_cast<const uint32_t*>(src + 16 * (lane + 32) + j4);
-                    v[i].z = *reinterpret_cast<const uint32_t*>(src + 16 * (lane + 64) + j4);
-                    v[i].w = *reinterpret_cast<const uint32_t*>(src + 16 * (lane + 96) + j4);
+                    v[i].x = *reinterpret_cast<const uint32_t*>(src + SF_KB * (lane + 0) + j4);
+                    v[i].y = *reinterpret_cast<const uint32_t*>(src + SF_KB * (lane + 32) + j4);
+                    v[i].z = *reinterpret_cast<const uint32_t*>(src + SF_KB * (lane + 64) + j4);
+                    v[i].w = *reinterpret_cast<const uint32_t*>(src + SF_KB * (lane + 96) + j4);
                 }
-                __syncwarp();  // in place: every lane has read the tiles before they are overwritten
-                if (C::SF_RING && (kb & 3) == 3) {
+                if (kb % SF_STAGES == SF_STAGES - 1 || kb == KB - 1) {
+                    __syncwarp();
                     if (lane == 0) mbar_arrive(&sf_empty[sfs]);
                     if (++sfs == 2) { sfs = 0; sf_phase ^= 1; }
                 }
 #pragma unroll
-                for (int i = 0; i < 2 * C::NPAIR; ++i) {
-                    uint8_t* dst = atoms + (i >> 1) * 2 * SF_TILE + (i & 1) * SF_TILE;
-#pragma unroll
-                    for (int r = 0; r < 4; ++r)
-                        *reinterpret_cast<uint4*>(dst + 16 * (lane + 32 * r)) = v[i];
-                }
-                if (C::NOPS & 1)
-                    *reinterpret_cast<uint4*>(atoms + 2 * C::NPAIR * SF_TILE + 16 * lane) =
-                        v[C::NOPS - 1];
-                fence_proxy_async_smem();
+                for (int i = 0; i < C::NOPS; ++i) tmem_st4(lane_cols + set * C::SET_COLS + 4 * i, v[i]);
+                tmem_st_wait();
+                tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sf_ready[stage]);
-                if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+                if (++stage == C::STAGES) stage = 0;
+                if (++set == C::NSETS) set = 0;
+                ++g;
             }
-            if (!ok) break;
         }
     } else if (GEMM == 2) {
-        epilogue_loop<2, C::ACC_COLS, C::ACCB>(p, pref, total, tmem_base, tfull, tempty, abort_flag,
-                                               warp, lane);
+        // down epilogue: NA accumulators of BNX columns, lane = output feature.
+        // Group grp takes the 16-token chunks grp, grp + EG, ... Per chunk each
+        // warp converts its 32 features to bf16 into the group's shared
+        // [16 tokens][128 features] tile (two, alternating), the group's four
+        // warps meet at an mbarrier, and warp q writes token rows 4q..4q+3 as
+        // 256 contiguous bytes each, 16 bytes per lane.
+        const int q = warp & 3;
+        const int grp = (warp - 2) >> 2;
+        const int row = q * 32 + lane;
+        __nv_bfloat16* gbuf = ep_buf + grp * 2 * 16 * BM;
+        uint64_t* gbar = ep_bar + 2 * grp;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        int chunk = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+            const Unit t = decode_unit(p, pref, u);
+            if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int w = 0; w < C::NA && ok; ++w) {
+                const uint32_t taddr =
+                    tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::ACC_COLS + w * C::BNX;
+                __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(t.out) + t.mt * p.tile_rows + w * BM;
+                for (int c0 = 16 * grp; c0 < t.n_valid; c0 += 16 * C::EG, ++chunk) {
+                    uint32_t g[16];
+                    tmem_ld16(taddr + c0, g);
+                    tmem_ld_wait(g);
+                    __nv_bfloat16* buf = gbuf + (chunk & 1) * 16 * BM;
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) buf[j * BM + row] = __float2bfloat16_rn(__uint_as_float(g[j]));
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&gbar[chunk & 1]);
+                    if (!mbar_wait(&gbar[chunk & 1], (uint32_t)(chunk >> 1) & 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int r = 4 * q + 2 * h + (lane >> 4);  // token row of the chunk
+                        const int col = (lane & 15) * 8;            // first of 8 features
+                        if (c0 + r < t.n_valid)
+                            *reinterpret_cast<uint4*>(out + (size_t)(c0 + r) * p.ld_out + col) =
+                                *reinterpret_cast<const uint4*>(buf + r * BM + col);
+                    }
+                }
+            }
+            if (!ok) break;
+            tc_fence_before();
+            mbar_arrive(&tempty[acc]);
+            if (++acc == C::ACCB) { acc = 0; acc_phase ^= 1; }
+        }
     } else {
         // GEMM1 epilogue: SwiGLU, then E4M3 + E8M0 block quantisation along I.
         // Group grp takes the 16-column chunks grp, grp + EG, ...
@@ -449,13 +499,13 @@ __global__ void __launch_bounds__(TileMX<GEMM, BNX_, ACCB_>::THREADS, 1)
 
 }  // namespace
 
-template <int GEMM, int AFMT, int BNX_, int ACCB_>
+template <int GEMM, int AFMT, int NA_, int BNX_, int ACCB_>
 cudaError_t launch_mx(const GroupedGemmArgs& a, cudaStream_t st) {
-    using C = TileMX<GEMM, BNX_, ACCB_>;
+    using C = TileMX<GEMM, NA_, BNX_, ACCB_>;
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(grouped_gemm_mx_kernel<GEMM, AFMT, BNX_, ACCB_>,
+        attr_err = cudaFuncSetAttribute(grouped_gemm_mx_kernel<GEMM, AFMT, NA_, BNX_, ACCB_>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     });
     if (attr_err != cudaSuccess) return attr_err;
@@ -466,6 +516,11 @@ cudaError_t launch_mx(const GroupedGemmArgs& a, cudaStream_t st) {
         p.out_esize = 1;  // E4M3 intermediate
         p.sc_routed = a.out_routed_scale;
         p.sc_shared = a.out_shared_scale;
+    } else if (C::NA == 2) {
+        // two consecutive 128-row blocks of the down projection per unit
+        if (p.M % (2 * BM)) return cudaErrorInvalidValue;
+        p.tile_rows = 2 * BM;
+        p.a_up_offset = BM;
     }
     const int S = a.S;
     const uint64_t K = p.K, rowsA = (uint64_t)a.E * p.a_rows_per_mat;
@@ -480,31 +535,33 @@ cudaError_t launch_mx(const GroupedGemmArgs& a, cudaStream_t st) {
                       CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_tmap_2d(&tmAs, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, wAs, rowsAs, K, K / 2, MX_BK, BM,
                       CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_tmap_2d(&tmSFA, CU_TENSOR_MAP_DATA_TYPE_UINT8, sA, rowsA, K / 32, K / 32, 16, 128,
+        !make_tmap_2d(&tmSFA, CU_TENSOR_MAP_DATA_TYPE_UINT8, sA, rowsA, K / 32, K / 32, SF_KB, 128,
                       CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_tmap_2d(&tmSFAs, CU_TENSOR_MAP_DATA_TYPE_UINT8, sAs, rowsAs, K / 32, K / 32, 16, 128,
+        !make_tmap_2d(&tmSFAs, CU_TENSOR_MAP_DATA_TYPE_UINT8, sAs, rowsAs, K / 32, K / 32, SF_KB, 128,
                       CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     if (b_rows == 0) return cudaSuccess;
     if (!make_bmaps(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.b_rows, b_rows, K, MX_BK) ||
-        !make_tmap_2d(&tmSFB, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.b_scale, b_rows, K / 32, K / 32, 16,
+        !make_tmap_2d(&tmSFB, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.b_scale, b_rows, K / 32, K / 32, SF_KB,
                       C::SFB_ROWS, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    grouped_gemm_mx_kernel<GEMM, AFMT, BNX_, ACCB_><<<grid_for(p), C::THREADS, C::SMEM_BYTES, st>>>(
+    grouped_gemm_mx_kernel<GEMM, AFMT, NA_, BNX_, ACCB_><<<grid_for(p), C::THREADS, C::SMEM_BYTES, st>>>(
         tmA, tmAs, tmSFA, tmSFAs, tmB, tmSFB, p);
     return cudaGetLastError();
 }
 
 template <int AFMT>
 cudaError_t launch_mx_tiles(const GroupedGemmArgs& a, cudaStream_t st) {
-    // When experts average many tokens: 240-token tiles (gate/up single-buffered
-    // with two epilogue groups, down double-buffered). Otherwise gate/up takes
-    // 112-token tiles with double-buffered accumulators, so the quantising
-    // epilogue overlaps the next tile, and down 128-token tiles with a deeper ring.
+    // When experts average many tokens: 224-token tiles (gate/up single-buffered
+    // with three epilogue groups, down double-buffered with one weight tile;
+    // at 224 both keep one TMEM scale set per pipeline stage).
+    // Otherwise 112-token tiles with double-buffered accumulators, so the
+    // epilogue overlaps the next tile, and two weight tiles (two MMA threads)
+    // per unit in both GEMMs.
     const bool wide = a.N >= 128L * a.E;
     if (a.gemm == 1)
-        return wide ? launch_mx<1, AFMT, 240, 1>(a, st) : launch_mx<1, AFMT, 112, 2>(a, st);
-    return wide ? launch_mx<2, AFMT, 240, 2>(a, st) : launch_mx<2, AFMT, 128, 2>(a, st);
+        return wide ? launch_mx<1, AFMT, 2, 224, 1>(a, st) : launch_mx<1, AFMT, 2, 112, 2>(a, st);
+    return wide ? launch_mx<2, AFMT, 1, 224, 2>(a, st) : launch_mx<2, AFMT, 2, 112, 2>(a, st);
 }
 
 cudaError_t launch_gemm_mx(const GroupedGemmArgs& a, cudaStream_t st) {

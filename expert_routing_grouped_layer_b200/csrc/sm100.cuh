@@ -219,6 +219,20 @@ __device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t src_
                  : "memory");
 }
 
+// Registers -> tensor memory: thread i of the warp writes v to 4 consecutive
+// 32-bit columns of lane (base lane + i). A warp may address only its own lane
+// quadrant (warp index mod 4).
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, uint4 v) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr),
+                 "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// Wait until this thread's tcgen05.st have completed.
+__device__ __forceinline__ void tmem_st_wait() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 // Matrix descriptor of a K-major, unswizzled operand whose 8-row x 16-byte core
 // matrices are stored back to back (128 bytes apart): the scale-factor tiles.
 __device__ __forceinline__ uint64_t sdesc_kmajor_noswizzle_rows16(uint32_t smem_addr) {
