@@ -13,10 +13,15 @@ namespace {
 // E4M3 weights with one fp32 scale per 128x128 block ("DeepSeek-V4-Pro 架构与代码概述",
 // 文件说明: Linear with block-scaled FP8 weights; block 128x128). There is no
 // tensor-core instruction for E4M3 times bf16, so a converter warpgroup turns
-// each TMA-staged E4M3 weight tile (64-byte swizzled rows) into 16-bit values
-// times the tile's block scale, written straight into the 128B-swizzled
-// K-major layout tcgen05.mma reads. With BK = 64 inside a 128-wide scale block
-// and M tiles aligned to the 128-row blocks, one scalar scale covers a tile.
+// each TMA-staged E4M3 weight tile into 16-bit values times the tile's block
+// scale, written straight into the 128B-swizzled K-major layout tcgen05.mma
+// reads. A staged tile spans RKM MMA stages of BK = 64 (RKM = 2: 128-byte
+// swizzled rows; RKM = 1: 64-byte rows): the TMA unit keeps a bounded number
+// of row requests in flight and an HBM row holds its slot for the DRAM
+// latency whatever its width, so full 128-byte rows halve the weight stream's
+// cost there, where shared memory leaves room for the larger staging slots.
+// With a staged tile inside one 128-wide scale block and M tiles aligned to
+// the 128-row blocks, one scalar scale covers a tile.
 //  * gate/up: f16 operands (see the f16 path below): one cvt and one f16x2
 //    multiply per two weights; token rows come in as f16 with a power-of-two
 //    row scale.
@@ -35,7 +40,7 @@ static_assert(512 % CVT_THREADS == 0, "converter tasks: whole tiles per round");
 // as soon as the converters have read a slot, so it can run many stages ahead
 // of the tensor cores; the MMA ring holds the converted bf16 weight tiles and
 // the token tile, freed by the MMA commit.
-template <int GEMM, int BNF_, int ACCB_, int MST_>
+template <int GEMM, int BNF_, int ACCB_, int MST_, int RKM_>
 struct TileF8 {
     // gate/up (f16 path, ~86 registers) affords a second group of 4 epilogue
     // warps, which halves the drain of its single accumulator buffer
@@ -44,13 +49,15 @@ struct TileF8 {
     static constexpr int NA = (GEMM == 1) ? 2 : 1;
     static constexpr int BNF = BNF_;
     static constexpr int ACCB = ACCB_;
-    static constexpr int A8_BYTES = BM * BK;      // e4m3 staging tile
+    static constexpr int RKM = RKM_;
+    static constexpr int RK = RKM * BK;           // K of a staged e4m3 tile (RKM MMA stages)
+    static constexpr int A8_BYTES = BM * RK;      // e4m3 staging tile, RK-byte rows
     static constexpr int A_BYTES = BM * BK * 2;   // bf16 MMA tile
     static constexpr int B_BYTES = BNF * BK * 2;
     static constexpr int CVT_OFF = 0;                       // NA bf16 A tiles
     static constexpr int B_OFF = NA * A_BYTES;              // token tile
     static constexpr int MSLOT_BYTES = (B_OFF + B_BYTES + 1023) / 1024 * 1024;
-    static constexpr int RSLOT_BYTES = NA * A8_BYTES;       // NA e4m3 tiles
+    static constexpr int RSLOT_BYTES = NA * A8_BYTES;       // NA e4m3 tiles (RKM MMA stages)
     static constexpr int MSTAGES = MST_;
     static constexpr int FIXED_BYTES = 1024 + 8 * (2 * 8 + 3 * MSTAGES + 5) + 16 + 4 * (MAX_SEG + 1);
     static constexpr int RSTAGES_FIT = (232448 - FIXED_BYTES - MSTAGES * MSLOT_BYTES) / RSLOT_BYTES;
@@ -185,15 +192,15 @@ __device__ __forceinline__ void epilogue_f16_gate_up(const KParams& p, const int
     }
 }
 
-template <int GEMM, int BNF_, int ACCB_, int MST_>
-__global__ void __launch_bounds__(TileF8<GEMM, BNF_, ACCB_, MST_>::THREADS, 1)
+template <int GEMM, int BNF_, int ACCB_, int MST_, int RKM_>
+__global__ void __launch_bounds__(TileF8<GEMM, BNF_, ACCB_, MST_, RKM_>::THREADS, 1)
     grouped_gemm_fp8w_kernel(const __grid_constant__ CUtensorMap tmA_routed,
                              const __grid_constant__ CUtensorMap tmA_shared,
                              const __grid_constant__ BMaps tmB, const KParams p,
                              const float* __restrict__ scale_routed,
                              const float* __restrict__ scale_shared,
                              const int8_t* __restrict__ row_exp) {
-    using C = TileF8<GEMM, BNF_, ACCB_, MST_>;
+    using C = TileF8<GEMM, BNF_, ACCB_, MST_, RKM_>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -249,7 +256,7 @@ __global__ void __launch_bounds__(TileF8<GEMM, BNF_, ACCB_, MST_>::THREADS, 1)
     const int KB = p.K / BK;
 
     if (warp == 0) {
-        // producer: e4m3 weight tiles into the raw ring
+        // producer: e4m3 weight tiles (RK each) into the raw ring
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
@@ -258,13 +265,13 @@ __global__ void __launch_bounds__(TileF8<GEMM, BNF_, ACCB_, MST_>::THREADS, 1)
                 const Unit t = decode_unit(p, pref, u);
                 const CUtensorMap* tmA = (t.seg < p.E) ? &tmA_routed : &tmA_shared;
                 bool ok = true;
-                for (int kb = 0; kb < KB; ++kb) {
+                for (int kr = 0; kr < KB / C::RKM; ++kr) {
                     if (!mbar_wait(&raw_empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
                     uint8_t* rs = rring + stage * C::RSLOT_BYTES;
                     mbar_arrive_expect_tx(&raw_full[stage], C::RSLOT_BYTES);
-                    tma_load_2d(rs, tmA, kb * BK, t.a_row, &raw_full[stage]);
+                    tma_load_2d(rs, tmA, kr * C::RK, t.a_row, &raw_full[stage]);
                     if (GEMM == 1)
-                        tma_load_2d(rs + C::A8_BYTES, tmA, kb * BK, t.a_row + p.a_up_offset,
+                        tma_load_2d(rs + C::A8_BYTES, tmA, kr * C::RK, t.a_row + p.a_up_offset,
                                     &raw_full[stage]);
                     ++issued;
                     if (++stage == C::RSTAGES) { stage = 0; phase ^= 1; }
@@ -393,8 +400,9 @@ __global__ void __launch_bounds__(TileF8<GEMM, BNF_, ACCB_, MST_>::THREADS, 1)
                         if (GEMM == 1) u_nxt = s_up[nj];
                     }
                 }
+                const int h = kb % C::RKM;  // MMA stage within the staged tile
                 if (!mbar_wait(&m_empty[mstage], mphase ^ 1, abort_flag)) { ok = false; break; }
-                if (!mbar_wait(&raw_full[rstage], rphase, abort_flag)) { ok = false; break; }
+                if (h == 0 && !mbar_wait(&raw_full[rstage], rphase, abort_flag)) { ok = false; break; }
                 uint8_t* ms = mring + mstage * C::MSLOT_BYTES;
                 const uint8_t* rs = rring + rstage * C::RSLOT_BYTES;
                 const float sc[2] = {g_cur, u_cur};
@@ -405,7 +413,9 @@ __global__ void __launch_bounds__(TileF8<GEMM, BNF_, ACCB_, MST_>::THREADS, 1)
                     const int tile = (i * CVT_THREADS) >> 9;  // 512 tasks per tile, ct < CVT_THREADS
                     const int r = task & 127;
                     const int c = (task >> 7) & 3;
-                    const uint8_t* src = rs + tile * C::A8_BYTES + r * 64 + ((c ^ ((r >> 1) & 3)) << 4);
+                    const uint8_t* src =
+                        C::RKM == 2 ? rs + tile * C::A8_BYTES + r * 128 + (((4 * h + c) ^ (r & 7)) << 4)
+                                    : rs + tile * C::A8_BYTES + r * 64 + ((c ^ ((r >> 1) & 3)) << 4);
                     uint8_t* dst = ms + C::CVT_OFF + tile * C::A_BYTES + r * 128;
                     uint4 lo, hi;
                     if (GEMM == 1)
@@ -415,10 +425,10 @@ __global__ void __launch_bounds__(TileF8<GEMM, BNF_, ACCB_, MST_>::THREADS, 1)
                     *reinterpret_cast<uint4*>(dst + (((2 * c) ^ (r & 7)) << 4)) = lo;
                     *reinterpret_cast<uint4*>(dst + (((2 * c + 1) ^ (r & 7)) << 4)) = hi;
                 }
-                mbar_arrive(&raw_empty[rstage]);
+                if (h == C::RKM - 1) mbar_arrive(&raw_empty[rstage]);
                 fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
                 mbar_arrive(&cvt_full[mstage]);
-                if (++rstage == C::RSTAGES) { rstage = 0; rphase ^= 1; }
+                if (h == C::RKM - 1 && ++rstage == C::RSTAGES) { rstage = 0; rphase ^= 1; }
                 if (++mstage == C::MSTAGES) { mstage = 0; mphase ^= 1; }
             }
             if (!ok) break;
@@ -436,13 +446,13 @@ __global__ void __launch_bounds__(TileF8<GEMM, BNF_, ACCB_, MST_>::THREADS, 1)
 
 }  // namespace
 
-template <int GEMM, int BNF_, int ACCB_, int MST_>
+template <int GEMM, int BNF_, int ACCB_, int MST_, int RKM_>
 cudaError_t launch_fp8w(const GroupedGemmArgs& a, cudaStream_t st) {
-    using C = TileF8<GEMM, BNF_, ACCB_, MST_>;
+    using C = TileF8<GEMM, BNF_, ACCB_, MST_, RKM_>;
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(grouped_gemm_fp8w_kernel<GEMM, BNF_, ACCB_, MST_>,
+        attr_err = cudaFuncSetAttribute(grouped_gemm_fp8w_kernel<GEMM, BNF_, ACCB_, MST_, RKM_>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     });
     if (attr_err != cudaSuccess) return attr_err;
@@ -452,17 +462,18 @@ cudaError_t launch_fp8w(const GroupedGemmArgs& a, cudaStream_t st) {
     CUtensorMap tmAr, tmAs;
     BMaps tmB;
     const int S = a.S;
-    if (!make_tmap_u8_sw64(&tmAr, a.w_routed, (uint64_t)a.E * p.a_rows_per_mat, p.K, BM))
-        return cudaErrorInvalidValue;
-    if (!make_tmap_u8_sw64(&tmAs, S > 0 ? a.w_shared : a.w_routed,
-                           (uint64_t)(S > 0 ? S : a.E) * p.a_rows_per_mat, p.K, BM))
+    if (!make_tmap_2d(&tmAr, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.w_routed, (uint64_t)a.E * p.a_rows_per_mat,
+                      p.K, p.K, C::RK, BM, C::RKM == 2 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !make_tmap_2d(&tmAs, CU_TENSOR_MAP_DATA_TYPE_UINT8, S > 0 ? a.w_shared : a.w_routed,
+                      (uint64_t)(S > 0 ? S : a.E) * p.a_rows_per_mat, p.K, p.K, C::RK, BM,
+                      C::RKM == 2 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
         return cudaErrorInvalidValue;
     if (b_rows == 0) return cudaSuccess;
     // gate/up reads f16 token rows (x * 2^-e), down reads the bf16 SwiGLU output
     if (!make_bmaps(&tmB, GEMM == 1 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
                     2, a.b_rows, b_rows, p.K, BK))
         return cudaErrorInvalidValue;
-    grouped_gemm_fp8w_kernel<GEMM, BNF_, ACCB_, MST_><<<grid_for(p), C::THREADS, C::SMEM_BYTES, st>>>(
+    grouped_gemm_fp8w_kernel<GEMM, BNF_, ACCB_, MST_, RKM_><<<grid_for(p), C::THREADS, C::SMEM_BYTES, st>>>(
         tmAr, tmAs, tmB, p, static_cast<const float*>(a.w_routed_scale),
         static_cast<const float*>(S > 0 ? a.w_shared_scale : a.w_routed_scale),
         reinterpret_cast<const int8_t*>(a.b_scale));
@@ -472,12 +483,14 @@ cudaError_t launch_fp8w(const GroupedGemmArgs& a, cudaStream_t st) {
 cudaError_t launch_gemm_fp8w(const GroupedGemmArgs& a, cudaStream_t st) {
     // many tokens per expert: wide token tiles (each weight tile converted once
     // per expert); few tokens per expert: narrower double-buffered tiles. The
-    // last argument is the MMA-ring depth; the raw ring takes the rest of
-    // shared memory (up to 8 slots).
+    // fourth argument is the MMA-ring depth; the raw ring takes the rest of
+    // shared memory (up to 8 slots of RKM MMA stages each, the last argument).
+    // Wide gate/up keeps 64-byte staged rows: the 128-byte ones leave room for
+    // two MMA slots only, which measured slower.
     const bool wide = a.N >= 128L * a.E;
     if (a.gemm == 1)
-        return wide ? launch_fp8w<1, 240, 1, 3>(a, st) : launch_fp8w<1, 128, 2, 3>(a, st);
-    return wide ? launch_fp8w<2, 240, 2, 3>(a, st) : launch_fp8w<2, 128, 2, 3>(a, st);
+        return wide ? launch_fp8w<1, 240, 1, 3, 1>(a, st) : launch_fp8w<1, 128, 2, 3, 2>(a, st);
+    return wide ? launch_fp8w<2, 240, 2, 3, 2>(a, st) : launch_fp8w<2, 128, 2, 3, 2>(a, st);
 }
 
 }  // namespace gemm
