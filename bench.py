@@ -219,6 +219,14 @@ def replica_seed(seed: int, rank: int) -> int:
 
 
 # ------------------------------------------------------------------ our arm
+def clock_log_path(pattern, device_index):
+    """The clock-sample file for one device: the pattern with %d replaced by the
+    device index when it has one, else the pattern itself (None: a temporary file)."""
+    if not pattern:
+        return None
+    return pattern % device_index if "%d" in pattern else pattern
+
+
 def run_ours(args, rank, world, dev):
     import torch
     import expert_routing_grouped_layer_b200 as moe
@@ -282,7 +290,7 @@ def run_ours(args, rank, world, dev):
     events = [mk() for _ in range(args.steps)]
     di = dev.index if dev.index is not None else 0
     clocks = ClockSampler(di, enabled=not args.no_clocks,
-                          log_path=args.clock_log % di if args.clock_log else None)
+                          log_path=clock_log_path(args.clock_log, di))
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
