@@ -183,6 +183,40 @@ def layer_flops(cfg, T):
     return 2.0 * (N + T * cfg.n_shared_experts) * 3 * cfg.hidden * cfg.moe_intermediate_size
 
 
+def gate_up_flops(cfg, T):
+    """FLOPs of one gate/up launch: 2 of the 3 H x I products of every (token,
+    expert) pair and of every token through each shared expert."""
+    return layer_flops(cfg, T) * 2.0 / 3.0
+
+
+# Nominal dense tensor rates relative to bf16. The expert GEMMs run bf16/f16
+# MMAs when the activations are bf16 (FP8 weights are converted to 16 bits),
+# else block-scaled E2M1 x E4M3 MMAs at the FP8 rate.
+NOMINAL_RATE_VS_BF16 = {"bf16": 1.0, "fp8": 2.0}
+
+
+def tensor_peak(peaks, peak_src, cfg):
+    """(TFLOP/s, source) of the tensor rate the expert GEMMs run at: the
+    measured bf16 figure, times the nominal ratio for FP8-rate MMAs."""
+    kind = "bf16" if cfg.afmt == "bf16" else "fp8"
+    ratio = NOMINAL_RATE_VS_BF16[kind]
+    src = peak_src if ratio == 1.0 else "%s bf16 x nominal %s/bf16 ratio %g" % (peak_src, kind, ratio)
+    return peaks["bf16_tflops"] * ratio, src
+
+
+def roofline(bytes_, flops, ms, hbm, tpeak):
+    """The binding roof (the larger of bytes / HBM and FLOPs / tensor peak) and the
+    achieved fraction of it, with both fractions."""
+    s = ms / 1e3
+    hbm_frac = bytes_ / s / 1e9 / hbm
+    tensor_frac = flops / s / 1e12 / tpeak
+    if flops / (tpeak * 1e12) > bytes_ / (hbm * 1e9):
+        return {"bound": "tensor", "achieved": flops / s / 1e12, "peak": tpeak, "unit": "TFLOP/s",
+                "frac": tensor_frac, "hbm_frac": hbm_frac, "tensor_frac": tensor_frac}
+    return {"bound": "hbm", "achieved": bytes_ / s / 1e9, "peak": hbm, "unit": "GB/s",
+            "frac": hbm_frac, "hbm_frac": hbm_frac, "tensor_frac": tensor_frac}
+
+
 def ncu_traffic(kernel: str, workload: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
     the current source of the kernel (else None)."""
@@ -348,9 +382,25 @@ def run_ours(args, rank, world, dev):
     gu_bytes = gate_up_bytes(cfg, active, T)
     gu_ms = stage_ms["gate_up"]
     hbm = peaks["hbm_gbs"]
-    achieved = gu_bytes / (gu_ms / 1e3) / 1e9
+    tpeak, tpeak_src = tensor_peak(peaks, peak_src, cfg)
     lb = layer_bytes(cfg, active, T)
+    lf = layer_flops(cfg, T)
     ewb = expert_weight_bytes(cfg, active)
+    kroof = roofline(gu_bytes, gate_up_flops(cfg, T), gu_ms, hbm, tpeak)
+    kroof.update({"kernel": "gate_up (grouped SwiGLU GEMM1)",
+                  "peak_source": peak_src if kroof["bound"] == "hbm" else tpeak_src,
+                  "traffic": ncu_traffic("gate_up", args.workload)
+                  if not (args.tokens or args.experts) else None,
+                  "algorithmic_bytes_per_launch": gu_bytes,
+                  "algorithmic_flops_per_launch": gate_up_flops(cfg, T)})
+    lroof = roofline(lb, lf, ms, hbm, tpeak)
+    lroof.update({"bytes": lb, "achieved_gbs": lb / (ms / 1e3) / 1e9,
+                  # the activated and shared experts' weights alone (no router
+                  # weight, no activations)
+                  "expert_weight_bytes": ewb,
+                  "expert_weight_frac": ewb / (ms / 1e3) / 1e9 / hbm,
+                  "flops": lf, "tflops": lf / (ms / 1e3) / 1e12,
+                  "tensor_peak": tpeak, "tensor_peak_source": tpeak_src})
     line = {
         "metric": METRIC,
         "value": world * T / (ms / 1e3),
@@ -372,19 +422,8 @@ def run_ours(args, rank, world, dev):
                    "shared_experts": S, "active_experts": active,
                    "parallelism": "replicas x%d" % world,
                    "l2": "256 MiB write before every timed step, outside the timed events"},
-        "roofline": {"bound": "hbm", "kernel": "gate_up (grouped SwiGLU GEMM1)",
-                     "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                     "peak_source": peak_src, "traffic": ncu_traffic("gate_up", args.workload)
-                     if not (args.tokens or args.experts) else None,
-                     "algorithmic_bytes_per_launch": gu_bytes},
-        "layer_roofline": {"bound": "hbm", "bytes": lb, "achieved_gbs": lb / (ms / 1e3) / 1e9,
-                           "frac": lb / (ms / 1e3) / 1e9 / hbm,
-                           # the activated and shared experts' weights alone (no router
-                           # weight, no activations)
-                           "expert_weight_bytes": ewb,
-                           "expert_weight_frac": ewb / (ms / 1e3) / 1e9 / hbm,
-                           "flops": layer_flops(cfg, T),
-                           "tflops": layer_flops(cfg, T) / (ms / 1e3) / 1e12},
+        "roofline": kroof,
+        "layer_roofline": lroof,
         "stage_ms": stage_ms,
         "gpu_launches": launches_per_step(cfg, T, torch.cuda.get_device_properties(dev).multi_processor_count) * args.steps,
         "wall_s_timed_loop": wall,
