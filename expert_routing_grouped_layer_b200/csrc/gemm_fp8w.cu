@@ -15,11 +15,10 @@ namespace {
 // tensor-core instruction for E4M3 times bf16, so a converter warpgroup turns
 // each TMA-staged E4M3 weight tile into 16-bit values times the tile's block
 // scale, written straight into the 128B-swizzled K-major layout tcgen05.mma
-// reads. A staged tile spans RKM MMA stages of BK = 64 (RKM = 2: 128-byte
-// swizzled rows; RKM = 1: 64-byte rows): the TMA unit keeps a bounded number
-// of row requests in flight and an HBM row holds its slot for the DRAM
-// latency whatever its width, so full 128-byte rows halve the weight stream's
-// cost there, where shared memory leaves room for the larger staging slots.
+// reads. A staged tile spans two MMA stages of BK = 64 (128-byte swizzled
+// rows): the TMA unit keeps a bounded number of row requests in flight and an
+// HBM row holds its slot for the DRAM latency whatever its width, so full
+// 128-byte rows halve the weight stream's cost there against 64-byte ones.
 // With a staged tile inside one 128-wide scale block and M tiles aligned to
 // the 128-row blocks, one scalar scale covers a tile.
 //  * gate/up: f16 operands (see the f16 path below): one cvt and one f16x2
@@ -40,7 +39,7 @@ static_assert(512 % CVT_THREADS == 0, "converter tasks: whole tiles per round");
 // as soon as the converters have read a slot, so it can run many stages ahead
 // of the tensor cores; the MMA ring holds the converted bf16 weight tiles and
 // the token tile, freed by the MMA commit.
-template <int GEMM, int BNF_, int ACCB_, int MST_, int RKM_>
+template <int GEMM, int BNF_, int ACCB_, int MST_>
 struct TileF8 {
     // gate/up (f16 path, ~86 registers) affords a second group of 4 epilogue
     // warps, which halves the drain of its single accumulator buffer
@@ -49,15 +48,14 @@ struct TileF8 {
     static constexpr int NA = (GEMM == 1) ? 2 : 1;
     static constexpr int BNF = BNF_;
     static constexpr int ACCB = ACCB_;
-    static constexpr int RKM = RKM_;
-    static constexpr int RK = RKM * BK;           // K of a staged e4m3 tile (RKM MMA stages)
-    static constexpr int A8_BYTES = BM * RK;      // e4m3 staging tile, RK-byte rows
+    static constexpr int RK = 2 * BK;             // K of a staged e4m3 tile (two MMA stages)
+    static constexpr int A8_BYTES = BM * RK;      // e4m3 staging tile, 128-byte rows
     static constexpr int A_BYTES = BM * BK * 2;   // bf16 MMA tile
     static constexpr int B_BYTES = BNF * BK * 2;
     static constexpr int CVT_OFF = 0;                       // NA bf16 A tiles
     static constexpr int B_OFF = NA * A_BYTES;              // token tile
     static constexpr int MSLOT_BYTES = (B_OFF + B_BYTES + 1023) / 1024 * 1024;
-    static constexpr int RSLOT_BYTES = NA * A8_BYTES;       // NA e4m3 tiles (RKM MMA stages)
+    static constexpr int RSLOT_BYTES = NA * A8_BYTES;       // NA e4m3 tiles (two MMA stages)
     static constexpr int MSTAGES = MST_;
     static constexpr int FIXED_BYTES = 1024 + 8 * (2 * 8 + 3 * MSTAGES + 5) + 16 + 4 * (MAX_SEG + 1);
     static constexpr int RSTAGES_FIT = (232448 - FIXED_BYTES - MSTAGES * MSLOT_BYTES) / RSLOT_BYTES;
@@ -192,15 +190,15 @@ __device__ __forceinline__ void epilogue_f16_gate_up(const KParams& p, const int
     }
 }
 
-template <int GEMM, int BNF_, int ACCB_, int MST_, int RKM_>
-__global__ void __launch_bounds__(TileF8<GEMM, BNF_, ACCB_, MST_, RKM_>::THREADS, 1)
+template <int GEMM, int BNF_, int ACCB_, int MST_>
+__global__ void __launch_bounds__(TileF8<GEMM, BNF_, ACCB_, MST_>::THREADS, 1)
     grouped_gemm_fp8w_kernel(const __grid_constant__ CUtensorMap tmA_routed,
                              const __grid_constant__ CUtensorMap tmA_shared,
                              const __grid_constant__ BMaps tmB, const KParams p,
                              const float* __restrict__ scale_routed,
                              const float* __restrict__ scale_shared,
                              const int8_t* __restrict__ row_exp) {
-    using C = TileF8<GEMM, BNF_, ACCB_, MST_, RKM_>;
+    using C = TileF8<GEMM, BNF_, ACCB_, MST_>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -265,7 +263,7 @@ __global__ void __launch_bounds__(TileF8<GEMM, BNF_, ACCB_, MST_, RKM_>::THREADS
                 const Unit t = decode_unit(p, pref, u);
                 const CUtensorMap* tmA = (t.seg < p.E) ? &tmA_routed : &tmA_shared;
                 bool ok = true;
-                for (int kr = 0; kr < KB / C::RKM; ++kr) {
+                for (int kr = 0; kr < KB / 2; ++kr) {
                     if (!mbar_wait(&raw_empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
                     uint8_t* rs = rring + stage * C::RSLOT_BYTES;
                     mbar_arrive_expect_tx(&raw_full[stage], C::RSLOT_BYTES);
@@ -400,7 +398,7 @@ __global__ void __launch_bounds__(TileF8<GEMM, BNF_, ACCB_, MST_, RKM_>::THREADS
                         if (GEMM == 1) u_nxt = s_up[nj];
                     }
                 }
-                const int h = kb % C::RKM;  // MMA stage within the staged tile
+                const int h = kb & 1;  // half of the staged 128-K tile
                 if (!mbar_wait(&m_empty[mstage], mphase ^ 1, abort_flag)) { ok = false; break; }
                 if (h == 0 && !mbar_wait(&raw_full[rstage], rphase, abort_flag)) { ok = false; break; }
                 uint8_t* ms = mring + mstage * C::MSLOT_BYTES;
@@ -413,9 +411,7 @@ __global__ void __launch_bounds__(TileF8<GEMM, BNF_, ACCB_, MST_, RKM_>::THREADS
                     const int tile = (i * CVT_THREADS) >> 9;  // 512 tasks per tile, ct < CVT_THREADS
                     const int r = task & 127;
                     const int c = (task >> 7) & 3;
-                    const uint8_t* src =
-                        C::RKM == 2 ? rs + tile * C::A8_BYTES + r * 128 + (((4 * h + c) ^ (r & 7)) << 4)
-                                    : rs + tile * C::A8_BYTES + r * 64 + ((c ^ ((r >> 1) & 3)) << 4);
+                    const uint8_t* src = rs + tile * C::A8_BYTES + r * 128 + (((4 * h + c) ^ (r & 7)) << 4);
                     uint8_t* dst = ms + C::CVT_OFF + tile * C::A_BYTES + r * 128;
                     uint4 lo, hi;
                     if (GEMM == 1)
@@ -425,10 +421,10 @@ __global__ void __launch_bounds__(TileF8<GEMM, BNF_, ACCB_, MST_, RKM_>::THREADS
                     *reinterpret_cast<uint4*>(dst + (((2 * c) ^ (r & 7)) << 4)) = lo;
                     *reinterpret_cast<uint4*>(dst + (((2 * c + 1) ^ (r & 7)) << 4)) = hi;
                 }
-                if (h == C::RKM - 1) mbar_arrive(&raw_empty[rstage]);
+                if (h == 1) mbar_arrive(&raw_empty[rstage]);
                 fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
                 mbar_arrive(&cvt_full[mstage]);
-                if (h == C::RKM - 1 && ++rstage == C::RSTAGES) { rstage = 0; rphase ^= 1; }
+                if (h == 1 && ++rstage == C::RSTAGES) { rstage = 0; rphase ^= 1; }
                 if (++mstage == C::MSTAGES) { mstage = 0; mphase ^= 1; }
             }
             if (!ok) break;
@@ -444,15 +440,307 @@ __global__ void __launch_bounds__(TileF8<GEMM, BNF_, ACCB_, MST_, RKM_>::THREADS
 }
 
 
+// ---------------------------------------------------------------- gate/up, weights in TMEM
+// tcgen05.mma can read its A operand from tensor memory (row i in lane i, two K
+// elements per 32-bit column). Here the converter warps (two per lane quadrant:
+// gate rows, up rows) turn each E4M3 weight row into f16 values times m, as in
+// the f16 path above, and store them there with tcgen05.st, one thread per row:
+// the converted tiles never cross shared memory. Per MMA stage that takes the
+// converters' 32 KB of stores and the tensor core's 32 KB of A reads off the
+// shared-memory traffic that capped the variant above (~186 KB against ~128
+// bytes per cycle). TMEM holds the gate and up accumulators (2 x BNT columns,
+// single-buffered) and two A stages of 64 columns (gate 32, up 32), which
+// limits the token tile to 192. The staged E4M3 tiles span two MMA stages
+// (128-byte rows); shared memory holds only those and the token tiles.
+
+// D[tmem] (+)= A[tmem] * B[smem]^T, kind::f16.
+__device__ __forceinline__ void mma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Registers -> tensor memory: thread i of the warp writes r[0..31] to columns
+// col..col+31 of lane (base lane + i).
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]) : "memory");
+}
+
+template <int BNT_, int MST_>
+struct TileGU {
+    static constexpr int BNT = BNT_;
+    static constexpr int EG = 2;
+    static constexpr int THREADS = 64 + 128 + CVT_THREADS + 32 + 128;  // warps as in TileF8<1, ...>
+    static constexpr int RK = 2 * BK;                 // K of a staged e4m3 tile (two MMA stages)
+    static constexpr int A8_BYTES = BM * RK;          // one staged tile, 128-byte rows
+    static constexpr int RSLOT_BYTES = 2 * A8_BYTES;  // gate + up
+    static constexpr int B_BYTES = BNT * BK * 2;
+    static constexpr int MSLOT_BYTES = (B_BYTES + 1023) / 1024 * 1024;
+    static constexpr int MSTAGES = MST_;
+    static constexpr int FIXED_BYTES = 1024 + 8 * (2 * 8 + 3 * MSTAGES + 5) + 16 + 4 * (MAX_SEG + 1);
+    static constexpr int RSTAGES_FIT = (232448 - FIXED_BYTES - MSTAGES * MSLOT_BYTES) / RSLOT_BYTES;
+    static constexpr int RSTAGES = RSTAGES_FIT < 8 ? RSTAGES_FIT : 8;
+    static constexpr int ACC_COLS = 2 * BNT;  // gate at 0, up at BNT
+    static constexpr int A_COL = ACC_COLS;    // A stage s at A_COL + 64 s: gate, then up
+    static constexpr int TMEM_COLS = 512;
+    static_assert(A_COL + 2 * 64 <= TMEM_COLS, "tensor memory budget");
+    static constexpr int RING_BYTES = MSTAGES * MSLOT_BYTES + RSTAGES * RSLOT_BYTES;
+    static constexpr int BAR_BYTES = 8 * (2 * RSTAGES + 3 * MSTAGES + 5) + 16;
+    static constexpr int SMEM_BYTES = 1024 + RING_BYTES + BAR_BYTES + 4 * (MAX_SEG + 1);
+    static_assert(RSTAGES >= 2 && MSTAGES >= 2 && SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+template <int BNT_, int MST_>
+__global__ void __launch_bounds__(TileGU<BNT_, MST_>::THREADS, 1)
+    grouped_gemm_fp8w_gu_kernel(const __grid_constant__ CUtensorMap tmA_routed,
+                                const __grid_constant__ CUtensorMap tmA_shared,
+                                const __grid_constant__ BMaps tmB, const KParams p,
+                                const float* __restrict__ scale_routed,
+                                const float* __restrict__ scale_shared,
+                                const int8_t* __restrict__ row_exp) {
+    using C = TileGU<BNT_, MST_>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t* mring = smem;                                // [MSTAGES][MSLOT_BYTES]: token tiles
+    uint8_t* rring = smem + C::MSTAGES * C::MSLOT_BYTES;  // [RSTAGES][RSLOT_BYTES]: e4m3 tiles
+    uint64_t* raw_full = reinterpret_cast<uint64_t*>(smem + C::RING_BYTES);
+    uint64_t* raw_empty = raw_full + C::RSTAGES;
+    uint64_t* b_full = raw_empty + C::RSTAGES;  // token tile landed
+    uint64_t* cvt_full = b_full + C::MSTAGES;   // the stage's weight tiles are in their TMEM stage
+    uint64_t* m_empty = cvt_full + C::MSTAGES;  // the stage's MMAs completed
+    uint64_t* tfull = m_empty + C::MSTAGES;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* mma_done = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* pref = reinterpret_cast<int*>(tmem_slot + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::RSTAGES; ++s) {
+            mbar_init(&raw_full[s], 1);
+            mbar_init(&raw_empty[s], CVT_THREADS);
+        }
+        for (int s = 0; s < C::MSTAGES; ++s) {
+            mbar_init(&b_full[s], 1);
+            mbar_init(&cvt_full[s], CVT_THREADS);
+            mbar_init(&m_empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], 128 * C::EG);
+        }
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&tmA_routed);
+        tma_prefetch_desc(&tmA_shared);
+        prefetch_bmaps(tmB);
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    const int MT = p.M / BM;
+    if (warp == 1) build_schedule(p, pref, MT, lane);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int total = pref[p.nseg];
+    const int KB = p.K / BK;
+
+    if (warp == 0) {
+        // producer: e4m3 gate and up tiles (128 K each) into the raw ring
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued = 0;
+            for (int u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x) {
+                const Unit t = decode_unit(p, pref, u);
+                const CUtensorMap* tmA = (t.seg < p.E) ? &tmA_routed : &tmA_shared;
+                bool ok = true;
+                for (int kr = 0; kr < KB / 2; ++kr) {
+                    if (!mbar_wait(&raw_empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+                    uint8_t* rs = rring + stage * C::RSLOT_BYTES;
+                    mbar_arrive_expect_tx(&raw_full[stage], C::RSLOT_BYTES);
+                    tma_load_2d(rs, tmA, kr * C::RK, t.a_row, &raw_full[stage]);
+                    tma_load_2d(rs + C::A8_BYTES, tmA, kr * C::RK, t.a_row + p.a_up_offset, &raw_full[stage]);
+                    ++issued;
+                    if (++stage == C::RSTAGES) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+            }
+            if (*abort_flag) {
+                int s = stage;
+                uint32_t ph = phase;
+                for (int i = 0; i < min(issued, C::RSTAGES); ++i) {
+                    if (--s < 0) { s = C::RSTAGES - 1; ph ^= 1; }
+                    volatile int no_abort = 0;
+                    mbar_wait(&raw_full[s], ph, &no_abort);
+                }
+                status_or(p.status, MOE_DEV_TIMEOUT);
+            }
+        }
+    } else if (warp == 1) {
+        // MMA thread: A (gate, up) from the stage's TMEM columns, B from the token tile
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int g = 0;
+            uint32_t acc_phase = 0;
+            for (int u = blockIdx.x; u < total; u += gridDim.x) {
+                const Unit t = decode_unit(p, pref, u);
+                const int n_mma = (t.n_valid + 15) & ~15;
+                const uint32_t idesc = idesc_f16(BM, n_mma);
+                if (!mbar_wait(&tempty[0], acc_phase ^ 1, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t d0 = tmem_base;
+                bool ok = true;
+                for (int kb = 0; kb < KB; ++kb, ++g) {
+                    if (!mbar_wait(&b_full[stage], phase, abort_flag) ||
+                        !mbar_wait(&cvt_full[stage], phase, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a0 = tmem_base + C::A_COL + 64 * (g & 1);
+                    const uint32_t sb = smem_u32(mring + stage * C::MSLOT_BYTES);
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        const uint32_t acc_flag = (kb | kk) != 0;
+                        const uint64_t bd = sdesc_kmajor_sw128(sb + kk * 32);
+                        mma_f16_tmem_a(d0, a0 + 8 * kk, bd, idesc, acc_flag);
+                        mma_f16_tmem_a(d0 + C::BNT, a0 + 32 + 8 * kk, bd, idesc, acc_flag);
+                    }
+                    mma_commit(&m_empty[stage]);
+                    if (++stage == C::MSTAGES) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                mma_commit(&tfull[0]);
+                acc_phase ^= 1;
+            }
+            mma_commit(mma_done);
+            volatile int no_abort = 0;
+            mbar_wait(mma_done, 0, &no_abort);
+            if (*abort_flag) status_or(p.status, MOE_DEV_TIMEOUT);
+        }
+    } else if (warp == B_WARP) {
+        // token-tile loader: fills each slot's token tile as soon as it is free
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued = 0;
+            for (int u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x) {
+                const Unit t = decode_unit(p, pref, u);
+                const int n_mma = (t.n_valid + 15) & ~15;
+                bool ok = true;
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(&m_empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&b_full[stage], (uint32_t)(n_mma * BK * 2));
+                    load_b_rows(mring + stage * C::MSLOT_BYTES, tmB, kb * BK, t.b_row, n_mma, BK * 2,
+                                &b_full[stage]);
+                    ++issued;
+                    if (++stage == C::MSTAGES) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+            }
+            if (*abort_flag) {
+                int s = stage;
+                uint32_t ph = phase;
+                for (int i = 0; i < min(issued, C::MSTAGES); ++i) {
+                    if (--s < 0) { s = C::MSTAGES - 1; ph ^= 1; }
+                    volatile int no_abort = 0;
+                    mbar_wait(&b_full[s], ph, &no_abort);
+                }
+            }
+        }
+    } else if (warp < 6 || warp >= EPI2_WARP) {
+        epilogue_f16_gate_up<C::ACC_COLS, 1, C::EG>(p, pref, total, tmem_base, tfull, tempty,
+                                                    abort_flag, warp, lane, warp < 6 ? 0 : 1,
+                                                    scale_routed, scale_shared, row_exp);
+    } else {
+        // converters: warps 6..9 gate rows, 10..13 up rows; thread = one weight row
+        // of its quadrant. The TMEM stage of MMA stage g was last read by stage
+        // g - 2, whose completion (its slot's empty barrier) is awaited first.
+        const int tile = (warp - 6) >> 2;
+        const int row = (warp & 3) * 32 + lane;
+        const uint32_t lane_cols = tmem_base + ((uint32_t)((warp & 3) * 32) << 16) + C::A_COL + 32 * tile;
+        const int KS = p.K / 128;  // scale blocks along K
+        const int RS = p.a_rows_per_mat / 128;
+        int rstage = 0, mstage = 0, g = 0;
+        uint32_t rphase = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+            const Unit t = decode_unit(p, pref, u);
+            const bool routed = t.seg < p.E;
+            const int mat = routed ? t.seg : t.seg - p.E;
+            const float* sbase = (routed ? scale_routed : scale_shared) + (size_t)mat * RS * KS;
+            const float* srow = sbase + (size_t)(tile == 0 ? t.mt : p.a_up_offset / 128 + t.mt) * KS;
+            // block scales relative to the tile's power of two; the scale of K
+            // block j serves stages 2j and 2j+1, the next one is loaded ahead
+            const float inv = pow2f(-tile_exp(srow, KS, lane));
+            float s_cur = srow[0];
+            float s_nxt = KS > 1 ? srow[1] : 0.f;
+            for (int kb = 0; kb < KB; ++kb, ++g) {
+                if (kb > 0 && (kb & 1) == 0) {
+                    s_cur = s_nxt;
+                    const int nj = (kb >> 1) + 1;
+                    if (nj < KS) s_nxt = srow[nj];
+                }
+                const int h = kb & 1;  // half of the staged 128-K tile
+                if (h == 0 && !mbar_wait(&raw_full[rstage], rphase, abort_flag)) { ok = false; break; }
+                if (g >= 2) {
+                    const int gp = g - 2;
+                    if (!mbar_wait(&m_empty[gp % C::MSTAGES], (uint32_t)(gp / C::MSTAGES) & 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                }
+                tc_fence_after();
+                const __half2 m2 = __float2half2_rn(s_cur * inv);
+                const uint8_t* src = rring + rstage * C::RSLOT_BYTES + tile * C::A8_BYTES + row * 128;
+                uint32_t v[32];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint4 lo, hi;
+                    e4m3x16_to_f16_scaled(*reinterpret_cast<const uint4*>(src + (((4 * h + c) ^ (row & 7)) << 4)),
+                                          m2, lo, hi);
+                    v[8 * c + 0] = lo.x; v[8 * c + 1] = lo.y; v[8 * c + 2] = lo.z; v[8 * c + 3] = lo.w;
+                    v[8 * c + 4] = hi.x; v[8 * c + 5] = hi.y; v[8 * c + 6] = hi.z; v[8 * c + 7] = hi.w;
+                }
+                if (h == 1) mbar_arrive(&raw_empty[rstage]);
+                tmem_st32(lane_cols + 64 * (g & 1), v);
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(&cvt_full[mstage]);
+                if (h == 1 && ++rstage == C::RSTAGES) { rstage = 0; rphase ^= 1; }
+                if (++mstage == C::MSTAGES) mstage = 0;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
 }  // namespace
 
-template <int GEMM, int BNF_, int ACCB_, int MST_, int RKM_>
+template <int GEMM, int BNF_, int ACCB_, int MST_>
 cudaError_t launch_fp8w(const GroupedGemmArgs& a, cudaStream_t st) {
-    using C = TileF8<GEMM, BNF_, ACCB_, MST_, RKM_>;
+    using C = TileF8<GEMM, BNF_, ACCB_, MST_>;
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(grouped_gemm_fp8w_kernel<GEMM, BNF_, ACCB_, MST_, RKM_>,
+        attr_err = cudaFuncSetAttribute(grouped_gemm_fp8w_kernel<GEMM, BNF_, ACCB_, MST_>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     });
     if (attr_err != cudaSuccess) return attr_err;
@@ -463,17 +751,49 @@ cudaError_t launch_fp8w(const GroupedGemmArgs& a, cudaStream_t st) {
     BMaps tmB;
     const int S = a.S;
     if (!make_tmap_2d(&tmAr, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.w_routed, (uint64_t)a.E * p.a_rows_per_mat,
-                      p.K, p.K, C::RK, BM, C::RKM == 2 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B) ||
+                      p.K, p.K, C::RK, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_tmap_2d(&tmAs, CU_TENSOR_MAP_DATA_TYPE_UINT8, S > 0 ? a.w_shared : a.w_routed,
                       (uint64_t)(S > 0 ? S : a.E) * p.a_rows_per_mat, p.K, p.K, C::RK, BM,
-                      C::RKM == 2 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
+                      CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     if (b_rows == 0) return cudaSuccess;
     // gate/up reads f16 token rows (x * 2^-e), down reads the bf16 SwiGLU output
     if (!make_bmaps(&tmB, GEMM == 1 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
                     2, a.b_rows, b_rows, p.K, BK))
         return cudaErrorInvalidValue;
-    grouped_gemm_fp8w_kernel<GEMM, BNF_, ACCB_, MST_, RKM_><<<grid_for(p), C::THREADS, C::SMEM_BYTES, st>>>(
+    grouped_gemm_fp8w_kernel<GEMM, BNF_, ACCB_, MST_><<<grid_for(p), C::THREADS, C::SMEM_BYTES, st>>>(
+        tmAr, tmAs, tmB, p, static_cast<const float*>(a.w_routed_scale),
+        static_cast<const float*>(S > 0 ? a.w_shared_scale : a.w_routed_scale),
+        reinterpret_cast<const int8_t*>(a.b_scale));
+    return cudaGetLastError();
+}
+
+template <int BNT_, int MST_>
+cudaError_t launch_fp8w_gu(const GroupedGemmArgs& a, cudaStream_t st) {
+    using C = TileGU<BNT_, MST_>;
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(grouped_gemm_fp8w_gu_kernel<BNT_, MST_>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    uint64_t b_rows;
+    KParams p = make_params(a, 1, &b_rows);
+    p.bn = C::BNT;
+    CUtensorMap tmAr, tmAs;
+    BMaps tmB;
+    const int S = a.S;
+    if (!make_tmap_2d(&tmAr, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.w_routed, (uint64_t)a.E * p.a_rows_per_mat,
+                      p.K, p.K, C::RK, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap_2d(&tmAs, CU_TENSOR_MAP_DATA_TYPE_UINT8, S > 0 ? a.w_shared : a.w_routed,
+                      (uint64_t)(S > 0 ? S : a.E) * p.a_rows_per_mat, p.K, p.K, C::RK, BM,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    if (b_rows == 0) return cudaSuccess;
+    if (!make_bmaps(&tmB, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.b_rows, b_rows, p.K, BK))
+        return cudaErrorInvalidValue;
+    grouped_gemm_fp8w_gu_kernel<BNT_, MST_><<<grid_for(p), C::THREADS, C::SMEM_BYTES, st>>>(
         tmAr, tmAs, tmB, p, static_cast<const float*>(a.w_routed_scale),
         static_cast<const float*>(S > 0 ? a.w_shared_scale : a.w_routed_scale),
         reinterpret_cast<const int8_t*>(a.b_scale));
@@ -483,14 +803,14 @@ cudaError_t launch_fp8w(const GroupedGemmArgs& a, cudaStream_t st) {
 cudaError_t launch_gemm_fp8w(const GroupedGemmArgs& a, cudaStream_t st) {
     // many tokens per expert: wide token tiles (each weight tile converted once
     // per expert); few tokens per expert: narrower double-buffered tiles. The
-    // fourth argument is the MMA-ring depth; the raw ring takes the rest of
-    // shared memory (up to 8 slots of RKM MMA stages each, the last argument).
-    // Wide gate/up keeps 64-byte staged rows: the 128-byte ones leave room for
-    // two MMA slots only, which measured slower.
+    // last argument is the MMA-ring depth; the raw ring takes the rest of
+    // shared memory (up to 8 slots of two MMA stages each).
+    // Wide gate/up runs the variant with its weight tiles in tensor memory
+    // (192-token tiles, four token slots).
     const bool wide = a.N >= 128L * a.E;
     if (a.gemm == 1)
-        return wide ? launch_fp8w<1, 240, 1, 3, 1>(a, st) : launch_fp8w<1, 128, 2, 3, 2>(a, st);
-    return wide ? launch_fp8w<2, 240, 2, 3, 2>(a, st) : launch_fp8w<2, 128, 2, 3, 2>(a, st);
+        return wide ? launch_fp8w_gu<192, 4>(a, st) : launch_fp8w<1, 128, 2, 3>(a, st);
+    return wide ? launch_fp8w<2, 240, 2, 3>(a, st) : launch_fp8w<2, 128, 2, 3>(a, st);
 }
 
 }  // namespace gemm
