@@ -94,7 +94,7 @@ WsLayout ws_layout(const moe_config* c, int T) {
     L.xa = take((N + T) * H * act_bytes);
     L.xa_scale = take(act_bytes == 1 ? (N + T) * (H / 32) : (f16_gate_up(c) ? (N + T) : 0));
     L.hbuf = take((N + S * T) * I * act_bytes);
-    L.h_scale = take(act_bytes == 1 ? (N + S * T) * (I / 32) : 0);
+    L.h_scale = take(act_bytes == 1 ? (N + S * T) * (I / 32) : (f16_gate_up(c) ? (N + S * T) : 0));
     L.y = take(N * H * 2);
     L.shared_y = take(S * T * H * 2);
     L.total = off;
@@ -251,7 +251,7 @@ moe_status moe_expert_gate_up(const moe_config* cfg, const void* xa, const void*
     const bool q = cfg->afmt != MOE_A_BF16;
     if (!xa || !expert_offsets || !h || !aligned16(xa) || !aligned16(h)) return MOE_ERR_INVALID_ARG;
     if (q && (!xa_scale || !h_scale)) return MOE_ERR_INVALID_ARG;
-    if (f16_gate_up(cfg) && !xa_scale) return MOE_ERR_INVALID_ARG;
+    if (f16_gate_up(cfg) && (!xa_scale || !h_scale)) return MOE_ERR_INVALID_ARG;
     if (!weights_ok(cfg, w, true)) return MOE_ERR_INVALID_ARG;
     GroupedGemmArgs a = gemm_args(cfg, T, expert_offsets, dev_status);
     const size_t hrow = (size_t)a.I * (q ? 1 : 2);
@@ -266,7 +266,10 @@ moe_status moe_expert_gate_up(const moe_config* cfg, const void* xa, const void*
     a.out_shared = static_cast<char*>(h) + (size_t)a.N * hrow;
     a.out_routed_scale = static_cast<uint8_t*>(h_scale);
     a.out_shared_scale = q ? static_cast<uint8_t*>(h_scale) + (size_t)a.N * (a.I / 32) : nullptr;
-    return cuda_status(launch_grouped_gemm(a, as_stream(stream)));
+    cudaError_t e = launch_grouped_gemm(a, as_stream(stream));
+    if (e == cudaSuccess && f16_gate_up(cfg))  // the down projection's f16 input rows
+        e = launch_rows_to_f16(h, a.I, a.N + a.S * a.T, static_cast<int8_t*>(h_scale), as_stream(stream));
+    return cuda_status(e);
 }
 
 moe_status moe_expert_down(const moe_config* cfg, const void* h, const void* h_scale, int32_t T,
@@ -279,7 +282,7 @@ moe_status moe_expert_down(const moe_config* cfg, const void* h, const void* h_s
     const bool q = cfg->afmt != MOE_A_BF16;
     if (!h || !expert_offsets || !y || !aligned16(h) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
     if (cfg->n_shared_experts > 0 && (!shared_y || !aligned16(shared_y))) return MOE_ERR_INVALID_ARG;
-    if (q && !h_scale) return MOE_ERR_INVALID_ARG;
+    if ((q || f16_gate_up(cfg)) && !h_scale) return MOE_ERR_INVALID_ARG;
     if (!weights_ok(cfg, w, false)) return MOE_ERR_INVALID_ARG;
     GroupedGemmArgs a = gemm_args(cfg, T, expert_offsets, dev_status);
     a.gemm = 2;

@@ -21,38 +21,38 @@ namespace {
 // 128-byte rows halve the weight stream's cost there against 64-byte ones.
 // With a staged tile inside one 128-wide scale block and M tiles aligned to
 // the 128-row blocks, one scalar scale covers a tile.
-//  * gate/up: f16 operands (see the f16 path below): one cvt and one f16x2
-//    multiply per two weights; token rows come in as f16 with a power-of-two
-//    row scale.
-//  * down: bf16 operands, since its input h is the bf16 SwiGLU output; E4M3 ->
-//    bf16 is exact and the product with the fp32 scale is rounded once to bf16
-//    (relative error <= 2^-9 per weight).
+// Both GEMMs run on f16 operands (see the f16 path below): one cvt and one
+// f16x2 multiply per two weights. Token rows come in as f16 with a power-of-two
+// row scale, and so does the SwiGLU output h (the gate/up call rewrites its
+// bf16 rows in place).
 constexpr int CVT_WARPS = 8;
 constexpr int CVT_THREADS = CVT_WARPS * 32;
 constexpr int B_WARP = 6 + CVT_WARPS;  // token-tile loader, after the converters
 constexpr int EPI2_WARP = B_WARP + 1;  // second epilogue group (gate/up), after the loader
 static_assert(512 % CVT_THREADS == 0, "converter tasks: whole tiles per round");
 
-// GEMM: 1 gate/up, 2 down. BNF_: tokens per tile. ACCB_: accumulator buffers in
-// tensor memory (2 overlaps a tile's epilogue with the next main loop).
-// Two rings: the raw ring holds the TMA-staged e4m3 weight tiles and is freed
-// as soon as the converters have read a slot, so it can run many stages ahead
-// of the tensor cores; the MMA ring holds the converted bf16 weight tiles and
-// the token tile, freed by the MMA commit.
+// Gate/up with the converted weight tiles in shared memory (the narrow-tile
+// variant; wide tiles keep them in tensor memory, below). GEMM: 1 (gate/up).
+// BNF_: tokens per tile. ACCB_: accumulator buffers in tensor memory (2
+// overlaps a tile's epilogue with the next main loop). Two rings: the raw ring
+// holds the TMA-staged e4m3 weight tiles and is freed as soon as the converters
+// have read a slot, so it can run many stages ahead of the tensor cores; the
+// MMA ring holds the converted f16 weight tiles and the token tile, freed by
+// the MMA commit.
 template <int GEMM, int BNF_, int ACCB_, int MST_>
 struct TileF8 {
-    // gate/up (f16 path, ~86 registers) affords a second group of 4 epilogue
-    // warps, which halves the drain of its single accumulator buffer
-    static constexpr int EG = (GEMM == 1) ? 2 : 1;
+    static_assert(GEMM == 1, "the shared-memory variant serves the gate/up GEMM");
+    // a second group of 4 epilogue warps halves the drain of the accumulator
+    static constexpr int EG = 2;
     static constexpr int THREADS = 64 + 128 + CVT_THREADS + 32 + 128 * (EG - 1);
-    static constexpr int NA = (GEMM == 1) ? 2 : 1;
+    static constexpr int NA = 2;
     static constexpr int BNF = BNF_;
     static constexpr int ACCB = ACCB_;
     static constexpr int RK = 2 * BK;             // K of a staged e4m3 tile (two MMA stages)
     static constexpr int A8_BYTES = BM * RK;      // e4m3 staging tile, 128-byte rows
-    static constexpr int A_BYTES = BM * BK * 2;   // bf16 MMA tile
+    static constexpr int A_BYTES = BM * BK * 2;   // f16 MMA tile
     static constexpr int B_BYTES = BNF * BK * 2;
-    static constexpr int CVT_OFF = 0;                       // NA bf16 A tiles
+    static constexpr int CVT_OFF = 0;                       // NA f16 A tiles
     static constexpr int B_OFF = NA * A_BYTES;              // token tile
     static constexpr int MSLOT_BYTES = (B_OFF + B_BYTES + 1023) / 1024 * 1024;
     static constexpr int RSLOT_BYTES = NA * A8_BYTES;       // NA e4m3 tiles (two MMA stages)
@@ -68,25 +68,6 @@ struct TileF8 {
     static constexpr int SMEM_BYTES = 1024 + RING_BYTES + BAR_BYTES + 4 * (MAX_SEG + 1);
     static_assert(RSTAGES >= 2 && SMEM_BYTES <= 232448, "shared memory budget");
 };
-
-// 16 E4M3 values -> 16 bf16 values of (value * scale), in element order.
-__device__ __forceinline__ void e4m3x16_to_bf16_scaled(uint4 v, float scale, uint4& lo, uint4& hi) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    uint32_t o[8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const __nv_fp8x2_storage_t pair = (__nv_fp8x2_storage_t)((w[i] >> (16 * h)) & 0xFFFFu);
-            const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
-            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
-            const __nv_bfloat162 b = __floats2bfloat162_rn(f.x * scale, f.y * scale);
-            o[2 * i + h] = *reinterpret_cast<const uint32_t*>(&b);
-        }
-    }
-    lo = make_uint4(o[0], o[1], o[2], o[3]);
-    hi = make_uint4(o[4], o[5], o[6], o[7]);
-}
 
 // ---- f16 path of the gate/up GEMM. The tensor-core operands are f16: token
 // rows arrive as x * 2^-e (exact, see pack_f16_kernel) and each weight tile is
@@ -190,6 +171,52 @@ __device__ __forceinline__ void epilogue_f16_gate_up(const KParams& p, const int
     }
 }
 
+// Down epilogue of the f16 path: per unit, wait for the accumulator, read it 16
+// token columns at a time (lane = output feature), restore 2^E (the W2 tile) and
+// 2^e (the token's h row), store bf16, release the buffer.
+template <int ACC_COLS, int ACCB>
+__device__ __forceinline__ void epilogue_f16_down(const KParams& p, const int* pref, int total,
+                                                  uint32_t tmem_base, uint64_t* tfull, uint64_t* tempty,
+                                                  volatile int* abort_flag, int warp, int lane,
+                                                  const float* __restrict__ scale_routed,
+                                                  const float* __restrict__ scale_shared,
+                                                  const int8_t* __restrict__ row_exp) {
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const int KS = p.K / 128;
+    const int RS = p.a_rows_per_mat / 128;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int u = blockIdx.x; u < total; u += gridDim.x) {
+        const Unit t = decode_unit(p, pref, u);
+        const bool routed = t.seg < p.E;
+        const int mat = routed ? t.seg : t.seg - p.E;
+        const float* sbase = (routed ? scale_routed : scale_shared) + (size_t)mat * RS * KS;
+        const float fw = pow2f(tile_exp(sbase + (size_t)t.mt * KS, KS, lane));
+        if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * ACC_COLS;
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(t.out) + t.mt * BM + row;
+        for (int c0 = 0; c0 < t.n_valid; c0 += 16) {
+            uint32_t g[16];
+            tmem_ld16(taddr + c0, g);
+            // 2^e of this lane's token column (e in [-127, 114]; 2^-127 is subnormal)
+            const int ex_l = (lane < 16 && c0 + lane < t.n_valid) ? row_exp[t.b_row + c0 + lane] : 0;
+            const float fe_l = ex_l >= -126 ? pow2f(ex_l) : __uint_as_float(0x00400000u);
+            tmem_ld_wait(g);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const float fe = __shfl_sync(0xffffffffu, fe_l, j);
+                if (c0 + j < t.n_valid)  // exact power-of-two factors
+                    out[(size_t)(c0 + j) * p.ld_out] = __float2bfloat16_rn(__uint_as_float(g[j]) * fw * fe);
+            }
+        }
+        tc_fence_before();
+        mbar_arrive(&tempty[acc]);
+        if (++acc == ACCB) { acc = 0; acc_phase ^= 1; }
+    }
+}
+
 template <int GEMM, int BNF_, int ACCB_, int MST_>
 __global__ void __launch_bounds__(TileF8<GEMM, BNF_, ACCB_, MST_>::THREADS, 1)
     grouped_gemm_fp8w_kernel(const __grid_constant__ CUtensorMap tmA_routed,
@@ -268,9 +295,7 @@ __global__ void __launch_bounds__(TileF8<GEMM, BNF_, ACCB_, MST_>::THREADS, 1)
                     uint8_t* rs = rring + stage * C::RSLOT_BYTES;
                     mbar_arrive_expect_tx(&raw_full[stage], C::RSLOT_BYTES);
                     tma_load_2d(rs, tmA, kr * C::RK, t.a_row, &raw_full[stage]);
-                    if (GEMM == 1)
-                        tma_load_2d(rs + C::A8_BYTES, tmA, kr * C::RK, t.a_row + p.a_up_offset,
-                                    &raw_full[stage]);
+                    tma_load_2d(rs + C::A8_BYTES, tmA, kr * C::RK, t.a_row + p.a_up_offset, &raw_full[stage]);
                     ++issued;
                     if (++stage == C::RSTAGES) { stage = 0; phase ^= 1; }
                 }
@@ -296,7 +321,7 @@ __global__ void __launch_bounds__(TileF8<GEMM, BNF_, ACCB_, MST_>::THREADS, 1)
             for (int u = blockIdx.x; u < total; u += gridDim.x) {
                 const Unit t = decode_unit(p, pref, u);
                 const int n_mma = (t.n_valid + 15) & ~15;
-                const uint32_t idesc = GEMM == 1 ? idesc_f16(BM, n_mma) : idesc_bf16(BM, n_mma);
+                const uint32_t idesc = idesc_f16(BM, n_mma);
                 if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag)) break;
                 tc_fence_after();
                 const uint32_t d0 = tmem_base + acc * C::ACC_COLS;
@@ -312,9 +337,8 @@ __global__ void __launch_bounds__(TileF8<GEMM, BNF_, ACCB_, MST_>::THREADS, 1)
                         const uint32_t acc_flag = (kb | kk) != 0;
                         const uint64_t bd = sdesc_kmajor_sw128(sb + kk * 32);
                         mma_bf16(d0, sdesc_kmajor_sw128(st + C::CVT_OFF + kk * 32), bd, idesc, acc_flag);
-                        if (GEMM == 1)
-                            mma_bf16(d0 + C::BNF, sdesc_kmajor_sw128(st + C::CVT_OFF + C::A_BYTES + kk * 32),
-                                     bd, idesc, acc_flag);
+                        mma_bf16(d0 + C::BNF, sdesc_kmajor_sw128(st + C::CVT_OFF + C::A_BYTES + kk * 32), bd,
+                                 idesc, acc_flag);
                     }
                     mma_commit(&m_empty[stage]);
                     if (++stage == C::MSTAGES) { stage = 0; phase ^= 1; }
@@ -359,15 +383,11 @@ __global__ void __launch_bounds__(TileF8<GEMM, BNF_, ACCB_, MST_>::THREADS, 1)
             }
         }
     } else if (warp < 6 || warp >= EPI2_WARP) {
-        if (GEMM == 1)
-            epilogue_f16_gate_up<C::ACC_COLS, C::ACCB, C::EG>(
-                p, pref, total, tmem_base, tfull, tempty, abort_flag, warp, lane,
-                warp < 6 ? 0 : 1, scale_routed, scale_shared, row_exp);
-        else
-            epilogue_loop<2, C::ACC_COLS, C::ACCB>(p, pref, total, tmem_base, tfull, tempty,
-                                                   abort_flag, warp, lane);
+        epilogue_f16_gate_up<C::ACC_COLS, C::ACCB, C::EG>(p, pref, total, tmem_base, tfull, tempty,
+                                                          abort_flag, warp, lane, warp < 6 ? 0 : 1,
+                                                          scale_routed, scale_shared, row_exp);
     } else {
-        // converters: e4m3 raw slot -> scaled bf16 tiles of the MMA slot
+        // converters: e4m3 raw slot -> scaled f16 tiles of the MMA slot
         const int ct = threadIdx.x - 192;
         const int KS = p.K / 128;  // scale blocks along K
         const int RS = p.a_rows_per_mat / 128;
@@ -380,13 +400,13 @@ __global__ void __launch_bounds__(TileF8<GEMM, BNF_, ACCB_, MST_>::THREADS, 1)
             const float* sbase = (routed ? scale_routed : scale_shared) + (size_t)mat * RS * KS;
             const float* s_gate = sbase + (size_t)(t.mt) * KS;
             const float* s_up = sbase + (size_t)(p.a_up_offset / 128 + t.mt) * KS;
-            // gate/up (f16 path): block scales relative to the tile's power of two
-            const float inv_g = GEMM == 1 ? pow2f(-tile_exp(s_gate, KS, lane)) : 1.f;
-            const float inv_u = GEMM == 1 ? pow2f(-tile_exp(s_up, KS, lane)) : 1.f;
+            // block scales relative to the tile's power of two
+            const float inv_g = pow2f(-tile_exp(s_gate, KS, lane));
+            const float inv_u = pow2f(-tile_exp(s_up, KS, lane));
             // the scales of K block j serve stages 2j and 2j+1; the next block's are
             // loaded two stages ahead so the load never stalls a conversion
-            float g_cur = s_gate[0], u_cur = GEMM == 1 ? s_up[0] : 0.f;
-            float g_nxt = KS > 1 ? s_gate[1] : 0.f, u_nxt = (GEMM == 1 && KS > 1) ? s_up[1] : 0.f;
+            float g_cur = s_gate[0], u_cur = s_up[0];
+            float g_nxt = KS > 1 ? s_gate[1] : 0.f, u_nxt = KS > 1 ? s_up[1] : 0.f;
             bool ok = true;
             for (int kb = 0; kb < KB; ++kb) {
                 if (kb > 0 && (kb & 1) == 0) {
@@ -395,7 +415,7 @@ __global__ void __launch_bounds__(TileF8<GEMM, BNF_, ACCB_, MST_>::THREADS, 1)
                     const int nj = (kb >> 1) + 1;
                     if (nj < KS) {
                         g_nxt = s_gate[nj];
-                        if (GEMM == 1) u_nxt = s_up[nj];
+                        u_nxt = s_up[nj];
                     }
                 }
                 const int h = kb & 1;  // half of the staged 128-K tile
@@ -403,7 +423,6 @@ __global__ void __launch_bounds__(TileF8<GEMM, BNF_, ACCB_, MST_>::THREADS, 1)
                 if (h == 0 && !mbar_wait(&raw_full[rstage], rphase, abort_flag)) { ok = false; break; }
                 uint8_t* ms = mring + mstage * C::MSLOT_BYTES;
                 const uint8_t* rs = rring + rstage * C::RSLOT_BYTES;
-                const float sc[2] = {g_cur, u_cur};
                 const __half2 m2[2] = {__float2half2_rn(g_cur * inv_g), __float2half2_rn(u_cur * inv_u)};
 #pragma unroll
                 for (int i = 0; i < C::NA * 512 / CVT_THREADS; ++i) {
@@ -414,10 +433,7 @@ __global__ void __launch_bounds__(TileF8<GEMM, BNF_, ACCB_, MST_>::THREADS, 1)
                     const uint8_t* src = rs + tile * C::A8_BYTES + r * 128 + (((4 * h + c) ^ (r & 7)) << 4);
                     uint8_t* dst = ms + C::CVT_OFF + tile * C::A_BYTES + r * 128;
                     uint4 lo, hi;
-                    if (GEMM == 1)
-                        e4m3x16_to_f16_scaled(*reinterpret_cast<const uint4*>(src), m2[tile], lo, hi);
-                    else
-                        e4m3x16_to_bf16_scaled(*reinterpret_cast<const uint4*>(src), sc[tile], lo, hi);
+                    e4m3x16_to_f16_scaled(*reinterpret_cast<const uint4*>(src), m2[tile], lo, hi);
                     *reinterpret_cast<uint4*>(dst + (((2 * c) ^ (r & 7)) << 4)) = lo;
                     *reinterpret_cast<uint4*>(dst + (((2 * c + 1) ^ (r & 7)) << 4)) = hi;
                 }
@@ -440,18 +456,25 @@ __global__ void __launch_bounds__(TileF8<GEMM, BNF_, ACCB_, MST_>::THREADS, 1)
 }
 
 
-// ---------------------------------------------------------------- gate/up, weights in TMEM
+// ---------------------------------------------------------------- weights in TMEM
 // tcgen05.mma can read its A operand from tensor memory (row i in lane i, two K
-// elements per 32-bit column). Here the converter warps (two per lane quadrant:
-// gate rows, up rows) turn each E4M3 weight row into f16 values times m, as in
-// the f16 path above, and store them there with tcgen05.st, one thread per row:
-// the converted tiles never cross shared memory. Per MMA stage that takes the
-// converters' 32 KB of stores and the tensor core's 32 KB of A reads off the
-// shared-memory traffic that capped the variant above (~186 KB against ~128
-// bytes per cycle). TMEM holds the gate and up accumulators (2 x BNT columns,
-// single-buffered) and two A stages of 64 columns (gate 32, up 32), which
-// limits the token tile to 192. The staged E4M3 tiles span two MMA stages
-// (128-byte rows); shared memory holds only those and the token tiles.
+// elements per 32-bit column). In this variant the converter warps turn each
+// E4M3 weight row into f16 values times m, as in the f16 path above, and store
+// them there with tcgen05.st, so the converted tiles never cross shared memory.
+// Per MMA stage that takes the converters' stores and the tensor core's A
+// reads (32 KB each for gate/up, 16 KB for down) off the shared-memory traffic
+// that bounds the shared-memory variant (for wide gate/up ~186 KB against ~128
+// bytes per cycle per 960-cycle stage). TMEM holds the accumulators and two A
+// stages:
+//  * gate/up: gate and up accumulators (2 x 192 columns, single-buffered), A
+//    stages of 64 columns (gate 32, up 32); converter warps 6..9 take gate
+//    rows, 10..13 up rows, one thread per row.
+//  * down (every tile width): two accumulators of up to 224 columns (double-
+//    buffered), A stages of 32 columns; converter warps 6..9 take the first 32
+//    K of a row, 10..13 the last 32. Its token rows are the f16 h rows (h times
+//    2^-e, e per row), restored by the epilogue with the tile's 2^E.
+// The staged E4M3 tiles span two MMA stages (128-byte rows); shared memory
+// holds only those and the token tiles.
 
 // D[tmem] (+)= A[tmem] * B[smem]^T, kind::f16.
 __device__ __forceinline__ void mma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
@@ -470,39 +493,48 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
     asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]) : "memory");
 }
 
-template <int BNT_, int MST_>
-struct TileGU {
+template <int GEMM, int BNT_, int MST_>
+struct TileTA {
+    static constexpr int NA = (GEMM == 1) ? 2 : 1;
+    static constexpr int EG = (GEMM == 1) ? 2 : 1;
+    static constexpr int ACCB = (GEMM == 1) ? 1 : 2;
     static constexpr int BNT = BNT_;
-    static constexpr int EG = 2;
-    static constexpr int THREADS = 64 + 128 + CVT_THREADS + 32 + 128;  // warps as in TileF8<1, ...>
-    static constexpr int RK = 2 * BK;                 // K of a staged e4m3 tile (two MMA stages)
-    static constexpr int A8_BYTES = BM * RK;          // one staged tile, 128-byte rows
-    static constexpr int RSLOT_BYTES = 2 * A8_BYTES;  // gate + up
+    static constexpr int THREADS = 64 + 128 + CVT_THREADS + 32 + 128 * (EG - 1);  // warps as in TileF8
+    static constexpr int RK = 2 * BK;                  // K of a staged e4m3 tile (two MMA stages)
+    static constexpr int A8_BYTES = BM * RK;           // one staged tile, 128-byte rows
+    static constexpr int RSLOT_BYTES = NA * A8_BYTES;
     static constexpr int B_BYTES = BNT * BK * 2;
     static constexpr int MSLOT_BYTES = (B_BYTES + 1023) / 1024 * 1024;
     static constexpr int MSTAGES = MST_;
     static constexpr int FIXED_BYTES = 1024 + 8 * (2 * 8 + 3 * MSTAGES + 5) + 16 + 4 * (MAX_SEG + 1);
     static constexpr int RSTAGES_FIT = (232448 - FIXED_BYTES - MSTAGES * MSLOT_BYTES) / RSLOT_BYTES;
     static constexpr int RSTAGES = RSTAGES_FIT < 8 ? RSTAGES_FIT : 8;
-    static constexpr int ACC_COLS = 2 * BNT;  // gate at 0, up at BNT
-    static constexpr int A_COL = ACC_COLS;    // A stage s at A_COL + 64 s: gate, then up
+    static constexpr int ACC_COLS = NA * BNT;       // gate at 0, up at BNT (gate/up)
+    static constexpr int A_COL = ACCB * ACC_COLS;   // A stage s at A_COL + s * A_STAGE_COLS
+    static constexpr int A_STAGE_COLS = 32 * NA;    // 64 K of 16-bit values per weight tile
     static constexpr int TMEM_COLS = 512;
-    static_assert(A_COL + 2 * 64 <= TMEM_COLS, "tensor memory budget");
+    static_assert(A_COL + 2 * A_STAGE_COLS <= TMEM_COLS, "tensor memory budget");
     static constexpr int RING_BYTES = MSTAGES * MSLOT_BYTES + RSTAGES * RSLOT_BYTES;
     static constexpr int BAR_BYTES = 8 * (2 * RSTAGES + 3 * MSTAGES + 5) + 16;
     static constexpr int SMEM_BYTES = 1024 + RING_BYTES + BAR_BYTES + 4 * (MAX_SEG + 1);
     static_assert(RSTAGES >= 2 && MSTAGES >= 2 && SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-template <int BNT_, int MST_>
-__global__ void __launch_bounds__(TileGU<BNT_, MST_>::THREADS, 1)
-    grouped_gemm_fp8w_gu_kernel(const __grid_constant__ CUtensorMap tmA_routed,
+// Registers -> tensor memory: thread i of the warp writes r[0..15] to columns
+// col..col+15 of lane (base lane + i).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]) : "memory");
+}
+
+template <int GEMM, int BNT_, int MST_>
+__global__ void __launch_bounds__(TileTA<GEMM, BNT_, MST_>::THREADS, 1)
+    grouped_gemm_fp8w_ta_kernel(const __grid_constant__ CUtensorMap tmA_routed,
                                 const __grid_constant__ CUtensorMap tmA_shared,
                                 const __grid_constant__ BMaps tmB, const KParams p,
                                 const float* __restrict__ scale_routed,
                                 const float* __restrict__ scale_shared,
                                 const int8_t* __restrict__ row_exp) {
-    using C = TileGU<BNT_, MST_>;
+    using C = TileTA<GEMM, BNT_, MST_>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -558,7 +590,7 @@ __global__ void __launch_bounds__(TileGU<BNT_, MST_>::THREADS, 1)
     const int KB = p.K / BK;
 
     if (warp == 0) {
-        // producer: e4m3 gate and up tiles (128 K each) into the raw ring
+        // producer: e4m3 weight tiles (gate and up, or one down tile; 128 K each) into the raw ring
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
@@ -572,7 +604,9 @@ __global__ void __launch_bounds__(TileGU<BNT_, MST_>::THREADS, 1)
                     uint8_t* rs = rring + stage * C::RSLOT_BYTES;
                     mbar_arrive_expect_tx(&raw_full[stage], C::RSLOT_BYTES);
                     tma_load_2d(rs, tmA, kr * C::RK, t.a_row, &raw_full[stage]);
-                    tma_load_2d(rs + C::A8_BYTES, tmA, kr * C::RK, t.a_row + p.a_up_offset, &raw_full[stage]);
+                    if (GEMM == 1)
+                        tma_load_2d(rs + C::A8_BYTES, tmA, kr * C::RK, t.a_row + p.a_up_offset,
+                                    &raw_full[stage]);
                     ++issued;
                     if (++stage == C::RSTAGES) { stage = 0; phase ^= 1; }
                 }
@@ -590,39 +624,40 @@ __global__ void __launch_bounds__(TileGU<BNT_, MST_>::THREADS, 1)
             }
         }
     } else if (warp == 1) {
-        // MMA thread: A (gate, up) from the stage's TMEM columns, B from the token tile
+        // MMA thread: A from the stage's TMEM columns, B from the token tile
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
             int g = 0;
+            int acc = 0;
             uint32_t acc_phase = 0;
             for (int u = blockIdx.x; u < total; u += gridDim.x) {
                 const Unit t = decode_unit(p, pref, u);
                 const int n_mma = (t.n_valid + 15) & ~15;
                 const uint32_t idesc = idesc_f16(BM, n_mma);
-                if (!mbar_wait(&tempty[0], acc_phase ^ 1, abort_flag)) break;
+                if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag)) break;
                 tc_fence_after();
-                const uint32_t d0 = tmem_base;
+                const uint32_t d0 = tmem_base + acc * C::ACC_COLS;
                 bool ok = true;
                 for (int kb = 0; kb < KB; ++kb, ++g) {
                     if (!mbar_wait(&b_full[stage], phase, abort_flag) ||
                         !mbar_wait(&cvt_full[stage], phase, abort_flag)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t a0 = tmem_base + C::A_COL + 64 * (g & 1);
+                    const uint32_t a0 = tmem_base + C::A_COL + C::A_STAGE_COLS * (g & 1);
                     const uint32_t sb = smem_u32(mring + stage * C::MSLOT_BYTES);
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
                         const uint32_t acc_flag = (kb | kk) != 0;
                         const uint64_t bd = sdesc_kmajor_sw128(sb + kk * 32);
                         mma_f16_tmem_a(d0, a0 + 8 * kk, bd, idesc, acc_flag);
-                        mma_f16_tmem_a(d0 + C::BNT, a0 + 32 + 8 * kk, bd, idesc, acc_flag);
+                        if (GEMM == 1) mma_f16_tmem_a(d0 + C::BNT, a0 + 32 + 8 * kk, bd, idesc, acc_flag);
                     }
                     mma_commit(&m_empty[stage]);
                     if (++stage == C::MSTAGES) { stage = 0; phase ^= 1; }
                 }
                 if (!ok) break;
-                mma_commit(&tfull[0]);
-                acc_phase ^= 1;
+                mma_commit(&tfull[acc]);
+                if (++acc == C::ACCB) { acc = 0; acc_phase ^= 1; }
             }
             mma_commit(mma_done);
             volatile int no_abort = 0;
@@ -660,16 +695,23 @@ __global__ void __launch_bounds__(TileGU<BNT_, MST_>::THREADS, 1)
             }
         }
     } else if (warp < 6 || warp >= EPI2_WARP) {
-        epilogue_f16_gate_up<C::ACC_COLS, 1, C::EG>(p, pref, total, tmem_base, tfull, tempty,
-                                                    abort_flag, warp, lane, warp < 6 ? 0 : 1,
-                                                    scale_routed, scale_shared, row_exp);
+        if (GEMM == 1)
+            epilogue_f16_gate_up<C::ACC_COLS, 1, C::EG>(p, pref, total, tmem_base, tfull, tempty,
+                                                        abort_flag, warp, lane, warp < 6 ? 0 : 1,
+                                                        scale_routed, scale_shared, row_exp);
+        else
+            epilogue_f16_down<C::ACC_COLS, C::ACCB>(p, pref, total, tmem_base, tfull, tempty, abort_flag,
+                                                    warp, lane, scale_routed, scale_shared, row_exp);
     } else {
-        // converters: warps 6..9 gate rows, 10..13 up rows; thread = one weight row
-        // of its quadrant. The TMEM stage of MMA stage g was last read by stage
-        // g - 2, whose completion (its slot's empty barrier) is awaited first.
-        const int tile = (warp - 6) >> 2;
+        // converters, thread = one weight row of its lane quadrant. gate/up: warps
+        // 6..9 gate rows, 10..13 up rows, 64 K each; down: warps 6..9 the first
+        // 32 K of a row, 10..13 the last 32. The TMEM stage of MMA stage g was
+        // last read by stage g - 2, whose completion (its slot's empty barrier)
+        // is awaited first.
+        const int tile = (warp - 6) >> 2;  // gate/up: which tile; down: which half of the row
         const int row = (warp & 3) * 32 + lane;
-        const uint32_t lane_cols = tmem_base + ((uint32_t)((warp & 3) * 32) << 16) + C::A_COL + 32 * tile;
+        const uint32_t lane_cols = tmem_base + ((uint32_t)((warp & 3) * 32) << 16) + C::A_COL +
+                                   (GEMM == 1 ? 32 : 16) * tile;
         const int KS = p.K / 128;  // scale blocks along K
         const int RS = p.a_rows_per_mat / 128;
         int rstage = 0, mstage = 0, g = 0;
@@ -680,8 +722,9 @@ __global__ void __launch_bounds__(TileGU<BNT_, MST_>::THREADS, 1)
             const bool routed = t.seg < p.E;
             const int mat = routed ? t.seg : t.seg - p.E;
             const float* sbase = (routed ? scale_routed : scale_shared) + (size_t)mat * RS * KS;
-            const float* srow = sbase + (size_t)(tile == 0 ? t.mt : p.a_up_offset / 128 + t.mt) * KS;
-            // block scales relative to the tile's power of two; the scale of K
+            const float* srow =
+                sbase + (size_t)((GEMM == 1 && tile == 1) ? p.a_up_offset / 128 + t.mt : t.mt) * KS;
+            // block scales relative to the tile's power of two. The scale of K
             // block j serves stages 2j and 2j+1, the next one is loaded ahead
             const float inv = pow2f(-tile_exp(srow, KS, lane));
             float s_cur = srow[0];
@@ -703,18 +746,34 @@ __global__ void __launch_bounds__(TileGU<BNT_, MST_>::THREADS, 1)
                 }
                 tc_fence_after();
                 const __half2 m2 = __float2half2_rn(s_cur * inv);
-                const uint8_t* src = rring + rstage * C::RSLOT_BYTES + tile * C::A8_BYTES + row * 128;
-                uint32_t v[32];
+                if (GEMM == 1) {
+                    const uint8_t* src = rring + rstage * C::RSLOT_BYTES + tile * C::A8_BYTES + row * 128;
+                    uint32_t v[32];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint4 lo, hi;
-                    e4m3x16_to_f16_scaled(*reinterpret_cast<const uint4*>(src + (((4 * h + c) ^ (row & 7)) << 4)),
-                                          m2, lo, hi);
-                    v[8 * c + 0] = lo.x; v[8 * c + 1] = lo.y; v[8 * c + 2] = lo.z; v[8 * c + 3] = lo.w;
-                    v[8 * c + 4] = hi.x; v[8 * c + 5] = hi.y; v[8 * c + 6] = hi.z; v[8 * c + 7] = hi.w;
+                    for (int c = 0; c < 4; ++c) {
+                        uint4 lo, hi;
+                        e4m3x16_to_f16_scaled(
+                            *reinterpret_cast<const uint4*>(src + (((4 * h + c) ^ (row & 7)) << 4)), m2, lo, hi);
+                        v[8 * c + 0] = lo.x; v[8 * c + 1] = lo.y; v[8 * c + 2] = lo.z; v[8 * c + 3] = lo.w;
+                        v[8 * c + 4] = hi.x; v[8 * c + 5] = hi.y; v[8 * c + 6] = hi.z; v[8 * c + 7] = hi.w;
+                    }
+                    if (h == 1) mbar_arrive(&raw_empty[rstage]);
+                    tmem_st32(lane_cols + C::A_STAGE_COLS * (g & 1), v);
+                } else {
+                    const uint8_t* src = rring + rstage * C::RSLOT_BYTES + row * 128;
+                    uint32_t v[16];
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        const int c = 2 * tile + i;  // 16-K chunk of the stage
+                        uint4 lo, hi;
+                        e4m3x16_to_f16_scaled(
+                            *reinterpret_cast<const uint4*>(src + (((4 * h + c) ^ (row & 7)) << 4)), m2, lo, hi);
+                        v[8 * i + 0] = lo.x; v[8 * i + 1] = lo.y; v[8 * i + 2] = lo.z; v[8 * i + 3] = lo.w;
+                        v[8 * i + 4] = hi.x; v[8 * i + 5] = hi.y; v[8 * i + 6] = hi.z; v[8 * i + 7] = hi.w;
+                    }
+                    if (h == 1) mbar_arrive(&raw_empty[rstage]);
+                    tmem_st16(lane_cols + C::A_STAGE_COLS * (g & 1), v);
                 }
-                if (h == 1) mbar_arrive(&raw_empty[rstage]);
-                tmem_st32(lane_cols + 64 * (g & 1), v);
                 tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(&cvt_full[mstage]);
@@ -757,9 +816,8 @@ cudaError_t launch_fp8w(const GroupedGemmArgs& a, cudaStream_t st) {
                       CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     if (b_rows == 0) return cudaSuccess;
-    // gate/up reads f16 token rows (x * 2^-e), down reads the bf16 SwiGLU output
-    if (!make_bmaps(&tmB, GEMM == 1 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                    2, a.b_rows, b_rows, p.K, BK))
+    // f16 token rows (x * 2^-e)
+    if (!make_bmaps(&tmB, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.b_rows, b_rows, p.K, BK))
         return cudaErrorInvalidValue;
     grouped_gemm_fp8w_kernel<GEMM, BNF_, ACCB_, MST_><<<grid_for(p), C::THREADS, C::SMEM_BYTES, st>>>(
         tmAr, tmAs, tmB, p, static_cast<const float*>(a.w_routed_scale),
@@ -768,18 +826,18 @@ cudaError_t launch_fp8w(const GroupedGemmArgs& a, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-template <int BNT_, int MST_>
-cudaError_t launch_fp8w_gu(const GroupedGemmArgs& a, cudaStream_t st) {
-    using C = TileGU<BNT_, MST_>;
+template <int GEMM, int BNT_, int MST_>
+cudaError_t launch_fp8w_ta(const GroupedGemmArgs& a, cudaStream_t st) {
+    using C = TileTA<GEMM, BNT_, MST_>;
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(grouped_gemm_fp8w_gu_kernel<BNT_, MST_>,
+        attr_err = cudaFuncSetAttribute(grouped_gemm_fp8w_ta_kernel<GEMM, BNT_, MST_>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     });
     if (attr_err != cudaSuccess) return attr_err;
     uint64_t b_rows;
-    KParams p = make_params(a, 1, &b_rows);
+    KParams p = make_params(a, GEMM, &b_rows);
     p.bn = C::BNT;
     CUtensorMap tmAr, tmAs;
     BMaps tmB;
@@ -791,9 +849,10 @@ cudaError_t launch_fp8w_gu(const GroupedGemmArgs& a, cudaStream_t st) {
                       CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     if (b_rows == 0) return cudaSuccess;
+    // f16 rows: token rows x * 2^-e (gate/up), SwiGLU output rows h * 2^-e (down)
     if (!make_bmaps(&tmB, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.b_rows, b_rows, p.K, BK))
         return cudaErrorInvalidValue;
-    grouped_gemm_fp8w_gu_kernel<BNT_, MST_><<<grid_for(p), C::THREADS, C::SMEM_BYTES, st>>>(
+    grouped_gemm_fp8w_ta_kernel<GEMM, BNT_, MST_><<<grid_for(p), C::THREADS, C::SMEM_BYTES, st>>>(
         tmAr, tmAs, tmB, p, static_cast<const float*>(a.w_routed_scale),
         static_cast<const float*>(S > 0 ? a.w_shared_scale : a.w_routed_scale),
         reinterpret_cast<const int8_t*>(a.b_scale));
@@ -805,12 +864,12 @@ cudaError_t launch_gemm_fp8w(const GroupedGemmArgs& a, cudaStream_t st) {
     // per expert); few tokens per expert: narrower double-buffered tiles. The
     // last argument is the MMA-ring depth; the raw ring takes the rest of
     // shared memory (up to 8 slots of two MMA stages each).
-    // Wide gate/up runs the variant with its weight tiles in tensor memory
-    // (192-token tiles, four token slots).
+    // Wide tiles run the variant with the weight tiles in tensor memory
+    // (gate/up: 192-token tiles, down: 224; four token slots).
     const bool wide = a.N >= 128L * a.E;
     if (a.gemm == 1)
-        return wide ? launch_fp8w_gu<192, 4>(a, st) : launch_fp8w<1, 128, 2, 3>(a, st);
-    return wide ? launch_fp8w<2, 240, 2, 3>(a, st) : launch_fp8w<2, 128, 2, 3>(a, st);
+        return wide ? launch_fp8w_ta<1, 192, 4>(a, st) : launch_fp8w<1, 128, 2, 3>(a, st);
+    return wide ? launch_fp8w_ta<2, 224, 4>(a, st) : launch_fp8w_ta<2, 128, 4>(a, st);
 }
 
 }  // namespace gemm

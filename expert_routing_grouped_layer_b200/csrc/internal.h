@@ -59,7 +59,10 @@ cudaError_t launch_pack_rows(int afmt, const void* x, int H, const int32_t* sort
 // f16 expert input rows with per-row power-of-two exponents (FP8-weight layers)
 cudaError_t launch_pack_f16_rows(const void* x, int H, const int32_t* sorted_pair, int N, int k,
                                  int T, int n_rows, void* out, int8_t* xs, cudaStream_t st);
-// true when the gate/up GEMM runs on f16 operands (FP8 weights, bf16 activations)
+// bf16 rows [n_rows][C] -> f16 rows times 2^-e in place, e per row in xs (C % 8 == 0).
+cudaError_t launch_rows_to_f16(void* rows, int C, int n_rows, int8_t* xs, cudaStream_t st);
+// true when the expert GEMMs run on f16 operands (FP8 weights, bf16 activations):
+// token rows and the SwiGLU output travel as f16 rows with per-row exponents
 inline bool f16_gate_up(const moe_config* c) {
     return c->wfmt == MOE_W_FP8_E4M3_B128x128 && c->afmt == MOE_A_BF16;
 }

@@ -204,6 +204,45 @@ __global__ void __launch_bounds__(256) pack_f16_kernel(const uint4* __restrict__
     if (lane == 0) xs[r] = (int8_t)e;
 }
 
+// In place: bf16 rows [n_rows][C] become f16 rows holding the row times 2^-e,
+// e per row in xs, by the rule pack_f16_kernel uses (the row's largest
+// magnitude scaled into [2^13, 2^14); exact for every element within 2^-30 of
+// it). One warp per row; each lane rewrites only the vectors it read.
+__global__ void __launch_bounds__(256) rows_to_f16_kernel(uint4* __restrict__ rows, int C8, int n_rows,
+                                                          int8_t* __restrict__ xs) {
+    const int lane = threadIdx.x & 31;
+    const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (r >= n_rows) return;
+    uint4* row = rows + (size_t)r * C8;
+    uint32_t m = 0;
+    for (int v = lane; v < C8; v += 32) {
+        const uint4 u = row[v];
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) m = max(m, max(w[i] & 0x7FFFu, (w[i] >> 16) & 0x7FFFu));
+    }
+    m = __reduce_max_sync(0xffffffffu, m);
+    int e = 0;
+    if (m != 0) {
+        const int E = ilogbf(__uint_as_float(m << 16));  // floor(log2(amax)), exact
+        e = min(max(E - 13, -127), 114);
+    }
+    const float sc = __uint_as_float((uint32_t)(127 - e) << 23);  // 2^-e, a normal float
+    for (int v = lane; v < C8; v += 32) {
+        const uint4 u = row[v];
+        const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&u);
+        uint4 o;
+        __half2* h = reinterpret_cast<__half2*>(&o);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(b[i]);
+            h[i] = __floats2half2_rn(f.x * sc, f.y * sc);
+        }
+        row[v] = o;
+    }
+    if (lane == 0) xs[r] = (int8_t)e;
+}
+
 // Large batches: one CTA per token, threads striding over the row's 16-byte
 // columns, the k expert rows and S shared rows of a column summed in order.
 __global__ void __launch_bounds__(128) combine_token_kernel(const __nv_bfloat16* __restrict__ y,
@@ -385,6 +424,12 @@ cudaError_t launch_pack_f16_rows(const void* x, int H, const int32_t* sorted_pai
             static_cast<const uint4*>(out), N, H / 8, nullptr, 0, sorted_pair, N, k, T, N,
             static_cast<uint4*>(out), nullptr, xs, xs);
     }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rows_to_f16(void* rows, int C, int n_rows, int8_t* xs, cudaStream_t st) {
+    if (n_rows == 0) return cudaSuccess;
+    rows_to_f16_kernel<<<(n_rows + 7) / 8, 256, 0, st>>>(static_cast<uint4*>(rows), C / 8, n_rows, xs);
     return cudaGetLastError();
 }
 

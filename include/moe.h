@@ -203,10 +203,13 @@ moe_status moe_pack_expert_inputs(const moe_config *cfg, const void *x, int32_t 
  * shared experts in one launch: for every row r of expert e's block
  * [expert_offsets[e], expert_offsets[e+1]) and for the shared rows,
  *   a = SiLU(W1 xa[r]) * (W3 xa[r])   (fp32 accumulation on the tensor cores)
- * written to h as bf16 (BF16 activations) or E4M3 + E8M0 block scales along I
- * (quantised activations). h is [N + S*T][I]: rows 0..N-1 follow xa, rows
- * N + s*T + t belong to shared expert s and token t; h_scale [N + S*T][I/32]
- * (one E8M0 code per 32 features, per-128 codes repeated as for xa_scale).
+ * written to h as bf16 (BF16 activations with BF16 weights), as f16 rows holding
+ * the bf16-rounded row times 2^-e with e in h_scale int8 [N + S*T] (FP8 weights:
+ * the same rule as for xa, the input of the f16 down GEMM), or as E4M3 + E8M0
+ * block scales along I (quantised activations). h is [N + S*T][I]: rows 0..N-1
+ * follow xa, rows N + s*T + t belong to shared expert s and token t; for
+ * quantised activations h_scale is [N + S*T][I/32] (one E8M0 code per 32
+ * features, per-128 codes repeated as for xa_scale).
  * xa / xa_scale as written by moe_pack_expert_inputs for the same config.
  * E2M1 / MXFP4 weights need E4M3 activations and H, I multiples of 512.
  * A pipeline wait past its time limit sets MOE_DEV_TIMEOUT. */
