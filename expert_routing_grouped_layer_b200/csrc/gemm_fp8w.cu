@@ -493,6 +493,74 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
     asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]) : "memory");
 }
 
+// Gate/up epilogue of the f16 path, staged: as epilogue_f16_gate_up, but each
+// 16-token chunk goes as bf16 into the group's shared [16 tokens][128
+// features] tile (two, alternating), the group's four warps meet at an
+// mbarrier, and warp q writes token rows 4q..4q+3 as 256 contiguous bytes
+// each, 16 bytes per lane (scalar 2-byte stores had made the drain of the
+// single accumulator stall the tensor cores).
+template <int ACC_COLS, int GROUPS>
+__device__ __forceinline__ void epilogue_f16_gate_up_staged(
+    const KParams& p, const int* pref, int total, uint32_t tmem_base, uint64_t* tfull,
+    uint64_t* tempty, volatile int* abort_flag, int warp, int lane, int group,
+    const float* __restrict__ scale_routed, const float* __restrict__ scale_shared,
+    const int8_t* __restrict__ row_exp, __nv_bfloat16* buf2, uint64_t* bar2) {
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const int KS = p.K / 128;
+    const int RS = p.a_rows_per_mat / 128;
+    uint32_t acc_phase = 0;
+    int chunk = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+        const Unit t = decode_unit(p, pref, u);
+        const bool routed = t.seg < p.E;
+        const int mat = routed ? t.seg : t.seg - p.E;
+        const float* sbase = (routed ? scale_routed : scale_shared) + (size_t)mat * RS * KS;
+        const float fg = pow2f(tile_exp(sbase + (size_t)t.mt * KS, KS, lane));
+        const float fu = pow2f(tile_exp(sbase + (size_t)(p.a_up_offset / 128 + t.mt) * KS, KS, lane));
+        if (!mbar_wait(&tfull[0], acc_phase, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16);
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(t.out) + t.mt * BM;
+        for (int c0 = 16 * group; c0 < t.n_valid; c0 += 16 * GROUPS, ++chunk) {
+            uint32_t g[16], uu[16];
+            tmem_ld16(taddr + c0, g);
+            tmem_ld16(taddr + ACC_COLS / 2 + c0, uu);
+            // 2^e of this lane's token column (e in [-127, 114]; 2^-127 is subnormal)
+            const int ex_l = (lane < 16 && c0 + lane < t.n_valid) ? row_exp[t.b_row + c0 + lane] : 0;
+            const float fe_l = ex_l >= -126 ? pow2f(ex_l) : __uint_as_float(0x00400000u);
+            tmem_ld_wait(g, uu);
+            __nv_bfloat16* b = buf2 + (chunk & 1) * 16 * BM;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const float fe = __shfl_sync(0xffffffffu, fe_l, j);
+                const float gv = __uint_as_float(g[j]) * fg * fe;  // exact power-of-two factors
+                const float uv = __uint_as_float(uu[j]) * fu * fe;
+                b[j * BM + row] = __float2bfloat16_rn(swiglu(gv, uv, p.swiglu_limit));
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar2[chunk & 1]);
+            if (!mbar_wait(&bar2[chunk & 1], (uint32_t)(chunk >> 1) & 1u, abort_flag)) {
+                ok = false;
+                break;
+            }
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+                const int r = 4 * q + 2 * h2 + (lane >> 4);  // token row of the chunk
+                const int col = (lane & 15) * 8;             // first of 8 features
+                if (c0 + r < t.n_valid)
+                    *reinterpret_cast<uint4*>(out + (size_t)(c0 + r) * p.ld_out + col) =
+                        *reinterpret_cast<const uint4*>(b + r * BM + col);
+            }
+        }
+        if (!ok) break;
+        tc_fence_before();
+        mbar_arrive(&tempty[0]);
+        acc_phase ^= 1;
+    }
+}
+
 template <int GEMM, int BNT_, int MST_>
 struct TileTA {
     static constexpr int NA = (GEMM == 1) ? 2 : 1;
@@ -506,7 +574,10 @@ struct TileTA {
     static constexpr int B_BYTES = BNT * BK * 2;
     static constexpr int MSLOT_BYTES = (B_BYTES + 1023) / 1024 * 1024;
     static constexpr int MSTAGES = MST_;
-    static constexpr int FIXED_BYTES = 1024 + 8 * (2 * 8 + 3 * MSTAGES + 5) + 16 + 4 * (MAX_SEG + 1);
+    // gate/up: each epilogue group stages 16-token chunks of h, [2][16][128] bf16
+    static constexpr int EPI_BYTES = GEMM == 1 ? EG * 2 * 16 * BM * 2 + 128 : 0;
+    static constexpr int FIXED_BYTES =
+        1024 + 8 * (2 * 8 + 3 * MSTAGES + 5 + 2 * EG) + 16 + 4 * (MAX_SEG + 1) + EPI_BYTES;
     static constexpr int RSTAGES_FIT = (232448 - FIXED_BYTES - MSTAGES * MSLOT_BYTES) / RSLOT_BYTES;
     static constexpr int RSTAGES = RSTAGES_FIT < 8 ? RSTAGES_FIT : 8;
     static constexpr int ACC_COLS = NA * BNT;       // gate at 0, up at BNT (gate/up)
@@ -515,8 +586,8 @@ struct TileTA {
     static constexpr int TMEM_COLS = 512;
     static_assert(A_COL + 2 * A_STAGE_COLS <= TMEM_COLS, "tensor memory budget");
     static constexpr int RING_BYTES = MSTAGES * MSLOT_BYTES + RSTAGES * RSLOT_BYTES;
-    static constexpr int BAR_BYTES = 8 * (2 * RSTAGES + 3 * MSTAGES + 5) + 16;
-    static constexpr int SMEM_BYTES = 1024 + RING_BYTES + BAR_BYTES + 4 * (MAX_SEG + 1);
+    static constexpr int BAR_BYTES = 8 * (2 * RSTAGES + 3 * MSTAGES + 5 + 2 * EG) + 16;
+    static constexpr int SMEM_BYTES = 1024 + RING_BYTES + BAR_BYTES + 4 * (MAX_SEG + 1) + EPI_BYTES;
     static_assert(RSTAGES >= 2 && MSTAGES >= 2 && SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -548,9 +619,12 @@ __global__ void __launch_bounds__(TileTA<GEMM, BNT_, MST_>::THREADS, 1)
     uint64_t* tfull = m_empty + C::MSTAGES;
     uint64_t* tempty = tfull + 2;
     uint64_t* mma_done = tempty + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+    uint64_t* ep_bar = mma_done + 1;  // [group][parity]: a gate/up epilogue group's staged chunk
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ep_bar + 2 * C::EG);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* pref = reinterpret_cast<int*>(tmem_slot + 4);
+    __nv_bfloat16* ep_buf = reinterpret_cast<__nv_bfloat16*>(  // [group][2][16][128], 128-byte aligned
+        (reinterpret_cast<uintptr_t>(pref + MAX_SEG + 1) + 127) & ~static_cast<uintptr_t>(127));
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -570,6 +644,7 @@ __global__ void __launch_bounds__(TileTA<GEMM, BNT_, MST_>::THREADS, 1)
             mbar_init(&tempty[a], 128 * C::EG);
         }
         mbar_init(mma_done, 1);
+        for (int i = 0; i < 2 * C::EG; ++i) mbar_init(&ep_bar[i], 4);
         *abort_flag = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tmA_routed);
@@ -695,10 +770,12 @@ __global__ void __launch_bounds__(TileTA<GEMM, BNT_, MST_>::THREADS, 1)
             }
         }
     } else if (warp < 6 || warp >= EPI2_WARP) {
-        if (GEMM == 1)
-            epilogue_f16_gate_up<C::ACC_COLS, 1, C::EG>(p, pref, total, tmem_base, tfull, tempty,
-                                                        abort_flag, warp, lane, warp < 6 ? 0 : 1,
-                                                        scale_routed, scale_shared, row_exp);
+        if (GEMM == 1) {
+            const int grp = warp < 6 ? 0 : 1;
+            epilogue_f16_gate_up_staged<C::ACC_COLS, C::EG>(
+                p, pref, total, tmem_base, tfull, tempty, abort_flag, warp, lane, grp, scale_routed,
+                scale_shared, row_exp, ep_buf + grp * 2 * 16 * BM, ep_bar + 2 * grp);
+        }
         else
             epilogue_f16_down<C::ACC_COLS, C::ACCB>(p, pref, total, tmem_base, tfull, tempty, abort_flag,
                                                     warp, lane, scale_routed, scale_shared, row_exp);

@@ -196,6 +196,63 @@ def test_fp8_weights_extreme_row_magnitudes():
     assert err.max() <= LAYER_TOL["bf16"], (err.max(), int(err.argmax()))
 
 
+def test_fp8_weights_h_rows_are_f16_with_row_exponents():
+    """With FP8 weights the gate/up call leaves h as f16 rows holding the bf16
+    SwiGLU output times 2^-e, e per row in h_scale: the row's largest magnitude
+    lands in [2^13, 2^14), every element within 2^-30 of it converts back to a
+    bf16 value exactly, and the rows match the oracle's SwiGLU output (its
+    expert computation with an identity down projection, E4M3 1.0 on the
+    diagonal with unit block scales) to bf16 rounding plus fp32 summation."""
+    cfg = FP8_TINY.replace(T=80, hidden=512, moe_intermediate_size=256, shared_intermediate_size=256,
+                           n_routed_experts=8, num_experts_per_tok=3, n_shared_experts=1)
+    T, H, I, k, S = cfg.T, cfg.hidden, cfg.moe_intermediate_size, cfg.num_experts_per_tok, 1
+    N = T * k
+    dev = torch.device("cuda")
+    inp = W.make_inputs(cfg, dev)
+    wts = W.make_weights(cfg, dev)
+    r = oracle_route(cfg, inp, T=T)
+    layer = moe.MoELayer(cfg, wts, inp["gate_w"], inp["gate_bias"], max_tokens=T, device=dev)
+    P = lambda which: layer.ws_ptr(T, which)
+    st, ws, ccfg, cw = layer.status, layer.ws, layer.ccfg, layer.cw
+    idx = torch.as_tensor(r["idx"], dtype=torch.int32, device=dev).contiguous()
+    moe.moe_permute(ccfg, idx, T, P(moe.WS_OFFSETS), P(moe.WS_SORTED_PAIR), P(moe.WS_ROW_OF), st,
+                    ws, ws.numel())
+    moe.moe_pack_expert_inputs(ccfg, inp["x"], T, P(moe.WS_SORTED_PAIR), P(moe.WS_XA),
+                               P(moe.WS_XA_SCALE))
+    moe.moe_expert_gate_up(ccfg, P(moe.WS_XA), P(moe.WS_XA_SCALE), T, P(moe.WS_OFFSETS), cw,
+                           P(moe.WS_H), P(moe.WS_H_SCALE), st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    view = lambda which, n, dt: ws[P(which) - ws.data_ptr():][: n * torch.tensor([], dtype=dt).element_size()].view(dt)
+    h = view(moe.WS_H, (N + S * T) * I, torch.float16).view(N + S * T, I).double().cpu().numpy()
+    e = view(moe.WS_H_SCALE, N + S * T, torch.int8).cpu().numpy().astype(np.int64)
+    sp = view(moe.WS_SORTED_PAIR, N, torch.int32).cpu().numpy()
+    rec = h * np.exp2(e)[:, None]
+    # the oracle's SwiGLU rows: identity down projection in the weights' own format
+    w2_id = np.zeros((1, H, I), np.uint8)
+    w2_id[0, np.arange(I), np.arange(I)] = oracle.e4m3_encode(np.ones(1))[0]
+    w2s_id = np.ones((1, H // 128, I // 128), np.float32)
+    xin, _, _ = oracle.expert_input(cfg.afmt, W.bf16_codes(inp["x"]))
+    want = np.zeros_like(rec)
+    for row in range(N + S * T):
+        t, ex = (sp[row] // k, int(r["idx"][sp[row] // k][sp[row] % k])) if row < N else (row - N, None)
+        w13, w13s, _, _ = W.expert_slice(wts, ex) if ex is not None else W.expert_slice(wts, 0, shared=True)
+        want[row] = oracle.expert_rows(cfg.wfmt, cfg.afmt, w13, w13s, w2_id, w2s_id, 0, I, H,
+                                       xin[t:t + 1])[0, :I]
+    for row in range(N + S * T):
+        m = np.abs(rec[row]).max()
+        if m == 0:
+            assert e[row] == 0
+            continue
+        if e[row] > -127:
+            assert 2.0 ** 13 <= np.abs(h[row]).max() < 2.0 ** 14, row
+        big = np.abs(rec[row]) >= m * 2.0 ** -30
+        as_bf16 = torch.tensor(rec[row][big]).to(torch.bfloat16).double().numpy()
+        assert np.array_equal(as_bf16, rec[row][big]), row
+    err = np.linalg.norm(rec - want, axis=1) / np.maximum(np.linalg.norm(want, axis=1), 1e-300)
+    assert err.max() <= 2.0 ** -7, (err.max(), int(err.argmax()))
+
+
 @pytest.mark.parametrize("name", ["bf16", "fp8w", "fp4", "mx"])
 def test_swiglu_limit_every_format(name):
     """swiglu_limit = 0.25, below the typical |g| and |u| of these inputs, so the
