@@ -44,19 +44,22 @@ constexpr int SF_TILE = 128 * SF_KB;  // scale tile: 128 rows x 32 k-blocks
 // tile's epilogue with the next tile's main loop; 1 lets gate/up use
 // 224-token tiles). Warps: 0 TMA, 1 MMA (tile 0), then EG groups of 4
 // epilogue warps (one per TMEM lane quadrant), then the 4 scale warps, then
-// the MMA warp of tile 1. Single-buffered gate/up tiles take three epilogue
-// groups, since there the quantising epilogue is not overlapped with the
-// next tile's main loop.
+// the MMA warp of tile 1. Wide tiles take two epilogue groups on alternating
+// 16-token chunks (the single-buffered gate/up drain is not overlapped with
+// the next tile's main loop).
 template <int GEMM, int NA_, int BNX_, int ACCB_>
 struct TileMX {
     static constexpr int NA = NA_;
-    // epilogue groups: single-buffered gate/up 3; wide double-buffered down 2
-    static constexpr int EG = (GEMM == 1 && ACCB_ == 1) ? 3 : (GEMM == 2 && BNX_ > 128) ? 2 : 1;
+    // epilogue groups: two for the wide tiles (single-buffered gate/up, double-buffered down)
+    static constexpr int EG = (ACCB_ == 1 || BNX_ > 128) ? 2 : 1;
     static constexpr int SCALE_WARP = 2 + 4 * EG;     // first of the 4 scale warps
     static constexpr int MMA2_WARP = SCALE_WARP + 4;  // MMA thread of tile 1 (NA == 2)
     static constexpr int THREADS = 32 * (MMA2_WARP + (NA == 2 ? 1 : 0));
     static constexpr int RED_BYTES = EG * 2 * 4 * 16 * 4;  // [group][parity][warp][16 columns]
-    static constexpr int EPI_BYTES = GEMM == 2 ? EG * 2 * 16 * BM * 2 + 128 : 0;  // down: [group][2][16][128] bf16
+    // staged epilogue chunks, per group and parity: down [16 tokens][128] bf16;
+    // gate/up [16][128] E4M3 bytes, then [16][4] E8M0 codes
+    static constexpr int G1_STAGE = 16 * BM + 16 * 4;
+    static constexpr int EPI_BYTES = (GEMM == 2 ? EG * 2 * 16 * BM * 2 : EG * 2 * G1_STAGE) + 128;
     static constexpr int BNX = BNX_;
     static constexpr int ACCB = ACCB_;
     static constexpr int SFB_ROWS = (BNX + 127) / 128 * 128;  // token rows of the scale tile
@@ -148,7 +151,7 @@ __global__ void __launch_bounds__(TileMX<GEMM, NA_, BNX_, ACCB_>::THREADS, 1)
     uint64_t* sf_full = mma_done + 1;  // [2] scale ring slots
     uint64_t* sf_empty = sf_full + 2;  // [2] released by the 4 scale warps
     uint64_t* red_bar = sf_empty + 2;  // [group][parity]: the amax exchange of a group's 4 warps
-    uint64_t* ep_bar = red_bar + 2 * C::EG;  // [group][parity]: the down epilogue's staged chunk
+    uint64_t* ep_bar = red_bar + 2 * C::EG;  // [group][parity]: an epilogue group's staged chunk
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ep_bar + 2 * C::EG);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* pref = reinterpret_cast<int*>(tmem_slot + 4);
@@ -415,10 +418,16 @@ __global__ void __launch_bounds__(TileMX<GEMM, NA_, BNX_, ACCB_>::THREADS, 1)
         }
     } else {
         // GEMM1 epilogue: SwiGLU, then E4M3 + E8M0 block quantisation along I.
-        // Group grp takes the 16-column chunks grp, grp + EG, ...
+        // Group grp takes the 16-column chunks grp, grp + EG, ... Each chunk's
+        // bytes and codes are staged in shared memory; after the group's four
+        // warps meet, every lane writes one 16-byte piece of a 128-byte token row
+        // (one-byte stores had made the single accumulator's drain stall the
+        // tensor cores), and 16 lanes the rows' four scale codes.
         const int q = warp & 3;
         const int grp = (warp - 2) >> 2;
         const int row = q * 32 + lane;
+        uint8_t* gstage = reinterpret_cast<uint8_t*>(ep_buf) + grp * 2 * C::G1_STAGE;
+        uint64_t* gbar = ep_bar + 2 * grp;
         float* red_g = red + grp * 128;
         uint64_t* red_bar_g = red_bar + 2 * grp;
         int acc = 0;
@@ -430,9 +439,8 @@ __global__ void __launch_bounds__(TileMX<GEMM, NA_, BNX_, ACCB_>::THREADS, 1)
             if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::ACC_COLS;
-            const int feat = t.mt * BM + row;  // output feature (column of h)
-            uint8_t* out = t.out + feat;
-            uint8_t* sc = t.sc + (t.mt * BM + q * 32) / 32;
+            uint8_t* hrow = t.out + t.mt * BM;     // first feature of the tile, row of the first token
+            uint8_t* srow = t.sc + t.mt * BM / 32;  // its four 32-feature codes
             const int ld_sc = p.ld_out / 32;
             for (int c0 = 16 * grp; c0 < t.n_valid; c0 += 16 * C::EG, ++chunk) {
                 uint32_t g[16], uu[16];
@@ -472,15 +480,25 @@ __global__ void __launch_bounds__(TileMX<GEMM, NA_, BNX_, ACCB_>::THREADS, 1)
                         e[j] = pow2_exp448(m);
                     }
                 }
+                uint8_t* b = gstage + (chunk & 1) * C::G1_STAGE;
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
-                    if (c0 + j < t.n_valid) {
-                        const int ej = min(max(e[j], -127), 127);
-                        const float inv = __uint_as_float((uint32_t)(127 - ej) << 23);
-                        out[(size_t)(c0 + j) * p.ld_out] = e4m3_sat(a[j] * inv);
-                        if (lane == 0) sc[(size_t)(c0 + j) * ld_sc] = (uint8_t)(ej + 127);
-                    }
+                    const int ej = min(max(e[j], -127), 127);
+                    const float inv = __uint_as_float((uint32_t)(127 - ej) << 23);
+                    b[j * BM + row] = e4m3_sat(a[j] * inv);
+                    if (lane == 0) b[16 * BM + j * 4 + q] = (uint8_t)(ej + 127);
                 }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&gbar[chunk & 1]);
+                if (!mbar_wait(&gbar[chunk & 1], (uint32_t)(chunk >> 1) & 1u, abort_flag)) { ok = false; break; }
+                const int f = q * 32 + lane;  // 16 token rows x 8 pieces of 16 bytes
+                const int r = f >> 3, pc = f & 7;
+                if (c0 + r < t.n_valid)
+                    *reinterpret_cast<uint4*>(hrow + (size_t)(c0 + r) * p.ld_out + pc * 16) =
+                        *reinterpret_cast<const uint4*>(b + r * BM + pc * 16);
+                if (q == 0 && lane < 16 && c0 + lane < t.n_valid)
+                    *reinterpret_cast<uint32_t*>(srow + (size_t)(c0 + lane) * ld_sc) =
+                        *reinterpret_cast<const uint32_t*>(b + 16 * BM + lane * 4);
             }
             if (!ok) break;
             tc_fence_before();
