@@ -248,21 +248,6 @@ inline bool make_tmap_bf16(CUtensorMap* tm, const void* ptr, uint64_t rows, uint
     return r == CUDA_SUCCESS;
 }
 
-// 2-D row-major uint8 tensor [rows][cols], box = box_rows x 64 bytes, 64B swizzle.
-inline bool make_tmap_u8_sw64(CUtensorMap* tm, const void* ptr, uint64_t rows, uint64_t cols,
-                       uint32_t box_rows) {
-    auto enc = get_encode();
-    if (!enc) return false;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols};
-    cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides,
-                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
 // The four B maps of one row-major tensor [rows][cols] of esize-byte elements,
 // box = box_x elements x (16 << i) rows, 128-byte swizzle.
 inline bool make_bmaps(BMaps* bm, CUtensorMapDataType dtype, int esize, const void* ptr,

@@ -1,6 +1,6 @@
 // sm100.cuh -- thin inline-PTX wrappers for the Blackwell (sm_100a) features
 // the kernels use: mbarriers with bounded waits, TMA tiled loads, tcgen05
-// tensor-memory allocation, MMA issue, commit and loads. Written from the PTX
+// tensor-memory allocation, MMA issue, commit, loads and stores. Written from the PTX
 // ISA's descriptions of these instructions.
 #pragma once
 
@@ -211,14 +211,6 @@ __device__ __forceinline__ void mma_mx(uint32_t d_tmem, uint64_t a_desc, uint64_
         : "memory");
 }
 
-// Shared memory -> tensor memory copy of a 32-row x 16-byte matrix, written to
-// lanes 0..31 of all four lane quadrants: row r's 16 bytes land in lane r (and
-// r+32, r+64, r+96) as 4 consecutive 32-bit columns.
-__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t src_desc) {
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(src_desc)
-                 : "memory");
-}
-
 // Registers -> tensor memory: thread i of the warp writes v to 4 consecutive
 // 32-bit columns of lane (base lane + i). A warp may address only its own lane
 // quadrant (warp index mod 4).
@@ -233,17 +225,6 @@ __device__ __forceinline__ void tmem_st_wait() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-// Matrix descriptor of a K-major, unswizzled operand whose 8-row x 16-byte core
-// matrices are stored back to back (128 bytes apart): the scale-factor tiles.
-__device__ __forceinline__ uint64_t sdesc_kmajor_noswizzle_rows16(uint32_t smem_addr) {
-    uint64_t d = 0;
-    d |= static_cast<uint64_t>((smem_addr & 0x3FFFFu) >> 4);
-    d |= static_cast<uint64_t>(2048 >> 4) << 16;  // leading byte offset (one core matrix along K: unused)
-    d |= static_cast<uint64_t>(128 >> 4) << 32;   // stride byte offset: next 8 rows
-    d |= static_cast<uint64_t>(1) << 46;
-    return d;  // layout type 0: no swizzle
-}
-
 // Instruction descriptor, kind::mxf8f6f4 block-scaled: A E2M1 (format 5), B E4M3
 // (format 0), both K-major, E8M0 scales (bit 23), shape M x N, scale-factor byte
 // selectors for A (bits 29-30) and B (bits 4-5).
@@ -251,10 +232,6 @@ __host__ __device__ __forceinline__ uint32_t idesc_mx_e2m1_e4m3(uint32_t M, uint
                                                               uint32_t a_sf_id, uint32_t b_sf_id) {
     return (b_sf_id << 4) | (5u << 7) | (0u << 10) | ((N >> 3) << 17) | (1u << 23) |
            ((M >> 4) << 24) | (a_sf_id << 29);
-}
-
-__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t threads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
 __device__ __forceinline__ void status_or(int32_t* status, int32_t bits) {
