@@ -37,19 +37,32 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 def launches_per_step(cfg, T, n_sms):
-    """Kernels one layer step launches: router plane split, router GEMM, its
-    split-K reduction when K is split, top-k, 3 permutation kernels, the input
-    pack (quantise + gather for quantised activations with shared experts),
-    gate/up, down, combine. Mirrors the library's router split rule."""
+    """Kernels one layer step launches, mirroring the library's launch rules:
+    router plane split, router GEMM, its split-K reduction when K is split;
+    top-k; the permutation (one kernel up to 4096 pairs, else count, scan and
+    scatter); the expert-input pack (a gather of bf16 rows, or, for quantised
+    activations and for the f16 rows of FP8 weights, the token rows converted
+    once and then gathered); gate/up (FP8 weights: plus the in-place f16 repack
+    of h); down; combine."""
     E, H = cfg.n_routed_experts, cfg.hidden
+    N = T * cfg.num_experts_per_tok
     epad = (E + 127) // 128 * 128
     kb = H // 64
     base = (epad // 128) * ((T + 127) // 128)
     s = max(1, min((n_sms + base - 1) // base, kb // 4))
     kbps = (kb + s - 1) // s
     splits = (kb + kbps - 1) // kbps
-    two_pass = cfg.afmt != "bf16" and cfg.n_shared_experts > 0
-    return 2 + (1 if splits > 1 else 0) + 1 + 3 + (2 if two_pass else 1) + 3
+    router = 2 + (1 if splits > 1 else 0)
+    permute = 1 if N <= 4096 else 3
+    fp8w = cfg.wfmt == "fp8_e4m3_b128x128" and cfg.afmt == "bf16"
+    if fp8w:
+        pack = 2
+    elif cfg.afmt == "bf16":
+        pack = 1
+    else:  # quantise the token rows once, gather when the scale rows are whole 16-byte vectors
+        pack = 2 if (H // 32) % 16 == 0 else 1
+    gate_up = 2 if fp8w else 1
+    return router + 1 + permute + pack + gate_up + 1 + 1
 
 
 def parse():
