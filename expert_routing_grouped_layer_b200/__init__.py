@@ -30,7 +30,7 @@ AFMT = {"bf16": 0, "fp8_e4m3_pow2_b128": 1, "mxfp8": 2}
 EXPORTS = ("moe_workspace_bytes", "moe_gate_topk", "moe_permute", "moe_quantize_activations",
            "moe_pack_expert_inputs", "moe_expert_gate_up", "moe_expert_down",
            "moe_grouped_swiglu", "moe_combine", "moe_layer_forward", "moe_workspace_offset",
-           "moe_status_string", "moe_permute_noalloc")
+           "moe_status_string", "moe_permute_noalloc", "moe_selftest_wait_limit")
 
 # capacity (int32 counts) of the static scratch behind moe_permute_noalloc
 MOE_PERMUTE_NOALLOC_MAX_COUNTS = 262144
@@ -85,6 +85,8 @@ def lib() -> ctypes.CDLL:
             l.moe_workspace_bytes.argtypes = [CP, _I32]
             l.moe_workspace_offset.restype = _SZ
             l.moe_workspace_offset.argtypes = [CP, _I32, _I32]
+            l.moe_selftest_wait_limit.restype = ctypes.c_int
+            l.moe_selftest_wait_limit.argtypes = [_P, _P]
             l.moe_status_string.restype = ctypes.c_char_p
             l.moe_status_string.argtypes = [ctypes.c_int]
             l.moe_gate_topk.restype = ctypes.c_int
@@ -239,6 +241,12 @@ def moe_grouped_swiglu(cfg, x, T, sorted_pair, expert_offsets, weights, y, share
 def moe_combine(cfg, y, shared_y, row_of, topk_w, T, out, stream=None):
     _check(lib().moe_combine(ctypes.byref(_cfg(cfg)), _ptr(y), _ptr(shared_y), _ptr(row_of),
                              _ptr(topk_w), int(T), _ptr(out), _stream(stream)), "moe_combine")
+
+
+def moe_selftest_wait_limit(dev_status, stream=None):
+    """Launch the wait-limit self-test: MOE_DEV_TIMEOUT lands in dev_status
+    (device int32) about 2 s later, and the stream continues normally."""
+    _check(lib().moe_selftest_wait_limit(_ptr(dev_status), _stream(stream)), "moe_selftest_wait_limit")
 
 
 def moe_layer_forward(cfg, x, T, weights, out, ws, dev_status, ws_bytes=None, stream=None):

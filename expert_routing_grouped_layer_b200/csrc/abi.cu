@@ -368,4 +368,9 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* x, int32_t T, co
     return s;
 }
 
+moe_status moe_selftest_wait_limit(int32_t* dev_status, void* stream) {
+    if (!dev_status) return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_wait_limit_selftest(dev_status, as_stream(stream)));
+}
+
 }  // extern "C"

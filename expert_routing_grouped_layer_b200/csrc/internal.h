@@ -68,6 +68,9 @@ inline bool f16_gate_up(const moe_config* c) {
 }
 cudaError_t launch_combine(const void* y, const void* shared_y, int S, const int32_t* row_of,
                            const float* w, int T, int k, int H, void* out, cudaStream_t st);
+// one warp waits on a barrier nothing arrives on until the pipeline wait limit;
+// sets MOE_DEV_TIMEOUT in *status
+cudaError_t launch_wait_limit_selftest(int32_t* status, cudaStream_t st);
 
 struct GroupedGemmArgs {
     // problem

@@ -261,6 +261,14 @@ moe_status moe_layer_forward(const moe_config *cfg, const void *x, int32_t T,
  *  Returns (size_t)-1 for an invalid config or which. */
 size_t moe_workspace_offset(const moe_config *cfg, int32_t T, int32_t which);
 
+/* Self-test of the pipeline waits' time limit: one warp waits, with the same
+ * bounded mbarrier wait every GEMM pipeline uses, on a barrier that nothing
+ * arrives on; once the limit (2 s) has passed it sets MOE_DEV_TIMEOUT in
+ * *dev_status (device int32, OR-ed into) and returns normally, so the context
+ * stays usable. Asynchronous on `stream`. MOE_ERR_INVALID_ARG for a null
+ * dev_status, MOE_ERR_CUDA if the launch fails. */
+moe_status moe_selftest_wait_limit(int32_t *dev_status, void *stream);
+
 /* Human-readable name of a status code (static string). */
 const char *moe_status_string(moe_status s);
 

@@ -2,7 +2,10 @@
 no routing in the loop: the dispatch permutation on both sides of its
 one-chunk path, the weighted combine on both sides of its small-batch path,
 and the f16 expert-input rows that FP8-weight layers feed to the f16
-tensor-core gate/up GEMM."""
+tensor-core gate/up GEMM. Also the pipeline waits' time limit: a wait that
+nothing ends reports a timeout and leaves the context usable."""
+import time
+
 import numpy as np
 import pytest
 import torch
@@ -114,3 +117,31 @@ def test_pack_f16_rows_are_exact():
         big = np.abs(want[r]) >= rmax[r] * 2.0 ** -30
         assert np.array_equal(rec[r][big], want[r][big]), r
         assert np.all(np.abs(rec[r] - want[r]) <= 2.0 ** (e[r] - 25)), r
+
+
+def test_wait_limit_reports_timeout_and_context_stays_usable():
+    """A bounded pipeline wait on a barrier nothing arrives on gives up after its
+    limit (2 s) and reports MOE_DEV_TIMEOUT in the status word, without a trap;
+    the same context then runs a layer that still matches the oracle."""
+    dev = torch.device("cuda")
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    moe.moe_selftest_wait_limit(st)
+    torch.cuda.synchronize()
+    waited = time.perf_counter() - t0
+    assert int(st.item()) & moe.MOE_DEV_TIMEOUT
+    assert 1.5 < waited < 60.0, waited
+    cfg = TINY
+    inp = W.make_inputs(cfg, dev)
+    wts = W.make_weights(cfg, dev)
+    layer = moe.MoELayer(cfg, wts, inp["gate_w"], inp["gate_bias"], max_tokens=cfg.T, device=dev)
+    out = layer.forward(inp["x"])
+    torch.cuda.synchronize()
+    assert int(layer.status.item()) == 0
+    r = oracle.route(cfg, W.bf16_codes(inp["x"]), inp["gate_w"].cpu().numpy(),
+                     inp["gate_bias"].cpu().numpy())
+    want = oracle.layer(cfg, W.bf16_codes(inp["x"]), r["idx"], r["w"],
+                        lambda e: W.expert_slice(wts, e), lambda s: W.expert_slice(wts, s, shared=True))
+    got = out.double().cpu().numpy()
+    assert np.linalg.norm(got - want) / np.linalg.norm(want) <= 1e-2
