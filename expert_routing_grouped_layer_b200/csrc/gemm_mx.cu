@@ -119,6 +119,11 @@ __device__ __forceinline__ uint8_t e4m3_sat(float v) {
     return (uint8_t)(__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3));
 }
 
+// Word w (0..3) of a 16-byte vector.
+__device__ __forceinline__ uint32_t word_of(const uint4& u, int w) {
+    return w == 0 ? u.x : (w == 1 ? u.y : (w == 2 ? u.z : u.w));
+}
+
 // Wait by lane 0 only, the outcome shared with the warp.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int lane) {
     int ok = 1;
@@ -315,8 +320,12 @@ __global__ void __launch_bounds__(TileMX<GEMM, NA_, BNX_, ACCB_>::THREADS, 1)
         // ring slot and stores them to columns 0..3 of the operand in the
         // stage's TMEM set. A set is rewritten only after the MMAs that read it
         // completed (the empty barrier of the stage that last used it). A ring
-        // slot serves eight stages (fewer at the end of a unit), then is released.
+        // slot serves eight stages (fewer at the end of a unit): every four stages
+        // each lane loads the 16 bytes covering them of each of its rows (one
+        // vector load per row instead of one 4-byte load per row per stage), and
+        // the slot is released after the group's last such load.
         const uint32_t lane_cols = tmem_base + ((uint32_t)((warp & 3) * 32) << 16) + C::SF_COL;
+        uint4 cache[C::NOPS][4];  // rows lane + 32 r: 16 bytes, the k-blocks of four stages
         int stage = 0;
         int set = 0;
         int g = 0;  // stages processed
@@ -336,22 +345,27 @@ __global__ void __launch_bounds__(TileMX<GEMM, NA_, BNX_, ACCB_>::THREADS, 1)
                         break;
                     }
                 }
-                const uint8_t* raw = sf_ring + sfs * C::RAW_BYTES;
-                const int j4 = (kb % SF_STAGES) * 4;  // byte offset of this stage's k-blocks in a row
+                if ((kb & 3) == 0) {
+                    // the next four stages' bytes of this lane's four rows, one 16-byte
+                    // load per row; after the group's last such load the slot is free
+                    const uint8_t* raw = sf_ring + sfs * C::RAW_BYTES + 16 * ((kb % SF_STAGES) >> 2);
+#pragma unroll
+                    for (int i = 0; i < C::NOPS; ++i)
+#pragma unroll
+                        for (int r = 0; r < 4; ++r)
+                            cache[i][r] = *reinterpret_cast<const uint4*>(raw + i * SF_TILE + SF_KB * (lane + 32 * r));
+                    if (kb % SF_STAGES == SF_STAGES - 4 || kb + 4 >= KB) {
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&sf_empty[sfs]);
+                        if (++sfs == 2) { sfs = 0; sf_phase ^= 1; }
+                    }
+                }
+                const int w = kb & 3;  // this stage's word: its 4 k-block bytes
                 uint4 v[C::NOPS];
 #pragma unroll
-                for (int i = 0; i < C::NOPS; ++i) {
-                    const uint8_t* src = raw + i * SF_TILE;
-                    v[i].x = *reinterpret_cast<const uint32_t*>(src + SF_KB * (lane + 0) + j4);
-                    v[i].y = *reinterpret_cast<const uint32_t*>(src + SF_KB * (lane + 32) + j4);
-                    v[i].z = *reinterpret_cast<const uint32_t*>(src + SF_KB * (lane + 64) + j4);
-                    v[i].w = *reinterpret_cast<const uint32_t*>(src + SF_KB * (lane + 96) + j4);
-                }
-                if (kb % SF_STAGES == SF_STAGES - 1 || kb == KB - 1) {
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&sf_empty[sfs]);
-                    if (++sfs == 2) { sfs = 0; sf_phase ^= 1; }
-                }
+                for (int i = 0; i < C::NOPS; ++i)
+                    v[i] = make_uint4(word_of(cache[i][0], w), word_of(cache[i][1], w), word_of(cache[i][2], w),
+                                      word_of(cache[i][3], w));
 #pragma unroll
                 for (int i = 0; i < C::NOPS; ++i) tmem_st4(lane_cols + set * C::SET_COLS + 4 * i, v[i]);
                 tmem_st_wait();
