@@ -125,6 +125,24 @@ def test_workspace_grows_with_tokens_and_offsets_fit(lib):
         assert moe.moe_workspace_offset(c, T, 11) == 2 ** 64 - 1
 
 
+def test_fp8_weight_steps_need_h_scale_and_the_workspace_holds_it(lib):
+    """With FP8 weights the gate/up call leaves h as f16 rows with one int8
+    exponent per row in h_scale, which the down call reads: both reject a null
+    h_scale before launching, and the workspace reserves N + S*T bytes for it."""
+    base = W.CONFIGS["tiny_bf16"].replace(wfmt="fp8_e4m3_b128x128")
+    c = moe.make_config(base)
+    w = moe.moe_weights(256, 256, 256, 256, 256, 256, 256, 256, 256, 256)
+    T = 64
+    assert lib.moe_expert_gate_up(ctypes.byref(c), 256, 256, T, 256, ctypes.byref(w), 256, None,
+                                  None, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_expert_down(ctypes.byref(c), 256, None, T, 256, ctypes.byref(w), 256, 256,
+                               None, None) == moe.MOE_ERR_INVALID_ARG
+    N, S = T * base.num_experts_per_tok, base.n_shared_experts
+    total = moe.moe_workspace_bytes(c, T)
+    hs = moe.moe_workspace_offset(c, T, 10)
+    assert hs != 2 ** 64 - 1 and hs + N + S * T <= total
+
+
 def test_status_strings(lib):
     assert moe.lib().moe_status_string(0) == b"ok"
     assert moe.lib().moe_status_string(3) == b"workspace too small"
