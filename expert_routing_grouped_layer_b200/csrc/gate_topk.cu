@@ -20,13 +20,22 @@ namespace moe {
 namespace {
 
 // logits = sum over splits of the partial sums, added in split order; written
-// over split 0 so the selection kernel reads one slab.
+// over split 0 so the selection kernel reads one slab. Eight splits' loads are
+// issued before their adds, which still run in split order.
 __global__ void __launch_bounds__(256) router_reduce_kernel(float* __restrict__ part, long n,
                                                             int splits) {
     const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= n) return;
     float l = 0.f;
-    for (int s = 0; s < splits; ++s) l += part[(size_t)s * n + i];
+    int s = 0;
+    for (; s + 8 <= splits; s += 8) {
+        float v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = part[(size_t)(s + j) * n + i];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) l += v[j];
+    }
+    for (; s < splits; ++s) l += part[(size_t)s * n + i];
     part[i] = l;
 }
 

@@ -142,9 +142,12 @@ __global__ void __launch_bounds__(PERM_WARPS * 32) perm_scatter_kernel(
 }
 
 // All pairs in one chunk (N <= PERM_CHUNK): count, scan and scatter in one CTA,
-// the same per-warp histograms and in-warp ranks as the three launches, so the
-// order is the same. Each lane loads its PERM_PER_WARP / 32 expert ids once, up
-// front (independent loads), and both passes run on the registers.
+// with per-warp histograms and in-warp ranks as in the three launches. The pairs
+// are split evenly over the warps (span pairs each, a multiple of 32, in pair
+// order), so small batches keep every warp busy; any split into contiguous
+// ranges in warp order gives the same stable order. Each lane loads its
+// span / 32 expert ids once, up front (independent loads), and both passes run
+// on the registers.
 __global__ void __launch_bounds__(PERM_WARPS * 32) perm_single_kernel(
     const int32_t* __restrict__ idx, long N, int E, int32_t* __restrict__ offsets,
     int32_t* __restrict__ sorted_pair, int32_t* __restrict__ row_of, int32_t* status) {
@@ -153,18 +156,21 @@ __global__ void __launch_bounds__(PERM_WARPS * 32) perm_single_kernel(
     __shared__ int32_t excl[PERM_MAX_E];
     __shared__ int32_t part[PERM_WARPS * 32];
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-    const long wstart = (long)w * PERM_PER_WARP;
+    const int span = (int)((N + PERM_WARPS * 32 - 1) / (PERM_WARPS * 32)) * 32;  // <= PERM_PER_WARP
+    const int n_it = span / 32;
+    const long wstart = (long)w * span;
     int ev[PER_LANE];  // expert id of pair wstart + 32*i + lane, or -1 past N
 #pragma unroll
     for (int i = 0; i < PER_LANE; ++i) {
         const long p = wstart + 32 * i + lane;
-        ev[i] = p < N ? idx[p] : -1;
+        ev[i] = (i < n_it && p < N) ? idx[p] : -1;
     }
     for (int i = tid; i < PERM_WARPS * E; i += blockDim.x) wbase[i / E][i % E] = 0;
     __syncthreads();
     bool bad = false;
 #pragma unroll
     for (int i = 0; i < PER_LANE; ++i) {
+        if (i >= n_it) break;  // warp-uniform
         const long p = wstart + 32 * i + lane;
         const int e = ev[i];
         const bool ok = p < N && e >= 0 && e < E;
@@ -213,6 +219,7 @@ __global__ void __launch_bounds__(PERM_WARPS * 32) perm_single_kernel(
     const unsigned lt = (1u << lane) - 1u;
 #pragma unroll
     for (int i = 0; i < PER_LANE; ++i) {
+        if (i >= n_it) break;  // warp-uniform
         const long p = wstart + 32 * i + lane;
         const int e = ev[i];
         const bool valid = p < N;

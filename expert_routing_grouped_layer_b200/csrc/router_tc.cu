@@ -64,22 +64,46 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* tmap, in
         : "memory");
 }
 
-// hi / mid / lo bf16 planes of the fp32 router weight, rows padded to Epad with zeros.
-__global__ void __launch_bounds__(256) router_split_kernel(const float* __restrict__ wg,
-                                                           __nv_bfloat16* __restrict__ planes,
-                                                           int E, int Epad, int H) {
-    const long n = (long)Epad * H;
-    for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+// hi / mid / lo bf16 planes of the fp32 router weight, rows padded to Epad with
+// zeros. Eight consecutive weights per thread (H is a multiple of 64, so the eight
+// share a row): two 16-byte loads and one 16-byte store per plane. Element i of
+// [Epad][H] is a real weight exactly when i < E*H, so the padding needs no divide.
+__device__ __forceinline__ uint32_t pack_bf16x2(__nv_bfloat16 a, __nv_bfloat16 b) {
+    return (uint32_t)__bfloat16_as_ushort(a) | ((uint32_t)__bfloat16_as_ushort(b) << 16);
+}
+
+__global__ void __launch_bounds__(256) router_split_kernel(const float4* __restrict__ wg,
+                                                           uint4* __restrict__ planes,
+                                                           long n_valid8, long n8) {
+    for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
          i += (long)gridDim.x * blockDim.x) {
-        const long e = i / H;
-        const float w = e < E ? wg[i] : 0.0f;
-        const __nv_bfloat16 hi = __float2bfloat16_rn(w);
-        const float r1 = w - __bfloat162float(hi);
-        const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
-        const float r2 = r1 - __bfloat162float(mid);
-        planes[i] = hi;
-        planes[n + i] = mid;
-        planes[2 * n + i] = __float2bfloat16_rn(r2);
+        float w[8];
+        if (i < n_valid8) {
+            const float4 a = wg[2 * i], b = wg[2 * i + 1];
+            w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+            w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+        } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) w[j] = 0.0f;
+        }
+        uint32_t hi[4], mid[4], lo[4];
+#pragma unroll
+        for (int j = 0; j < 8; j += 2) {
+            __nv_bfloat16 h[2], m[2], l[2];
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                h[q] = __float2bfloat16_rn(w[j + q]);
+                const float r1 = w[j + q] - __bfloat162float(h[q]);
+                m[q] = __float2bfloat16_rn(r1);
+                l[q] = __float2bfloat16_rn(r1 - __bfloat162float(m[q]));
+            }
+            hi[j / 2] = pack_bf16x2(h[0], h[1]);
+            mid[j / 2] = pack_bf16x2(m[0], m[1]);
+            lo[j / 2] = pack_bf16x2(l[0], l[1]);
+        }
+        planes[i] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        planes[n8 + i] = make_uint4(mid[0], mid[1], mid[2], mid[3]);
+        planes[2 * n8 + i] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
     }
 }
 
@@ -270,8 +294,9 @@ cudaError_t launch_router_tc(const void* x, const float* gate_w, void* planes, f
     if (attr_err != cudaSuccess) return attr_err;
     const RouterPlan plan = router_plan(T, E, H);
     const long n = (long)plan.Epad * H;
-    router_split_kernel<<<(unsigned)std::min<long>((n + 255) / 256, 4L * num_sms()), 256, 0, st>>>(
-        gate_w, static_cast<__nv_bfloat16*>(planes), E, plan.Epad, H);
+    const long n8 = n / 8;
+    router_split_kernel<<<(unsigned)std::min<long>((n8 + 255) / 256, 8L * num_sms()), 256, 0, st>>>(
+        reinterpret_cast<const float4*>(gate_w), static_cast<uint4*>(planes), (long)E * H / 8, n8);
     CUtensorMap tmW;
     BMaps tmX;
     if (!make_tmap_planes(&tmW, planes, plan.Epad, H) ||
