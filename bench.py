@@ -7,7 +7,10 @@
 A step is one pass of the whole layer (router + top-k, dispatch permutation,
 expert input gather, gate/up + SwiGLU, down projection, combine) over one
 batch of the workload's tokens, run through the library's C ABI. Inputs are
-resident in HBM when the timed region starts. Multi-GPU runs are replicas
+resident in HBM when the timed region starts. The timed steps are whole-layer
+calls (``moe_layer_forward``), so the layer's kernels follow one another with
+programmatic dependent launch; the per-stage split comes from a separate pass
+of the staged entry points with CUDA events between them. Multi-GPU runs are replicas
 (weak scaling): every rank holds all experts and runs its own batch; there is
 no data-path collective, only a barrier and a max over ranks of the timing.
 
@@ -334,7 +337,8 @@ def run_ours(args, rank, world, dev):
     assert torch.equal(ref.view(torch.int16), out.view(torch.int16)), "staged != layer forward"
     assert st.item() == 0, "device status %d" % st.item()
 
-    events = [mk() for _ in range(args.steps)]
+    events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
     di = dev.index if dev.index is not None else 0
     clocks = ClockSampler(di, enabled=not args.no_clocks,
                           log_path=clock_log_path(args.clock_log, di))
@@ -342,19 +346,30 @@ def run_ours(args, rank, world, dev):
         torch.distributed.barrier()
     torch.cuda.synchronize()
     t_wall = time.perf_counter()
-    for i in range(args.steps):
+    for e0, e1 in events:
         flush.zero_()  # L2 flush outside the timed events
-        step(events[i])
+        e0.record(stream)
+        layer.forward(x, out=out, stream=sp)
+        e1.record(stream)
     torch.cuda.synchronize()
     wall = time.perf_counter() - t_wall
     if world > 1:
         torch.distributed.barrier()
     clk = clocks.stop()
-
-    stage = [[events[i][j].elapsed_time(events[i][j + 1]) for i in range(args.steps)]
-             for j in range(6)]
-    step_ms = [sum(stage[j][i] for j in range(6)) for i in range(args.steps)]
+    step_ms = [e0.elapsed_time(e1) for e0, e1 in events]
     total_ms = max_over_ranks(sum(step_ms), dev)
+    assert torch.equal(ref.view(torch.int16), out.view(torch.int16)), "timed steps changed output"
+
+    # per-stage split: the staged entry points with events between them (not
+    # part of the timed steps above)
+    n_stage = max(1, min(args.steps, 100))
+    sevents = [mk() for _ in range(n_stage)]
+    for i in range(n_stage):
+        flush.zero_()
+        step(sevents[i])
+    torch.cuda.synchronize()
+    stage = [[sevents[i][j].elapsed_time(sevents[i][j + 1]) for i in range(n_stage)]
+             for j in range(6)]
     offsets = layer.intermediate(T, moe.WS_OFFSETS, torch.int32, (E + 1,)).cpu()
     active = int((offsets[1:] - offsets[:-1] > 0).sum())
 
@@ -438,6 +453,8 @@ def run_ours(args, rank, world, dev):
         "roofline": kroof,
         "layer_roofline": lroof,
         "stage_ms": stage_ms,
+        "stage_ms_source": "staged entry points with events between them, %d separate steps"
+                           % n_stage,
         "gpu_launches": launches_per_step(cfg, T, torch.cuda.get_device_properties(dev).multi_processor_count) * args.steps,
         "wall_s_timed_loop": wall,
         "clocks": clk,

@@ -24,6 +24,8 @@ namespace {
 // issued before their adds, which still run in split order.
 __global__ void __launch_bounds__(256) router_reduce_kernel(float* __restrict__ part, long n,
                                                             int splits) {
+    pdl_wait();
+    pdl_trigger();
     const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= n) return;
     float l = 0.f;
@@ -61,6 +63,8 @@ struct TopkParams {
 // One warp per token. Lane l holds experts e = l + 32*j, j < MAXJ.
 template <int MAXJ>
 __global__ void __launch_bounds__(256) topk_kernel(TopkParams p) {
+    pdl_wait();
+    pdl_trigger();
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (t >= p.T) return;
@@ -207,7 +211,7 @@ __global__ void __launch_bounds__(256) topk_kernel(TopkParams p) {
 }  // namespace
 
 cudaError_t launch_router_reduce(float* part, long n, int splits, cudaStream_t st) {
-    router_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(part, n, splits);
+    launch_pdl(router_reduce_kernel, (unsigned)((n + 255) / 256), 256, 0, st, part, n, splits);
     return cudaGetLastError();
 }
 
@@ -229,10 +233,10 @@ cudaError_t launch_topk(const moe_config* c, const float* part, const float* bia
     p.w = w;
     const int warps = 8;
     dim3 grid((T + warps - 1) / warps);
-    if (p.E <= 32) topk_kernel<1><<<grid, warps * 32, 0, st>>>(p);
-    else if (p.E <= 128) topk_kernel<4><<<grid, warps * 32, 0, st>>>(p);
-    else if (p.E <= 512) topk_kernel<16><<<grid, warps * 32, 0, st>>>(p);
-    else topk_kernel<32><<<grid, warps * 32, 0, st>>>(p);
+    if (p.E <= 32) launch_pdl(topk_kernel<1>, grid, warps * 32, 0, st, p);
+    else if (p.E <= 128) launch_pdl(topk_kernel<4>, grid, warps * 32, 0, st, p);
+    else if (p.E <= 512) launch_pdl(topk_kernel<16>, grid, warps * 32, 0, st, p);
+    else launch_pdl(topk_kernel<32>, grid, warps * 32, 0, st, p);
     return cudaGetLastError();
 }
 

@@ -34,6 +34,8 @@ __global__ void __launch_bounds__(192, 1)
     grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA_routed,
                              const __grid_constant__ CUtensorMap tmA_shared,
                              const __grid_constant__ CUtensorMap tmB, const KParams p) {
+    pdl_wait();
+    pdl_trigger();
     using C = Tile<GEMM>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -200,7 +202,7 @@ cudaError_t launch_bf16(const GroupedGemmArgs& a, cudaStream_t st) {
     if (b_rows == 0) return cudaSuccess;
     if (!make_tmap_bf16(&tmB, a.b_rows, b_rows, p.K, B_BOX)) return cudaErrorInvalidValue;
     const int grid = grid_for(p);
-    grouped_gemm_bf16_kernel<GEMM><<<grid, 192, C::SMEM_BYTES, st>>>(tmAr, tmAs, tmB, p);
+    launch_pdl(grouped_gemm_bf16_kernel<GEMM>, grid, 192, C::SMEM_BYTES, st, tmAr, tmAs, tmB, p);
     return cudaGetLastError();
 }
 

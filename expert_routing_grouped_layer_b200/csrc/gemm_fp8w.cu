@@ -225,6 +225,8 @@ __global__ void __launch_bounds__(TileF8<GEMM, BNF_, ACCB_, MST_>::THREADS, 1)
                              const float* __restrict__ scale_routed,
                              const float* __restrict__ scale_shared,
                              const int8_t* __restrict__ row_exp) {
+    pdl_wait();
+    pdl_trigger();
     using C = TileF8<GEMM, BNF_, ACCB_, MST_>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -605,6 +607,8 @@ __global__ void __launch_bounds__(TileTA<GEMM, BNT_, MST_>::THREADS, 1)
                                 const float* __restrict__ scale_routed,
                                 const float* __restrict__ scale_shared,
                                 const int8_t* __restrict__ row_exp) {
+    pdl_wait();
+    pdl_trigger();
     using C = TileTA<GEMM, BNT_, MST_>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -896,10 +900,9 @@ cudaError_t launch_fp8w(const GroupedGemmArgs& a, cudaStream_t st) {
     // f16 token rows (x * 2^-e)
     if (!make_bmaps(&tmB, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.b_rows, b_rows, p.K, BK))
         return cudaErrorInvalidValue;
-    grouped_gemm_fp8w_kernel<GEMM, BNF_, ACCB_, MST_><<<grid_for(p), C::THREADS, C::SMEM_BYTES, st>>>(
-        tmAr, tmAs, tmB, p, static_cast<const float*>(a.w_routed_scale),
-        static_cast<const float*>(S > 0 ? a.w_shared_scale : a.w_routed_scale),
-        reinterpret_cast<const int8_t*>(a.b_scale));
+    launch_pdl(grouped_gemm_fp8w_kernel<GEMM, BNF_, ACCB_, MST_>, grid_for(p), C::THREADS,
+        C::SMEM_BYTES, st, tmAr, tmAs, tmB, p, static_cast<const float*>(a.w_routed_scale),
+        static_cast<const float*>(S > 0 ? a.w_shared_scale : a.w_routed_scale), reinterpret_cast<const int8_t*>(a.b_scale));
     return cudaGetLastError();
 }
 
@@ -929,10 +932,9 @@ cudaError_t launch_fp8w_ta(const GroupedGemmArgs& a, cudaStream_t st) {
     // f16 rows: token rows x * 2^-e (gate/up), SwiGLU output rows h * 2^-e (down)
     if (!make_bmaps(&tmB, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.b_rows, b_rows, p.K, BK))
         return cudaErrorInvalidValue;
-    grouped_gemm_fp8w_ta_kernel<GEMM, BNT_, MST_><<<grid_for(p), C::THREADS, C::SMEM_BYTES, st>>>(
-        tmAr, tmAs, tmB, p, static_cast<const float*>(a.w_routed_scale),
-        static_cast<const float*>(S > 0 ? a.w_shared_scale : a.w_routed_scale),
-        reinterpret_cast<const int8_t*>(a.b_scale));
+    launch_pdl(grouped_gemm_fp8w_ta_kernel<GEMM, BNT_, MST_>, grid_for(p), C::THREADS,
+        C::SMEM_BYTES, st, tmAr, tmAs, tmB, p, static_cast<const float*>(a.w_routed_scale),
+        static_cast<const float*>(S > 0 ? a.w_shared_scale : a.w_routed_scale), reinterpret_cast<const int8_t*>(a.b_scale));
     return cudaGetLastError();
 }
 

@@ -142,6 +142,8 @@ __global__ void __launch_bounds__(TileMX<GEMM, NA_, BNX_, ACCB_>::THREADS, 1)
                            const __grid_constant__ CUtensorMap tmSFA_shared,
                            const __grid_constant__ BMaps tmB,
                            const __grid_constant__ CUtensorMap tmSFB, const KParams p) {
+    pdl_wait();
+    pdl_trigger();
     using C = TileMX<GEMM, NA_, BNX_, ACCB_>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -577,8 +579,8 @@ cudaError_t launch_mx(const GroupedGemmArgs& a, cudaStream_t st) {
         !make_tmap_2d(&tmSFB, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.b_scale, b_rows, K / 32, K / 32, SF_KB,
                       C::SFB_ROWS, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    grouped_gemm_mx_kernel<GEMM, AFMT, NA_, BNX_, ACCB_><<<grid_for(p), C::THREADS, C::SMEM_BYTES, st>>>(
-        tmA, tmAs, tmSFA, tmSFAs, tmB, tmSFB, p);
+    launch_pdl(grouped_gemm_mx_kernel<GEMM, AFMT, NA_, BNX_, ACCB_>, grid_for(p), C::THREADS,
+        C::SMEM_BYTES, st, tmA, tmAs, tmSFA, tmSFAs, tmB, tmSFB, p);
     return cudaGetLastError();
 }
 

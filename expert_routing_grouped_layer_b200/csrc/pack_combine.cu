@@ -54,6 +54,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(
     const uint4* src, int src_row0, int row16, const uint4* ssrc, int srow16,
     const int32_t* __restrict__ sorted_pair, int N, int k, int T, int n_rows, uint4* dst,
     uint4* sdst, const int8_t* esrc, int8_t* edst) {
+    pdl_wait();
+    pdl_trigger();
     const int lane = threadIdx.x & 31;
     const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
     if (r >= n_rows) return;
@@ -118,6 +120,8 @@ __global__ void __launch_bounds__(256) pack_fp8_kernel(const __nv_bfloat16* __re
                                                        uint8_t* __restrict__ out,
                                                        uint8_t* __restrict__ out_scale, int per32,
                                                        int row0) {
+    pdl_wait();
+    pdl_trigger();
     constexpr int BLK = (AFMT == MOE_A_FP8_E4M3_POW2_B128) ? 128 : 32;
     const int SBLK = per32 ? 32 : BLK;  // elements per stored scale
     const int lane = threadIdx.x & 31;
@@ -163,6 +167,8 @@ __global__ void __launch_bounds__(256) pack_f16_kernel(const uint4* __restrict__
                                                        int N, int k, int T, int n_rows, int row0,
                                                        uint4* __restrict__ out,
                                                        int8_t* __restrict__ xs) {
+    pdl_wait();
+    pdl_trigger();
     const int lane = threadIdx.x & 31;
     const int r = row0 + blockIdx.x * 8 + (threadIdx.x >> 5);
     if (r >= n_rows) return;
@@ -210,6 +216,8 @@ __global__ void __launch_bounds__(256) pack_f16_kernel(const uint4* __restrict__
 // it). One warp per row; each lane rewrites only the vectors it read.
 __global__ void __launch_bounds__(256) rows_to_f16_kernel(uint4* __restrict__ rows, int C8, int n_rows,
                                                           int8_t* __restrict__ xs) {
+    pdl_wait();
+    pdl_trigger();
     const int lane = threadIdx.x & 31;
     const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
     if (r >= n_rows) return;
@@ -250,6 +258,8 @@ __global__ void __launch_bounds__(128) combine_token_kernel(const __nv_bfloat16*
                                                       int S, const int32_t* __restrict__ row_of,
                                                       const float* __restrict__ w, int T, int k,
                                                       int H, __nv_bfloat16* __restrict__ out) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ int32_t rows[32];
     __shared__ float wts[32];
     const int t = blockIdx.x;
@@ -305,6 +315,8 @@ __global__ void __launch_bounds__(128) combine_kernel(const __nv_bfloat16* __res
                                                       int S, const int32_t* __restrict__ row_of,
                                                       const float* __restrict__ w, int T, int k,
                                                       int H, __nv_bfloat16* __restrict__ out) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ int32_t rows[32];
     __shared__ float wts[32];
     // column blocks of one token are consecutive CTAs, so each token's rows are
@@ -372,9 +384,9 @@ cudaError_t launch_pack_rows(int afmt, const void* x, int H, const int32_t* sort
                              cudaStream_t st) {
     if (n_rows == 0) return cudaSuccess;
     if (afmt == MOE_A_BF16) {
-        gather_rows_kernel<<<(n_rows + 7) / 8, 256, 0, st>>>(
-            static_cast<const uint4*>(x), 0, H / 8, nullptr, 0, sorted_pair, N, k, T, n_rows,
-            static_cast<uint4*>(out), nullptr, nullptr, nullptr);
+        launch_pdl(gather_rows_kernel, (n_rows + 7) / 8, 256, 0, st, static_cast<const uint4*>(x),
+            0, H / 8, nullptr, 0, sorted_pair, N, k, T, n_rows, static_cast<uint4*>(out), nullptr,
+            nullptr, nullptr);
         return cudaGetLastError();
     }
     const int blk = (afmt == MOE_A_FP8_E4M3_POW2_B128) ? 128 : 32;
@@ -389,21 +401,19 @@ cudaError_t launch_pack_rows(int afmt, const void* x, int H, const int32_t* sort
     const int q_rows = n_rows - row0;
     dim3 grid((q_rows + 7) / 8);
     if (afmt == MOE_A_FP8_E4M3_POW2_B128)
-        pack_fp8_kernel<MOE_A_FP8_E4M3_POW2_B128><<<grid, 256, 0, st>>>(
+        launch_pdl(pack_fp8_kernel<MOE_A_FP8_E4M3_POW2_B128>, grid, 256, 0, st,
             static_cast<const __nv_bfloat16*>(x), H, sorted_pair, N, k, T, n_rows,
             static_cast<uint8_t*>(out), out_scale, per32, row0);
     else
-        pack_fp8_kernel<MOE_A_MXFP8><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), H,
-                                                           sorted_pair, N, k, T, n_rows,
-                                                           static_cast<uint8_t*>(out), out_scale,
-                                                           per32, row0);
+        launch_pdl(pack_fp8_kernel<MOE_A_MXFP8>, grid, 256, 0, st,
+            static_cast<const __nv_bfloat16*>(x), H, sorted_pair, N, k, T, n_rows,
+            static_cast<uint8_t*>(out), out_scale, per32, row0);
     if (two_pass && N > 0) {
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
-        gather_rows_kernel<<<(N + 7) / 8, 256, 0, st>>>(
-            static_cast<const uint4*>(out), N, H / 16, reinterpret_cast<const uint4*>(out_scale),
-            sbytes / 16, sorted_pair, N, k, T, N, static_cast<uint4*>(out),
-            reinterpret_cast<uint4*>(out_scale), nullptr, nullptr);
+        launch_pdl(gather_rows_kernel, (N + 7) / 8, 256, 0, st, static_cast<const uint4*>(out), N,
+            H / 16, reinterpret_cast<const uint4*>(out_scale), sbytes / 16, sorted_pair, N, k, T, N,
+            static_cast<uint4*>(out), reinterpret_cast<uint4*>(out_scale), nullptr, nullptr);
     }
     return cudaGetLastError();
 }
@@ -414,22 +424,21 @@ cudaError_t launch_pack_f16_rows(const void* x, int H, const int32_t* sorted_pai
     // with shared-expert rows, convert the T token rows once and gather the rest
     const bool two_pass = n_rows == N + T && T > 0;
     const int row0 = two_pass ? N : 0;
-    pack_f16_kernel<<<(n_rows - row0 + 7) / 8, 256, 0, st>>>(static_cast<const uint4*>(x), H / 8,
-                                                            sorted_pair, N, k, T, n_rows, row0,
-                                                            static_cast<uint4*>(out), xs);
+    launch_pdl(pack_f16_kernel, (n_rows - row0 + 7) / 8, 256, 0, st, static_cast<const uint4*>(x),
+        H / 8, sorted_pair, N, k, T, n_rows, row0, static_cast<uint4*>(out), xs);
     if (two_pass && N > 0) {
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
-        gather_rows_kernel<<<(N + 7) / 8, 256, 0, st>>>(
-            static_cast<const uint4*>(out), N, H / 8, nullptr, 0, sorted_pair, N, k, T, N,
-            static_cast<uint4*>(out), nullptr, xs, xs);
+        launch_pdl(gather_rows_kernel, (N + 7) / 8, 256, 0, st, static_cast<const uint4*>(out), N,
+            H / 8, nullptr, 0, sorted_pair, N, k, T, N, static_cast<uint4*>(out), nullptr, xs, xs);
     }
     return cudaGetLastError();
 }
 
 cudaError_t launch_rows_to_f16(void* rows, int C, int n_rows, int8_t* xs, cudaStream_t st) {
     if (n_rows == 0) return cudaSuccess;
-    rows_to_f16_kernel<<<(n_rows + 7) / 8, 256, 0, st>>>(static_cast<uint4*>(rows), C / 8, n_rows, xs);
+    launch_pdl(rows_to_f16_kernel, (n_rows + 7) / 8, 256, 0, st, static_cast<uint4*>(rows), C / 8,
+        n_rows, xs);
     return cudaGetLastError();
 }
 
@@ -443,15 +452,15 @@ cudaError_t launch_combine(const void* y, const void* shared_y, int S, const int
     // enough tokens to fill the GPU with one CTA each (the column-split CTAs
     // are latency-bound: measured slower at 16384 tokens, faster at 128)
     if (T >= 8 * num_sms()) {
-        combine_token_kernel<<<T, 128, 0, st>>>(yy, sy, S, row_of, w, T, k, H, o);
+        launch_pdl(combine_token_kernel, T, 128, 0, st, yy, sy, S, row_of, w, T, k, H, o);
         return cudaGetLastError();
     }
     if (k + S <= 12)
-        combine_kernel<12><<<grid, 128, 0, st>>>(yy, sy, S, row_of, w, T, k, H, o);
+        launch_pdl(combine_kernel<12>, grid, 128, 0, st, yy, sy, S, row_of, w, T, k, H, o);
     else if (k + S <= 20)
-        combine_kernel<20><<<grid, 128, 0, st>>>(yy, sy, S, row_of, w, T, k, H, o);
+        launch_pdl(combine_kernel<20>, grid, 128, 0, st, yy, sy, S, row_of, w, T, k, H, o);
     else
-        combine_kernel<36><<<grid, 128, 0, st>>>(yy, sy, S, row_of, w, T, k, H, o);
+        launch_pdl(combine_kernel<36>, grid, 128, 0, st, yy, sy, S, row_of, w, T, k, H, o);
     return cudaGetLastError();
 }
 

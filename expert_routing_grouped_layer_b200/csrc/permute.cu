@@ -29,6 +29,8 @@ constexpr int PERM_MAX_E = 1024;
 __global__ void __launch_bounds__(256) perm_count_kernel(const int32_t* __restrict__ idx, long N,
                                                          int E, int32_t* __restrict__ chunk,
                                                          int32_t* status) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ int32_t cnt[PERM_MAX_E];
     for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
     __syncthreads();
@@ -49,6 +51,8 @@ __global__ void __launch_bounds__(256) perm_count_kernel(const int32_t* __restri
 // Single CTA of 1024 threads; thread e owns expert e.
 __global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t* __restrict__ chunk, int n_chunks,
                                                          int E, int32_t* __restrict__ offsets) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ int32_t warp_sums[32];
     const int e = threadIdx.x;
     int total = 0;
@@ -90,6 +94,8 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t* __restrict__ c
 __global__ void __launch_bounds__(PERM_WARPS * 32) perm_scatter_kernel(
     const int32_t* __restrict__ idx, long N, int E, const int32_t* __restrict__ chunk,
     int32_t* __restrict__ sorted_pair, int32_t* __restrict__ row_of) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ int32_t wbase[PERM_WARPS][PERM_MAX_E];
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     for (int i = threadIdx.x; i < PERM_WARPS * E; i += blockDim.x) wbase[i / E][i % E] = 0;
@@ -151,6 +157,8 @@ __global__ void __launch_bounds__(PERM_WARPS * 32) perm_scatter_kernel(
 __global__ void __launch_bounds__(PERM_WARPS * 32) perm_single_kernel(
     const int32_t* __restrict__ idx, long N, int E, int32_t* __restrict__ offsets,
     int32_t* __restrict__ sorted_pair, int32_t* __restrict__ row_of, int32_t* status) {
+    pdl_wait();
+    pdl_trigger();
     constexpr int PER_LANE = PERM_PER_WARP / 32;
     __shared__ int32_t wbase[PERM_WARPS][PERM_MAX_E];
     __shared__ int32_t excl[PERM_MAX_E];
@@ -248,13 +256,14 @@ cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int n_chunks
                            int32_t* status, cudaStream_t st) {
     const long N = (long)T * k;
     if (n_chunks <= 1) {
-        perm_single_kernel<<<1, PERM_WARPS * 32, 0, st>>>(idx, N, E, offsets, sorted_pair, row_of,
-                                                          status);
+        launch_pdl(perm_single_kernel, 1, PERM_WARPS * 32, 0, st, idx, N, E, offsets, sorted_pair,
+            row_of, status);
         return cudaGetLastError();
     }
-    perm_count_kernel<<<n_chunks, 256, 0, st>>>(idx, N, E, chunk, status);
-    perm_scan_kernel<<<1, 1024, 0, st>>>(chunk, n_chunks, E, offsets);
-    perm_scatter_kernel<<<n_chunks, PERM_WARPS * 32, 0, st>>>(idx, N, E, chunk, sorted_pair, row_of);
+    launch_pdl(perm_count_kernel, n_chunks, 256, 0, st, idx, N, E, chunk, status);
+    launch_pdl(perm_scan_kernel, 1, 1024, 0, st, chunk, n_chunks, E, offsets);
+    launch_pdl(perm_scatter_kernel, n_chunks, PERM_WARPS * 32, 0, st, idx, N, E, chunk, sorted_pair,
+        row_of);
     return cudaGetLastError();
 }
 

@@ -75,6 +75,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(__nv_bfloat16 a, __nv_bfloat16 b
 __global__ void __launch_bounds__(256) router_split_kernel(const float4* __restrict__ wg,
                                                            uint4* __restrict__ planes,
                                                            long n_valid8, long n8) {
+    pdl_wait();
+    pdl_trigger();
     for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
          i += (long)gridDim.x * blockDim.x) {
         float w[8];
@@ -110,6 +112,8 @@ __global__ void __launch_bounds__(256) router_split_kernel(const float4* __restr
 __global__ void __launch_bounds__(192, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ BMaps tmX,
                      const RouterParams p) {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -295,8 +299,9 @@ cudaError_t launch_router_tc(const void* x, const float* gate_w, void* planes, f
     const RouterPlan plan = router_plan(T, E, H);
     const long n = (long)plan.Epad * H;
     const long n8 = n / 8;
-    router_split_kernel<<<(unsigned)std::min<long>((n8 + 255) / 256, 8L * num_sms()), 256, 0, st>>>(
-        reinterpret_cast<const float4*>(gate_w), static_cast<uint4*>(planes), (long)E * H / 8, n8);
+    launch_pdl(router_split_kernel, (unsigned)std::min<long>((n8 + 255) / 256, 8L * num_sms()), 256,
+        0, st, reinterpret_cast<const float4*>(gate_w), static_cast<uint4*>(planes),
+        (long)E * H / 8, n8);
     CUtensorMap tmW;
     BMaps tmX;
     if (!make_tmap_planes(&tmW, planes, plan.Epad, H) ||
@@ -314,7 +319,7 @@ cudaError_t launch_router_tc(const void* x, const float* gate_w, void* planes, f
     p.part = part;
     p.status = status;
     const int units = p.mtiles * p.ntiles * p.ksplit;
-    router_tc_kernel<<<std::min(units, num_sms()), 192, RT_SMEM_BYTES, st>>>(tmW, tmX, p);
+    launch_pdl(router_tc_kernel, std::min(units, num_sms()), 192, RT_SMEM_BYTES, st, tmW, tmX, p);
     cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess && plan.splits > 1) e = launch_router_reduce(part, (long)T * E, plan.splits, st);
     return e;

@@ -1,7 +1,7 @@
 // sm100.cuh -- thin inline-PTX wrappers for the Blackwell (sm_100a) features
 // the kernels use: mbarriers with bounded waits, TMA tiled loads, tcgen05
-// tensor-memory allocation, MMA issue, commit, loads and stores. Written from the PTX
-// ISA's descriptions of these instructions.
+// tensor-memory allocation, MMA issue, commit, loads and stores, and programmatic
+// dependent launch. Written from the PTX ISA's descriptions of these instructions.
 #pragma once
 
 #include <cstdint>
@@ -10,6 +10,37 @@
 #include "moe.h"
 
 namespace moe {
+
+// ------------------------------------------------------------------ launches
+// Programmatic dependent launch. A kernel started by launch_pdl may begin while
+// the previous kernel in the stream is still running; pdl_wait() returns once
+// that kernel has completed and its memory writes are visible. Every kernel of
+// the layer calls pdl_wait() before its first global-memory access, read or
+// write, so the order of memory effects is that of plain stream order and only
+// the launch itself overlaps. pdl_trigger() lets the next kernel be scheduled
+// once every CTA of this grid has called it. Both are no-ops in a grid launched
+// without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
 
 // ------------------------------------------------------------------ timers
 __device__ __forceinline__ uint64_t globaltimer_ns() {
