@@ -23,6 +23,12 @@
  *    the SM count and the set of kernels whose shared-memory limit was raised.
  *  - `stream` is a cudaStream_t (NULL = legacy default stream). All work is
  *    enqueued on it in order; outputs are valid once the stream reaches them.
+ *    Kernels are launched with programmatic stream serialization: one may be
+ *    scheduled while the kernel before it on the stream is finishing, but it
+ *    waits on the device for that kernel to complete (and its writes to become
+ *    visible) before touching memory, so the ordering is that of the stream.
+ *  - The shared-memory limit of a kernel is raised once per process, on the
+ *    device current at the first call: drive one GPU per process.
  *  - Arguments are checked on the host before anything is launched; a bad
  *    argument returns MOE_ERR_INVALID_ARG (or MOE_ERR_UNSUPPORTED for a valid
  *    but unimplemented combination, MOE_ERR_WORKSPACE for a short workspace)
