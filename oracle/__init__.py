@@ -14,8 +14,11 @@ itself; see ``tests/test_oracle_*.py``): format decoders/encoders, the activatio
 quantisers, scoring, routing (brute force, library top-k, invariants), the
 permutation (library stable argsort, bijection), one expert's SwiGLU (one-hot
 closed forms, zero gate, linearity) and the combine (identical-expert identity).
-The composed layer output has no worked example on the pages: its parity rests
-on the pinned parts ("parity unpinned" beyond their composition).
+The composed layer output has no worked example on the pages. It is pinned by
+properties its definition fixes for any weights (each token's output depends on
+that token alone; relabelling the experts changes nothing; the routed part
+scales exactly with routed_scaling_factor; a common bias shift changes nothing),
+with planted index mistakes shown to break them.
 """
 from __future__ import annotations
 
