@@ -27,6 +27,10 @@
  *    scheduled while the kernel before it on the stream is finishing, but it
  *    waits on the device for that kernel to complete (and its writes to become
  *    visible) before touching memory, so the ordering is that of the stream.
+ *    Each kernel signals its dependents as it starts: a caller's kernel launched
+ *    next on the same stream WITH programmatic serialization must itself wait
+ *    (griddepcontrol.wait) before reading outputs; one launched without it, any
+ *    copy, and any event or host synchronisation see finished results.
  *  - The shared-memory limit of a kernel is raised once per process, on the
  *    device current at the first call: drive one GPU per process.
  *  - Arguments are checked on the host before anything is launched; a bad
