@@ -3,9 +3,9 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
-#include <mutex>
-
+#include <atomic>
 #include <cmath>
+#include <mutex>
 
 #include "internal.h"
 
@@ -13,17 +13,19 @@ namespace moe {
 
 int permute_chunks(long N);
 
+// SM count of the current device, cached per device (host threads may race to
+// fill an entry; they all store the same value).
 int num_sms() {
-    static int cache[64] = {0};
+    static std::atomic<int> cache[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-    if (cache[dev] == 0) {
-        int n = 0;
+    int n = cache[dev].load(std::memory_order_relaxed);
+    if (n == 0) {
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
             n = 148;
-        cache[dev] = n;
+        cache[dev].store(n, std::memory_order_relaxed);
     }
-    return cache[dev];
+    return n;
 }
 
 bool config_valid(const moe_config* c) {
