@@ -13,7 +13,10 @@ Pinned functions (each has ``-m "not gpu"`` tests against something other than
 itself; see ``tests/test_oracle_*.py``): format decoders/encoders, the activation
 quantisers, scoring, routing (brute force, library top-k, invariants), the
 permutation (library stable argsort, bijection), one expert's SwiGLU (one-hot
-closed forms, zero gate, linearity) and the combine (identical-expert identity).
+closed forms, zero gate, linearity), the combine (identical-expert identity),
+and the post-attention RMSNorm in front of the layer with its one-step
+double -> bf16 rounding (brute force over the bf16 grid, a 60-digit evaluation
+of the definition, closed forms, scale and permutation invariance).
 The composed layer output has no worked example on the pages. It is pinned by
 properties its definition fixes for any weights (each token's output depends on
 that token alone; relabelling the experts changes nothing; the routed part
@@ -92,6 +95,10 @@ def lib() -> ctypes.CDLL:
             l.or_expert_rows.argtypes = [_I, _I, _P, _P, _P, _P, _I, _I, _I, _P, _I, _D, _P]
             l.or_combine.restype = None
             l.or_combine.argtypes = [_I, _I, _I, _I, _P, _P, _P, _P]
+            l.or_bf16_encode.restype = ctypes.c_uint16
+            l.or_bf16_encode.argtypes = [_D, _D, _P]
+            l.or_rmsnorm.restype = _I
+            l.or_rmsnorm.argtypes = [_P, _I, _I, _P, _D, _D, _P, _P]
             _lib = l
     return _lib
 
@@ -168,6 +175,38 @@ def weight_value(wfmt: str, w, s, rows: int, cols: int, e: int, r: int, c: int) 
     w = np.ascontiguousarray(w)
     s = None if s is None else np.ascontiguousarray(s)
     return lib().or_weight_value(W_FMT[wfmt], _ptr(w), _ptr(s), rows, cols, e, r, c)
+
+
+def bf16_encode(vals, tie_rel: float = 0.0):
+    """Round doubles to bf16 codes (RNE, one rounding); also returns the flags of
+    values within tie_rel of a rounding midpoint."""
+    l = lib()
+    flat = np.ravel(np.asarray(vals, dtype=np.float64))
+    codes = np.zeros(flat.shape, np.uint16)
+    near = np.zeros(flat.shape, bool)
+    f = ctypes.c_uint8(0)
+    for i, v in enumerate(flat):
+        codes[i] = l.or_bf16_encode(float(v), float(tie_rel), ctypes.byref(f))
+        near[i] = bool(f.value)
+    return codes.reshape(np.shape(vals)), near.reshape(np.shape(vals))
+
+
+RMSNORM_TIE_REL = 2.0 ** -36  # a rounding near-tie: within this of a bf16 midpoint
+
+
+def rmsnorm(x_u16, w, eps: float, tie_rel: float = RMSNORM_TIE_REL):
+    """Post-attention RMSNorm of bf16 rows x [n, H] with fp32 weight w [H].
+
+    Returns (out bf16 codes [n, H], near_tie bool [n, H])."""
+    x = _c(x_u16, np.uint16)
+    w = _c(w, np.float32)
+    n, H = x.shape
+    out = np.zeros((n, H), np.uint16)
+    near = np.zeros((n, H), np.uint8)
+    if lib().or_rmsnorm(_ptr(x), n, H, _ptr(w), float(eps), float(tie_rel), _ptr(out),
+                        _ptr(near)) != 0:
+        raise ValueError("bad RMSNorm arguments")
+    return out, near.astype(bool)
 
 
 # ----------------------------------------------------------------- config

@@ -21,6 +21,9 @@
  *         e2m1 -> e4m3 lossless conversion).
  *   [MX]  "开源巨头开放2.8T MoE权重:架构创新与本地部署实践指南", section
  *         "存储与量化策略：MXFP格式下的1.56TB精粹" (MXFP4 weights, MXFP8 activations).
+ *   The post-attention RMSNorm in front of the layer follows [V3] 三 (the
+ *   decoder layer: post_attention_layernorm -> MoE) and [V4] 文件说明
+ *   (model.py RMSNorm, weight kept in fp32).
  *
  * Where the pages are silent the oracle takes one stated reading; each such
  * place is marked READING below.
@@ -491,4 +494,76 @@ void or_combine(int n, int K, int n_shared, int H, const double *w, const double
             for (int s = 0; s < n_shared; s++) acc += ys[((size_t)s * n + t) * H + h];
             out[(size_t)t * H + h] = acc;
         }
+}
+
+/* ------------------------------------------------- post-attention RMSNorm */
+/* Round-to-nearest-even of a double onto the bfloat16 grid in one step (no
+ * intermediate binary32 rounding). bfloat16 keeps 8 significant bits with the
+ * binary32 exponent range: in [2^(E), 2^(E+1)) with E >= -126 its spacing is
+ * 2^(E-7); below 2^-126 (subnormal) it is 2^-133. q = |v| / spacing is exact
+ * (a power-of-two division), so the two neighbours are floor(q) and
+ * floor(q) + 1 spacings; an exact midpoint goes to the even multiple (the code
+ * whose last bit is 0). Magnitudes that round past the largest finite value
+ * (2 - 2^-7) * 2^127 become infinity. *near (if given) is set to 1 when |v|
+ * lies within tie_rel * |v| of a midpoint between two neighbours. */
+uint16_t or_bf16_encode(double v, double tie_rel, uint8_t *near) {
+    if (near) *near = 0;
+    if (isnan(v)) return 0x7FC0;
+    uint16_t sign = signbit(v) ? 0x8000 : 0x0000;
+    double a = fabs(v);
+    if (a == 0.0) return sign;
+    if (isinf(v)) return sign | 0x7F80;
+    int e;
+    frexp(a, &e); /* a = f * 2^e, f in [0.5, 1): leading bit 2^(e-1) */
+    int lead = e - 1;
+    if (lead < -126) lead = -126; /* subnormal spacing */
+    double spacing = ldexp(1.0, lead - 7);
+    double q = a / spacing; /* exact */
+    double lo = floor(q);
+    double frac = q - lo; /* exact */
+    if (near && fabs(a - (lo + 0.5) * spacing) <= tie_rel * a) *near = 1;
+    double n;
+    if (frac > 0.5) n = lo + 1.0;
+    else if (frac < 0.5) n = lo;
+    else n = (fmod(lo, 2.0) == 0.0) ? lo : lo + 1.0;
+    double r = n * spacing; /* a bfloat16 value (or 2^128) */
+    if (r >= ldexp(1.0, 128)) return sign | 0x7F80;
+    float f = (float)r; /* exact: r has at most 8 significant bits in range */
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    return sign | (uint16_t)(u >> 16);
+}
+
+/* The post-attention RMSNorm in front of the MoE block ([V3] 三, the decoder
+ * layer: post_attention_layernorm -> MoE/MLP; [V4] 文件说明, model.py RMSNorm:
+ * the standard form with its weight kept in fp32):
+ *   r = 1 / sqrt( (sum_h x_h^2) / H + eps ),   y_h = (x_h * r) * w_h,
+ * READING: the pages fix neither the working precision nor eps. Here every
+ * step is evaluated in double in the order written (the sum sequentially over
+ * h, then the mean, eps, sqrt and reciprocal, then the two products), and y_h
+ * is rounded once to bf16 (RNE) -- the output the router and the expert
+ * inputs read. x [n][H] bf16 codes, w [H] fp32, out [n][H] bf16 codes;
+ * near[n][H] (if given) flags outputs within tie_rel * |y| of a bf16 rounding
+ * midpoint, where an implementation summing the squares in another order may
+ * round the other way. Returns OR_ERR_ARG for n < 0, H < 1 or eps < 0. */
+int or_rmsnorm(const uint16_t *x, int n, int H, const float *w, double eps, double tie_rel,
+               uint16_t *out, uint8_t *near) {
+    if (n < 0 || H < 1 || !(eps >= 0.0)) return OR_ERR_ARG;
+#pragma omp parallel for schedule(static)
+    for (int t = 0; t < n; t++) {
+        const uint16_t *xr = x + (size_t)t * H;
+        double ss = 0.0;
+        for (int h = 0; h < H; h++) {
+            double v = or_bf16_value(xr[h]);
+            ss += v * v;
+        }
+        double r = 1.0 / sqrt(ss / (double)H + eps);
+        for (int h = 0; h < H; h++) {
+            double y = (or_bf16_value(xr[h]) * r) * (double)w[h];
+            uint8_t nt = 0;
+            out[(size_t)t * H + h] = or_bf16_encode(y, tie_rel, &nt);
+            if (near) near[(size_t)t * H + h] = nt;
+        }
+    }
+    return OR_OK;
 }
