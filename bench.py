@@ -86,6 +86,11 @@ def parse():
     ap.add_argument("--clock-log", default=None,
                     help="keep the raw nvidia-smi samples here (%%d = device index)")
     ap.add_argument("--cpu-sample-tokens", type=int, default=128)
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="time only the headline workload (N=1 runs otherwise also time the "
+                         "prefill-shaped workloads)")
+    ap.add_argument("--per-workload-steps", type=int, default=20)
+    ap.add_argument("--per-workload-cpu-tokens", type=int, default=12)
     return ap.parse_args()
 
 
@@ -207,19 +212,69 @@ def gate_up_flops(cfg, T):
     return layer_flops(cfg, T) * 2.0 / 3.0
 
 
-# Nominal dense tensor rates relative to bf16. The expert GEMMs run bf16/f16
-# MMAs when the activations are bf16 (FP8 weights are converted to 16 bits),
-# else block-scaled E2M1 x E4M3 MMAs at the FP8 rate.
+# Nominal dense tensor rates relative to bf16 (context: the FP8 rate is the
+# one the block-scaled E2M1 x E4M3 MMAs run at).
 NOMINAL_RATE_VS_BF16 = {"bf16": 1.0, "fp8": 2.0}
+NOMINAL_HBM_GBS = 7700.0  # B200 HGX datasheet figure, for context beside the measured copy rate
 
 
-def tensor_peak(peaks, peak_src, cfg):
+def measure_fp8_peaks(dev, n=8192, reps=10):
+    """Measured FP8-rate tensor throughput of cuBLAS on this GPU (TFLOP/s, best of
+    `reps` back-to-back n^3 products, CUDA events): E4M3 x E4M3 with per-tensor
+    scales, and the block-scaled MXFP8 form (E8M0 scale per 32 elements) when
+    this torch exposes it. These are library GEMMs used only as the denominator
+    of the block-scaled layers' tensor fraction, the way the bf16 peak is."""
+    import torch
+    out = {}
+    a = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn)
+    b = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn).t()  # column-major operand
+    one = torch.ones((), device=dev)
+
+    def best(fn):
+        fn()
+        torch.cuda.synchronize()
+        t = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            t.append(e0.elapsed_time(e1))
+        return 2.0 * n ** 3 / (min(t) / 1e3) / 1e12
+
+    try:
+        out["fp8_e4m3_tensorwise"] = best(
+            lambda: torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16))
+    except Exception as e:  # noqa: BLE001 - report why, keep the bench line
+        out["fp8_e4m3_tensorwise_error"] = str(e).splitlines()[0][:160]
+    try:
+        e8 = getattr(torch, "float8_e8m0fnu")
+        sa = torch.full((n * (n // 32),), 127, dtype=torch.uint8, device=dev).view(e8)
+        sb = torch.full((n * (n // 32),), 127, dtype=torch.uint8, device=dev).view(e8)
+        out["mxfp8_block32"] = best(
+            lambda: torch._scaled_mm(a, b, scale_a=sa, scale_b=sb, out_dtype=torch.bfloat16))
+    except Exception as e:  # noqa: BLE001
+        out["mxfp8_block32_error"] = str(e).splitlines()[0][:160]
+    del a, b
+    torch.cuda.empty_cache()
+    return out
+
+
+def tensor_peak(peaks, peak_src, cfg, fp8_measured=None):
     """(TFLOP/s, source) of the tensor rate the expert GEMMs run at: the
-    measured bf16 figure, times the nominal ratio for FP8-rate MMAs."""
+    measured bf16 figure for bf16/f16 MMAs; for FP8-rate MMAs the best measured
+    FP8 cuBLAS rate when one was measured in this run, else the bf16 figure
+    times the nominal ratio."""
     kind = "bf16" if cfg.afmt == "bf16" else "fp8"
+    if kind == "bf16":
+        return peaks["bf16_tflops"], peak_src
+    meas = {k: v for k, v in (fp8_measured or {}).items() if isinstance(v, float)}
+    if meas:
+        name = max(meas, key=meas.get)
+        return meas[name], "measured in this run: cuBLAS %s 8192^3, best of 10" % name
     ratio = NOMINAL_RATE_VS_BF16[kind]
-    src = peak_src if ratio == 1.0 else "%s bf16 x nominal %s/bf16 ratio %g" % (peak_src, kind, ratio)
-    return peaks["bf16_tflops"] * ratio, src
+    return peaks["bf16_tflops"] * ratio, "%s bf16 x nominal %s/bf16 ratio %g" % (peak_src, kind, ratio)
 
 
 def roofline(bytes_, flops, ms, hbm, tpeak):
@@ -229,10 +284,17 @@ def roofline(bytes_, flops, ms, hbm, tpeak):
     hbm_frac = bytes_ / s / 1e9 / hbm
     tensor_frac = flops / s / 1e12 / tpeak
     if flops / (tpeak * 1e12) > bytes_ / (hbm * 1e9):
-        return {"bound": "tensor", "achieved": flops / s / 1e12, "peak": tpeak, "unit": "TFLOP/s",
-                "frac": tensor_frac, "hbm_frac": hbm_frac, "tensor_frac": tensor_frac}
-    return {"bound": "hbm", "achieved": bytes_ / s / 1e9, "peak": hbm, "unit": "GB/s",
-            "frac": hbm_frac, "hbm_frac": hbm_frac, "tensor_frac": tensor_frac}
+        r = {"bound": "tensor", "achieved": flops / s / 1e12, "peak": tpeak, "unit": "TFLOP/s",
+             "frac": tensor_frac, "hbm_frac": hbm_frac, "tensor_frac": tensor_frac}
+    else:
+        # the measured peak is a read+write copy; a read-mostly stream can pass it,
+        # so the fraction of the datasheet bandwidth is given beside it
+        r = {"bound": "hbm", "achieved": bytes_ / s / 1e9, "peak": hbm, "unit": "GB/s",
+             "frac": hbm_frac, "hbm_frac": hbm_frac, "tensor_frac": tensor_frac,
+             "frac_of_nominal_hbm": bytes_ / s / 1e9 / NOMINAL_HBM_GBS,
+             "nominal_hbm_gbs": NOMINAL_HBM_GBS}
+    r["above_measured_peak"] = r["frac"] > 1.0
+    return r
 
 
 def ncu_traffic(kernel: str, workload: str):
@@ -279,16 +341,31 @@ def clock_log_path(pattern, device_index):
     return pattern % device_index if "%d" in pattern else pattern
 
 
-def run_ours(args, rank, world, dev):
+def workload_config(cfg, world):
+    """The config dict both arms print for a workload (identical keys and values)."""
+    return {"workload": "%s: T=%d tokens, hidden %d, %d routed experts top-%d, intermediate %d, "
+                        "%d shared, %s weights, %s activations"
+                        % (cfg.name, cfg.T, cfg.hidden, cfg.n_routed_experts,
+                           cfg.num_experts_per_tok, cfg.moe_intermediate_size,
+                           cfg.n_shared_experts, cfg.wfmt, cfg.afmt),
+            "T": cfg.T, "hidden": cfg.hidden, "experts": cfg.n_routed_experts,
+            "top_k": cfg.num_experts_per_tok, "n_group": cfg.n_group,
+            "topk_group": cfg.topk_group, "intermediate": cfg.moe_intermediate_size,
+            "shared_experts": cfg.n_shared_experts, "score_fn": cfg.score_fn,
+            "weights": cfg.wfmt, "activations": cfg.afmt, "routing": cfg.routing,
+            "seed": cfg.seed, "parallelism": "replicas x%d" % world,
+            "l2": "256 MiB write before every timed step, outside the timed events"}
+
+
+def measure(args, cfg, rank, world, dev, steps, warmup, n_stage, n_e2e, workload_key,
+            fp8_measured=None):
+    """Time `steps` layer steps of one workload on this rank (staged ABI calls,
+    L2 flushed before each), plus the per-stage split and the end-to-end form.
+    Returns (line fields, inputs, weights)."""
     import torch
     import expert_routing_grouped_layer_b200 as moe
     from expert_routing_grouped_layer_b200 import workloads as W
 
-    cfg = W.CONFIGS[args.workload]
-    if args.tokens:
-        cfg = cfg.replace(T=args.tokens)
-    if args.experts:
-        cfg = cfg.replace(n_routed_experts=args.experts)
     T, k, E, H, I, S = (cfg.T, cfg.num_experts_per_tok, cfg.n_routed_experts, cfg.hidden,
                         cfg.moe_intermediate_size, cfg.n_shared_experts)
     inp = W.make_inputs(cfg, dev)
@@ -333,7 +410,7 @@ def run_ours(args, rank, world, dev):
 
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(7)]
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         flush.zero_()
         step(mk())
     torch.cuda.synchronize()
@@ -344,7 +421,7 @@ def run_ours(args, rank, world, dev):
     assert st.item() == 0, "device status %d" % st.item()
 
     # per timed step: start, gate/up start, gate/up end, end
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
     di = dev.index if dev.index is not None else 0
     clocks = ClockSampler(di, enabled=not args.no_clocks,
                           log_path=clock_log_path(args.clock_log, di))
@@ -367,7 +444,6 @@ def run_ours(args, rank, world, dev):
 
     # per-stage split: the staged entry points with events between them (not
     # part of the timed steps above)
-    n_stage = max(1, min(args.steps, 100))
     sevents = [mk() for _ in range(n_stage)]
     for i in range(n_stage):
         flush.zero_()
@@ -376,11 +452,12 @@ def run_ours(args, rank, world, dev):
     stage = [[sevents[i][j].elapsed_time(sevents[i][j + 1]) for i in range(n_stage)]
              for j in range(6)]
     offsets = layer.intermediate(T, moe.WS_OFFSETS, torch.int32, (E + 1,)).cpu()
-    active = int((offsets[1:] - offsets[:-1] > 0).sum())
+    counts = offsets[1:] - offsets[:-1]
+    active = int((counts > 0).sum())
 
     # end to end: host tokens in (pinned), layer through the public API, host result out
     e2e = None
-    if not args.no_e2e:
+    if n_e2e > 0:
         xh = x.cpu().pin_memory()
         oh = torch.empty(T, H, dtype=torch.bfloat16).pin_memory()
         xd = torch.empty_like(x)
@@ -392,7 +469,6 @@ def run_ours(args, rank, world, dev):
             torch.distributed.barrier()
         # each step: L2 flushed first (outside the timed events), then the
         # pinned-host copy in, the layer, and the copy of the result back out
-        n_e2e = max(1, min(args.steps, 100))
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(n_e2e)]
         for e0, e1 in evs:
@@ -408,24 +484,25 @@ def run_ours(args, rank, world, dev):
                "ms_per_step": e2e_ms, "includes_l2_flush": False}
 
     peaks, peak_src = load_peaks()
-    ms = total_ms / args.steps
+    ms = total_ms / steps
     mean = lambda j: statistics.fmean(stage[j])
     names = ["gate_topk", "permute", "pack_inputs", "gate_up", "down", "combine"]
     stage_ms = {n: mean(j) for j, n in enumerate(names)}
     gu_bytes = gate_up_bytes(cfg, active, T)
     gu_ms = statistics.fmean(gate_up_ms)  # the dominant kernel, over the timed steps
     hbm = peaks["hbm_gbs"]
-    tpeak, tpeak_src = tensor_peak(peaks, peak_src, cfg)
+    tpeak, tpeak_src = tensor_peak(peaks, peak_src, cfg, fp8_measured)
     lb = layer_bytes(cfg, active, T)
     lf = layer_flops(cfg, T)
     ewb = expert_weight_bytes(cfg, active)
     kroof = roofline(gu_bytes, gate_up_flops(cfg, T), gu_ms, hbm, tpeak)
     kroof.update({"kernel": "gate_up (grouped SwiGLU GEMM1)",
                   "peak_source": peak_src if kroof["bound"] == "hbm" else tpeak_src,
-                  "traffic": ncu_traffic("gate_up", args.workload)
+                  "traffic": ncu_traffic("gate_up", workload_key)
                   if not (args.tokens or args.experts) else None,
                   "algorithmic_bytes_per_launch": gu_bytes,
-                  "algorithmic_flops_per_launch": gate_up_flops(cfg, T)})
+                  "algorithmic_flops_per_launch": gate_up_flops(cfg, T),
+                  "ms_per_launch": gu_ms})
     lroof = roofline(lb, lf, ms, hbm, tpeak)
     lroof.update({"bytes": lb, "achieved_gbs": lb / (ms / 1e3) / 1e9,
                   # the activated and shared experts' weights alone (no router
@@ -434,39 +511,114 @@ def run_ours(args, rank, world, dev):
                   "expert_weight_frac": ewb / (ms / 1e3) / 1e9 / hbm,
                   "flops": lf, "tflops": lf / (ms / 1e3) / 1e12,
                   "tensor_peak": tpeak, "tensor_peak_source": tpeak_src})
-    line = {
-        "metric": METRIC,
+    if cfg.afmt == "bf16":
+        lroof["tensor_frac_sustained_peak"] = lf / (ms / 1e3) / 1e12 / peaks.get(
+            "bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    cfgd = workload_config(cfg, world)
+    routing_stats = {"active_experts": active,
+                     "max_over_mean_load": float(counts.max()) / max(1e-9, float(counts.float().mean())),
+                     "max_tokens_per_expert": int(counts.max())}
+    fields = {
         "value": world * T / (ms / 1e3),
-        "unit": UNIT,
-        "n_gpus": world,
-        "steps": args.steps,
-        "warmup": args.warmup,
         "ms_per_step": ms,
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
+        "steps": steps,
+        "warmup": warmup,
         "dtype": "bf16" if cfg.wfmt == "bf16" else cfg.wfmt,
-        "data": "synthetic (seeded; x ~ N(0,1), router N(0,0.02), bias U[-0.1,0.1], "
-                "experts N(0,0.02)); random-init weights",
-        "config": {"workload": "%s: T=%d tokens, hidden %d, %d routed experts top-%d, "
-                               "intermediate %d, %d shared, %s weights, %s activations"
-                               % (cfg.name, T, H, E, k, I, S, cfg.wfmt, cfg.afmt),
-                   "T": T, "hidden": H, "experts": E, "top_k": k, "intermediate": I,
-                   "shared_experts": S, "active_experts": active,
-                   "parallelism": "replicas x%d" % world,
-                   "l2": "256 MiB write before every timed step, outside the timed events"},
+        "config": cfgd,
+        "routing_stats": routing_stats,
         "roofline": kroof,
         "layer_roofline": lroof,
         "stage_ms": stage_ms,
         "stage_ms_source": "staged entry points with events between them, %d separate steps "
                            "(the timed steps record events only at their ends and around "
                            "gate_up)" % n_stage,
-        "gpu_launches": launches_per_step(cfg, T, torch.cuda.get_device_properties(dev).multi_processor_count) * args.steps,
+        "gpu_launches": launches_per_step(
+            cfg, T, torch.cuda.get_device_properties(dev).multi_processor_count) * steps,
         "wall_s_timed_loop": wall,
         "clocks": clk,
         "e2e": e2e,
     }
-    return line, cfg, inp, wts
+    del layer, ws, out, flush, ref
+    return fields, inp, wts
+
+
+def cpu_baseline(cfg, inp, wts, tokens, seed=3):
+    tok = min(tokens, cfg.T)
+    times = oracle_timing(cfg, inp, wts, tok, 1, seed=seed)
+    return {"value": tok / times[0], "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+            "sample": "%d seeded tokens of the %d-token batch (route + layer, float64), %.1f s"
+                      % (tok, cfg.T, times[0])}
+
+
+# prefill-shaped workloads timed after the headline in an N=1 run
+PER_WORKLOADS = ("k2_prefill_fp8w", "v4_fp4", "mx896")
+
+
+def run_ours(args, rank, world, dev):
+    import torch
+    from expert_routing_grouped_layer_b200 import workloads as W
+
+    cfg = W.CONFIGS[args.workload]
+    if args.tokens:
+        cfg = cfg.replace(T=args.tokens)
+    if args.experts:
+        cfg = cfg.replace(n_routed_experts=args.experts)
+    fp8_measured = None
+    if world == 1 and (cfg.afmt != "bf16" or not args.no_per_workload):
+        fp8_measured = measure_fp8_peaks(dev)
+    fields, inp, wts = measure(args, cfg, rank, world, dev, args.steps, args.warmup,
+                               max(1, min(args.steps, 100)),
+                               0 if args.no_e2e else max(1, min(args.steps, 100)),
+                               args.workload, fp8_measured)
+    line = {
+        "metric": METRIC,
+        "value": fields["value"],
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": fields["ms_per_step"],
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": fields["dtype"],
+        "data": "synthetic (seeded; x ~ N(0,1), router N(0,0.02), bias U[-0.1,0.1], "
+                "experts N(0,0.02)); random-init weights",
+    }
+    line.update({k: v for k, v in fields.items() if k not in line})
+    if fp8_measured is not None:
+        line["fp8_peaks_tflops"] = fp8_measured
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, inp, wts, args.cpu_sample_tokens)
+    del inp, wts
+    torch.cuda.empty_cache()
+
+    if world == 1 and not args.no_per_workload and not (args.tokens or args.experts):
+        per = {}
+        for name in PER_WORKLOADS:
+            if name == args.workload:
+                continue
+            c = W.CONFIGS[name]
+            f, inp, wts = measure(args, c, rank, world, dev, args.per_workload_steps,
+                                  max(3, min(args.warmup, 5)), args.per_workload_steps,
+                                  0 if args.no_e2e else min(args.per_workload_steps, 10),
+                                  name, fp8_measured)
+            keep = ("value", "ms_per_step", "steps", "warmup", "dtype", "config", "routing_stats",
+                    "roofline",
+                    "layer_roofline", "stage_ms", "gpu_launches", "clocks", "e2e")
+            per[name] = {k: f[k] for k in keep}
+            per[name]["unit"] = UNIT
+            if not args.no_cpu_baseline:
+                per[name]["cpu_baseline"] = cpu_baseline(c, inp, wts,
+                                                         args.per_workload_cpu_tokens)
+            del inp, wts
+            torch.cuda.empty_cache()
+        line["per_workload"] = per
+        line["per_workload_note"] = ("each prefill-shaped workload timed at full size after the "
+                                     "headline, %d steps, same L2 flush and clock sampling; the "
+                                     "headline value/config above is the decode workload"
+                                     % args.per_workload_steps)
+    return line
 
 
 # ------------------------------------------------------------------ oracle arm
@@ -516,7 +668,7 @@ def cpu_cores():
         return os.cpu_count()
 
 
-def run_reference(args, dev):
+def run_reference(args, dev, world=1):
     import torch
     from expert_routing_grouped_layer_b200 import workloads as W
     cfg = W.CONFIGS[args.workload]
@@ -535,8 +687,7 @@ def run_reference(args, dev):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded, same workload as the CUDA arm)",
-        "config": {"workload": cfg.name, "T": cfg.T, "hidden": cfg.hidden,
-                   "experts": cfg.n_routed_experts, "top_k": cfg.num_experts_per_tok},
+        "config": workload_config(cfg, world),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -554,7 +705,7 @@ def main():
             return 0
         dev = torch.device("cuda", local)
         torch.cuda.set_device(dev)
-        print(json.dumps(run_reference(args, dev)), flush=True)
+        print(json.dumps(run_reference(args, dev, world)), flush=True)
         return 0
 
     dev = torch.device("cuda", local)
@@ -563,14 +714,7 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", device_id=dev,
                                              timeout=datetime.timedelta(seconds=300))
-    line, cfg, inp, wts = run_ours(args, rank, world, dev)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tok = min(args.cpu_sample_tokens, cfg.T)
-        times = oracle_timing(cfg, inp, wts, tok, 1, seed=3)
-        line["cpu_baseline"] = {"value": tok / times[0], "unit": UNIT, "cores": cpu_cores(),
-                                "kind": "oracle",
-                                "sample": "%d seeded tokens of the %d-token batch (route + layer, "
-                                          "float64), %.1f s" % (tok, cfg.T, times[0])}
+    line = run_ours(args, rank, world, dev)
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()

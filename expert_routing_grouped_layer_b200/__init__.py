@@ -30,14 +30,15 @@ AFMT = {"bf16": 0, "fp8_e4m3_pow2_b128": 1, "mxfp8": 2}
 EXPORTS = ("moe_workspace_bytes", "moe_gate_topk", "moe_permute", "moe_quantize_activations",
            "moe_pack_expert_inputs", "moe_expert_gate_up", "moe_expert_down",
            "moe_grouped_swiglu", "moe_combine", "moe_layer_forward", "moe_workspace_offset",
-           "moe_status_string", "moe_permute_noalloc", "moe_selftest_wait_limit")
+           "moe_status_string", "moe_permute_noalloc", "moe_selftest_wait_limit",
+           "moe_rmsnorm_prologue", "moe_layer_forward_prenorm")
 
 # capacity (int32 counts) of the static scratch behind moe_permute_noalloc
 MOE_PERMUTE_NOALLOC_MAX_COUNTS = 262144
 
 # moe_workspace_offset selectors
 WS_TOPK_IDX, WS_TOPK_W, WS_OFFSETS, WS_SORTED_PAIR, WS_ROW_OF, WS_Y, WS_SHARED_Y, WS_XA, \
-    WS_XA_SCALE, WS_H, WS_H_SCALE = range(11)
+    WS_XA_SCALE, WS_H, WS_H_SCALE, WS_X_NORM = range(12)
 
 
 class MoEError(RuntimeError):
@@ -107,6 +108,11 @@ def lib() -> ctypes.CDLL:
             l.moe_grouped_swiglu.argtypes = [CP, _P, _I32, _P, _P, WP, _P, _P, _P, _SZ, _P, _P]
             l.moe_combine.restype = ctypes.c_int
             l.moe_combine.argtypes = [CP, _P, _P, _P, _P, _I32, _P, _P]
+            l.moe_rmsnorm_prologue.restype = ctypes.c_int
+            l.moe_rmsnorm_prologue.argtypes = [CP, _P, _I32, _P, ctypes.c_float, _P, _P, _P, _P]
+            l.moe_layer_forward_prenorm.restype = ctypes.c_int
+            l.moe_layer_forward_prenorm.argtypes = [CP, _P, _I32, _P, ctypes.c_float, WP, _P, _P,
+                                                    _SZ, _P, _P]
             l.moe_layer_forward.restype = ctypes.c_int
             l.moe_layer_forward.argtypes = [CP, _P, _I32, WP, _P, _P, _SZ, _P, _P]
             _lib = l
@@ -257,6 +263,22 @@ def moe_layer_forward(cfg, x, T, weights, out, ws, dev_status, ws_bytes=None, st
                                    _stream(stream)), "moe_layer_forward")
 
 
+def moe_rmsnorm_prologue(cfg, x, T, norm_w, eps, x_norm, xq=None, xq_scale=None, stream=None):
+    _check(lib().moe_rmsnorm_prologue(ctypes.byref(_cfg(cfg)), _ptr(x), int(T), _ptr(norm_w),
+                                      float(eps), _ptr(x_norm), _ptr(xq), _ptr(xq_scale),
+                                      _stream(stream)), "moe_rmsnorm_prologue")
+
+
+def moe_layer_forward_prenorm(cfg, x, T, norm_w, eps, weights, out, ws, dev_status, ws_bytes=None,
+                              stream=None):
+    ws_bytes = ws.numel() * ws.element_size() if ws_bytes is None else ws_bytes
+    w = weights if isinstance(weights, moe_weights) else make_weights(weights)
+    _check(lib().moe_layer_forward_prenorm(ctypes.byref(_cfg(cfg)), _ptr(x), int(T), _ptr(norm_w),
+                                           float(eps), ctypes.byref(w), _ptr(out), _ptr(ws),
+                                           ws_bytes, _ptr(dev_status), _stream(stream)),
+           "moe_layer_forward_prenorm")
+
+
 class MoELayer:
     """A layer bound to its device-resident parameters and a workspace.
 
@@ -293,6 +315,18 @@ class MoELayer:
         return out
 
     __call__ = forward
+
+    def forward_prenorm(self, x, norm_w, eps, out=None, stream=None):
+        """The layer from the un-normalised hidden state (moe_layer_forward_prenorm)."""
+        import torch
+        T = x.shape[0]
+        if T > self.max_tokens:
+            raise ValueError("more tokens than the workspace was sized for")
+        if out is None:
+            out = torch.empty(T, self.cfg.hidden, dtype=torch.bfloat16, device=self.device)
+        moe_layer_forward_prenorm(self.ccfg, x, T, norm_w, eps, self.cw, out, self.ws, self.status,
+                                  ws_bytes=self.ws.numel(), stream=stream)
+        return out
 
     def ws_ptr(self, T: int, which: int) -> int:
         """Device address of an intermediate inside the workspace."""

@@ -5,7 +5,9 @@
 #include <algorithm>
 #include <atomic>
 #include <cmath>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "internal.h"
 
@@ -26,6 +28,21 @@ int num_sms() {
         cache[dev].store(n, std::memory_order_relaxed);
     }
     return n;
+}
+
+cudaError_t ensure_smem_limit(const void* kernel, int bytes) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    static std::mutex mu;
+    static std::map<std::pair<const void*, int>, cudaError_t> done;
+    std::lock_guard<std::mutex> lock(mu);
+    const auto key = std::make_pair(kernel, dev);
+    const auto it = done.find(key);
+    if (it != done.end()) return it->second;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    done.emplace(key, e);
+    return e;
 }
 
 bool config_valid(const moe_config* c) {
@@ -99,6 +116,7 @@ WsLayout ws_layout(const moe_config* c, int T) {
     L.h_scale = take(act_bytes == 1 ? (N + S * T) * (I / 32) : (f16_gate_up(c) ? (N + S * T) : 0));
     L.y = take(N * H * 2);
     L.shared_y = take(S * T * H * 2);
+    L.x_norm = take((size_t)T * H * 2);
     L.total = off;
     return L;
 }
@@ -110,12 +128,6 @@ using namespace moe;
 static inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
 static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
-
-static moe_status cuda_status(cudaError_t e) {
-    if (e == cudaSuccess) return MOE_OK;
-    if (e == cudaErrorNotSupported) return MOE_ERR_UNSUPPORTED;
-    return MOE_ERR_CUDA;
-}
 
 extern "C" {
 
@@ -139,6 +151,7 @@ size_t moe_workspace_offset(const moe_config* cfg, int32_t T, int32_t which) {
     case 8: return L.xa_scale;
     case 9: return L.hbuf;
     case 10: return L.h_scale;
+    case 11: return L.x_norm;
     }
     return (size_t)-1;
 }
@@ -366,6 +379,83 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* x, int32_t T, co
     if (s == MOE_OK) s = moe_permute(cfg, idx, T, off, sp, ro, dev_status, ws, ws_bytes, stream);
     if (s == MOE_OK)
         s = moe_grouped_swiglu(cfg, x, T, sp, off, w, y, sy, ws, ws_bytes, dev_status, stream);
+    if (s == MOE_OK) s = moe_combine(cfg, y, sy, ro, tw, T, out, stream);
+    return s;
+}
+
+moe_status moe_rmsnorm_prologue(const moe_config* cfg, const void* x, int32_t T, const float* norm_w,
+                                float eps, void* x_norm, void* xq, void* xq_scale, void* stream) {
+    if (!config_valid(cfg) || T < 0) return MOE_ERR_INVALID_ARG;
+    if (!(eps >= 0.0f) || isinf(eps)) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!x || !norm_w || !x_norm || !aligned16(x) || !aligned16(norm_w) || !aligned16(x_norm))
+        return MOE_ERR_INVALID_ARG;
+    const bool q = cfg->afmt != MOE_A_BF16;
+    if (q && (cfg->hidden % 512 || !xq || !xq_scale || !aligned16(xq) || !aligned16(xq_scale)))
+        return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_rmsnorm_quant(cfg->afmt, x, cfg->hidden, norm_w, eps, T, x_norm,
+                                            q ? xq : nullptr,
+                                            static_cast<uint8_t*>(q ? xq_scale : nullptr),
+                                            as_stream(stream)));
+}
+
+moe_status moe_layer_forward_prenorm(const moe_config* cfg, const void* x, int32_t T,
+                                     const float* norm_w, float eps, const moe_weights* w,
+                                     void* out, void* ws, size_t ws_bytes, int32_t* dev_status,
+                                     void* stream) {
+    if (!config_valid(cfg) || T < 0 || !w) return MOE_ERR_INVALID_ARG;
+    const moe_status sup = config_supported(cfg);
+    if (sup != MOE_OK) return sup;
+    if (!(eps >= 0.0f) || isinf(eps)) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    // everything is checked before the first launch
+    if (!x || !norm_w || !out || !ws || !w->gate_w || !w->gate_bias) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(norm_w) || !aligned16(out) || !aligned16(w->gate_w))
+        return MOE_ERR_INVALID_ARG;
+    if (!weights_ok(cfg, w, true) || !weights_ok(cfg, w, false)) return MOE_ERR_INVALID_ARG;
+    if ((long)T * cfg->num_experts_per_tok > 0x7fffffffL) return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(cfg, T);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+    char* base = static_cast<char*>(ws);
+    int32_t* idx = reinterpret_cast<int32_t*>(base + L.topk_idx);
+    float* tw = reinterpret_cast<float*>(base + L.topk_w);
+    int32_t* off = reinterpret_cast<int32_t*>(base + L.offsets);
+    int32_t* sp = reinterpret_cast<int32_t*>(base + L.sorted_pair);
+    int32_t* ro = reinterpret_cast<int32_t*>(base + L.row_of);
+    void* xn = base + L.x_norm;
+    void* y = base + L.y;
+    void* sy = base + L.shared_y;
+    const int k = cfg->num_experts_per_tok, H = cfg->hidden, N = T * k;
+    cudaStream_t st = as_stream(stream);
+    if (cfg->afmt == MOE_A_BF16) {
+        // bf16 expert inputs: the prologue's output feeds the unchanged layer
+        moe_status s = cuda_status(launch_rmsnorm_quant(MOE_A_BF16, x, H, norm_w, eps, T, xn,
+                                                        nullptr, nullptr, st));
+        if (s == MOE_OK)
+            s = moe_layer_forward(cfg, xn, T, w, out, ws, ws_bytes, dev_status, stream);
+        return s;
+    }
+    // quantised expert inputs: the prologue writes the token rows (rows N..N+T-1
+    // of the expert input, the shared experts' rows) once; the routed rows are
+    // gathered from them after the permutation
+    uint8_t* xa = reinterpret_cast<uint8_t*>(base + L.xa);
+    uint8_t* xas = reinterpret_cast<uint8_t*>(base + L.xa_scale);
+    uint8_t* qrows = xa + (size_t)N * H;
+    uint8_t* qscales = xas + (size_t)N * (H / 32);
+    moe_status s = cuda_status(launch_rmsnorm_quant(cfg->afmt, x, H, norm_w, eps, T, xn, qrows,
+                                                    qscales, st));
+    if (s == MOE_OK)
+        s = moe_gate_topk(cfg, xn, T, w->gate_w, w->gate_bias, idx, tw, dev_status, ws, ws_bytes,
+                          stream);
+    if (s == MOE_OK) s = moe_permute(cfg, idx, T, off, sp, ro, dev_status, ws, ws_bytes, stream);
+    if (s == MOE_OK)
+        s = cuda_status(launch_gather_token_rows(qrows, qscales, H, sp, N, k, T, xa, xas, st));
+    if (s == MOE_OK)
+        s = moe_expert_gate_up(cfg, xa, xas, T, off, w, base + L.hbuf, base + L.h_scale, dev_status,
+                               stream);
+    if (s == MOE_OK)
+        s = moe_expert_down(cfg, base + L.hbuf, base + L.h_scale, T, off, w, y, sy, dev_status,
+                            stream);
     if (s == MOE_OK) s = moe_combine(cfg, y, sy, ro, tw, T, out, stream);
     return s;
 }

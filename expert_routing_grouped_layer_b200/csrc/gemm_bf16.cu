@@ -182,12 +182,8 @@ __global__ void __launch_bounds__(192, 1)
 template <int GEMM>
 cudaError_t launch_bf16(const GroupedGemmArgs& a, cudaStream_t st) {
     using C = Tile<GEMM>;
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(grouped_gemm_bf16_kernel<GEMM>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-    });
+    const cudaError_t attr_err =
+        ensure_smem_limit(reinterpret_cast<const void*>(grouped_gemm_bf16_kernel<GEMM>), C::SMEM_BYTES);
     if (attr_err != cudaSuccess) return attr_err;
 
     uint64_t b_rows;

@@ -877,12 +877,8 @@ __global__ void __launch_bounds__(TileTA<GEMM, BNT_, MST_>::THREADS, 1)
 template <int GEMM, int BNF_, int ACCB_, int MST_>
 cudaError_t launch_fp8w(const GroupedGemmArgs& a, cudaStream_t st) {
     using C = TileF8<GEMM, BNF_, ACCB_, MST_>;
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(grouped_gemm_fp8w_kernel<GEMM, BNF_, ACCB_, MST_>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-    });
+    const cudaError_t attr_err = ensure_smem_limit(
+        reinterpret_cast<const void*>(grouped_gemm_fp8w_kernel<GEMM, BNF_, ACCB_, MST_>), C::SMEM_BYTES);
     if (attr_err != cudaSuccess) return attr_err;
     uint64_t b_rows;
     KParams p = make_params(a, GEMM, &b_rows);
@@ -909,12 +905,8 @@ cudaError_t launch_fp8w(const GroupedGemmArgs& a, cudaStream_t st) {
 template <int GEMM, int BNT_, int MST_>
 cudaError_t launch_fp8w_ta(const GroupedGemmArgs& a, cudaStream_t st) {
     using C = TileTA<GEMM, BNT_, MST_>;
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(grouped_gemm_fp8w_ta_kernel<GEMM, BNT_, MST_>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-    });
+    const cudaError_t attr_err = ensure_smem_limit(
+        reinterpret_cast<const void*>(grouped_gemm_fp8w_ta_kernel<GEMM, BNT_, MST_>), C::SMEM_BYTES);
     if (attr_err != cudaSuccess) return attr_err;
     uint64_t b_rows;
     KParams p = make_params(a, GEMM, &b_rows);

@@ -536,12 +536,8 @@ __global__ void __launch_bounds__(TileMX<GEMM, NA_, BNX_, ACCB_>::THREADS, 1)
 template <int GEMM, int AFMT, int NA_, int BNX_, int ACCB_>
 cudaError_t launch_mx(const GroupedGemmArgs& a, cudaStream_t st) {
     using C = TileMX<GEMM, NA_, BNX_, ACCB_>;
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(grouped_gemm_mx_kernel<GEMM, AFMT, NA_, BNX_, ACCB_>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-    });
+    const cudaError_t attr_err = ensure_smem_limit(
+        reinterpret_cast<const void*>(grouped_gemm_mx_kernel<GEMM, AFMT, NA_, BNX_, ACCB_>), C::SMEM_BYTES);
     if (attr_err != cudaSuccess) return attr_err;
     uint64_t b_rows;
     KParams p = make_params(a, GEMM, &b_rows);

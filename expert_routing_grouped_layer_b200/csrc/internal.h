@@ -33,12 +33,23 @@ struct WsLayout {
     size_t h_scale;       // uint8 E8M0 [(N+S*T)][I/32]
     size_t y;             // bf16 [N][H]
     size_t shared_y;      // bf16 [S][T][H]
+    size_t x_norm;        // bf16 [T][H] RMSNorm output (layer calls with the prologue)
     size_t total;
     int router_splits;
     int n_chunks;
 };
 
 bool config_valid(const moe_config* c);
+// Raises a kernel's opt-in dynamic shared-memory limit on the current device,
+// once per (kernel, device) pair; later calls return the first call's result.
+cudaError_t ensure_smem_limit(const void* kernel, int bytes);
+// Status of a launch error: MOE_ERR_UNSUPPORTED for an operation the device or
+// driver does not support, MOE_ERR_CUDA for any other failure.
+inline moe_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return MOE_OK;
+    if (e == cudaErrorNotSupported) return MOE_ERR_UNSUPPORTED;
+    return MOE_ERR_CUDA;
+}
 moe_status config_supported(const moe_config* c);
 WsLayout ws_layout(const moe_config* c, int T);
 int num_sms();
@@ -66,6 +77,16 @@ cudaError_t launch_rows_to_f16(void* rows, int C, int n_rows, int8_t* xs, cudaSt
 inline bool f16_gate_up(const moe_config* c) {
     return c->wfmt == MOE_W_FP8_E4M3_B128x128 && c->afmt == MOE_A_BF16;
 }
+// Post-attention RMSNorm (double arithmetic, one bf16 rounding) of x bf16
+// [T][H] with weight w fp32 [H] into xn bf16 [T][H]; for a quantised afmt also
+// E4M3 rows q [T][H] and E8M0 scales qs [T][H/32] of xn in one pass.
+cudaError_t launch_rmsnorm_quant(int afmt, const void* x, int H, const float* w, float eps, int T,
+                                 void* xn, void* q, uint8_t* qs, cudaStream_t st);
+// 8-bit token rows [T][H] with their per-32 scale rows [T][H/32] gathered into
+// expert order: out row r < N is token sorted_pair[r] / k (H % 512 == 0).
+cudaError_t launch_gather_token_rows(const void* rows, const uint8_t* scales, int H,
+                                     const int32_t* sorted_pair, int N, int k, int T, void* out,
+                                     uint8_t* out_scale, cudaStream_t st);
 cudaError_t launch_combine(const void* y, const void* shared_y, int S, const int32_t* row_of,
                            const float* w, int T, int k, int H, void* out, cudaStream_t st);
 // one warp waits on a barrier nothing arrives on until the pipeline wait limit;

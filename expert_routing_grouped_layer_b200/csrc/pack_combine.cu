@@ -377,6 +377,116 @@ __global__ void __launch_bounds__(128) combine_kernel(const __nv_bfloat16* __res
     *reinterpret_cast<uint4*>(out + (size_t)t * H + (size_t)v * 8) = o;
 }
 
+// Post-attention RMSNorm fused with the expert-input quantisation: the prologue
+// in front of the router ("DeepSeek V3架构拆解：Kimi-K2-Thinking-NVFP4的MLA注意力
+// 与MoE路由实现原理", 三: the decoder layer runs post_attention_layernorm then the
+// MoE block; "DeepSeek-V4-Pro 架构与代码概述", 文件说明: model.py RMSNorm keeps its
+// weight in fp32, kernel.py act_quant_kernel quantises the activations).
+// Row t: r = 1 / sqrt(sum_h x_h^2 / H + eps) and xn_h = bf16((x_h * r) * w_h),
+// every step in double and one round-to-nearest-even to bf16, so the bf16
+// decision is taken at a precision where only values within ~2^-40 of a
+// rounding midpoint can depend on the order of the sum. With a quantised
+// activation format the same pass also writes the row's E4M3 codes and E8M0
+// scales (per 32 elements; a 128-element block's code repeated over its four
+// sub-blocks), by the rule pack_fp8_kernel applies, computed from the bf16 xn.
+// One warp per row, two passes over it (sum of squares, then normalise); the
+// second reads the row again from L2. Lane l covers 8 consecutive elements
+// per 256-element step: a 128-element block is 16 lanes, a 32-element one 4.
+template <int AFMT>
+__global__ void __launch_bounds__(256) rmsnorm_quant_kernel(const uint4* __restrict__ x, int H,
+                                                            const float4* __restrict__ w,
+                                                            double eps, int T,
+                                                            uint4* __restrict__ xn,
+                                                            uint2* __restrict__ q,
+                                                            uint8_t* __restrict__ qs) {
+    pdl_wait();
+    pdl_trigger();
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (t >= T) return;
+    const int H8 = H / 8;
+    const uint4* row = x + (size_t)t * H8;
+    double ss = 0.0;
+    int v = lane;
+    for (; v + 96 < H8; v += 128) {
+        const uint4 u[4] = {row[v], row[v + 32], row[v + 64], row[v + 96]};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&u[j]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 f = __bfloat1622float2(b[i]);
+                ss = fma((double)f.x, (double)f.x, ss);
+                ss = fma((double)f.y, (double)f.y, ss);
+            }
+        }
+    }
+    for (; v < H8; v += 32) {
+        const uint4 u = row[v];
+        const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(b[i]);
+            ss = fma((double)f.x, (double)f.x, ss);
+            ss = fma((double)f.y, (double)f.y, ss);
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    const double r = 1.0 / sqrt(ss / (double)H + eps);
+    uint4* orow = xn + (size_t)t * H8;
+    for (int base = 0; base < H8; base += 32) {  // every lane runs every step (shuffles below)
+        const int vv = base + lane;
+        const bool act = vv < H8;
+        uint4 u = make_uint4(0, 0, 0, 0);
+        float4 w0 = make_float4(0.f, 0.f, 0.f, 0.f), w1 = w0;
+        if (act) {
+            u = row[vv];
+            w0 = w[2 * vv];
+            w1 = w[2 * vv + 1];
+        }
+        const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&u);
+        uint4 o;
+        __nv_bfloat16* ob = reinterpret_cast<__nv_bfloat16*>(&o);
+        float f[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 p = __bfloat1622float2(b[i]);
+            ob[2 * i] = __double2bfloat16(((double)p.x * r) * (double)wv[2 * i]);
+            ob[2 * i + 1] = __double2bfloat16(((double)p.y * r) * (double)wv[2 * i + 1]);
+            f[2 * i] = __bfloat162float(ob[2 * i]);
+            f[2 * i + 1] = __bfloat162float(ob[2 * i + 1]);
+        }
+        if (act) orow[vv] = o;
+        if (AFMT != MOE_A_BF16) {
+            constexpr int LANES = (AFMT == MOE_A_FP8_E4M3_POW2_B128) ? 16 : 4;  // lanes per block
+            float amax = 0.f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+#pragma unroll
+            for (int off = LANES / 2; off > 0; off >>= 1)
+                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+            int e = (AFMT == MOE_A_FP8_E4M3_POW2_B128) ? pow2_scale_exp(amax) : mx_scale_exp(amax);
+            e = min(max(e, -127), 127);
+            const float inv = __uint_as_float((uint32_t)(127 - e) << 23);  // 2^-e, e in [-127, 126]
+            uint32_t pk[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const __nv_fp8x2_storage_t a = __nv_cvt_float2_to_fp8x2(
+                    make_float2(f[4 * h] * inv, f[4 * h + 1] * inv), __NV_SATFINITE, __NV_E4M3);
+                const __nv_fp8x2_storage_t c = __nv_cvt_float2_to_fp8x2(
+                    make_float2(f[4 * h + 2] * inv, f[4 * h + 3] * inv), __NV_SATFINITE, __NV_E4M3);
+                pk[h] = (uint32_t)a | ((uint32_t)c << 16);
+            }
+            if (act) {
+                q[(size_t)t * H8 + vv] = make_uint2(pk[0], pk[1]);
+                if ((lane & 3) == 0) qs[(size_t)t * (H / 32) + vv / 4] = (uint8_t)(e + 127);
+            }
+        }
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_pack_rows(int afmt, const void* x, int H, const int32_t* sorted_pair, int N,
@@ -461,6 +571,36 @@ cudaError_t launch_combine(const void* y, const void* shared_y, int S, const int
         launch_pdl(combine_kernel<20>, grid, 128, 0, st, yy, sy, S, row_of, w, T, k, H, o);
     else
         launch_pdl(combine_kernel<36>, grid, 128, 0, st, yy, sy, S, row_of, w, T, k, H, o);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rmsnorm_quant(int afmt, const void* x, int H, const float* w, float eps, int T,
+                                 void* xn, void* q, uint8_t* qs, cudaStream_t st) {
+    if (T == 0) return cudaSuccess;
+    const unsigned grid = (unsigned)((T + 7) / 8);
+    const auto* xx = static_cast<const uint4*>(x);
+    const auto* ww = reinterpret_cast<const float4*>(w);
+    auto* o = static_cast<uint4*>(xn);
+    auto* qq = static_cast<uint2*>(q);
+    if (afmt == MOE_A_FP8_E4M3_POW2_B128)
+        launch_pdl(rmsnorm_quant_kernel<MOE_A_FP8_E4M3_POW2_B128>, grid, 256, 0, st, xx, H, ww,
+            (double)eps, T, o, qq, qs);
+    else if (afmt == MOE_A_MXFP8)
+        launch_pdl(rmsnorm_quant_kernel<MOE_A_MXFP8>, grid, 256, 0, st, xx, H, ww, (double)eps, T, o,
+            qq, qs);
+    else
+        launch_pdl(rmsnorm_quant_kernel<MOE_A_BF16>, grid, 256, 0, st, xx, H, ww, (double)eps, T, o,
+            qq, qs);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather_token_rows(const void* rows, const uint8_t* scales, int H,
+                                     const int32_t* sorted_pair, int N, int k, int T, void* out,
+                                     uint8_t* out_scale, cudaStream_t st) {
+    if (N == 0) return cudaSuccess;
+    launch_pdl(gather_rows_kernel, (N + 7) / 8, 256, 0, st, static_cast<const uint4*>(rows), 0,
+        H / 16, reinterpret_cast<const uint4*>(scales), H / 32 / 16, sorted_pair, N, k, T, N,
+        static_cast<uint4*>(out), reinterpret_cast<uint4*>(out_scale), nullptr, nullptr);
     return cudaGetLastError();
 }
 

@@ -311,5 +311,5 @@ extern "C" moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* 
                                          cfg->n_routed_experts, n_chunks, counts, expert_offsets,
                                          sorted_pair, row_of, dev_status,
                                          static_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return cuda_status(e);
 }

@@ -289,12 +289,8 @@ RouterPlan router_plan(int T, int E, int H) {
 cudaError_t launch_router_tc(const void* x, const float* gate_w, void* planes, float* part, int T,
                              int E, int H, int32_t* status, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        RT_SMEM_BYTES);
-    });
+    const cudaError_t attr_err =
+        ensure_smem_limit(reinterpret_cast<const void*>(router_tc_kernel), RT_SMEM_BYTES);
     if (attr_err != cudaSuccess) return attr_err;
     const RouterPlan plan = router_plan(T, E, H);
     const long n = (long)plan.Epad * H;

@@ -165,6 +165,28 @@ def make_inputs(cfg: MoEConfig, device="cpu"):
             "gate_bias": bias.float().contiguous()}
 
 
+# Input recipe of the prologue (the post-attention RMSNorm in front of the
+# layer): the hidden state before the norm is the workload's x with every row
+# scaled by 2^u * (1 + v), u uniform on the integers -6..6 and v ~ U[0, 1), so
+# rows span about four decades of magnitude; the norm weight is drawn
+# N(1, 0.2) in fp32; eps = 1e-6.
+PRENORM_EPS = 1e-6
+PRENORM_WEIGHT_STD = 0.2
+
+
+def make_prenorm_inputs(cfg: MoEConfig, x: torch.Tensor):
+    """(x_resid bf16 [T,H], norm_w fp32 [H], eps) for the prologue, drawn from
+    the workload's own x (same device) and the config's seed."""
+    dev = x.device
+    g = _gen(cfg, dev, 7)
+    T, H = x.shape
+    u = torch.randint(-6, 7, (T, 1), generator=g, device=dev).to(torch.float32)
+    v = torch.rand(T, 1, generator=g, device=dev)
+    x_resid = (x.float() * torch.exp2(u) * (1.0 + v)).to(torch.bfloat16).contiguous()
+    norm_w = (1.0 + PRENORM_WEIGHT_STD * torch.randn(H, generator=g, device=dev)).float().contiguous()
+    return x_resid, norm_w, PRENORM_EPS
+
+
 # ------------------------------------------------------------- weight encoding
 _E2M1_GRID = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)
 
@@ -290,7 +312,8 @@ def config_summary(cfg: MoEConfig) -> dict:
     return {k: v for k, v in dataclasses.asdict(cfg).items() if k != "description"}
 
 
-__all__ = ["MoEConfig", "CONFIGS", "make_inputs", "make_weights", "encode_weight", "expert_slice",
+__all__ = ["MoEConfig", "CONFIGS", "make_inputs", "make_prenorm_inputs", "make_weights",
+           "encode_weight", "expert_slice",
            "bf16_codes", "weight_bytes_per_matrix", "config_summary"]
 
 assert math.isclose(CONFIGS["k2_decode_bf16"].routed_scaling_factor, 2.827)

@@ -20,7 +20,8 @@
  *    moe_config and moe_weights structs themselves live in host memory and are
  *    read during the call only. The library never allocates, frees or
  *    synchronises; it keeps no state across calls except a per-device cache of
- *    the SM count and the set of kernels whose shared-memory limit was raised.
+ *    the SM count and the set of (kernel, device) pairs whose shared-memory limit
+ *    was raised.
  *  - `stream` is a cudaStream_t (NULL = legacy default stream). All work is
  *    enqueued on it in order; outputs are valid once the stream reaches them.
  *    Kernels are launched with programmatic stream serialization: one may be
@@ -31,8 +32,9 @@
  *    next on the same stream WITH programmatic serialization must itself wait
  *    (griddepcontrol.wait) before reading outputs; one launched without it, any
  *    copy, and any event or host synchronisation see finished results.
- *  - The shared-memory limit of a kernel is raised once per process, on the
- *    device current at the first call: drive one GPU per process.
+ *  - A kernel's shared-memory limit is raised on each device the first time
+ *    the kernel is launched there (the device current at the call), so one
+ *    process may drive several GPUs, switching with cudaSetDevice.
  *  - Arguments are checked on the host before anything is launched; a bad
  *    argument returns MOE_ERR_INVALID_ARG (or MOE_ERR_UNSUPPORTED for a valid
  *    but unimplemented combination, MOE_ERR_WORKSPACE for a short workspace)
@@ -264,10 +266,46 @@ moe_status moe_layer_forward(const moe_config *cfg, const void *x, int32_t T,
                              const moe_weights *w, void *out, void *ws, size_t ws_bytes,
                              int32_t *dev_status, void *stream);
 
+/* Post-attention RMSNorm fused with the expert-input quantisation: the
+ * prologue in front of the router ([V3] 三, the decoder layer: input_layernorm
+ * -> attention -> residual -> post_attention_layernorm -> MoE; [V4] 文件说明,
+ * model.py RMSNorm, its weight kept in fp32, and kernel.py act_quant_kernel).
+ *  x bf16 [T][H]: the hidden state after the attention residual (the norm's
+ *  input); norm_w fp32 [H]; eps >= 0 (finite).
+ *  x_norm bf16 [T][H]: per token r = 1 / sqrt(sum_h x_h^2 / H + eps) and
+ *  x_norm_h = (x_h * r) * norm_w_h, evaluated in double precision and rounded
+ *  once to bf16 (round to nearest even). The sum's order is the kernel's own,
+ *  so a value within ~2^-40 (relative) of a bf16 rounding midpoint may round
+ *  either way; every other value is fixed by the formula.
+ *  For afmt FP8_E4M3_POW2_B128 / MXFP8 the same pass writes the quantised rows
+ *  of x_norm: xq uint8 E4M3 [T][H] and xq_scale uint8 E8M0 [T][H/32] (one code
+ *  per 32 elements, the power-of-two format's per-128 code repeated over its
+ *  four sub-blocks -- the row layout moe_pack_expert_inputs writes), by the
+ *  rule of moe_quantize_activations; H must then be a multiple of 512. For
+ *  afmt BF16, xq and xq_scale are ignored (may be NULL).
+ *  All pointers 16-byte aligned. One read of x, writes of x_norm (and xq). */
+moe_status moe_rmsnorm_prologue(const moe_config *cfg, const void *x, int32_t T,
+                                const float *norm_w, float eps, void *x_norm, void *xq,
+                                void *xq_scale, void *stream);
+
+/* The whole layer from the un-normalised hidden state: moe_rmsnorm_prologue,
+ * then the router and top-k on x_norm, the permutation, the expert-input
+ * gather (quantised activations: a byte gather of the rows the prologue
+ * quantised; bf16 activations: the inputs built from x_norm as in
+ * moe_pack_expert_inputs), the expert GEMMs and the combine. Equal to
+ * moe_layer_forward applied to the prologue's x_norm.
+ *  x bf16 [T][H] -> out bf16 [T][H]; norm_w fp32 [H]; ws >= moe_workspace_bytes
+ *  (which includes the x_norm buffer, offset selector 11). */
+moe_status moe_layer_forward_prenorm(const moe_config *cfg, const void *x, int32_t T,
+                                     const float *norm_w, float eps, const moe_weights *w,
+                                     void *out, void *ws, size_t ws_bytes, int32_t *dev_status,
+                                     void *stream);
+
 /* Byte offsets inside the workspace of the intermediate results that
  * moe_layer_forward leaves there (for inspection, tests and step-by-step use):
  *  which = 0 topk_idx, 1 topk_w, 2 expert_offsets, 3 sorted_pair, 4 row_of,
- *          5 y, 6 shared_y, 7 xa, 8 xa_scale, 9 h, 10 h_scale.
+ *          5 y, 6 shared_y, 7 xa, 8 xa_scale, 9 h, 10 h_scale,
+ *          11 x_norm (moe_layer_forward_prenorm's RMSNorm output).
  *  Returns (size_t)-1 for an invalid config or which. */
 size_t moe_workspace_offset(const moe_config *cfg, int32_t T, int32_t which);
 

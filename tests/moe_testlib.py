@@ -85,3 +85,69 @@ def oracle_layer_rows(cfg, inp, wts, idx, w, tokens):
 
 def rel_l2(a, b):
     return float(np.linalg.norm(a - b) / np.linalg.norm(b))
+
+
+def rel_l2_rows(a, b):
+    """Relative L2 error of every row (token) separately."""
+    return np.linalg.norm(a - b, axis=1) / np.maximum(np.linalg.norm(b, axis=1), 1e-300)
+
+
+def compare_permutation_exact(cfg, g, r):
+    """The GPU permutation against the oracle's (the oracle's stable sort of its
+    own routing), element by element: offsets, sorted_pair and row_of in full when
+    no token is a near-tie, else the block of every expert that no near-tie token
+    (by either side's choice) touches. Returns the number of experts compared."""
+    E = cfg.n_routed_experts
+    off, sp, ro = oracle.permute(r["idx"], E)
+    tie = np.nonzero(r["near_tie"])[0]
+    if tie.size == 0:
+        assert np.array_equal(g["offsets"], off)
+        assert np.array_equal(g["sorted_pair"], sp)
+        assert np.array_equal(g["row_of"], ro)
+        return E
+    touched = set(g["idx"][tie].ravel().tolist()) | set(r["idx"][tie].ravel().tolist())
+    n = 0
+    for e in range(E):
+        if e in touched:
+            continue
+        a = g["sorted_pair"][g["offsets"][e]:g["offsets"][e + 1]]
+        b = sp[off[e]:off[e + 1]]
+        assert np.array_equal(a, b), "expert %d block differs" % e
+        n += 1
+    return n
+
+
+def chosen_tokens(cfg, g, r, sample, seed):
+    """Tokens whose layer output is checked one by one: a seeded random sample,
+    plus tokens at the places where tiles end raggedly -- the first and last
+    rows of the most loaded expert's block (its last, partial token tile), the
+    rows of the least loaded non-empty expert (a one-token expert when there is
+    one), the last rows of the last non-empty expert, and the first and last
+    tokens (the shared experts' rows run in token order, so these sit in the
+    shared segment's first and last tiles). Near-tie tokens are left out."""
+    T, k = len(g["idx"]), cfg.num_experts_per_tok
+    counts = np.diff(g["offsets"])
+    sp = g["sorted_pair"]
+    rows = []
+    hot = int(counts.argmax())
+    rows += [g["offsets"][hot], g["offsets"][hot + 1] - 2, g["offsets"][hot + 1] - 1]
+    nz = np.nonzero(counts)[0]
+    cold = int(nz[counts[nz].argmin()])
+    rows += list(range(g["offsets"][cold], g["offsets"][cold + 1]))[:2]
+    last = int(nz[-1])
+    rows += [g["offsets"][last + 1] - 1]
+    toks = {int(sp[x]) // k for x in rows if 0 <= x < len(sp)}
+    toks |= {0, T - 1, max(0, T - 2)}
+    rng = np.random.default_rng(seed)
+    toks |= set(rng.choice(T, min(sample, T), replace=False).tolist())
+    toks = np.array(sorted(t for t in toks if not r["near_tie"][t]), dtype=np.int64)
+    return toks
+
+
+def check_layer_tokens(cfg, inp, wts, g, r, toks, tol):
+    """Per-token rel-L2 of the GPU output against the oracle (its own routing)
+    on the listed tokens: the largest must be within tol. Returns the errors."""
+    want = oracle_layer_rows(cfg, inp, wts, r["idx"][toks], r["w"][toks], toks)
+    err = rel_l2_rows(g["out"][toks], want)
+    assert err.max() <= tol, (float(err.max()), int(toks[err.argmax()]))
+    return err

@@ -122,7 +122,8 @@ def test_workspace_grows_with_tokens_and_offsets_fit(lib):
             W.CONFIGS[name].n_shared_experts
         assert moe.moe_workspace_offset(c, T, 5) + T * k * H * 2 <= total
         assert moe.moe_workspace_offset(c, T, 6) + S * T * H * 2 <= total
-        assert moe.moe_workspace_offset(c, T, 11) == 2 ** 64 - 1
+        assert moe.moe_workspace_offset(c, T, 11) + T * H * 2 <= total  # x_norm
+        assert moe.moe_workspace_offset(c, T, 12) == 2 ** 64 - 1
 
 
 def test_fp8_weight_steps_need_h_scale_and_the_workspace_holds_it(lib):
@@ -141,6 +142,39 @@ def test_fp8_weight_steps_need_h_scale_and_the_workspace_holds_it(lib):
     total = moe.moe_workspace_bytes(c, T)
     hs = moe.moe_workspace_offset(c, T, 10)
     assert hs != 2 ** 64 - 1 and hs + N + S * T <= total
+
+
+def test_prologue_arguments_are_checked_on_the_host(lib):
+    """The RMSNorm prologue and the layer from the un-normalised hidden state
+    reject bad eps, null or misaligned pointers and a short workspace before
+    launching; quantised formats need their code and scale rows and H % 512.
+    Every call here is refused (or has T = 0), so none reaches a kernel."""
+    c = cfg()
+    f = ctypes.c_float
+    ok = lambda *a: lib.moe_rmsnorm_prologue(ctypes.byref(c), *a)
+    assert ok(256, 64, 256, f(-1.0), 256, None, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert ok(256, 64, 256, f(float("inf")), 256, None, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert ok(256, 64, 256, f(float("nan")), 256, None, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert ok(None, 64, 256, f(1e-6), 256, None, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert ok(256, 64, 8, f(1e-6), 256, None, None, None) == moe.MOE_ERR_INVALID_ARG  # misaligned w
+    assert ok(256, 0, None, f(1e-6), None, None, None, None) == moe.MOE_OK
+    cq = cfg(afmt="mxfp8", wfmt="mxfp4", hidden=512, moe_intermediate_size=512,
+             shared_intermediate_size=512)
+    assert lib.moe_rmsnorm_prologue(ctypes.byref(cq), 256, 4, 256, f(1e-6), 256, None, 256,
+                                    None) == moe.MOE_ERR_INVALID_ARG  # no code rows
+    c256 = cfg(afmt="mxfp8", wfmt="mxfp4", hidden=256)
+    assert lib.moe_rmsnorm_prologue(ctypes.byref(c256), 256, 4, 256, f(1e-6), 256, 256, 256,
+                                    None) == moe.MOE_ERR_INVALID_ARG  # H % 512
+    need = moe.moe_workspace_bytes(c, 64)
+    w = moe.moe_weights(256, None, 256, None, 256, None, 256, None, 256, 256)
+    lf = lambda *a: lib.moe_layer_forward_prenorm(ctypes.byref(c), *a)
+    assert lf(256, 64, 256, f(1e-6), ctypes.byref(w), 256, 256, need - 1, None, None) == \
+        moe.MOE_ERR_WORKSPACE
+    assert lf(256, 64, None, f(1e-6), ctypes.byref(w), 256, 256, need, None, None) == \
+        moe.MOE_ERR_INVALID_ARG
+    assert lf(256, 64, 256, f(-1e-6), ctypes.byref(w), 256, 256, need, None, None) == \
+        moe.MOE_ERR_INVALID_ARG
+    assert lf(None, 0, None, f(1e-6), ctypes.byref(w), None, None, 0, None, None) == moe.MOE_OK
 
 
 def test_status_strings(lib):

@@ -79,3 +79,36 @@ def test_launch_count_matches_the_launch_lists(name, count):
     to 4096 pairs; two-pass packs; the FP8-weight h repack)."""
     cfg = W.CONFIGS[name]
     assert bench.launches_per_step(cfg, cfg.T, 148) == count
+
+
+def test_tensor_peak_prefers_a_measured_fp8_rate():
+    """Block-scaled layers take the best FP8 cuBLAS rate measured in the run;
+    failed measurements (error strings) are ignored."""
+    peaks = {"bf16_tflops": 1651.4}
+    meas = {"fp8_e4m3_tensorwise": 3000.0, "mxfp8_block32": 3100.0,
+            "nvfp4_block16_error": "not supported"}
+    p, src = bench.tensor_peak(peaks, "measured", W.CONFIGS["v4_fp4"], meas)
+    assert p == 3100.0 and "mxfp8_block32" in src
+    # bf16-rate layers keep the bf16 figure
+    p, _ = bench.tensor_peak(peaks, "measured", W.CONFIGS["k2_prefill_fp8w"], meas)
+    assert p == 1651.4
+
+
+def test_roofline_flags_fractions_above_the_measured_peak():
+    # 7 GB in 1 ms = 7000 GB/s: above the measured copy rate, below the datasheet
+    r = bench.roofline(7e9, 1e9, 1.0, 6542.4, 1651.4)
+    assert r["bound"] == "hbm" and r["above_measured_peak"]
+    assert r["frac_of_nominal_hbm"] == pytest.approx(7000.0 / bench.NOMINAL_HBM_GBS)
+    r = bench.roofline(6e9, 1e9, 1.0, 6542.4, 1651.4)
+    assert not r["above_measured_peak"]
+
+
+def test_both_arms_build_the_config_from_one_function():
+    """The CUDA arm and the reference arm print the same config dict for a
+    workload: both take it from workload_config, unchanged."""
+    import inspect
+    src = inspect.getsource(bench.measure) + inspect.getsource(bench.run_reference)
+    assert src.count("workload_config(cfg, world)") == 2
+    assert "cfgd[" not in src
+    d = bench.workload_config(W.CONFIGS["mx896"], 1)
+    assert d["T"] == 16384 and d["experts"] == 896 and d["weights"] == "mxfp4"

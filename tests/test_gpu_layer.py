@@ -7,8 +7,8 @@ import torch
 import expert_routing_grouped_layer_b200 as moe
 import oracle
 from expert_routing_grouped_layer_b200 import workloads as W
-from moe_testlib import (LAYER_TOL, check_permutation_properties, compare_routing, gpu_forward,
-                         oracle_layer_rows, oracle_route, rel_l2)
+from moe_testlib import (LAYER_TOL, check_layer_tokens, check_permutation_properties,
+                         compare_permutation_exact, compare_routing, gpu_forward, oracle_route)
 
 pytestmark = pytest.mark.gpu
 
@@ -19,24 +19,19 @@ def _data(cfg):
     return inp, wts
 
 
-def _full_check(cfg, inp, wts, T=None, exact_perm=True):
+def _full_check(cfg, inp, wts, T=None):
+    """Routing of every token (sets and weights, near-ties excepted), the
+    permutation element by element, and every token's output against the oracle."""
     T = cfg.T if T is None else T
     g = gpu_forward(cfg, inp, wts, T)
     assert g["status"] == 0
     r = oracle_route(cfg, inp, T=T)
-    toks = np.arange(T)
-    n_tie = compare_routing(cfg, g, r, toks)
+    compare_routing(cfg, g, r, np.arange(T))
     check_permutation_properties(cfg, g, T)
-    if exact_perm and n_tie == 0 and np.array_equal(g["idx"], r["idx"]):
-        off, sp, ro = oracle.permute(r["idx"], cfg.n_routed_experts)
-        assert np.array_equal(g["offsets"], off)
-        assert np.array_equal(g["sorted_pair"], sp)
-        assert np.array_equal(g["row_of"], ro)
-    ok = ~r["near_tie"]
-    want = oracle_layer_rows(cfg, inp, wts, r["idx"], r["w"], toks)
-    err = rel_l2(g["out"][ok], want[ok])
-    assert err <= LAYER_TOL[cfg.afmt], err
-    return g, r, err
+    compare_permutation_exact(cfg, g, r)
+    toks = np.nonzero(~r["near_tie"])[0]
+    err = check_layer_tokens(cfg, inp, wts, g, r, toks, LAYER_TOL[cfg.afmt])
+    return g, r, float(err.max())
 
 
 def test_tiny_layer_full_parity():
@@ -106,6 +101,8 @@ def test_tiny_larger_shapes_span_tiles():
 
 
 def test_decode_bf16_full_size():
+    """The decode layer at full size: routing of all 128 tokens, the permutation
+    element by element, and the output of every token against the oracle."""
     cfg = W.CONFIGS["k2_decode_bf16"]
     inp, wts = _data(cfg)
     g = gpu_forward(cfg, inp, wts)
@@ -113,17 +110,11 @@ def test_decode_bf16_full_size():
     r = oracle_route(cfg, inp)  # routing of every token
     compare_routing(cfg, g, r, np.arange(cfg.T))
     check_permutation_properties(cfg, g)
-    if not r["near_tie"].any() and np.array_equal(g["idx"], r["idx"]):
-        off, sp, ro = oracle.permute(r["idx"], cfg.n_routed_experts)
-        assert np.array_equal(g["sorted_pair"], sp) and np.array_equal(g["offsets"], off)
+    compare_permutation_exact(cfg, g, r)
     active = int((np.diff(g["offsets"]) > 0).sum())
     assert 100 <= active <= 384
-    # layer output on a seeded sample of tokens
-    toks = np.sort(np.random.default_rng(0).choice(cfg.T, 12, replace=False))
-    ok = ~r["near_tie"][toks]
-    want = oracle_layer_rows(cfg, inp, wts, r["idx"][toks], r["w"][toks], toks)
-    err = rel_l2(g["out"][toks][ok], want[ok])
-    assert err <= LAYER_TOL["bf16"], err
+    toks = np.nonzero(~r["near_tie"])[0]
+    check_layer_tokens(cfg, inp, wts, g, r, toks, LAYER_TOL["bf16"])
 
 
 def test_step_entry_points_match_layer():
@@ -197,3 +188,45 @@ def test_softmax_scoring_wide_expert_counts(E, k):
     g, r, _ = _full_check(cfg, inp, wts)
     ok = ~r["near_tie"]
     assert (np.abs(g["w"][ok] - r["w"][ok]) <= 1e-5 * np.abs(r["w"][ok])).all()
+
+
+_REORDER_CASES = {
+    # several token tiles per expert with ragged ends, several M tiles
+    "bf16": W.CONFIGS["tiny_bf16"].replace(T=700, hidden=512, moe_intermediate_size=256,
+                                           shared_intermediate_size=256, n_routed_experts=8,
+                                           num_experts_per_tok=3),
+    "fp8w": W.CONFIGS["tiny_bf16"].replace(T=700, hidden=512, moe_intermediate_size=256,
+                                           shared_intermediate_size=256, n_routed_experts=8,
+                                           num_experts_per_tok=3, n_shared_experts=2,
+                                           wfmt="fp8_e4m3_b128x128"),
+    "fp4": W.CONFIGS["tiny_bf16"].replace(T=700, hidden=1024, moe_intermediate_size=512,
+                                          shared_intermediate_size=512, n_routed_experts=8,
+                                          num_experts_per_tok=3, wfmt="fp4_e2m1_ue8m0_b32",
+                                          afmt="fp8_e4m3_pow2_b128", score_fn="sqrtsoftplus",
+                                          routed_scaling_factor=2.5),
+    "mx": W.CONFIGS["tiny_bf16"].replace(T=700, hidden=1024, moe_intermediate_size=512,
+                                         shared_intermediate_size=512, n_routed_experts=8,
+                                         num_experts_per_tok=3, wfmt="mxfp4", afmt="mxfp8",
+                                         n_shared_experts=2),
+    "decode_full": W.CONFIGS["k2_decode_bf16"],
+}
+
+
+@pytest.mark.parametrize("name", list(_REORDER_CASES))
+def test_token_order_permutes_output_bit_for_bit(name):
+    """Each token's output depends on that token alone ([V3] 三.4: every token is
+    routed and combined on its own): at a fixed token count, feeding the tokens
+    in another order must give the same rows in that order, bit for bit. The
+    tokens land in other tiles and at other rows of them, so this checks that
+    no kernel lets a row's arithmetic depend on its neighbours or its place."""
+    cfg = _REORDER_CASES[name]
+    inp, wts = _data(cfg)
+    T = cfg.T
+    layer = moe.MoELayer(cfg, wts, inp["gate_w"], inp["gate_bias"], max_tokens=T, device="cuda")
+    out = layer.forward(inp["x"]).clone()
+    g = torch.Generator(device="cpu").manual_seed(17)
+    perm = torch.randperm(T, generator=g).to("cuda")
+    out_p = layer.forward(inp["x"][perm].contiguous()).clone()
+    torch.cuda.synchronize()
+    assert layer.status.item() == 0
+    assert torch.equal(out_p.view(torch.int16), out[perm].view(torch.int16))

@@ -62,11 +62,25 @@ def test_no_alloc_permute_matches_workspace_version_twice():
 
 @pytest.mark.gpu
 def test_no_alloc_permute_rejects_sizes_past_its_array():
+    """One chunk past the array's limit is refused on the host before any launch.
+    The buffers are real and full-sized, and topk_idx holds valid expert ids, so
+    even a broken size check would only produce a wrong status, never a bad
+    address."""
     cfg = W.CONFIGS["mx896"]  # 896 experts: the array holds 292 chunks of 4096 pairs
     k, E = cfg.num_experts_per_tok, cfg.n_routed_experts
     T = (moe.MOE_PERMUTE_NOALLOC_MAX_COUNTS // E + 1) * 4096 // k
+    idx = _routing(T, k, E, 3)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    off = torch.full((E + 1,), -9, dtype=torch.int32, device="cuda")
+    sp = torch.full((T * k,), -9, dtype=torch.int32, device="cuda")
+    ro = torch.full((T * k,), -9, dtype=torch.int32, device="cuda")
     c = moe.make_config(cfg)
-    s = moe.lib().moe_permute_noalloc(ctypes.byref(c), 256, T, 256, 256, 256, None, None)
+    s = moe.lib().moe_permute_noalloc(ctypes.byref(c), idx.data_ptr(), T, off.data_ptr(),
+                                      sp.data_ptr(), ro.data_ptr(), st.data_ptr(),
+                                      torch.cuda.current_stream().cuda_stream)
     assert s == moe.MOE_ERR_WORKSPACE
     with pytest.raises(moe.MoEError, match="workspace too small"):
-        moe.moe_permute_noalloc(cfg, 256, T, 256, 256, 256, None)
+        moe.moe_permute_noalloc(cfg, idx, T, off, sp, ro, st)
+    torch.cuda.synchronize()
+    # nothing was launched: every output still holds its fill value
+    assert (off == -9).all() and (sp == -9).all() and (ro == -9).all() and st.item() == 0
