@@ -38,8 +38,8 @@ _SO = os.path.join(_HERE, "libmoe_oracle.so")
 _lock = threading.Lock()
 _lib = None
 
-W_FMT = {"bf16": 0, "fp8_e4m3_b128x128": 1, "fp4_e2m1_ue8m0_b32": 2, "mxfp4": 3}
-A_FMT = {"bf16": 0, "fp8_e4m3_pow2_b128": 1, "mxfp8": 2}
+W_FMT = {"bf16": 0, "fp8_e4m3_b128x128": 1, "fp4_e2m1_ue8m0_b32": 2, "mxfp4": 3, "nvfp4": 4}
+A_FMT = {"bf16": 0, "fp8_e4m3_pow2_b128": 1, "mxfp8": 2, "nvfp4": 3}
 SCORE = {"sigmoid": 0, "sqrtsoftplus": 1, "softmax": 2}
 NEAR_TIE_REL = 1e-6  # relative score gap under which a selection counts as a near-tie
 
@@ -84,9 +84,9 @@ def lib() -> ctypes.CDLL:
             l.or_weight_value.restype = _D
             l.or_weight_value.argtypes = [_I, _P, _P, _I, _I, _I, _I, _I]
             l.or_route_token.restype = _I
-            l.or_route_token.argtypes = [_P, _D, _P, _P, _P, _D, _P, _P, _P, _P, _P]
+            l.or_route_token.argtypes = [_P, _D, _P, _P, _P, _D, _P, _P, _P, _P, _P, _P]
             l.or_route.restype = _I
-            l.or_route.argtypes = [_P, _D, _P, _I, _P, _I, _P, _P, _D, _P, _P, _P, _P]
+            l.or_route.argtypes = [_P, _D, _P, _I, _P, _I, _P, _P, _D, _P, _P, _P, _P, _P]
             l.or_permute.restype = _I
             l.or_permute.argtypes = [_P, _I, _I, _I, _P, _P, _P]
             l.or_expert_input.restype = _I
@@ -95,6 +95,17 @@ def lib() -> ctypes.CDLL:
             l.or_expert_rows.argtypes = [_I, _I, _P, _P, _P, _P, _I, _I, _I, _P, _I, _D, _P]
             l.or_combine.restype = None
             l.or_combine.argtypes = [_I, _I, _I, _I, _P, _P, _P, _P]
+            l.or_e2m1_encode.restype = ctypes.c_uint8
+            l.or_e2m1_encode.argtypes = [_D]
+            l.or_quant_nvfp4.restype = _I
+            l.or_quant_nvfp4.argtypes = [_P, _I, _D, _P, _P]
+            l.or_dequant_nvfp4.restype = _I
+            l.or_dequant_nvfp4.argtypes = [_P, _P, _I, _D, _P]
+            l.or_weight_value_nvfp4.restype = _D
+            l.or_weight_value_nvfp4.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I]
+            l.or_expert_rows_nvfp4.restype = _I
+            l.or_expert_rows_nvfp4.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _I, _D, _D,
+                                               _P]
             l.or_bf16_encode.restype = ctypes.c_uint16
             l.or_bf16_encode.argtypes = [_D, _D, _P]
             l.or_rmsnorm.restype = _I
@@ -209,6 +220,77 @@ def rmsnorm(x_u16, w, eps: float, tie_rel: float = RMSNORM_TIE_REL):
     return out, near.astype(bool)
 
 
+def e2m1_encode(vals):
+    """Round doubles to E2M1 codes (RNE, saturating at +-6)."""
+    l = lib()
+    return np.array([l.or_e2m1_encode(float(v)) for v in np.ravel(vals)],
+                    dtype=np.uint8).reshape(np.shape(vals))
+
+
+def quant_nvfp4(v, g: float):
+    """NVFP4 quantisation of one vector with tensor scale g: (E2M1 codes uint8[n]
+    one per byte, E4M3 scale codes uint8[n/16])."""
+    v = _c(v, np.float64)
+    n = v.shape[0]
+    q = np.zeros(n, np.uint8)
+    sc = np.zeros(max(1, n // 16), np.uint8)
+    if lib().or_quant_nvfp4(_ptr(v), n, float(g), _ptr(q), _ptr(sc)) < 0:
+        raise ValueError("bad NVFP4 length or tensor scale")
+    return q, sc[: n // 16].copy()
+
+
+def dequant_nvfp4(q, sc, g: float):
+    q = _c(q, np.uint8)
+    sc = _c(sc, np.uint8)
+    out = np.zeros(q.shape[0], np.float64)
+    if lib().or_dequant_nvfp4(_ptr(q), _ptr(sc), q.shape[0], float(g), _ptr(out)) < 0:
+        raise ValueError("bad NVFP4 length")
+    return out
+
+
+def weight_value_nvfp4(w, s, g, rows: int, cols: int, e: int, r: int, c: int) -> float:
+    w = np.ascontiguousarray(w, np.uint8)
+    s = np.ascontiguousarray(s, np.uint8)
+    g = np.ascontiguousarray(g, np.float32)
+    return lib().or_weight_value_nvfp4(_ptr(w), _ptr(s), _ptr(g), rows, cols, e, r, c)
+
+
+def expert_input_nvfp4(x_rows_u16, g: float):
+    """Rows of bf16 x as an NVFP4 expert sees them: (dequantised float64 [n,H],
+    codes uint8 [n,H], scale codes uint8 [n,H/16])."""
+    x = bf16_value_rows(x_rows_u16)
+    n, H = x.shape
+    q = np.zeros((n, H), np.uint8)
+    sc = np.zeros((n, H // 16), np.uint8)
+    xin = np.zeros((n, H), np.float64)
+    for r in range(n):
+        q[r], sc[r] = quant_nvfp4(x[r], g)
+        xin[r] = dequant_nvfp4(q[r], sc[r], g)
+    return xin, q, sc
+
+
+def bf16_value_rows(x_rows_u16):
+    """float64 values of bf16 codes (exact: a bf16 code is the top half of a float32)."""
+    x = _c(x_rows_u16, np.uint16)
+    return (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def expert_rows_nvfp4(w13, w13s, g13, w2, w2s, g2, e: int, I: int, H: int, xin, ga2: float,
+                      limit: float = 0.0):
+    """SwiGLU of NVFP4 expert e on dequantised input rows xin [n, H] -> y [n, H];
+    the intermediate is NVFP4-quantised with tensor scale ga2."""
+    xin = _c(xin, np.float64)
+    n = xin.shape[0]
+    y = np.zeros((n, H), np.float64)
+    a = [np.ascontiguousarray(t) for t in (w13, w13s, g13, w2, w2s, g2)]
+    rc = lib().or_expert_rows_nvfp4(_ptr(a[0]), _ptr(a[1]), _ptr(_c(a[2], np.float32)), _ptr(a[3]),
+                                    _ptr(a[4]), _ptr(_c(a[5], np.float32)), e, I, H, _ptr(xin), n,
+                                    float(ga2), float(limit), _ptr(y))
+    if rc != 0:
+        raise ValueError("bad NVFP4 expert arguments")
+    return y
+
+
 # ----------------------------------------------------------------- config
 def icfg(cfg) -> np.ndarray:
     return np.array([cfg.hidden, cfg.n_routed_experts, cfg.num_experts_per_tok, cfg.n_group,
@@ -221,7 +303,9 @@ def icfg(cfg) -> np.ndarray:
 def route(cfg, x_u16, wg, bias, tokens=None, tie_rel: float = NEAR_TIE_REL):
     """Route tokens (all, or the listed ones). x_u16: [T, H] bf16 codes.
 
-    Returns dict idx int32[n,k], w float64[n,k], near_tie bool[n], gap float64[n].
+    Returns dict idx int32[n,k], w float64[n,k], near_tie bool[n], gap float64[n],
+    order_gap float64[n] (smallest relative gap between consecutive slots' s') and
+    order_tie bool[n] (order_gap below tie_rel: the slot order is a near-tie).
     """
     x_u16 = _c(x_u16, np.uint16)
     wg = _c(wg, np.float32)
@@ -234,13 +318,15 @@ def route(cfg, x_u16, wg, bias, tokens=None, tie_rel: float = NEAR_TIE_REL):
     w = np.zeros((n, k), np.float64)
     nt = np.zeros(n, np.uint8)
     gap = np.zeros(n, np.float64)
+    og = np.zeros(n, np.float64)
     ic = icfg(cfg)
     rc = lib().or_route(_ptr(ic), float(cfg.routed_scaling_factor), _ptr(x_u16), T, _ptr(toks), n,
                         _ptr(wg), _ptr(bias), float(tie_rel), _ptr(idx), _ptr(w), _ptr(nt),
-                        _ptr(gap))
+                        _ptr(gap), _ptr(og))
     if rc != 0:
         raise ValueError("oracle routing failed (code %d)" % rc)
-    return {"idx": idx, "w": w, "near_tie": nt.astype(bool), "gap": gap}
+    return {"idx": idx, "w": w, "near_tie": nt.astype(bool), "gap": gap, "order_gap": og,
+            "order_tie": og < tie_rel}
 
 
 def route_token(cfg, xrow_u16, wg, bias, tie_rel: float = NEAR_TIE_REL):
@@ -254,13 +340,15 @@ def route_token(cfg, xrow_u16, wg, bias, tie_rel: float = NEAR_TIE_REL):
     nt = np.zeros(1, np.uint8)
     gap = np.zeros(1, np.float64)
     logits = np.zeros(E, np.float64)
+    og = np.zeros(1, np.float64)
     ic = icfg(cfg)
     rc = lib().or_route_token(_ptr(ic), float(cfg.routed_scaling_factor), _ptr(xrow_u16), _ptr(wg),
                               _ptr(bias), float(tie_rel), _ptr(idx), _ptr(w), _ptr(nt), _ptr(gap),
-                              _ptr(logits))
+                              _ptr(logits), _ptr(og))
     if rc != 0:
         raise ValueError("oracle routing failed (code %d)" % rc)
-    return {"idx": idx, "w": w, "near_tie": bool(nt[0]), "gap": float(gap[0]), "logits": logits}
+    return {"idx": idx, "w": w, "near_tie": bool(nt[0]), "gap": float(gap[0]), "logits": logits,
+            "order_gap": float(og[0]), "order_tie": bool(og[0] < tie_rel)}
 
 
 def permute(idx, n_experts: int):
@@ -324,6 +412,33 @@ def combine(w, y, ys):
     out = np.zeros((n, H), np.float64)
     lib().or_combine(n, k, ys.shape[0], H, _ptr(w), _ptr(y), _ptr(ys), _ptr(out))
     return out
+
+
+def layer_nvfp4(cfg, x_rows_u16, idx, w, get_expert, get_shared, act_gscales):
+    """Layer output with NVFP4 routed experts ([V3] 四): get_expert(e) returns
+    (w13, w13_scale, w2, w2_scale, g13, g2) of that one matrix (leading dimension
+    1), act_gscales = (tensor scale of the experts' input, of their
+    intermediate); the shared experts stay bf16 (the page's exclusion list) and
+    read the bf16 input unquantised; get_shared(s) returns bf16 (w13, None, w2,
+    None)."""
+    H, I, Ish = cfg.hidden, cfg.moe_intermediate_size, cfg.shared_intermediate_size
+    idx = np.asarray(idx)
+    n, k = idx.shape
+    ga13, ga2 = act_gscales
+    xin, _, _ = expert_input_nvfp4(x_rows_u16, ga13)
+    lim = float(getattr(cfg, "swiglu_limit", 0.0))
+    y = np.zeros((n, k, H), np.float64)
+    for e in np.unique(idx):
+        rows, slots = np.nonzero(idx == e)
+        w13, w13s, w2, w2s, g13, g2 = get_expert(int(e))
+        y[rows, slots] = expert_rows_nvfp4(w13, w13s, g13, w2, w2s, g2, 0, I, H, xin[rows], ga2,
+                                           lim)
+    xb, _, _ = expert_input("bf16", x_rows_u16)
+    ys = np.zeros((cfg.n_shared_experts, n, H), np.float64)
+    for s_ in range(cfg.n_shared_experts):
+        w13, _, w2, _ = get_shared(s_)
+        ys[s_] = expert_rows("bf16", "bf16", w13, None, w2, None, 0, Ish, H, xb, lim)
+    return combine(w, y, ys)
 
 
 def layer(cfg, x_rows_u16, idx, w, get_expert, get_shared):

@@ -261,10 +261,13 @@ static double rel_gap(double a, double b) {
  * Slot order: s' descending, ties to the lower expert index.
  * near_tie is set when the k-th and (k+1)-th candidate s' (or the topk_group-th
  * and next group score) differ by less than tie_rel relatively; gap_out gets the
- * smallest such relative gap (or +inf when no competitor exists). */
+ * smallest such relative gap (or +inf when no competitor exists).
+ * order_gap_out (if given) gets the smallest relative gap between the s' of two
+ * consecutive slots (+inf for k = 1): below tie_rel the slot order of the
+ * chosen experts is a near-tie, though their set is not. */
 int or_route_token(const int *icfg, double rsf, const uint16_t *xrow, const float *wg,
                    const float *bias, double tie_rel, int32_t *idx, double *w, uint8_t *near_tie,
-                   double *gap_out, double *logits_out) {
+                   double *gap_out, double *logits_out, double *order_gap_out) {
     const int H = icfg[C_H], E = icfg[C_E], K = icfg[C_K], NG = icfg[C_NG], TG = icfg[C_TG];
     double *s = (double *)malloc(sizeof(double) * E);
     double *sp = (double *)malloc(sizeof(double) * E);
@@ -335,6 +338,12 @@ int or_route_token(const int *icfg, double rsf, const uint16_t *xrow, const floa
         gap = fmin(gap, rel_gap(sp[idx[K - 1]], sp[nxt]));
     }
 
+    if (order_gap_out) {
+        double og = INFINITY;
+        for (int j = 0; j + 1 < K; j++) og = fmin(og, rel_gap(sp[idx[j]], sp[idx[j + 1]]));
+        *order_gap_out = og;
+    }
+
     /* weights */
     double sum = 0.0;
     for (int j = 0; j < K; j++) {
@@ -357,7 +366,7 @@ done:
 /* Routing of a list of tokens (independent per token). */
 int or_route(const int *icfg, double rsf, const uint16_t *x, int T, const int32_t *tokens,
              int ntok, const float *wg, const float *bias, double tie_rel, int32_t *idx, double *w,
-             uint8_t *near_tie, double *gap) {
+             uint8_t *near_tie, double *gap, double *order_gap) {
     const int H = icfg[C_H], K = icfg[C_K];
     if (icfg[C_NG] < 1 || icfg[C_E] % icfg[C_NG] || icfg[C_TG] < 1 || icfg[C_TG] > icfg[C_NG] ||
         K < 1)
@@ -368,7 +377,8 @@ int or_route(const int *icfg, double rsf, const uint16_t *x, int T, const int32_
         int t = tokens ? tokens[i] : i;
         if (t < 0 || t >= T) { rc = OR_ERR_ARG; continue; }
         int r = or_route_token(icfg, rsf, x + (size_t)t * H, wg, bias, tie_rel, idx + (size_t)i * K,
-                               w + (size_t)i * K, near_tie + i, gap + i, NULL);
+                               w + (size_t)i * K, near_tie + i, gap + i, NULL,
+                               order_gap ? order_gap + i : NULL);
         if (r != OR_OK) rc = r;
     }
     return rc;
@@ -565,5 +575,127 @@ int or_rmsnorm(const uint16_t *x, int n, int H, const float *w, double eps, doub
             if (near) near[(size_t)t * H + h] = nt;
         }
     }
+    return OR_OK;
+}
+
+/* ------------------------------------------------------------------ NVFP4 */
+/* [V3] 四 NVFP4 量化: the routed experts' weights and their input activations
+ * are 4-bit floats (E2M1) in groups of 16 sharing one FP8 (E4M3) scale; the
+ * shared experts, like attention and lm_head, stay in high precision.
+ * READING (the page gives the group size and the scale type only): NVIDIA's
+ * NVFP4 as it is usually stored -- value = e2m1(q) * e4m3(s) * g, with s the
+ * group's scale code (non-negative E4M3) and g one fp32 scale per tensor (per
+ * expert matrix for weights; one per layer input for activations, a calibrated
+ * constant).
+ * Round-to-nearest-even onto the E2M1 grid {0, 0.5, 1, 1.5, 2, 3, 4, 6},
+ * saturating to +-6; an exact midpoint goes to the code whose last bit is 0;
+ * the sign is copied from v. Plain search over the eight magnitudes. */
+uint8_t or_e2m1_encode(double v) {
+    uint8_t sign = signbit(v) ? 8 : 0;
+    double a = fabs(v);
+    if (isnan(v)) return 7; /* no NaN in E2M1: saturate */
+    if (a >= 6.0) return sign | 7;
+    int lo = 0;
+    while (lo < 7 && or_e2m1_value((uint8_t)(lo + 1)) <= a) lo++;
+    double below = or_e2m1_value((uint8_t)lo), above = or_e2m1_value((uint8_t)(lo + 1));
+    double mid = 0.5 * (below + above); /* exact */
+    int c;
+    if (a < mid) c = lo;
+    else if (a > mid) c = lo + 1;
+    else c = (lo & 1) ? lo + 1 : lo;
+    return sign | (uint8_t)c;
+}
+
+/* NVFP4 quantiser of one vector v[n] (n a multiple of 16) with tensor scale g:
+ * per group of 16, s = E4M3_RNE(amax / (6 g)) (the scale that maps the group's
+ * largest magnitude onto E2M1's largest value 6, rounded to its FP8 code,
+ * saturating at 448), then q_i = E2M1_RNE(v_i / (e4m3(s) g)); a group whose
+ * scale code decodes to 0 stores zero codes. READING: the quotients are formed
+ * in double (for bf16 inputs and fp32 g they decide each code exactly). q[n]
+ * codes (one per byte here), sc[n/16] codes. Returns 16, or -1 for bad n or
+ * g <= 0. */
+int or_quant_nvfp4(const double *v, int n, double g, uint8_t *q, uint8_t *sc) {
+    if (n % 16 || !(g > 0.0)) return -1;
+    for (int b = 0; b < n / 16; b++) {
+        double amax = 0.0;
+        for (int i = 0; i < 16; i++) {
+            double a = fabs(v[b * 16 + i]);
+            if (a > amax) amax = a;
+        }
+        uint8_t s = or_e4m3_encode(amax / (6.0 * g));
+        sc[b] = s;
+        double sv = or_e4m3_value(s);
+        for (int i = 0; i < 16; i++)
+            q[b * 16 + i] = (sv == 0.0) ? 0 : or_e2m1_encode(v[b * 16 + i] / (sv * g));
+    }
+    return 16;
+}
+
+/* Dequantised NVFP4 vector: e2m1(q_i) * e4m3(sc[i/16]) * g. */
+int or_dequant_nvfp4(const uint8_t *q, const uint8_t *sc, int n, double g, double *out) {
+    if (n % 16) return -1;
+    for (int i = 0; i < n; i++) out[i] = or_e2m1_value(q[i]) * or_e4m3_value(sc[i / 16]) * g;
+    return 16;
+}
+
+/* One NVFP4 weight element W[e][r][c]: E2M1 codes two per byte (even column in
+ * the low nibble), E4M3 scale codes [n_mat][rows][cols/16], tensor scale g[e]. */
+static inline double w_nvfp4(const uint8_t *w, const uint8_t *s, const float *g, int rows, int cols,
+                             int e, int r, int c) {
+    size_t idx = ((size_t)e * rows + r) * cols + c;
+    uint8_t byte = w[idx / 2];
+    uint8_t nib = (c & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 15);
+    size_t sidx = ((size_t)e * rows + r) * (cols / 16) + c / 16;
+    return or_e2m1_value(nib) * or_e4m3_value(s[sidx]) * (double)g[e];
+}
+
+double or_weight_value_nvfp4(const uint8_t *w, const uint8_t *s, const float *g, int rows, int cols,
+                             int e, int r, int c) {
+    return w_nvfp4(w, s, g, rows, cols, e, r, c);
+}
+
+/* One routed expert e on n input rows xin[n][H] (already the dequantised NVFP4
+ * activations, tensor scale ga13), [V3] 三.4 with the NVFP4 recipe of [V3] 四:
+ *   g = W1 x, u = W3 x  (dequantised NVFP4 weights, tensor scale g13[e]),
+ *   a = SiLU(g) * u  (limit > 0: SiLU(min(g, limit)) * clamp(u, -limit, limit)),
+ *   a quantised to NVFP4 with tensor scale ga2 and dequantised,
+ *   y = W2 a  (NVFP4 weights, tensor scale g2[e]).
+ * All in double. y [n][H]. */
+int or_expert_rows_nvfp4(const uint8_t *w13, const uint8_t *w13s, const float *g13,
+                         const uint8_t *w2, const uint8_t *w2s, const float *g2, int e, int I,
+                         int H, const double *xin, int n, double ga2, double limit, double *y) {
+    if (I % 16 || H % 16 || !(ga2 > 0.0)) return OR_ERR_ARG;
+    double *a = (double *)malloc(sizeof(double) * (size_t)n * I);
+    for (int r = 0; r < n; r++) {
+        const double *xr = xin + (size_t)r * H;
+        double *ar = a + (size_t)r * I;
+#pragma omp parallel for schedule(static)
+        for (int i = 0; i < I; i++) {
+            double gsum = 0.0, usum = 0.0;
+            for (int h = 0; h < H; h++) {
+                gsum += w_nvfp4(w13, w13s, g13, 2 * I, H, e, i, h) * xr[h];
+                usum += w_nvfp4(w13, w13s, g13, 2 * I, H, e, I + i, h) * xr[h];
+            }
+            if (limit > 0.0) {
+                gsum = fmin(gsum, limit);
+                usum = fmax(fmin(usum, limit), -limit);
+            }
+            ar[i] = gsum / (1.0 + exp(-gsum)) * usum;
+        }
+        uint8_t *q = (uint8_t *)malloc(I);
+        uint8_t *sc = (uint8_t *)malloc(I / 16);
+        or_quant_nvfp4(ar, I, ga2, q, sc);
+        or_dequant_nvfp4(q, sc, I, ga2, ar);
+        free(q);
+        free(sc);
+        double *yr = y + (size_t)r * H;
+#pragma omp parallel for schedule(static)
+        for (int o = 0; o < H; o++) {
+            double acc = 0.0;
+            for (int i = 0; i < I; i++) acc += w_nvfp4(w2, w2s, g2, H, I, e, o, i) * ar[i];
+            yr[o] = acc;
+        }
+    }
+    free(a);
     return OR_OK;
 }

@@ -186,6 +186,33 @@ def test_near_tie_reported():
     assert not r["near_tie"] and r["gap"] > 1e-3
 
 
+def test_slot_order_near_tie_reported():
+    """Two chosen experts whose biased scores sit within 1e-6 (relative) of each
+    other make the slot order a near-tie, not the set: the order gap is the
+    smallest relative gap between consecutive slots, by brute force over the
+    constructed scores."""
+    E, k = 8, 3
+    logits = np.zeros(E, np.float32)  # s = 0.5 everywhere
+    bias = np.array([0.30, 0.20, 0.20, 0.10, 0.0, -0.1, -0.2, -0.3], np.float32)
+    bias[2] = np.nextafter(np.float32(0.20), np.float32(1.0))  # one float32 ulp above expert 1
+    x, wg = onehot_router(logits)
+    r = oracle.route_token(cfg(E, k), x, wg, bias)
+    assert r["idx"].tolist() == [0, 2, 1]
+    sp = 0.5 + bias.astype(np.float64)
+    want = min(abs(sp[a] - sp[b]) / max(abs(sp[a]), abs(sp[b]))
+               for a, b in ((0, 2), (2, 1)))
+    assert r["order_gap"] == want and r["order_tie"]
+    assert not r["near_tie"]  # the k-th and (k+1)-th are 0.1 apart
+    many = oracle.route(cfg(E, k), x, wg, bias)
+    assert many["order_tie"][0] and many["order_gap"][0] == want
+    # well separated slots: no order near-tie; k = 1 has no consecutive pair
+    r = oracle.route_token(cfg(E, k), x, wg, np.array([0.3, 0.2, 0.1, 0, -0.1, -0.2, -0.3, -0.4],
+                                                      np.float32))
+    assert not r["order_tie"] and r["order_gap"] > 0.1
+    r = oracle.route_token(cfg(E, 1), x, wg, bias)
+    assert r["order_gap"] == math.inf
+
+
 def test_group_near_tie_reported():
     E, k, ng, tg = 8, 2, 4, 2
     # groups of 2: group sums 2s, with groups 1 and 2 equal -> tie at the kept/dropped boundary
