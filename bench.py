@@ -60,6 +60,9 @@ def launches_per_step(cfg, T, n_sms):
     router = 2 + (1 if splits > 1 else 0)
     permute = 1 if N <= 4096 else 3
     fp8w = cfg.wfmt == "fp8_e4m3_b128x128" and cfg.afmt == "bf16"
+    if cfg.afmt == "nvfp4":  # quantise the token rows, gather; bf16 shared experts launch apart
+        sh = 1 if cfg.n_shared_experts > 0 else 0
+        return router + 1 + permute + 2 + (1 + sh) + (1 + sh) + 1
     if fp8w:
         pack = 2
     elif cfg.afmt == "bf16":
@@ -171,7 +174,7 @@ def expert_bytes(cfg):
     """Bytes of one routed (and one shared) expert's stored weights."""
     from expert_routing_grouped_layer_b200 import workloads as W
     return (W.weight_bytes_per_matrix(cfg, cfg.moe_intermediate_size),
-            W.weight_bytes_per_matrix(cfg, cfg.shared_intermediate_size))
+            W.weight_bytes_per_matrix(cfg, cfg.shared_intermediate_size, shared=True))
 
 
 def gate_up_bytes(cfg, active, T):
@@ -180,7 +183,7 @@ def gate_up_bytes(cfg, active, T):
     (each read once) and the intermediate written once."""
     routed, shared = expert_bytes(cfg)
     frac = 2.0 / 3.0  # w13 holds 2 of the 3 H x I matrices
-    abytes = 2 if cfg.afmt == "bf16" else 1
+    abytes = {"bf16": 2, "nvfp4": 0.5 + 1 / 16}.get(cfg.afmt, 1)
     N = T * cfg.num_experts_per_tok
     S = cfg.n_shared_experts
     return (active * routed + S * shared) * frac + (N + T) * cfg.hidden * abytes + \
@@ -214,7 +217,7 @@ def gate_up_flops(cfg, T):
 
 # Nominal dense tensor rates relative to bf16 (context: the FP8 rate is the
 # one the block-scaled E2M1 x E4M3 MMAs run at).
-NOMINAL_RATE_VS_BF16 = {"bf16": 1.0, "fp8": 2.0}
+NOMINAL_RATE_VS_BF16 = {"bf16": 1.0, "fp8": 2.0, "fp4": 4.0}
 NOMINAL_HBM_GBS = 7700.0  # B200 HGX datasheet figure, for context beside the measured copy rate
 
 
@@ -249,6 +252,18 @@ def measure_fp8_peaks(dev, n=8192, reps=10):
     except Exception as e:  # noqa: BLE001 - report why, keep the bench line
         out["fp8_e4m3_tensorwise_error"] = str(e).splitlines()[0][:160]
     try:
+        a4 = torch.randint(0, 255, (n, n // 2), dtype=torch.uint8, device=dev).view(
+            torch.float4_e2m1fn_x2)
+        b4 = torch.randint(0, 255, (n, n // 2), dtype=torch.uint8, device=dev).view(
+            torch.float4_e2m1fn_x2)
+        s4 = torch.full((n * (n // 16),), 0x38, dtype=torch.uint8, device=dev).view(
+            torch.float8_e4m3fn)
+        out["nvfp4_block16"] = best(
+            lambda: torch._scaled_mm(a4, b4.t(), scale_a=s4, scale_b=s4, out_dtype=torch.bfloat16))
+        del a4, b4, s4
+    except Exception as e:  # noqa: BLE001
+        out["nvfp4_block16_error"] = str(e).splitlines()[0][:160]
+    try:
         e8 = getattr(torch, "float8_e8m0fnu")
         sa = torch.full((n * (n // 32),), 127, dtype=torch.uint8, device=dev).view(e8)
         sb = torch.full((n * (n // 32),), 127, dtype=torch.uint8, device=dev).view(e8)
@@ -266,10 +281,11 @@ def tensor_peak(peaks, peak_src, cfg, fp8_measured=None):
     measured bf16 figure for bf16/f16 MMAs; for FP8-rate MMAs the best measured
     FP8 cuBLAS rate when one was measured in this run, else the bf16 figure
     times the nominal ratio."""
-    kind = "bf16" if cfg.afmt == "bf16" else "fp8"
+    kind = "bf16" if cfg.afmt == "bf16" else ("fp4" if cfg.afmt == "nvfp4" else "fp8")
     if kind == "bf16":
         return peaks["bf16_tflops"], peak_src
-    meas = {k: v for k, v in (fp8_measured or {}).items() if isinstance(v, float)}
+    meas = {k: v for k, v in (fp8_measured or {}).items()
+            if isinstance(v, float) and k.startswith("nvfp4") == (kind == "fp4")}
     if meas:
         name = max(meas, key=meas.get)
         return meas[name], "measured in this run: cuBLAS %s 8192^3, best of 10" % name
@@ -551,7 +567,7 @@ def cpu_baseline(cfg, inp, wts, tokens, seed=3):
 
 
 # prefill-shaped workloads timed after the headline in an N=1 run
-PER_WORKLOADS = ("k2_prefill_fp8w", "v4_fp4", "mx896")
+PER_WORKLOADS = ("k2_prefill_fp8w", "v4_fp4", "mx896", "k2_nvfp4")
 
 
 def run_ours(args, rank, world, dev):
@@ -653,8 +669,12 @@ def oracle_timing(cfg, inp, wts, tokens_per_step, steps, seed=0):
         for s in range(cfg.n_shared_experts):
             get(s, True)
         t0 = time.perf_counter()
-        oracle.layer(cfg, x_all[toks], r["idx"], r["w"], lambda e: get(e),
-                     lambda s: get(s, True))
+        if cfg.wfmt == "nvfp4":
+            oracle.layer_nvfp4(cfg, x_all[toks], r["idx"], r["w"], lambda e: get(e),
+                               lambda s: get(s, True), W.nvfp4_act_scales())
+        else:
+            oracle.layer(cfg, x_all[toks], r["idx"], r["w"], lambda e: get(e),
+                         lambda s: get(s, True))
         times.append(t_route + time.perf_counter() - t0)
         if len(cache) > 64:  # bound host memory
             cache.clear()

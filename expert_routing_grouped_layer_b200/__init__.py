@@ -23,8 +23,8 @@ MOE_DEV_BAD_EXPERT = 1
 MOE_DEV_TIMEOUT = 2
 
 SCORE_FN = {"sigmoid": 0, "sqrtsoftplus": 1, "softmax": 2}
-WFMT = {"bf16": 0, "fp8_e4m3_b128x128": 1, "fp4_e2m1_ue8m0_b32": 2, "mxfp4": 3}
-AFMT = {"bf16": 0, "fp8_e4m3_pow2_b128": 1, "mxfp8": 2}
+WFMT = {"bf16": 0, "fp8_e4m3_b128x128": 1, "fp4_e2m1_ue8m0_b32": 2, "mxfp4": 3, "nvfp4": 4}
+AFMT = {"bf16": 0, "fp8_e4m3_pow2_b128": 1, "mxfp8": 2, "nvfp4": 3}
 
 # symbols include/moe.h declares
 EXPORTS = ("moe_workspace_bytes", "moe_gate_topk", "moe_permute", "moe_quantize_activations",
@@ -54,13 +54,14 @@ class moe_config(ctypes.Structure):
                 ("n_shared_experts", ctypes.c_int32), ("shared_intermediate_size", ctypes.c_int32),
                 ("norm_topk_prob", ctypes.c_int32), ("routed_scaling_factor", ctypes.c_float),
                 ("score_fn", ctypes.c_int32), ("wfmt", ctypes.c_int32), ("afmt", ctypes.c_int32),
-                ("swiglu_limit", ctypes.c_float)]
+                ("swiglu_limit", ctypes.c_float), ("nvfp4_x_scale", ctypes.c_float),
+                ("nvfp4_h_scale", ctypes.c_float)]
 
 
 class moe_weights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("w13", "w13_scale", "w2", "w2_scale", "sh_w13", "sh_w13_scale", "sh_w2",
-                 "sh_w2_scale", "gate_w", "gate_bias")]
+                 "sh_w2_scale", "gate_w", "gate_bias", "w13_gscale", "w2_gscale")]
 
 
 _lib = None
@@ -151,11 +152,20 @@ def _stream(stream) -> int | None:
 
 def make_config(cfg) -> moe_config:
     """moe_config from any object with the layer's field names (e.g. a MoEConfig)."""
+    xs, hs = 1.0, 1.0
+    if cfg.afmt == "nvfp4":
+        xs, hs = getattr(cfg, "nvfp4_act_scales", None) or _nvfp4_act_scales()
     return moe_config(cfg.hidden, cfg.n_routed_experts, cfg.num_experts_per_tok, cfg.n_group,
                       cfg.topk_group, cfg.moe_intermediate_size, cfg.n_shared_experts,
                       cfg.shared_intermediate_size, int(bool(cfg.norm_topk_prob)),
                       float(cfg.routed_scaling_factor), SCORE_FN[cfg.score_fn], WFMT[cfg.wfmt],
-                      AFMT[cfg.afmt], float(getattr(cfg, "swiglu_limit", 0.0)))
+                      AFMT[cfg.afmt], float(getattr(cfg, "swiglu_limit", 0.0)), float(xs),
+                      float(hs))
+
+
+def _nvfp4_act_scales():
+    from . import workloads
+    return workloads.nvfp4_act_scales()
 
 
 def make_weights(w: dict, gate_w=None, gate_bias=None) -> moe_weights:
@@ -163,7 +173,8 @@ def make_weights(w: dict, gate_w=None, gate_bias=None) -> moe_weights:
     return moe_weights(g("w13"), g("w13_scale"), g("w2"), g("w2_scale"), g("sh_w13"),
                        g("sh_w13_scale"), g("sh_w2"), g("sh_w2_scale"),
                        _ptr(gate_w if gate_w is not None else w.get("gate_w")),
-                       _ptr(gate_bias if gate_bias is not None else w.get("gate_bias")))
+                       _ptr(gate_bias if gate_bias is not None else w.get("gate_bias")),
+                       g("w13_gscale"), g("w2_gscale"))
 
 
 def _cfg(cfg):

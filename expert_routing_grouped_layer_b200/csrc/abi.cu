@@ -65,8 +65,12 @@ bool config_valid(const moe_config* c) {
         c->score_fn != MOE_SCORE_SOFTMAX)
         return false;
     if (!(c->swiglu_limit >= 0.0f) || isinf(c->swiglu_limit)) return false;
-    if (c->wfmt < MOE_W_BF16 || c->wfmt > MOE_W_MXFP4) return false;
-    if (c->afmt < MOE_A_BF16 || c->afmt > MOE_A_MXFP8) return false;
+    if (c->wfmt < MOE_W_BF16 || c->wfmt > MOE_W_NVFP4) return false;
+    if (c->afmt < MOE_A_BF16 || c->afmt > MOE_A_NVFP4) return false;
+    if (c->afmt == MOE_A_NVFP4 &&
+        !(c->nvfp4_x_scale > 0.0f && c->nvfp4_h_scale > 0.0f && !isinf(c->nvfp4_x_scale) &&
+          !isinf(c->nvfp4_h_scale)))
+        return false;
     return true;
 }
 
@@ -75,6 +79,11 @@ moe_status config_supported(const moe_config* c) {
     if (c->n_shared_experts > 0 && c->shared_intermediate_size != c->moe_intermediate_size)
         return MOE_ERR_UNSUPPORTED;
     if (c->afmt == MOE_A_BF16 && (c->wfmt == MOE_W_BF16 || c->wfmt == MOE_W_FP8_E4M3_B128x128))
+        return MOE_OK;
+    // NVFP4 routed experts: 256 packed E2M1 values per 128-byte row of a stage,
+    // two 128-row weight tiles per unit
+    if (c->wfmt == MOE_W_NVFP4 && c->afmt == MOE_A_NVFP4 && c->hidden % 256 == 0 &&
+        c->moe_intermediate_size % 256 == 0)
         return MOE_OK;
     // block-scaled tensor cores: E2M1 weights x E4M3 activations; the scale tiles
     // move by TMA in rows of 16 scales, so H and I must be multiples of 512
@@ -110,10 +119,19 @@ WsLayout ws_layout(const moe_config* c, int T) {
     L.sorted_pair = take(N * 4);
     L.row_of = take(N * 4);
     L.chunk_counts = take((size_t)L.n_chunks * E * 4);
-    L.xa = take((N + T) * H * act_bytes);
-    L.xa_scale = take(act_bytes == 1 ? (N + T) * (H / 32) : (f16_gate_up(c) ? (N + T) : 0));
-    L.hbuf = take((N + S * T) * I * act_bytes);
-    L.h_scale = take(act_bytes == 1 ? (N + S * T) * (I / 32) : (f16_gate_up(c) ? (N + S * T) : 0));
+    if (c->afmt == MOE_A_NVFP4) {
+        // packed routed rows (+ the token rows they are gathered from), then the
+        // bf16 token rows of the shared experts; h likewise with bf16 shared rows
+        L.xa = take(nvfp4_tail_offset((N + T) * H / 2) + (size_t)T * H * 2);
+        L.xa_scale = take((N + T) * (H / 16));
+        L.hbuf = take(nvfp4_tail_offset(N * I / 2) + S * T * I * 2);
+        L.h_scale = take(N * (I / 16));
+    } else {
+        L.xa = take((N + T) * H * act_bytes);
+        L.xa_scale = take(act_bytes == 1 ? (N + T) * (H / 32) : (f16_gate_up(c) ? (N + T) : 0));
+        L.hbuf = take((N + S * T) * I * act_bytes);
+        L.h_scale = take(act_bytes == 1 ? (N + S * T) * (I / 32) : (f16_gate_up(c) ? (N + S * T) : 0));
+    }
     L.y = take(N * H * 2);
     L.shared_y = take(S * T * H * 2);
     L.x_norm = take((size_t)T * H * 2);
@@ -207,6 +225,12 @@ moe_status moe_quantize_activations(const moe_config* cfg, const void* x, int32_
     if (!config_valid(cfg) || T < 0 || cfg->afmt == MOE_A_BF16) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
     if (!x || !xq || !xq_scale || !aligned16(x) || !aligned16(xq)) return MOE_ERR_INVALID_ARG;
+    if (cfg->afmt == MOE_A_NVFP4) {
+        if (cfg->hidden % 256) return MOE_ERR_INVALID_ARG;
+        return cuda_status(launch_pack_nvfp4(x, cfg->hidden, cfg->nvfp4_x_scale, T, xq,
+                                             static_cast<uint8_t*>(xq_scale), nullptr,
+                                             as_stream(stream)));
+    }
     return cuda_status(launch_pack_rows(cfg->afmt, x, cfg->hidden, nullptr, 0,
                                         cfg->num_experts_per_tok, T, T, xq,
                                         static_cast<uint8_t*>(xq_scale), 0, as_stream(stream)));
@@ -218,8 +242,11 @@ static bool weights_ok(const moe_config* cfg, const moe_weights* w, bool gate_up
     const void* sh = gate_up ? w->sh_w13 : w->sh_w2;
     const void* shs = gate_up ? w->sh_w13_scale : w->sh_w2_scale;
     const bool scaled = cfg->wfmt != MOE_W_BF16;
-    if (!r || !aligned16(r) || (scaled && !rs)) return false;
-    if (cfg->n_shared_experts > 0 && (!sh || !aligned16(sh) || (scaled && !shs))) return false;
+    const bool nvfp4 = cfg->wfmt == MOE_W_NVFP4;  // bf16 shared experts, tensor scales
+    if (!r || !aligned16(r) || (scaled && (!rs || !aligned16(rs)))) return false;
+    if (nvfp4 && !(gate_up ? w->w13_gscale : w->w2_gscale)) return false;
+    if (cfg->n_shared_experts > 0 && (!sh || !aligned16(sh) || (scaled && !nvfp4 && !shs)))
+        return false;
     return true;
 }
 
@@ -249,6 +276,21 @@ moe_status moe_pack_expert_inputs(const moe_config* cfg, const void* x, int32_t 
     if (!x || !sorted_pair || !xa || !aligned16(x) || !aligned16(xa)) return MOE_ERR_INVALID_ARG;
     if ((cfg->afmt != MOE_A_BF16 || f16_gate_up(cfg)) && !xa_scale) return MOE_ERR_INVALID_ARG;
     const int k = cfg->num_experts_per_tok, N = T * k;
+    if (cfg->afmt == MOE_A_NVFP4) {
+        // the token rows once (rows N..N+T-1, with the bf16 copy for the shared
+        // experts behind the packed rows), then the routed rows gathered from them
+        if (cfg->hidden % 256) return MOE_ERR_INVALID_ARG;
+        const int H = cfg->hidden;
+        uint8_t* q = static_cast<uint8_t*>(xa);
+        uint8_t* qs = static_cast<uint8_t*>(xa_scale);
+        void* xb = q + nvfp4_tail_offset((size_t)(N + T) * H / 2);
+        cudaError_t e = launch_pack_nvfp4(x, H, cfg->nvfp4_x_scale, T, q + (size_t)N * H / 2,
+                                          qs + (size_t)N * (H / 16), xb, as_stream(stream));
+        if (e == cudaSuccess)
+            e = launch_gather_nvfp4_rows(q + (size_t)N * H / 2, qs + (size_t)N * (H / 16), H,
+                                         sorted_pair, N, k, T, q, qs, as_stream(stream));
+        return cuda_status(e);
+    }
     if (f16_gate_up(cfg))
         return cuda_status(launch_pack_f16_rows(x, cfg->hidden, sorted_pair, N, k, T, N + T, xa,
                                                 static_cast<int8_t*>(xa_scale), as_stream(stream)));
@@ -269,6 +311,33 @@ moe_status moe_expert_gate_up(const moe_config* cfg, const void* xa, const void*
     if (f16_gate_up(cfg) && (!xa_scale || !h_scale)) return MOE_ERR_INVALID_ARG;
     if (!weights_ok(cfg, w, true)) return MOE_ERR_INVALID_ARG;
     GroupedGemmArgs a = gemm_args(cfg, T, expert_offsets, dev_status);
+    if (cfg->afmt == MOE_A_NVFP4) {
+        const int H = a.H, I = a.I, N = a.N;
+        a.gemm = 1;
+        a.w_routed = w->w13;
+        a.w_routed_scale = w->w13_scale;
+        a.w_gscale = w->w13_gscale;
+        a.a_gscale = cfg->nvfp4_x_scale;
+        a.out_gscale = cfg->nvfp4_h_scale;
+        a.b_rows = xa;
+        a.b_scale = static_cast<const uint8_t*>(xa_scale);
+        a.out_routed = h;
+        a.out_routed_scale = static_cast<uint8_t*>(h_scale);
+        cudaError_t e = launch_grouped_gemm(a, as_stream(stream));
+        if (e == cudaSuccess && a.S > 0) {  // bf16 shared experts on the bf16 token rows
+            GroupedGemmArgs b = gemm_args(cfg, T, expert_offsets, dev_status);
+            b.E = 0;
+            b.N = 0;
+            b.wfmt = MOE_W_BF16;
+            b.afmt = MOE_A_BF16;
+            b.gemm = 1;
+            b.w_routed = b.w_shared = w->sh_w13;
+            b.b_rows = static_cast<const uint8_t*>(xa) + nvfp4_tail_offset((size_t)(N + T) * H / 2);
+            b.out_shared = static_cast<uint8_t*>(h) + nvfp4_tail_offset((size_t)N * I / 2);
+            e = launch_grouped_gemm(b, as_stream(stream));
+        }
+        return cuda_status(e);
+    }
     const size_t hrow = (size_t)a.I * (q ? 1 : 2);
     a.gemm = 1;
     a.w_routed = w->w13;
@@ -300,6 +369,30 @@ moe_status moe_expert_down(const moe_config* cfg, const void* h, const void* h_s
     if ((q || f16_gate_up(cfg)) && !h_scale) return MOE_ERR_INVALID_ARG;
     if (!weights_ok(cfg, w, false)) return MOE_ERR_INVALID_ARG;
     GroupedGemmArgs a = gemm_args(cfg, T, expert_offsets, dev_status);
+    if (cfg->afmt == MOE_A_NVFP4) {
+        a.gemm = 2;
+        a.w_routed = w->w2;
+        a.w_routed_scale = w->w2_scale;
+        a.w_gscale = w->w2_gscale;
+        a.a_gscale = cfg->nvfp4_h_scale;
+        a.b_rows = h;
+        a.b_scale = static_cast<const uint8_t*>(h_scale);
+        a.out_routed = y;
+        cudaError_t e = launch_grouped_gemm(a, as_stream(stream));
+        if (e == cudaSuccess && a.S > 0) {  // bf16 shared experts on their bf16 rows of h
+            GroupedGemmArgs b = gemm_args(cfg, T, expert_offsets, dev_status);
+            b.E = 0;
+            b.N = 0;
+            b.wfmt = MOE_W_BF16;
+            b.afmt = MOE_A_BF16;
+            b.gemm = 2;
+            b.w_routed = b.w_shared = w->sh_w2;
+            b.b_rows = static_cast<const uint8_t*>(h) + nvfp4_tail_offset((size_t)a.N * a.I / 2);
+            b.out_shared = shared_y;
+            e = launch_grouped_gemm(b, as_stream(stream));
+        }
+        return cuda_status(e);
+    }
     a.gemm = 2;
     a.w_routed = w->w2;
     a.w_routed_scale = w->w2_scale;
@@ -390,7 +483,9 @@ moe_status moe_rmsnorm_prologue(const moe_config* cfg, const void* x, int32_t T,
     if (T == 0) return MOE_OK;
     if (!x || !norm_w || !x_norm || !aligned16(x) || !aligned16(norm_w) || !aligned16(x_norm))
         return MOE_ERR_INVALID_ARG;
-    const bool q = cfg->afmt != MOE_A_BF16;
+    // FP8 / MX activations: the quantised rows in the same pass (NVFP4 layers
+    // quantise their routed inputs from x_norm in the expert-input step)
+    const bool q = cfg->afmt == MOE_A_FP8_E4M3_POW2_B128 || cfg->afmt == MOE_A_MXFP8;
     if (q && (cfg->hidden % 512 || !xq || !xq_scale || !aligned16(xq) || !aligned16(xq_scale)))
         return MOE_ERR_INVALID_ARG;
     return cuda_status(launch_rmsnorm_quant(cfg->afmt, x, cfg->hidden, norm_w, eps, T, x_norm,
@@ -427,8 +522,8 @@ moe_status moe_layer_forward_prenorm(const moe_config* cfg, const void* x, int32
     void* sy = base + L.shared_y;
     const int k = cfg->num_experts_per_tok, H = cfg->hidden, N = T * k;
     cudaStream_t st = as_stream(stream);
-    if (cfg->afmt == MOE_A_BF16) {
-        // bf16 expert inputs: the prologue's output feeds the unchanged layer
+    if (cfg->afmt == MOE_A_BF16 || cfg->afmt == MOE_A_NVFP4) {
+        // bf16 / NVFP4 expert inputs: the prologue's output feeds the unchanged layer
         moe_status s = cuda_status(launch_rmsnorm_quant(MOE_A_BF16, x, H, norm_w, eps, T, xn,
                                                         nullptr, nullptr, st));
         if (s == MOE_OK)

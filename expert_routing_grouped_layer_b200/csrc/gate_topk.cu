@@ -6,7 +6,7 @@
 // from "DeepSeek-V4-Pro 架构与代码概述", 架构; softmax, the alternative 三.1
 // contrasts with sigmoid, over a token's logits): score, bias, group-limited top-k,
 // normalised and scaled weights. The reduction adds each logit's partials in
-// split order, so the logits are deterministic.
+// split order (in fp64), so the logits are deterministic.
 #include <cuda_bf16.h>
 
 #include <cfloat>
@@ -19,26 +19,27 @@ namespace moe {
 
 namespace {
 
-// logits = sum over splits of the partial sums, added in split order; written
-// over split 0 so the selection kernel reads one slab. Eight splits' loads are
-// issued before their adds, which still run in split order.
+// logits = sum over splits of the partial sums, added in split order in fp64
+// and rounded once to fp32; written over split 0 so the selection kernel reads
+// one slab. Eight splits' loads are issued before their adds, which still run
+// in split order.
 __global__ void __launch_bounds__(256) router_reduce_kernel(float* __restrict__ part, long n,
                                                             int splits) {
     pdl_wait();
     pdl_trigger();
     const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= n) return;
-    float l = 0.f;
+    double l = 0.0;
     int s = 0;
     for (; s + 8 <= splits; s += 8) {
         float v[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) v[j] = part[(size_t)(s + j) * n + i];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) l += v[j];
+        for (int j = 0; j < 8; ++j) l += (double)v[j];
     }
-    for (; s < splits; ++s) l += part[(size_t)s * n + i];
-    part[i] = l;
+    for (; s < splits; ++s) l += (double)part[(size_t)s * n + i];
+    part[i] = (float)l;
 }
 
 __device__ __forceinline__ float score_of(float l, int score_fn) {

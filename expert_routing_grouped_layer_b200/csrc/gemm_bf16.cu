@@ -190,10 +190,12 @@ cudaError_t launch_bf16(const GroupedGemmArgs& a, cudaStream_t st) {
     const KParams p = make_params(a, GEMM, &b_rows);
     const int E = a.E, S = a.S;
     CUtensorMap tmAr, tmAs, tmB;
-    if (!make_tmap_bf16(&tmAr, a.w_routed, (uint64_t)E * p.a_rows_per_mat, p.K, BM))
-        return cudaErrorInvalidValue;
     if (!make_tmap_bf16(&tmAs, S > 0 ? a.w_shared : a.w_routed,
                         (uint64_t)(S > 0 ? S : E) * p.a_rows_per_mat, p.K, BM))
+        return cudaErrorInvalidValue;
+    // a launch of shared experts alone (E == 0) never reads the routed map
+    if (E == 0) tmAr = tmAs;
+    else if (!make_tmap_bf16(&tmAr, a.w_routed, (uint64_t)E * p.a_rows_per_mat, p.K, BM))
         return cudaErrorInvalidValue;
     if (b_rows == 0) return cudaSuccess;
     if (!make_tmap_bf16(&tmB, a.b_rows, b_rows, p.K, B_BOX)) return cudaErrorInvalidValue;

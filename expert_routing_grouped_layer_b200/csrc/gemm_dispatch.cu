@@ -6,9 +6,14 @@ namespace gemm {
 cudaError_t launch_gemm_bf16(const GroupedGemmArgs& a, cudaStream_t st);
 cudaError_t launch_gemm_fp8w(const GroupedGemmArgs& a, cudaStream_t st);
 cudaError_t launch_gemm_mx(const GroupedGemmArgs& a, cudaStream_t st);
+cudaError_t launch_gemm_nvfp4(const GroupedGemmArgs& a, cudaStream_t st);
 }  // namespace gemm
 
 cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st) {
+    if (a.wfmt == MOE_W_NVFP4) {  // routed experts only; the caller runs the bf16 shared experts
+        if (a.afmt == MOE_A_NVFP4) return gemm::launch_gemm_nvfp4(a, st);
+        return cudaErrorNotSupported;
+    }
     if (a.wfmt == MOE_W_FP4_E2M1_UE8M0_B32 || a.wfmt == MOE_W_MXFP4) {
         if (a.afmt == MOE_A_MXFP8 || a.afmt == MOE_A_FP8_E4M3_POW2_B128)
             return gemm::launch_gemm_mx(a, st);

@@ -1,0 +1,533 @@
+// gemm_nvfp4.cu -- the routed experts' SwiGLU MLP in NVFP4 ("DeepSeek V3架构拆解：
+// Kimi-K2-Thinking-NVFP4的MLA注意力与MoE路由实现原理", 四 NVFP4 量化: weights and
+// input activations are 4-bit floats in groups of 16 sharing one FP8 scale; the
+// shared experts stay in high precision and run through the bf16 kernel).
+//
+// Both operands are E2M1 codes packed two per byte, so a 128-byte shared-memory
+// row holds 256 values of K and the TMA moves the stored bytes unchanged (no
+// expansion to one byte per value). tcgen05.mma kind::mxf4nvf4 with
+// scale_vec::4X reads, for every row of A and of B, one 32-bit tensor-memory
+// word per MMA (K = 64): its four bytes are the E4M3 scales of the four
+// 16-element groups. Row m = m0 + 32*m1 of an operand sits in lane m0 of every
+// lane quadrant, column m1; four scale warps (one per quadrant) store each
+// stage's 16 columns per operand ([MMA kk][m1]) with tcgen05.st. The per-tensor
+// fp32 scales (the expert's weight scale times the activation scale) multiply
+// the fp32 accumulator in the epilogue. GEMM1's epilogue quantises the SwiGLU
+// output back to NVFP4 along I (groups of 16 features = 16 lanes of a warp).
+//
+// Tile: two 128-row weight tiles per unit (gate and up for GEMM1, two
+// consecutive 128-row blocks of the down projection for GEMM2) sharing one
+// token tile of up to 96 rows, each with its own MMA-issuing thread and
+// accumulator, accumulators double-buffered. Warps: 0 TMA, 1 MMA (tile 0),
+// 2-5 epilogue, 6-9 scale warps, 10 MMA (tile 1).
+#include <cuda_fp4.h>
+
+#include "gemm_common.cuh"
+
+namespace moe {
+namespace gemm {
+namespace {
+
+constexpr int NV_BK = 256;          // K values per stage: one 128-byte smem row of packed E2M1
+constexpr int NV_ROW = NV_BK / 2;   // bytes per stage row
+constexpr int NV_SF_STAGES = 4;     // stages per scale box
+constexpr int NV_SF_W = 16 * NV_SF_STAGES;  // scale bytes per row per box (64)
+constexpr int NV_SF_TILE = 128 * NV_SF_W;   // one operand's scale box: 128 rows
+
+template <int GEMM>
+struct TileNV {
+    static constexpr int NA = 2;
+    static constexpr int BNX = 96;
+    static constexpr int ACCB = 2;
+    static constexpr int SCALE_WARP = 6;
+    static constexpr int MMA2_WARP = 10;
+    static constexpr int THREADS = 32 * 11;
+    static constexpr int NOPS = NA + 1;  // scale operands: the two A tiles, the token rows
+    static constexpr int A_BYTES = BM * NV_ROW;
+    static constexpr int B_BYTES = BNX * NV_ROW;
+    static constexpr int A_OFF = 0;
+    static constexpr int B_OFF = NA * A_BYTES;
+    static constexpr int STAGE_BYTES = (B_OFF + B_BYTES + 1023) / 1024 * 1024;
+    static constexpr int RAW_BYTES = NOPS * NV_SF_TILE;
+    static constexpr int RING_BYTES = 2 * RAW_BYTES;
+    // staged epilogue chunk, two per parity: down [16 tokens][128] bf16;
+    // gate/up [16 tokens][64] code bytes then [16][8] scale codes
+    static constexpr int G1_STAGE = 16 * 64 + 16 * 8;
+    static constexpr int EPI_BYTES = (GEMM == 2 ? 2 * 16 * BM * 2 : 2 * G1_STAGE) + 128;
+    static constexpr int FIXED_BYTES = 1024 + 8 * (3 * 6 + 13) + 16 + 4 * (MAX_SEG + 1) + EPI_BYTES;
+    static constexpr int STAGES = stages_for(STAGE_BYTES, FIXED_BYTES + RING_BYTES, 6);
+    static constexpr int ACC_COLS = NA * BNX;
+    static constexpr int TMEM_COLS = 512;
+    static constexpr int SF_COL = ACCB * ACC_COLS;  // scale sets: set s, operand i at SF_COL + s*SET_COLS + 16*i
+    static constexpr int SET_COLS = 16 * NOPS;
+    static constexpr int NSETS_FIT = (TMEM_COLS - SF_COL) / SET_COLS;
+    static constexpr int NSETS = NSETS_FIT < STAGES ? NSETS_FIT : STAGES;
+    static_assert(NSETS >= 2, "tensor memory budget: two scale sets");
+    static constexpr int BAR_BYTES = 8 * (3 * STAGES + 13) + 16;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + RING_BYTES + BAR_BYTES +
+                                      4 * (MAX_SEG + 1) + EPI_BYTES;
+    static_assert(STAGES >= 2 && SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+// Instruction descriptor, kind::mxf4nvf4 block-scaled: A and B E2M1 (format 1),
+// K-major, UE4M3 scales (bit 23 clear), dense K = 64, scale-factor ids 0.
+__host__ __device__ __forceinline__ uint32_t idesc_nvf4(uint32_t M, uint32_t N) {
+    return (1u << 7) | (1u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+
+// D[tmem] (+)= (A * sfA) * (B * sfB)^T with one E4M3 scale per 16 elements of K,
+// four per row per MMA, read from tensor memory.
+__device__ __forceinline__ void mma_nvf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], "
+        "[%6], p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
+// Registers -> tensor memory: 16 consecutive 32-bit columns of this thread's lane.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        : "memory");
+}
+
+__device__ __forceinline__ uint32_t word4(const uint4& u, int w) {
+    return w == 0 ? u.x : (w == 1 ? u.y : (w == 2 ? u.z : u.w));
+}
+
+// E2M1 code of v by round to nearest even onto {0, .5, 1, 1.5, 2, 3, 4, 6},
+// saturating: the magnitude code counts the midpoints below |v| (a midpoint
+// itself goes to the even code), the sign bit is v's.
+__device__ __forceinline__ uint32_t e2m1_code(float v) {
+    const float a = fabsf(v);
+    const uint32_t c = (a > 0.25f) + (a >= 0.75f) + (a > 1.25f) + (a >= 1.75f) + (a > 2.5f) +
+                       (a >= 3.5f) + (a > 5.0f);
+    return c | (signbit(v) ? 8u : 0u);
+}
+
+__device__ __forceinline__ bool warp_wait_nv(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                             int lane) {
+    int ok = 1;
+    if (lane == 0) ok = mbar_wait(bar, parity, abort) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok != 0;
+}
+
+struct NVScales {
+    const float* w_gscale;  // per routed expert matrix
+    float a_gscale;         // the B operand's tensor scale
+    float out_gscale;       // GEMM1: tensor scale of the quantised intermediate
+};
+
+template <int GEMM>
+__global__ void __launch_bounds__(TileNV<GEMM>::THREADS, 1)
+    grouped_gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmA,
+                              const __grid_constant__ CUtensorMap tmSFA,
+                              const __grid_constant__ BMaps tmB,
+                              const __grid_constant__ CUtensorMap tmSFB, const KParams p,
+                              const NVScales sc) {
+    pdl_wait();
+    pdl_trigger();
+    using C = TileNV<GEMM>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t* sf_ring = smem + C::STAGES * C::STAGE_BYTES;  // [2][RAW_BYTES]
+    uint64_t* full = reinterpret_cast<uint64_t*>(sf_ring + C::RING_BYTES);
+    uint64_t* empty = full + C::STAGES;
+    uint64_t* sf_ready = empty + C::STAGES;
+    uint64_t* tfull = sf_ready + C::STAGES;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* mma_done = tempty + 2;
+    uint64_t* sf_full = mma_done + 1;  // [2]
+    uint64_t* sf_empty = sf_full + 2;  // [2]
+    uint64_t* ep_bar = sf_empty + 2;   // [2] the epilogue warps' staged chunk
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ep_bar + 2);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* pref = reinterpret_cast<int*>(tmem_slot + 4);
+    uint8_t* ep_buf = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(pref + MAX_SEG + 1) + 127) & ~static_cast<uintptr_t>(127));
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], C::NA);
+            mbar_init(&sf_ready[s], 4);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], C::NA);
+            mbar_init(&tempty[a], 128);
+        }
+        mbar_init(mma_done, C::NA);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sf_full[i], 1);
+            mbar_init(&sf_empty[i], 4);
+            mbar_init(&ep_bar[i], 4);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmSFA);
+        prefetch_bmaps(tmB);
+        tma_prefetch_desc(&tmSFB);
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    const int MT = p.M / p.tile_rows;
+    if (warp == 1) build_schedule(p, pref, MT, lane);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int total = pref[p.nseg];
+    const int KB = p.K / NV_BK;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued = 0;
+            int sfs = 0, sf_issued = 0;
+            uint32_t sf_phase = 0;
+            for (int u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x) {
+                const Unit t = decode_unit(p, pref, u);
+                const int n_mma = (t.n_valid + 15) & ~15;
+                const uint32_t tx = C::NA * C::A_BYTES + n_mma * NV_ROW;
+                bool ok = true;
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (kb % NV_SF_STAGES == 0) {  // the scales of this stage and the next three
+                        if (!mbar_wait(&sf_empty[sfs], sf_phase ^ 1, abort_flag)) { ok = false; break; }
+                        uint8_t* sl = sf_ring + sfs * C::RAW_BYTES;
+                        const int sfx = kb * 16;  // first scale byte of the box
+                        mbar_arrive_expect_tx(&sf_full[sfs], C::RAW_BYTES);
+#pragma unroll
+                        for (int j = 0; j < C::NA; ++j)
+                            tma_load_2d(sl + j * NV_SF_TILE, &tmSFA, sfx, t.a_row + j * p.a_up_offset,
+                                        &sf_full[sfs]);
+                        tma_load_2d(sl + C::NA * NV_SF_TILE, &tmSFB, sfx, t.b_row, &sf_full[sfs]);
+                        ++sf_issued;
+                        if (++sfs == 2) { sfs = 0; sf_phase ^= 1; }
+                    }
+                    if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+                    uint8_t* st = smem + stage * C::STAGE_BYTES;
+                    mbar_arrive_expect_tx(&full[stage], tx);
+#pragma unroll
+                    for (int j = 0; j < C::NA; ++j)
+                        tma_load_2d(st + C::A_OFF + j * C::A_BYTES, &tmA, kb * NV_ROW,
+                                    t.a_row + j * p.a_up_offset, &full[stage]);
+                    load_b_rows(st + C::B_OFF, tmB, kb * NV_ROW, t.b_row, n_mma, NV_ROW, &full[stage]);
+                    ++issued;
+                    if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+            }
+            if (*abort_flag) {
+                volatile int no_abort = 0;
+                int s = stage;
+                uint32_t ph = phase;
+                for (int i = 0; i < min(issued, C::STAGES); ++i) {
+                    if (--s < 0) { s = C::STAGES - 1; ph ^= 1; }
+                    mbar_wait(&full[s], ph, &no_abort);
+                }
+                s = sfs;
+                ph = sf_phase;
+                for (int i = 0; i < min(sf_issued, 2); ++i) {
+                    if (--s < 0) { s = 1; ph ^= 1; }
+                    mbar_wait(&sf_full[s], ph, &no_abort);
+                }
+                status_or(p.status, MOE_DEV_TIMEOUT);
+            }
+        }
+    } else if (warp == 1 || warp == C::MMA2_WARP) {
+        if (lane == 0) {
+            const int w = (warp == 1) ? 0 : 1;
+            int stage = 0;
+            uint32_t phase = 0;
+            int set = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            for (int u = blockIdx.x; u < total; u += gridDim.x) {
+                const Unit t = decode_unit(p, pref, u);
+                const int n_mma = (t.n_valid + 15) & ~15;
+                const uint32_t idesc = idesc_nvf4(BM, n_mma);
+                if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t d0 = tmem_base + acc * C::ACC_COLS + w * C::BNX;
+                bool ok = true;
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, abort_flag) ||
+                        !mbar_wait(&sf_ready[stage], phase, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t st = smem_u32(smem + stage * C::STAGE_BYTES);
+                    const uint32_t sfs = tmem_base + C::SF_COL + set * C::SET_COLS;
+#pragma unroll
+                    for (int kk = 0; kk < NV_BK / 64; ++kk)
+                        mma_nvf4(d0, sdesc_kmajor_sw128(st + C::A_OFF + w * C::A_BYTES + kk * 32),
+                                 sdesc_kmajor_sw128(st + C::B_OFF + kk * 32), idesc,
+                                 sfs + 16 * w + 4 * kk, sfs + 16 * C::NA + 4 * kk, (kb | kk) != 0);
+                    mma_commit(&empty[stage]);
+                    if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+                    if (++set == C::NSETS) set = 0;
+                }
+                if (!ok) break;
+                mma_commit(&tfull[acc]);
+                if (++acc == C::ACCB) { acc = 0; acc_phase ^= 1; }
+            }
+            mma_commit(mma_done);
+            volatile int no_abort = 0;
+            mbar_wait(mma_done, 0, &no_abort);
+            if (*abort_flag) status_or(p.status, MOE_DEV_TIMEOUT);
+        }
+    } else if (warp >= C::SCALE_WARP && warp < C::SCALE_WARP + 4) {
+        // scale warps: per stage, lane m0 of quadrant q takes, for every operand,
+        // the stage's 16 scale bytes of rows m0 + 32*m1 (m1 = 0..3) from the ring
+        // slot and stores word kk of row m1 to column 4*kk + m1 of the operand in
+        // the stage's TMEM set. A set is rewritten only after the MMAs that read
+        // it completed; a ring slot serves four stages (fewer at a unit's end).
+        const uint32_t lane_cols = tmem_base + ((uint32_t)((warp & 3) * 32) << 16) + C::SF_COL;
+        int stage = 0;
+        int set = 0;
+        int g = 0;
+        int sfs = 0;
+        uint32_t sf_phase = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+            for (int kb = 0; kb < KB; ++kb) {
+                if (kb % NV_SF_STAGES == 0 &&
+                    !warp_wait_nv(&sf_full[sfs], sf_phase, abort_flag, lane)) {
+                    ok = false;
+                    break;
+                }
+                if (g >= C::NSETS) {
+                    const int gp = g - C::NSETS;
+                    if (!warp_wait_nv(&empty[gp % C::STAGES], (uint32_t)(gp / C::STAGES) & 1u,
+                                      abort_flag, lane)) {
+                        ok = false;
+                        break;
+                    }
+                }
+                const uint8_t* raw = sf_ring + sfs * C::RAW_BYTES + 16 * (kb % NV_SF_STAGES);
+                uint4 row[C::NOPS][4];
+#pragma unroll
+                for (int i = 0; i < C::NOPS; ++i)
+#pragma unroll
+                    for (int r = 0; r < 4; ++r)
+                        row[i][r] = *reinterpret_cast<const uint4*>(raw + i * NV_SF_TILE +
+                                                                    NV_SF_W * (lane + 32 * r));
+                if (kb % NV_SF_STAGES == NV_SF_STAGES - 1 || kb + 1 == KB) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sf_empty[sfs]);
+                    if (++sfs == 2) { sfs = 0; sf_phase ^= 1; }
+                }
+#pragma unroll
+                for (int i = 0; i < C::NOPS; ++i) {
+                    uint32_t v[16];
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) v[4 * kk + r] = word4(row[i][r], kk);
+                    tmem_st16(lane_cols + set * C::SET_COLS + 16 * i, v);
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sf_ready[stage]);
+                if (++stage == C::STAGES) stage = 0;
+                if (++set == C::NSETS) set = 0;
+                ++g;
+            }
+        }
+    } else if (GEMM == 2) {
+        // down epilogue: y = acc * (activation scale * expert scale), bf16; per
+        // 16-token chunk each warp converts its 32 features into the shared
+        // [16 tokens][128] tile (two, alternating), the four warps meet at an
+        // mbarrier, and warp q writes token rows 4q..4q+3 with 16-byte stores
+        const int q = warp & 3;
+        const int row = q * 32 + lane;
+        __nv_bfloat16* gbuf = reinterpret_cast<__nv_bfloat16*>(ep_buf);
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        int chunk = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+            const Unit t = decode_unit(p, pref, u);
+            const float f = sc.a_gscale * sc.w_gscale[t.seg];
+            if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int w = 0; w < C::NA && ok; ++w) {
+                const uint32_t taddr =
+                    tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::ACC_COLS + w * C::BNX;
+                __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(t.out) + t.mt * p.tile_rows + w * BM;
+                for (int c0 = 0; c0 < t.n_valid; c0 += 16, ++chunk) {
+                    uint32_t gq[16];
+                    tmem_ld16(taddr + c0, gq);
+                    tmem_ld_wait(gq);
+                    __nv_bfloat16* buf = gbuf + (chunk & 1) * 16 * BM;
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        buf[j * BM + row] = __float2bfloat16_rn(__uint_as_float(gq[j]) * f);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&ep_bar[chunk & 1]);
+                    if (!mbar_wait(&ep_bar[chunk & 1], (uint32_t)(chunk >> 1) & 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int r = 4 * q + 2 * h + (lane >> 4);
+                        const int col = (lane & 15) * 8;
+                        if (c0 + r < t.n_valid)
+                            *reinterpret_cast<uint4*>(out + (size_t)(c0 + r) * p.ld_out + col) =
+                                *reinterpret_cast<const uint4*>(buf + r * BM + col);
+                    }
+                }
+            }
+            if (!ok) break;
+            tc_fence_before();
+            mbar_arrive(&tempty[acc]);
+            if (++acc == C::ACCB) { acc = 0; acc_phase ^= 1; }
+        }
+    } else {
+        // GEMM1 epilogue: g and u = acc * (activation scale * expert scale),
+        // a = SwiGLU, then NVFP4 along I with the intermediate's tensor scale G:
+        // per 16 features (16 lanes) s = E4M3(amax / (6 G)) and
+        // q = E2M1(a / (e4m3(s) G)). Codes of features 2i, 2i+1 share a byte (low
+        // nibble even). Per 16-token chunk the bytes ([16][64]) and scale codes
+        // ([16][8]) are staged in shared memory; after the four warps meet, 64
+        // threads write one 16-byte piece of a token row each, 16 threads the
+        // rows' 8 scale bytes.
+        const int q = warp & 3;
+        const float G = sc.out_gscale;
+        const float inv6G = 1.0f / (6.0f * G);
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        int chunk = 0;
+        bool ok = true;
+        const int ld_row = p.ld_out / 2;   // bytes per intermediate row (I features)
+        const int ld_sc = p.ld_out / 16;   // scale bytes per intermediate row
+        for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+            const Unit t = decode_unit(p, pref, u);
+            const float f = sc.a_gscale * sc.w_gscale[t.seg];
+            if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) break;
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::ACC_COLS;
+            // intermediate row b_row (the unit's first token), the tile's first feature
+            uint8_t* hrow = p.out_routed + (size_t)t.b_row * ld_row + t.mt * (BM / 2);
+            uint8_t* srow = p.sc_routed + (size_t)t.b_row * ld_sc + t.mt * (BM / 16);
+            for (int c0 = 0; c0 < t.n_valid; c0 += 16, ++chunk) {
+                uint32_t gg[16], uu[16];
+                tmem_ld16(taddr + c0, gg);
+                tmem_ld16(taddr + C::BNX + c0, uu);
+                tmem_ld_wait(gg, uu);
+                uint8_t* b = ep_buf + (chunk & 1) * C::G1_STAGE;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const float a = swiglu(__uint_as_float(gg[j]) * f, __uint_as_float(uu[j]) * f,
+                                           p.swiglu_limit);
+                    float m = fabsf(a);
+#pragma unroll
+                    for (int off = 8; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+                    const __nv_fp8_storage_t s8 = __nv_cvt_float_to_fp8(m * inv6G, __NV_SATFINITE, __NV_E4M3);
+                    const float sv = __half2float(__nv_cvt_fp8_to_halfraw(s8, __NV_E4M3));
+                    const uint32_t code = sv > 0.0f ? e2m1_code(a / (sv * G)) : 0u;
+                    const uint32_t hi = __shfl_down_sync(0xffffffffu, code, 1);
+                    if ((lane & 1) == 0) b[j * 64 + q * 16 + (lane >> 1)] = (uint8_t)(code | (hi << 4));
+                    if ((lane & 15) == 0) b[16 * 64 + j * 8 + q * 2 + (lane >> 4)] = (uint8_t)s8;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ep_bar[chunk & 1]);
+                if (!mbar_wait(&ep_bar[chunk & 1], (uint32_t)(chunk >> 1) & 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const int fidx = q * 32 + lane;  // 16 token rows x 4 pieces of 16 bytes
+                if (fidx < 64) {
+                    const int r = fidx >> 2, pc = fidx & 3;
+                    if (c0 + r < t.n_valid)
+                        *reinterpret_cast<uint4*>(hrow + (size_t)(c0 + r) * ld_row + pc * 16) =
+                            *reinterpret_cast<const uint4*>(b + r * 64 + pc * 16);
+                } else if (fidx < 80) {
+                    const int r = fidx - 64;
+                    if (c0 + r < t.n_valid)
+                        *reinterpret_cast<uint2*>(srow + (size_t)(c0 + r) * ld_sc) =
+                            *reinterpret_cast<const uint2*>(b + 16 * 64 + r * 8);
+                }
+            }
+            if (!ok) break;
+            tc_fence_before();
+            mbar_arrive(&tempty[acc]);
+            if (++acc == C::ACCB) { acc = 0; acc_phase ^= 1; }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+}  // namespace
+
+template <int GEMM>
+cudaError_t launch_nvfp4(const GroupedGemmArgs& a, cudaStream_t st) {
+    using C = TileNV<GEMM>;
+    const cudaError_t attr_err = ensure_smem_limit(
+        reinterpret_cast<const void*>(grouped_gemm_nvfp4_kernel<GEMM>), C::SMEM_BYTES);
+    if (attr_err != cudaSuccess) return attr_err;
+    GroupedGemmArgs r = a;
+    r.S = 0;  // the shared experts are bf16: not part of this launch
+    uint64_t b_rows;
+    KParams p = make_params(r, GEMM, &b_rows);
+    p.bn = C::BNX;
+    if (p.M % (2 * BM)) return cudaErrorInvalidValue;
+    if (GEMM == 1) {
+        p.sc_routed = a.out_routed_scale;  // the epilogue addresses the packed rows itself
+    } else {
+        p.tile_rows = 2 * BM;  // two consecutive 128-row blocks of the down projection per unit
+        p.a_up_offset = BM;
+    }
+    const uint64_t K = p.K, rowsA = (uint64_t)a.E * p.a_rows_per_mat;
+    CUtensorMap tmA, tmSFA, tmSFB;
+    BMaps tmB;
+    if (!make_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.w_routed, rowsA, K / 2, K / 2, NV_ROW,
+                      BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap_2d(&tmSFA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.w_routed_scale, rowsA, K / 16, K / 16,
+                      NV_SF_W, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    if (a.N == 0) return cudaSuccess;
+    if (!make_bmaps(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.b_rows, (uint64_t)a.N, K / 2, NV_ROW) ||
+        !make_tmap_2d(&tmSFB, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.b_scale, (uint64_t)a.N, K / 16, K / 16,
+                      NV_SF_W, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    NVScales s;
+    s.w_gscale = a.w_gscale;
+    s.a_gscale = a.a_gscale;
+    s.out_gscale = a.out_gscale;
+    launch_pdl(grouped_gemm_nvfp4_kernel<GEMM>, grid_for(p), C::THREADS, C::SMEM_BYTES, st, tmA,
+        tmSFA, tmB, tmSFB, p, s);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_nvfp4(const GroupedGemmArgs& a, cudaStream_t st) {
+    return a.gemm == 1 ? launch_nvfp4<1>(a, st) : launch_nvfp4<2>(a, st);
+}
+
+}  // namespace gemm
+}  // namespace moe

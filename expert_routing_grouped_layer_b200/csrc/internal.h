@@ -87,6 +87,19 @@ cudaError_t launch_rmsnorm_quant(int afmt, const void* x, int H, const float* w,
 cudaError_t launch_gather_token_rows(const void* rows, const uint8_t* scales, int H,
                                      const int32_t* sorted_pair, int N, int k, int T, void* out,
                                      uint8_t* out_scale, cudaStream_t st);
+// NVFP4 expert input rows of x bf16 [T][H] with tensor scale g: codes q
+// [T][H/2] (two per byte), E4M3 scale codes qs [T][H/16]; xb (optional) gets a
+// copy of the bf16 rows. H % 256 == 0.
+cudaError_t launch_pack_nvfp4(const void* x, int H, float g, int T, void* q, uint8_t* qs, void* xb,
+                              cudaStream_t st);
+// NVFP4 token rows [T][H/2] with scale rows [T][H/16] gathered into expert order
+// (out row r < N is token sorted_pair[r] / k).
+cudaError_t launch_gather_nvfp4_rows(const void* rows, const uint8_t* scales, int H,
+                                     const int32_t* sorted_pair, int N, int k, int T, void* out,
+                                     uint8_t* out_scale, cudaStream_t st);
+// NVFP4 layers: byte offset of the bf16 rows that follow the packed rows in the
+// expert-input (xa) and intermediate (h) buffers
+inline size_t nvfp4_tail_offset(size_t packed_bytes) { return (packed_bytes + 255) & ~size_t(255); }
 cudaError_t launch_combine(const void* y, const void* shared_y, int S, const int32_t* row_of,
                            const float* w, int T, int k, int H, void* out, cudaStream_t st);
 // one warp waits on a barrier nothing arrives on until the pipeline wait limit;
@@ -113,6 +126,11 @@ struct GroupedGemmArgs {
     uint8_t* out_shared_scale;
     int32_t* status;
     float swiglu_limit;  // gemm1: 0 = off, else SiLU(min(g, L)) * clamp(u, -L, L)
+    // NVFP4 only: per routed expert fp32 tensor scale of the weight, the B
+    // operand's tensor scale, and (gemm1) the quantised intermediate's
+    const float* w_gscale;
+    float a_gscale;
+    float out_gscale;
 };
 cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st);
 

@@ -487,6 +487,67 @@ __global__ void __launch_bounds__(256) rmsnorm_quant_kernel(const uint4* __restr
     }
 }
 
+// NVFP4 expert input rows ("DeepSeek V3架构拆解：Kimi-K2-Thinking-NVFP4的MLA注意力与
+// MoE路由实现原理", 四 NVFP4 量化: the routed experts' input activations in 4-bit
+// floats, groups of 16 with an FP8 scale), with tensor scale g: per group
+// s = E4M3_RNE(amax / (6 g)) and q = E2M1_RNE(v / (e4m3(s) g)), saturating at
+// +-6, zero codes where s is 0. The quotients are formed in double: for bf16 v
+// and fp32 g they are exact enough that every code is the one the definition
+// gives. One warp per token row, one 16-element group per lane per step; the
+// row's codes go to q (two per byte, even element in the low nibble), its scale
+// codes to qs, and, when xb is set, the bf16 row itself to xb (the shared
+// experts' input).
+__device__ __forceinline__ uint32_t e2m1_code_d(double v) {
+    const double a = fabs(v);
+    const uint32_t c = (a > 0.25) + (a >= 0.75) + (a > 1.25) + (a >= 1.75) + (a > 2.5) +
+                       (a >= 3.5) + (a > 5.0);
+    return c | (signbit(v) ? 8u : 0u);
+}
+
+__global__ void __launch_bounds__(256) pack_nvfp4_kernel(const uint4* __restrict__ x, int H, double g,
+                                                         int T, uint2* __restrict__ q,
+                                                         uint8_t* __restrict__ qs,
+                                                         uint4* __restrict__ xb) {
+    pdl_wait();
+    pdl_trigger();
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (t >= T) return;
+    const int G = H / 16;  // groups per row
+    const uint4* row = x + (size_t)t * (H / 8);
+    for (int gi = lane; gi < G; gi += 32) {
+        const uint4 u0 = row[2 * gi], u1 = row[2 * gi + 1];
+        if (xb) {
+            xb[(size_t)t * (H / 8) + 2 * gi] = u0;
+            xb[(size_t)t * (H / 8) + 2 * gi + 1] = u1;
+        }
+        float v[16];
+        const __nv_bfloat162* b0 = reinterpret_cast<const __nv_bfloat162*>(&u0);
+        const __nv_bfloat162* b1 = reinterpret_cast<const __nv_bfloat162*>(&u1);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 f0 = __bfloat1622float2(b0[i]), f1 = __bfloat1622float2(b1[i]);
+            v[2 * i] = f0.x;
+            v[2 * i + 1] = f0.y;
+            v[8 + 2 * i] = f1.x;
+            v[8 + 2 * i + 1] = f1.y;
+        }
+        float amax = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+        const __nv_fp8_storage_t s8 =
+            __nv_cvt_double_to_fp8((double)amax / (6.0 * g), __NV_SATFINITE, __NV_E4M3);
+        const double sg = (double)__half2float(__nv_cvt_fp8_to_halfraw(s8, __NV_E4M3)) * g;
+        uint32_t w[2] = {0u, 0u};
+        if (sg > 0.0) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) w[i >> 3] |= e2m1_code_d((double)v[i] / sg) << (4 * (i & 7));
+        }
+        q[(size_t)t * G + gi] = make_uint2(w[0], w[1]);
+        qs[(size_t)t * G + gi] = (uint8_t)s8;
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_pack_rows(int afmt, const void* x, int H, const int32_t* sorted_pair, int N,
@@ -600,6 +661,24 @@ cudaError_t launch_gather_token_rows(const void* rows, const uint8_t* scales, in
     if (N == 0) return cudaSuccess;
     launch_pdl(gather_rows_kernel, (N + 7) / 8, 256, 0, st, static_cast<const uint4*>(rows), 0,
         H / 16, reinterpret_cast<const uint4*>(scales), H / 32 / 16, sorted_pair, N, k, T, N,
+        static_cast<uint4*>(out), reinterpret_cast<uint4*>(out_scale), nullptr, nullptr);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_pack_nvfp4(const void* x, int H, float g, int T, void* q, uint8_t* qs, void* xb,
+                              cudaStream_t st) {
+    if (T == 0) return cudaSuccess;
+    launch_pdl(pack_nvfp4_kernel, (unsigned)((T + 7) / 8), 256, 0, st, static_cast<const uint4*>(x),
+        H, (double)g, T, static_cast<uint2*>(q), qs, static_cast<uint4*>(xb));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather_nvfp4_rows(const void* rows, const uint8_t* scales, int H,
+                                     const int32_t* sorted_pair, int N, int k, int T, void* out,
+                                     uint8_t* out_scale, cudaStream_t st) {
+    if (N == 0) return cudaSuccess;
+    launch_pdl(gather_rows_kernel, (N + 7) / 8, 256, 0, st, static_cast<const uint4*>(rows), 0,
+        H / 32, reinterpret_cast<const uint4*>(scales), H / 256, sorted_pair, N, k, T, N,
         static_cast<uint4*>(out), reinterpret_cast<uint4*>(out_scale), nullptr, nullptr);
     return cudaGetLastError();
 }

@@ -4,15 +4,22 @@
 // logits = x . Wg^T with an fp32 router weight and fp32 arithmetic. The bf16
 // input x is exact in bf16; the fp32 weight is split exactly enough into three
 // bf16 planes, Wg = hi + mid + lo (hi = bf16(Wg), mid = bf16(Wg - hi),
-// lo = bf16(Wg - hi - mid): 24 significand bits), and one GEMM accumulates
-// x.hi + x.mid + x.lo into the same fp32 tensor-memory accumulator. Every
-// product of two bf16 values is exact in fp32, so the result has fp32-class
-// error like a plain fp32 dot product, at tensor-core throughput.
+// lo = bf16(Wg - hi - mid): 24 significand bits), and the MMAs accumulate
+// x.hi + x.mid + x.lo. Every product of two bf16 values is exact in fp32.
+//
+// Accumulating a whole 7168-wide row in one tensor-memory accumulator (1344
+// MMAs) measured errors that grow with the number of MMAs and lean one way:
+// the largest logits of the 896-expert layer came out up to 1.8e-4 low
+// (4e-5 rms), enough to reorder experts whose scores differ by 1e-5. Here each
+// 64-wide k-block is accumulated afresh (12 MMAs) and the epilogue warps add
+// the k-blocks' fp32 partial sums into fp64 registers, so only 12 MMAs'
+// accumulation error enters per k-block, with signs that vary across
+// k-blocks, plus one rounding of the final value to fp32.
 //
 // Layout: experts are the MMA M operand (128 per tile, the three planes of the
 // same 128 experts are three A tiles of one stage), tokens are N (<= 128).
 // Small batches split K across CTAs; partial sums go to part[split][T][E] and a
-// reduction kernel adds them in split order (deterministic).
+// reduction kernel adds them in split order in fp64 (deterministic).
 #include "gemm_common.cuh"
 
 namespace moe {
@@ -29,6 +36,8 @@ constexpr int RT_B_BYTES = RT_BN * BK * 2;
 constexpr int RT_STAGE_BYTES = 3 * RT_A_BYTES + RT_B_BYTES;
 constexpr int RT_TMEM_COLS = 2 * RT_BN;
 constexpr int RT_SMEM_BYTES = 1024 + RT_STAGES * RT_STAGE_BYTES + 8 * (2 * RT_STAGES + 5) + 16;
+constexpr int RT_EPI_WARPS = 8;  // two per TMEM lane quadrant, each 64 token columns
+constexpr int RT_THREADS = 64 + 32 * RT_EPI_WARPS;
 
 struct RouterParams {
     int T, E, Epad, H;
@@ -109,7 +118,7 @@ __global__ void __launch_bounds__(256) router_split_kernel(const float4* __restr
     }
 }
 
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(RT_THREADS, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ BMaps tmX,
                      const RouterParams p) {
     pdl_wait();
@@ -134,7 +143,7 @@ __global__ void __launch_bounds__(192, 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull[a], 1);
-            mbar_init(&tempty[a], 128);
+            mbar_init(&tempty[a], 32 * RT_EPI_WARPS);
         }
         mbar_init(mma_done, 1);
         *abort_flag = 0;
@@ -191,16 +200,16 @@ __global__ void __launch_bounds__(192, 1)
             uint32_t phase = 0;
             int acc = 0;
             uint32_t acc_phase = 0;
-            for (int u = blockIdx.x; u < total; u += gridDim.x) {
+            bool ok = true;
+            for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
                 const RUnit r = router_unit(p, u);
                 const uint32_t idesc = idesc_bf16(BM, (r.n_valid + 15) & ~15);
-                if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag)) break;
-                tc_fence_after();
-                const uint32_t d = tmem_base + acc * RT_BN;
-                bool ok = true;
                 for (int kb = r.kb0; kb < r.kb1; ++kb) {
+                    // a fresh accumulator per k-block: the epilogue promotes it to fp64
+                    if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag)) { ok = false; break; }
                     if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
                     tc_fence_after();
+                    const uint32_t d = tmem_base + acc * RT_BN;
                     const uint32_t st = smem_u32(smem + stage * RT_STAGE_BYTES);
                     const uint32_t sb = st + 3 * RT_A_BYTES;
 #pragma unroll
@@ -209,14 +218,13 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
                         for (int pl = 0; pl < 3; ++pl)
                             mma_bf16(d, sdesc_kmajor_sw128(st + pl * RT_A_BYTES + kk * 32), bd, idesc,
-                                     (kb != r.kb0 || kk != 0 || pl != 0) ? 1u : 0u);
+                                     (kk != 0 || pl != 0) ? 1u : 0u);
                     }
                     mma_commit(&empty[stage]);
+                    mma_commit(&tfull[acc]);
                     if (++stage == RT_STAGES) { stage = 0; phase ^= 1; }
+                    if (++acc == 2) { acc = 0; acc_phase ^= 1; }
                 }
-                if (!ok) break;
-                mma_commit(&tfull[acc]);
-                if (++acc == 2) { acc = 0; acc_phase ^= 1; }
             }
             mma_commit(mma_done);
             volatile int no_abort = 0;
@@ -224,30 +232,47 @@ __global__ void __launch_bounds__(192, 1)
             if (*abort_flag) status_or(p.status, MOE_DEV_TIMEOUT);
         }
     } else {
+        // epilogue: warp w reads TMEM lane quadrant w % 4 (experts 32*(w%4) ..) and
+        // token columns 64*h .. 64*h+63 of each k-block's accumulator, adding them
+        // into fp64 registers; the unit's sum is rounded once to fp32
         const int q = warp & 3;
+        const int h = (warp - 2) >> 2;
         const int e = q * 32 + lane;  // expert within the M tile
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int u = blockIdx.x; u < total; u += gridDim.x) {
+        bool ok = true;
+        for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
             const RUnit r = router_unit(p, u);
-            if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) break;
-            tc_fence_after();
-            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * RT_BN;
-            const int eg = r.mt * BM + e;
-            float* out = p.part + ((size_t)r.ks * p.T + r.t0) * p.E + eg;
-            for (int c0 = 0; c0 < r.n_valid; c0 += 16) {
-                uint32_t v[16];
-                tmem_ld16(taddr + c0, v);
-                tmem_ld_wait(v);
-                if (eg < p.E) {
+            double sum[64];
 #pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        if (c0 + j < r.n_valid) out[(size_t)(c0 + j) * p.E] = __uint_as_float(v[j]);
+            for (int j = 0; j < 64; ++j) sum[j] = 0.0;
+            for (int kb = r.kb0; kb < r.kb1; ++kb) {
+                if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t taddr =
+                    tmem_base + ((uint32_t)(q * 32) << 16) + acc * RT_BN + (uint32_t)(h * 64);
+#pragma unroll
+                for (int c0 = 0; c0 < 64; c0 += 16) {
+                    if (h * 64 + c0 < r.n_valid) {  // warp-uniform
+                        uint32_t v[16];
+                        tmem_ld16(taddr + c0, v);
+                        tmem_ld_wait(v);
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) sum[c0 + j] += (double)__uint_as_float(v[j]);
+                    }
                 }
+                tc_fence_before();
+                mbar_arrive(&tempty[acc]);
+                if (++acc == 2) { acc = 0; acc_phase ^= 1; }
             }
-            tc_fence_before();
-            mbar_arrive(&tempty[acc]);
-            if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+            if (!ok) break;
+            const int eg = r.mt * BM + e;
+            if (eg < p.E) {
+                float* out = p.part + ((size_t)r.ks * p.T + r.t0) * p.E + eg;
+#pragma unroll
+                for (int j = 0; j < 64; ++j)
+                    if (h * 64 + j < r.n_valid) out[(size_t)(h * 64 + j) * p.E] = (float)sum[j];
+            }
         }
     }
     tc_fence_before();
@@ -315,7 +340,8 @@ cudaError_t launch_router_tc(const void* x, const float* gate_w, void* planes, f
     p.part = part;
     p.status = status;
     const int units = p.mtiles * p.ntiles * p.ksplit;
-    launch_pdl(router_tc_kernel, std::min(units, num_sms()), 192, RT_SMEM_BYTES, st, tmW, tmX, p);
+    launch_pdl(router_tc_kernel, std::min(units, num_sms()), RT_THREADS, RT_SMEM_BYTES, st, tmW, tmX,
+        p);
     cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess && plan.splits > 1) e = launch_router_reduce(part, (long)T * E, plan.splits, st);
     return e;

@@ -49,8 +49,8 @@ class MoEConfig:
     norm_topk_prob: bool
     routed_scaling_factor: float
     score_fn: str  # "sigmoid" | "sqrtsoftplus" | "softmax"
-    wfmt: str  # "bf16" | "fp8_e4m3_b128x128" | "fp4_e2m1_ue8m0_b32" | "mxfp4"
-    afmt: str  # "bf16" | "fp8_e4m3_pow2_b128" | "mxfp8"
+    wfmt: str  # "bf16" | "fp8_e4m3_b128x128" | "fp4_e2m1_ue8m0_b32" | "mxfp4" | "nvfp4"
+    afmt: str  # "bf16" | "fp8_e4m3_pow2_b128" | "mxfp8" | "nvfp4"
     routing: str  # input recipe: "bias_uniform" | "balanced" | "zipf"
     seed: int
     description: str = ""
@@ -99,6 +99,13 @@ CONFIGS = {
         shared_intermediate_size=1024, norm_topk_prob=True, routed_scaling_factor=2.827,
         score_fn="sigmoid", wfmt="mxfp4", afmt="mxfp8", routing="zipf", seed=_SEED + 4,
         description="896 fine-grained experts top-16, 2 shared, MXFP8 x MXFP4, Zipf loads"),
+    "k2_nvfp4": MoEConfig(
+        "k2_nvfp4", T=4096, hidden=7168, n_routed_experts=384, num_experts_per_tok=8, n_group=1,
+        topk_group=1, moe_intermediate_size=2048, n_shared_experts=1,
+        shared_intermediate_size=2048, norm_topk_prob=True, routed_scaling_factor=2.827,
+        score_fn="sigmoid", wfmt="nvfp4", afmt="nvfp4", routing="bias_uniform", seed=_SEED + 5,
+        description="Kimi-K2 shaped, 4096 tokens, NVFP4 routed experts (W4A4, groups of 16 with "
+                    "E4M3 scales), bf16 shared expert"),
 }
 
 # Input recipe constants (see the routing recipes in make_inputs).
@@ -187,6 +194,20 @@ def make_prenorm_inputs(cfg: MoEConfig, x: torch.Tensor):
     return x_resid, norm_w, PRENORM_EPS
 
 
+# NVFP4 tensor scales of the routed experts' activations (calibration
+# constants of the recipe): the input x ~ N(0,1) is covered up to |x| = 16 and
+# the SwiGLU intermediate up to 128, i.e. g = amax / (6 * 448), so a group's
+# scale code stays in E4M3's range with room to spare.
+NVFP4_X_AMAX = 16.0
+NVFP4_H_AMAX = 128.0
+
+
+def nvfp4_act_scales():
+    """(tensor scale of the experts' input, of their intermediate), fp32 values."""
+    return (float(torch.tensor(NVFP4_X_AMAX / (6 * 448), dtype=torch.float32)),
+            float(torch.tensor(NVFP4_H_AMAX / (6 * 448), dtype=torch.float32)))
+
+
 # ------------------------------------------------------------- weight encoding
 _E2M1_GRID = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)
 
@@ -237,6 +258,19 @@ def encode_weight(w: torch.Tensor, wfmt: str):
         e = torch.where(amax > 0, e, torch.full_like(e, -127.0)).clamp(-127, 127)
         codes = _e2m1_codes((blk / torch.exp2(e)[..., None]).float()).reshape(m, rows, cols)
         return _pack_nibbles(codes), (e + 127).to(torch.uint8).contiguous()
+    if wfmt == "nvfp4":
+        # one fp32 tensor scale per matrix, g = amax / (6 * 448); per group of 16
+        # an E4M3 scale code nearest amax_group / (6 g); E2M1 codes of w / (s g)
+        blk = w.reshape(m, rows, cols // 16, 16).double()
+        g = (blk.abs().amax(dim=(1, 2, 3)) / (6 * 448)).float()
+        g = torch.where(g > 0, g, torch.ones_like(g))
+        gd = g.double()[:, None, None]
+        s = (blk.abs().amax(dim=3) / (6 * gd)).clamp(max=448).to(torch.float8_e4m3fn)
+        sv = s.double()
+        safe = torch.where(sv > 0, sv, torch.ones_like(sv))
+        codes = _e2m1_codes((blk / (safe * gd)[..., None]).float())
+        codes = torch.where((sv > 0)[..., None], codes, torch.zeros_like(codes)).reshape(m, rows, cols)
+        return _pack_nibbles(codes), (s.view(torch.uint8).contiguous(), g.contiguous())
     raise ValueError("unknown weight format " + wfmt)
 
 
@@ -259,35 +293,56 @@ def make_weights(cfg: MoEConfig, device="cpu", experts=None):
     out = {}
     for prefix, n_mat, inter, base in (("", E, I, 1000), ("sh_", S, Ish, 10_000_000)):
         which = range(n_mat) if (experts is None or prefix) else sorted(set(int(e) for e in experts))
+        fmt = shared_wfmt(cfg) if prefix else cfg.wfmt
         for name, rows, cols, off in (("w13", 2 * inter, H, 0), ("w2", H, inter, 1)):
-            data = scale = None
+            data = scale = gscale = None
             for e in which:
-                d, s = encode_weight(draw(base + 2 * e + off, rows, cols), cfg.wfmt)
+                d, s = encode_weight(draw(base + 2 * e + off, rows, cols), fmt)
+                g = None
+                if isinstance(s, tuple):  # NVFP4: (group scale codes, tensor scale)
+                    s, g = s
                 if data is None:
                     data = torch.zeros((n_mat,) + tuple(d.shape[1:]), dtype=d.dtype, device=dev)
                     if s is not None:
                         scale = torch.zeros((n_mat,) + tuple(s.shape[1:]), dtype=s.dtype, device=dev)
+                    if g is not None:
+                        gscale = torch.ones(n_mat, dtype=torch.float32, device=dev)
                 data[e] = d[0]
                 if s is not None:
                     scale[e] = s[0]
+                if g is not None:
+                    gscale[e] = g[0]
             out[prefix + name] = data
             out[prefix + name + "_scale"] = scale
+            if gscale is not None:
+                out[prefix + name + "_gscale"] = gscale
     return out
 
 
-def weight_bytes_per_matrix(cfg: MoEConfig, inter: int) -> int:
-    """Stored bytes (data + scales) of one expert's w13 plus w2."""
+def shared_wfmt(cfg: MoEConfig) -> str:
+    """Weight format of the shared experts: the routed experts' format, except
+    that NVFP4 layers keep them in bf16 (the NVFP4 recipe's exclusion list)."""
+    return "bf16" if cfg.wfmt == "nvfp4" else cfg.wfmt
+
+
+def weight_bytes_per_matrix(cfg: MoEConfig, inter: int, shared: bool = False) -> int:
+    """Stored bytes (data + scales) of one expert's w13 plus w2 (a shared expert's
+    when shared is set)."""
     P = 3 * cfg.hidden * inter
-    if cfg.wfmt == "bf16":
+    fmt = shared_wfmt(cfg) if shared else cfg.wfmt
+    if fmt == "bf16":
         return 2 * P
-    if cfg.wfmt == "fp8_e4m3_b128x128":
+    if fmt == "nvfp4":
+        return P // 2 + P // 16 + 8  # codes, group scales, two tensor scales
+    if fmt == "fp8_e4m3_b128x128":
         return P + 4 * (P // (128 * 128))
     return P // 2 + P // 32
 
 
 def expert_slice(weights: dict, e: int, shared: bool = False):
     """(w13, w13_scale, w2, w2_scale) of one matrix, as host numpy arrays with a
-    leading dimension of 1 (bf16 returned as uint16 codes)."""
+    leading dimension of 1 (bf16 returned as uint16 codes); NVFP4 routed experts
+    add their two tensor scales (w13_gscale, w2_gscale) as a 6-tuple."""
     p = "sh_" if shared else ""
 
     def host(t):
@@ -299,8 +354,11 @@ def expert_slice(weights: dict, e: int, shared: bool = False):
         a = t.cpu().numpy()
         return a.view("uint16") if a.dtype.name == "int16" else a
 
-    return (host(weights[p + "w13"]), host(weights[p + "w13_scale"]), host(weights[p + "w2"]),
-            host(weights[p + "w2_scale"]))
+    out = (host(weights[p + "w13"]), host(weights[p + "w13_scale"]), host(weights[p + "w2"]),
+           host(weights[p + "w2_scale"]))
+    if weights.get(p + "w13_gscale") is not None:
+        out = out + (host(weights[p + "w13_gscale"]), host(weights[p + "w2_gscale"]))
+    return out
 
 
 def bf16_codes(x: torch.Tensor):

@@ -87,6 +87,13 @@ typedef enum {
 #define MOE_W_FP8_E4M3_B128x128 1
 #define MOE_W_FP4_E2M1_UE8M0_B32 2
 #define MOE_W_MXFP4 3
+/* NVFP4 ([V3] 四 NVFP4 量化): routed experts only, with MOE_A_NVFP4. uint8, two
+ * E2M1 codes per byte (even column in the low nibble) + uint8 E4M3 scale code
+ * per 16 columns (w13_scale [E][2I][H/16], w2_scale [E][H][I/16]) + one fp32
+ * tensor scale per expert matrix (moe_weights.w13_gscale / w2_gscale [E]):
+ * value = e2m1 * e4m3(scale) * tensor scale. The shared experts stay bf16
+ * (the recipe's exclusion list): sh_w13 / sh_w2 hold bf16 values. */
+#define MOE_W_NVFP4 4
 
 /* activation formats the experts consume (the router always reads bf16 x)
  *  BF16:               no quantisation.
@@ -100,6 +107,14 @@ typedef enum {
 #define MOE_A_BF16 0
 #define MOE_A_FP8_E4M3_POW2_B128 1
 #define MOE_A_MXFP8 2
+/* NVFP4 activations of the routed experts (with MOE_W_NVFP4 only): E2M1 codes
+ * (two per byte) + E4M3 scale code per 16 elements + a per-tensor fp32 scale g
+ * (moe_config.nvfp4_x_scale for the experts' input, nvfp4_h_scale for their
+ * intermediate): per 16-group s = E4M3_RNE(amax / (6 g)) and
+ * q = E2M1_RNE(v / (e4m3(s) g)) (saturating at +-6; zero codes where s is 0),
+ * decided in double precision for the bf16 input rows. The shared experts read
+ * the bf16 input. */
+#define MOE_A_NVFP4 3
 
 /* Layer configuration; field names follow the configuration the pages quote. */
 typedef struct {
@@ -119,6 +134,10 @@ typedef struct {
     /* [V4] 架构 FFNSwiGLU's optional swiglu_limit: 0 = off; L > 0 computes
      * SiLU(min(g, L)) * clamp(u, -L, L) in every expert (finite, >= 0) */
     float swiglu_limit;
+    /* NVFP4 tensor scales of the routed experts' activations (used only with
+     * MOE_A_NVFP4; calibrated constants, > 0): the input x, the intermediate h */
+    float nvfp4_x_scale;
+    float nvfp4_h_scale;
 } moe_config;
 
 /* Device pointers to the layer's parameters.
@@ -131,6 +150,8 @@ typedef struct {
     const void *w13, *w13_scale, *w2, *w2_scale;
     const void *sh_w13, *sh_w13_scale, *sh_w2, *sh_w2_scale;
     const float *gate_w, *gate_bias;
+    /* NVFP4 only: fp32 tensor scale of each routed expert's w13 and w2 [E] */
+    const float *w13_gscale, *w2_gscale;
 } moe_weights;
 
 /* Bytes of device workspace that moe_layer_forward needs for T tokens; every

@@ -12,7 +12,8 @@ import oracle
 from expert_routing_grouped_layer_b200 import workloads as W
 
 WEIGHT_REL_TOL = 1e-5  # top-k weights: fp32 against float64
-LAYER_TOL = {"bf16": 1e-2, "fp8_e4m3_pow2_b128": 2e-2, "mxfp8": 2e-2}  # rel-L2 of the output
+LAYER_TOL = {"bf16": 1e-2, "fp8_e4m3_pow2_b128": 2e-2, "mxfp8": 2e-2,
+             "nvfp4": 2e-2}  # rel-L2 of the output
 
 
 def gpu_forward(cfg, inp, wts, T=None):
@@ -46,14 +47,19 @@ def oracle_route(cfg, inp, tokens=None, T=None):
 
 def compare_routing(cfg, g, r, tokens):
     """Expert sets equal and weights within tolerance for every token the oracle
-    does not report as a near-tie. Returns the number of near-tie tokens."""
+    does not report as a near-tie, and the slot order (biased score descending)
+    equal wherever the oracle does not report it as an order near-tie. Returns
+    the number of near-tie tokens."""
     n_tie = 0
+    otie = r.get("order_tie")
     for i, t in enumerate(tokens):
         if r["near_tie"][i]:
             n_tie += 1
             continue
         gi, oi = g["idx"][t], r["idx"][i]
         assert set(gi.tolist()) == set(oi.tolist()), "token %d: gpu %s oracle %s" % (t, gi, oi)
+        if otie is not None and not otie[i]:
+            assert np.array_equal(gi, oi), "token %d slot order: gpu %s oracle %s" % (t, gi, oi)
         gw = dict(zip(gi.tolist(), g["w"][t].tolist()))
         for e, w in zip(oi.tolist(), r["w"][i].tolist()):
             assert abs(gw[e] - w) <= WEIGHT_REL_TOL * abs(w), "token %d expert %d" % (t, e)
@@ -79,7 +85,17 @@ def check_permutation_properties(cfg, g, T=None):
 def oracle_layer_rows(cfg, inp, wts, idx, w, tokens):
     """Oracle output for the listed tokens with the oracle's own routing."""
     x = W.bf16_codes(inp["x"][torch.as_tensor(tokens, dtype=torch.long, device=inp["x"].device)])
-    return oracle.layer(cfg, x, idx, w, lambda e: W.expert_slice(wts, e),
+    return oracle_layer(cfg, x, idx, w, wts)
+
+
+def oracle_layer(cfg, x_codes, idx, w, wts):
+    """The oracle's layer output for bf16 token rows given their routing, in the
+    layer's weight format (NVFP4 layers: NVFP4 routed experts, bf16 shared)."""
+    if cfg.wfmt == "nvfp4":
+        return oracle.layer_nvfp4(cfg, x_codes, idx, w, lambda e: W.expert_slice(wts, e),
+                                  lambda s: W.expert_slice(wts, s, shared=True),
+                                  W.nvfp4_act_scales())
+    return oracle.layer(cfg, x_codes, idx, w, lambda e: W.expert_slice(wts, e),
                         lambda s: W.expert_slice(wts, s, shared=True))
 
 
@@ -94,25 +110,32 @@ def rel_l2_rows(a, b):
 
 def compare_permutation_exact(cfg, g, r):
     """The GPU permutation against the oracle's (the oracle's stable sort of its
-    own routing), element by element: offsets, sorted_pair and row_of in full when
-    no token is a near-tie, else the block of every expert that no near-tie token
-    (by either side's choice) touches. Returns the number of experts compared."""
-    E = cfg.n_routed_experts
+    own routing of every token), element by element, on the block of every
+    expert that no near-tie token (by either side's choice) touches: the tokens
+    of each block in order exactly, and each entry's pair index exactly unless
+    that token's slot order is itself an oracle-reported near-tie. With no
+    near-ties at all the offsets and the row_of inverse are compared whole.
+    Returns the number of experts compared."""
+    E, k = cfg.n_routed_experts, cfg.num_experts_per_tok
     off, sp, ro = oracle.permute(r["idx"], E)
     tie = np.nonzero(r["near_tie"])[0]
+    otie = r.get("order_tie", np.zeros(len(r["near_tie"]), bool))
+    touched = set(g["idx"][tie].ravel().tolist()) | set(r["idx"][tie].ravel().tolist())
     if tie.size == 0:
         assert np.array_equal(g["offsets"], off)
-        assert np.array_equal(g["sorted_pair"], sp)
-        assert np.array_equal(g["row_of"], ro)
-        return E
-    touched = set(g["idx"][tie].ravel().tolist()) | set(r["idx"][tie].ravel().tolist())
+        if not otie.any():
+            assert np.array_equal(g["sorted_pair"], sp)
+            assert np.array_equal(g["row_of"], ro)
+            return E
     n = 0
     for e in range(E):
         if e in touched:
             continue
         a = g["sorted_pair"][g["offsets"][e]:g["offsets"][e + 1]]
         b = sp[off[e]:off[e + 1]]
-        assert np.array_equal(a, b), "expert %d block differs" % e
+        assert np.array_equal(a // k, b // k), "expert %d: token order differs" % e
+        keep = ~otie[b // k]
+        assert np.array_equal(a[keep], b[keep]), "expert %d: slot indices differ" % e
         n += 1
     return n
 

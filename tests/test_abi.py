@@ -35,9 +35,10 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_struct_layouts_match_header():
-    assert ctypes.sizeof(moe.moe_config) == 14 * 4
+    assert ctypes.sizeof(moe.moe_config) == 16 * 4
     assert moe.moe_config.swiglu_limit.offset == 13 * 4  # appended after afmt
-    assert ctypes.sizeof(moe.moe_weights) == 10 * 8
+    assert moe.moe_config.nvfp4_h_scale.offset == 15 * 4
+    assert ctypes.sizeof(moe.moe_weights) == 12 * 8
 
 
 def cfg(**kw):

@@ -72,7 +72,7 @@ def test_clock_log_path():
 
 
 @pytest.mark.parametrize("name,count", [("k2_decode_bf16", 9), ("k2_prefill_fp8w", 12),
-                                        ("v4_fp4", 12), ("mx896", 11)])
+                                        ("v4_fp4", 12), ("mx896", 11), ("k2_nvfp4", 14)])
 def test_launch_count_matches_the_launch_lists(name, count):
     """The kernels one step of each workload launches on a 148-SM B200, as the
     ncu launch lists of the four workloads show them (one-kernel permutation up
@@ -92,6 +92,12 @@ def test_tensor_peak_prefers_a_measured_fp8_rate():
     # bf16-rate layers keep the bf16 figure
     p, _ = bench.tensor_peak(peaks, "measured", W.CONFIGS["k2_prefill_fp8w"], meas)
     assert p == 1651.4
+    # NVFP4 layers take the NVFP4 rate, never an FP8 one
+    p, src = bench.tensor_peak(peaks, "measured", W.CONFIGS["k2_nvfp4"],
+                               dict(meas, nvfp4_block16=6000.0))
+    assert p == 6000.0 and "nvfp4" in src
+    p, src = bench.tensor_peak(peaks, "measured", W.CONFIGS["k2_nvfp4"], meas)
+    assert p == pytest.approx(4 * 1651.4) and "nominal" in src
 
 
 def test_roofline_flags_fractions_above_the_measured_peak():

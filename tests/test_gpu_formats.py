@@ -7,36 +7,33 @@ import torch
 import expert_routing_grouped_layer_b200 as moe
 import oracle
 from expert_routing_grouped_layer_b200 import workloads as W
-from moe_testlib import (LAYER_TOL, check_permutation_properties, compare_routing, gpu_forward,
-                         oracle_layer_rows, oracle_route, rel_l2)
+from moe_testlib import (LAYER_TOL, check_layer_tokens, check_permutation_properties,
+                         chosen_tokens, compare_permutation_exact, compare_routing, gpu_forward,
+                         oracle_route)
 
 pytestmark = pytest.mark.gpu
 
 
 def _layer_check(cfg, T=None, sample=None, seed=0):
+    """Routing of every token against the oracle (sets and weights, near-ties
+    excepted), the permutation element by element, and the layer output token
+    by token: every token when sample is None, else the chosen tokens (a seeded
+    sample plus the tokens at ragged tile ends)."""
     T = cfg.T if T is None else T
     inp = W.make_inputs(cfg, "cuda")
     wts = W.make_weights(cfg, "cuda")
     g = gpu_forward(cfg, inp, wts, T)
     assert g["status"] == 0
-    if sample is None:
-        toks = np.arange(T)
-        r = oracle_route(cfg, inp, T=T)
-        rs = r
-    else:
-        toks = np.sort(np.random.default_rng(seed).choice(T, sample, replace=False))
-        r = oracle_route(cfg, inp, T=T) if T <= 8192 else None
-        rs = oracle_route(cfg, inp, tokens=toks.astype(np.int32), T=T)
-    if r is not None:
-        compare_routing(cfg, g, r, np.arange(T))
-    else:
-        compare_routing(cfg, g, rs, toks)
+    r = oracle_route(cfg, inp, T=T)  # every token
+    compare_routing(cfg, g, r, np.arange(T))
     check_permutation_properties(cfg, g, T)
-    ok = ~rs["near_tie"]
-    want = oracle_layer_rows(cfg, inp, wts, rs["idx"], rs["w"], toks)
-    err = rel_l2(g["out"][toks][ok], want[ok])
-    assert err <= LAYER_TOL[cfg.afmt], err
-    return g, err
+    compare_permutation_exact(cfg, g, r)
+    if sample is None:
+        toks = np.nonzero(~r["near_tie"])[0]
+    else:
+        toks = chosen_tokens(cfg, g, r, sample, seed)
+    err = check_layer_tokens(cfg, inp, wts, g, r, toks, LAYER_TOL[cfg.afmt])
+    return g, float(err.max())
 
 
 FP8_TINY = W.CONFIGS["tiny_bf16"].replace(wfmt="fp8_e4m3_b128x128")
