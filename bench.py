@@ -467,6 +467,24 @@ def measure(args, cfg, rank, world, dev, steps, warmup, n_stage, n_e2e, workload
     torch.cuda.synchronize()
     stage = [[sevents[i][j].elapsed_time(sevents[i][j + 1]) for i in range(n_stage)]
              for j in range(6)]
+    # the fused prologue (post-attention RMSNorm + activation quantisation) as its
+    # own stage, on the workload's x scaled into an un-normalised hidden state
+    xr, nw, eps = W.make_prenorm_inputs(cfg, x)
+    xn = torch.empty_like(x)
+    qa = cfg.afmt in ("fp8_e4m3_pow2_b128", "mxfp8")
+    xq = torch.empty(T, H, dtype=torch.uint8, device=dev) if qa else None
+    xqs = torch.empty(T, H // 32, dtype=torch.uint8, device=dev) if qa else None
+    pro_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(n_stage)]
+    for e0, e1 in pro_ev:
+        flush.zero_()
+        e0.record(stream)
+        moe.moe_rmsnorm_prologue(ccfg, xr, T, nw, eps, xn, xq, xqs, stream=sp)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    pro_ms = statistics.fmean(e0.elapsed_time(e1) for e0, e1 in pro_ev)
+    pro_bytes = 4 * T * H + ((T * H + T * H // 32) if qa else 0)
+    del xr, xn, xq, xqs
     offsets = layer.intermediate(T, moe.WS_OFFSETS, torch.int32, (E + 1,)).cpu()
     counts = offsets[1:] - offsets[:-1]
     active = int((counts > 0).sum())
@@ -545,6 +563,12 @@ def measure(args, cfg, rank, world, dev, steps, warmup, n_stage, n_e2e, workload
         "roofline": kroof,
         "layer_roofline": lroof,
         "stage_ms": stage_ms,
+        "prologue": {"kernel": "moe_rmsnorm_prologue (RMSNorm + act quant, one pass)",
+                     "ms": pro_ms, "bytes": pro_bytes,
+                     "achieved_gbs": pro_bytes / (pro_ms / 1e3) / 1e9,
+                     "hbm_frac": pro_bytes / (pro_ms / 1e3) / 1e9 / load_peaks()[0]["hbm_gbs"],
+                     "note": "not part of the timed layer step (the layer's input is the "
+                             "normalised x); timed separately, L2 flushed before each call"},
         "stage_ms_source": "staged entry points with events between them, %d separate steps "
                            "(the timed steps record events only at their ends and around "
                            "gate_up)" % n_stage,
@@ -620,7 +644,7 @@ def run_ours(args, rank, world, dev):
                                   0 if args.no_e2e else min(args.per_workload_steps, 10),
                                   name, fp8_measured)
             keep = ("value", "ms_per_step", "steps", "warmup", "dtype", "config", "routing_stats",
-                    "roofline",
+                    "prologue", "roofline",
                     "layer_roofline", "stage_ms", "gpu_launches", "clocks", "e2e")
             per[name] = {k: f[k] for k in keep}
             per[name]["unit"] = UNIT

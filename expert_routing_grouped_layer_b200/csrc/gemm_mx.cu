@@ -16,8 +16,8 @@ namespace {
 // tcgen05.mma kind::mxf8f6f4 applies both scales inside the MMA, so the FP4
 // weights are never dequantised in software: TMA expands each packed row of
 // 128 E2M1 values to the one-byte-per-value layout the MMA reads
-// (16U4_ALIGN16B). Scales travel by TMA as 128 rows x 32 bytes (32 k-blocks)
-// into a two-slot ring. The MMA reads row m's scale (m = m0 + 32*m1) from
+// (16U4_ALIGN16B). Scales travel by TMA as 128 rows x 32 bytes (32 k-blocks,
+// 32-byte swizzle) into a two-slot ring. The MMA reads row m's scale (m = m0 + 32*m1) from
 // TMEM lane m0 of every lane quadrant, column m1, one k-block per byte. Four
 // scale warps, one per lane quadrant, store each stage's 4 k-blocks in that
 // order (tcgen05.st) into a ring of TMEM column sets: a tcgen05.cp issued by
@@ -349,13 +349,19 @@ __global__ void __launch_bounds__(TileMX<GEMM, NA_, BNX_, ACCB_>::THREADS, 1)
                 }
                 if ((kb & 3) == 0) {
                     // the next four stages' bytes of this lane's four rows, one 16-byte
-                    // load per row; after the group's last such load the slot is free
-                    const uint8_t* raw = sf_ring + sfs * C::RAW_BYTES + 16 * ((kb % SF_STAGES) >> 2);
+                    // load per row; after the group's last such load the slot is free.
+                    // The boxes arrive with a 32-byte swizzle: 16-byte piece c of row m
+                    // sits at piece c ^ ((m >> 2) & 1), so the eight lanes of a load
+                    // phase hit distinct banks (rows 32 bytes apart unswizzled put
+                    // lanes m and m + 4 on one bank).
+                    const uint8_t* raw = sf_ring + sfs * C::RAW_BYTES;
+                    const int sf_swz = 16 * (((kb % SF_STAGES) >> 2) ^ ((lane >> 2) & 1));
 #pragma unroll
                     for (int i = 0; i < C::NOPS; ++i)
 #pragma unroll
                         for (int r = 0; r < 4; ++r)
-                            cache[i][r] = *reinterpret_cast<const uint4*>(raw + i * SF_TILE + SF_KB * (lane + 32 * r));
+                            cache[i][r] = *reinterpret_cast<const uint4*>(
+                                raw + i * SF_TILE + SF_KB * (lane + 32 * r) + sf_swz);
                     if (kb % SF_STAGES == SF_STAGES - 4 || kb + 4 >= KB) {
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&sf_empty[sfs]);
@@ -566,14 +572,14 @@ cudaError_t launch_mx(const GroupedGemmArgs& a, cudaStream_t st) {
         !make_tmap_2d(&tmAs, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, wAs, rowsAs, K, K / 2, MX_BK, BM,
                       CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_tmap_2d(&tmSFA, CU_TENSOR_MAP_DATA_TYPE_UINT8, sA, rowsA, K / 32, K / 32, SF_KB, 128,
-                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
+                      CU_TENSOR_MAP_SWIZZLE_32B) ||
         !make_tmap_2d(&tmSFAs, CU_TENSOR_MAP_DATA_TYPE_UINT8, sAs, rowsAs, K / 32, K / 32, SF_KB, 128,
-                      CU_TENSOR_MAP_SWIZZLE_NONE))
+                      CU_TENSOR_MAP_SWIZZLE_32B))
         return cudaErrorInvalidValue;
     if (b_rows == 0) return cudaSuccess;
     if (!make_bmaps(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.b_rows, b_rows, K, MX_BK) ||
         !make_tmap_2d(&tmSFB, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.b_scale, b_rows, K / 32, K / 32, SF_KB,
-                      C::SFB_ROWS, CU_TENSOR_MAP_SWIZZLE_NONE))
+                      C::SFB_ROWS, CU_TENSOR_MAP_SWIZZLE_32B))
         return cudaErrorInvalidValue;
     launch_pdl(grouped_gemm_mx_kernel<GEMM, AFMT, NA_, BNX_, ACCB_>, grid_for(p), C::THREADS,
         C::SMEM_BYTES, st, tmA, tmAs, tmSFA, tmSFAs, tmB, tmSFB, p);

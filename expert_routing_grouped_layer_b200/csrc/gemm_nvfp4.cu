@@ -8,7 +8,8 @@
 // expansion to one byte per value). tcgen05.mma kind::mxf4nvf4 with
 // scale_vec::4X reads, for every row of A and of B, one 32-bit tensor-memory
 // word per MMA (K = 64): its four bytes are the E4M3 scales of the four
-// 16-element groups. Row m = m0 + 32*m1 of an operand sits in lane m0 of every
+// 16-element groups (scale boxes of 128 rows x 64 bytes, 64-byte swizzle).
+// Row m = m0 + 32*m1 of an operand sits in lane m0 of every
 // lane quadrant, column m1; four scale warps (one per quadrant) store each
 // stage's 16 columns per operand ([MMA kk][m1]) with tcgen05.st. The per-tensor
 // fp32 scales (the expert's weight scale times the activation scale) multiply
@@ -17,9 +18,8 @@
 //
 // Tile: two 128-row weight tiles per unit (gate and up for GEMM1, two
 // consecutive 128-row blocks of the down projection for GEMM2) sharing one
-// token tile of up to 96 rows, each with its own MMA-issuing thread and
-// accumulator, accumulators double-buffered. Warps: 0 TMA, 1 MMA (tile 0),
-// 2-5 epilogue, 6-9 scale warps, 10 MMA (tile 1).
+// token tile (96 rows with double-buffered accumulators, or 128 with one
+// buffer), each weight tile with its own MMA-issuing thread and accumulator.
 #include <cuda_fp4.h>
 
 #include "gemm_common.cuh"
@@ -34,14 +34,20 @@ constexpr int NV_SF_STAGES = 4;     // stages per scale box
 constexpr int NV_SF_W = 16 * NV_SF_STAGES;  // scale bytes per row per box (64)
 constexpr int NV_SF_TILE = 128 * NV_SF_W;   // one operand's scale box: 128 rows
 
-template <int GEMM>
+// GEMM: 1 gate/up, 2 down. BNX_: tokens per tile. ACCB_: accumulator buffers
+// (2 overlaps a tile's epilogue with the next tile's main loop; 1 lets wider
+// token tiles fit tensor memory and takes two epilogue groups on alternating
+// 16-token chunks). Warps: 0 TMA, 1 MMA (tile 0), then EG groups of 4 epilogue
+// warps, then the 4 scale warps, then the MMA warp of tile 1.
+template <int GEMM, int BNX_, int ACCB_>
 struct TileNV {
     static constexpr int NA = 2;
-    static constexpr int BNX = 96;
-    static constexpr int ACCB = 2;
-    static constexpr int SCALE_WARP = 6;
-    static constexpr int MMA2_WARP = 10;
-    static constexpr int THREADS = 32 * 11;
+    static constexpr int BNX = BNX_;
+    static constexpr int ACCB = ACCB_;
+    static constexpr int EG = ACCB == 1 ? 2 : 1;
+    static constexpr int SCALE_WARP = 2 + 4 * EG;
+    static constexpr int MMA2_WARP = SCALE_WARP + 4;
+    static constexpr int THREADS = 32 * (MMA2_WARP + 1);
     static constexpr int NOPS = NA + 1;  // scale operands: the two A tiles, the token rows
     static constexpr int A_BYTES = BM * NV_ROW;
     static constexpr int B_BYTES = BNX * NV_ROW;
@@ -50,11 +56,13 @@ struct TileNV {
     static constexpr int STAGE_BYTES = (B_OFF + B_BYTES + 1023) / 1024 * 1024;
     static constexpr int RAW_BYTES = NOPS * NV_SF_TILE;
     static constexpr int RING_BYTES = 2 * RAW_BYTES;
-    // staged epilogue chunk, two per parity: down [16 tokens][128] bf16;
+    // staged epilogue chunks, per group and parity: down [16 tokens][128] bf16;
     // gate/up [16 tokens][64] code bytes then [16][8] scale codes
     static constexpr int G1_STAGE = 16 * 64 + 16 * 8;
-    static constexpr int EPI_BYTES = (GEMM == 2 ? 2 * 16 * BM * 2 : 2 * G1_STAGE) + 128;
-    static constexpr int FIXED_BYTES = 1024 + 8 * (3 * 6 + 13) + 16 + 4 * (MAX_SEG + 1) + EPI_BYTES;
+    static constexpr int GROUP_EPI = GEMM == 2 ? 2 * 16 * BM * 2 : 2 * G1_STAGE;
+    static constexpr int EPI_BYTES = EG * GROUP_EPI + 128;
+    static constexpr int NBARS = 11 + 2 * EG;  // besides the 3 per stage
+    static constexpr int FIXED_BYTES = 1024 + 8 * (3 * 6 + NBARS + 2) + 16 + 4 * (MAX_SEG + 1) + EPI_BYTES;
     static constexpr int STAGES = stages_for(STAGE_BYTES, FIXED_BYTES + RING_BYTES, 6);
     static constexpr int ACC_COLS = NA * BNX;
     static constexpr int TMEM_COLS = 512;
@@ -63,10 +71,12 @@ struct TileNV {
     static constexpr int NSETS_FIT = (TMEM_COLS - SF_COL) / SET_COLS;
     static constexpr int NSETS = NSETS_FIT < STAGES ? NSETS_FIT : STAGES;
     static_assert(NSETS >= 2, "tensor memory budget: two scale sets");
-    static constexpr int BAR_BYTES = 8 * (3 * STAGES + 13) + 16;
+    static constexpr int BAR_BYTES = 8 * (3 * STAGES + NBARS + 2) + 16;
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + RING_BYTES + BAR_BYTES +
                                       4 * (MAX_SEG + 1) + EPI_BYTES;
-    static_assert(STAGES >= 2 && SMEM_BYTES <= 232448, "shared memory budget");
+    static_assert(STAGES >= 3 && SMEM_BYTES <= 232448, "shared memory budget");
+    // one 128-row scale box (and four TMEM columns per MMA) covers the token rows
+    static_assert(BNX % 16 == 0 && BNX <= 128, "token tile");
 };
 
 // Instruction descriptor, kind::mxf4nvf4 block-scaled: A and B E2M1 (format 1),
@@ -128,8 +138,8 @@ struct NVScales {
     float out_gscale;       // GEMM1: tensor scale of the quantised intermediate
 };
 
-template <int GEMM>
-__global__ void __launch_bounds__(TileNV<GEMM>::THREADS, 1)
+template <int GEMM, int BNX_, int ACCB_>
+__global__ void __launch_bounds__(TileNV<GEMM, BNX_, ACCB_>::THREADS, 1)
     grouped_gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmA,
                               const __grid_constant__ CUtensorMap tmSFA,
                               const __grid_constant__ BMaps tmB,
@@ -137,7 +147,7 @@ __global__ void __launch_bounds__(TileNV<GEMM>::THREADS, 1)
                               const NVScales sc) {
     pdl_wait();
     pdl_trigger();
-    using C = TileNV<GEMM>;
+    using C = TileNV<GEMM, BNX_, ACCB_>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -150,8 +160,8 @@ __global__ void __launch_bounds__(TileNV<GEMM>::THREADS, 1)
     uint64_t* mma_done = tempty + 2;
     uint64_t* sf_full = mma_done + 1;  // [2]
     uint64_t* sf_empty = sf_full + 2;  // [2]
-    uint64_t* ep_bar = sf_empty + 2;   // [2] the epilogue warps' staged chunk
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ep_bar + 2);
+    uint64_t* ep_bar = sf_empty + 2;   // [group][parity]: an epilogue group's staged chunk
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ep_bar + 2 * C::EG);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* pref = reinterpret_cast<int*>(tmem_slot + 4);
     uint8_t* ep_buf = reinterpret_cast<uint8_t*>(
@@ -168,14 +178,14 @@ __global__ void __launch_bounds__(TileNV<GEMM>::THREADS, 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull[a], C::NA);
-            mbar_init(&tempty[a], 128);
+            mbar_init(&tempty[a], 128 * C::EG);
         }
         mbar_init(mma_done, C::NA);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sf_full[i], 1);
             mbar_init(&sf_empty[i], 4);
-            mbar_init(&ep_bar[i], 4);
         }
+        for (int i = 0; i < 2 * C::EG; ++i) mbar_init(&ep_bar[i], 4);
         *abort_flag = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tmA);
@@ -320,7 +330,11 @@ __global__ void __launch_bounds__(TileNV<GEMM>::THREADS, 1)
                         break;
                     }
                 }
-                const uint8_t* raw = sf_ring + sfs * C::RAW_BYTES + 16 * (kb % NV_SF_STAGES);
+                // the boxes arrive with a 64-byte swizzle: 16-byte piece c of row m sits
+                // at piece c ^ ((m >> 1) & 3), so the eight lanes of a load phase hit
+                // distinct banks (unswizzled, rows 64 bytes apart share banks 4 ways)
+                const uint8_t* raw = sf_ring + sfs * C::RAW_BYTES +
+                                     16 * ((kb % NV_SF_STAGES) ^ ((lane >> 1) & 3));
                 uint4 row[C::NOPS][4];
 #pragma unroll
                 for (int i = 0; i < C::NOPS; ++i)
@@ -357,8 +371,10 @@ __global__ void __launch_bounds__(TileNV<GEMM>::THREADS, 1)
         // [16 tokens][128] tile (two, alternating), the four warps meet at an
         // mbarrier, and warp q writes token rows 4q..4q+3 with 16-byte stores
         const int q = warp & 3;
+        const int grp = (warp - 2) >> 2;
         const int row = q * 32 + lane;
-        __nv_bfloat16* gbuf = reinterpret_cast<__nv_bfloat16*>(ep_buf);
+        __nv_bfloat16* gbuf = reinterpret_cast<__nv_bfloat16*>(ep_buf + grp * C::GROUP_EPI);
+        uint64_t* gbar = ep_bar + 2 * grp;
         int acc = 0;
         uint32_t acc_phase = 0;
         int chunk = 0;
@@ -373,7 +389,7 @@ __global__ void __launch_bounds__(TileNV<GEMM>::THREADS, 1)
                 const uint32_t taddr =
                     tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::ACC_COLS + w * C::BNX;
                 __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(t.out) + t.mt * p.tile_rows + w * BM;
-                for (int c0 = 0; c0 < t.n_valid; c0 += 16, ++chunk) {
+                for (int c0 = 16 * grp; c0 < t.n_valid; c0 += 16 * C::EG, ++chunk) {
                     uint32_t gq[16];
                     tmem_ld16(taddr + c0, gq);
                     tmem_ld_wait(gq);
@@ -382,8 +398,8 @@ __global__ void __launch_bounds__(TileNV<GEMM>::THREADS, 1)
                     for (int j = 0; j < 16; ++j)
                         buf[j * BM + row] = __float2bfloat16_rn(__uint_as_float(gq[j]) * f);
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&ep_bar[chunk & 1]);
-                    if (!mbar_wait(&ep_bar[chunk & 1], (uint32_t)(chunk >> 1) & 1u, abort_flag)) {
+                    if (lane == 0) mbar_arrive(&gbar[chunk & 1]);
+                    if (!mbar_wait(&gbar[chunk & 1], (uint32_t)(chunk >> 1) & 1u, abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -412,6 +428,9 @@ __global__ void __launch_bounds__(TileNV<GEMM>::THREADS, 1)
         // threads write one 16-byte piece of a token row each, 16 threads the
         // rows' 8 scale bytes.
         const int q = warp & 3;
+        const int grp = (warp - 2) >> 2;
+        uint8_t* gstage = ep_buf + grp * C::GROUP_EPI;
+        uint64_t* gbar = ep_bar + 2 * grp;
         const float G = sc.out_gscale;
         const float inv6G = 1.0f / (6.0f * G);
         int acc = 0;
@@ -429,12 +448,12 @@ __global__ void __launch_bounds__(TileNV<GEMM>::THREADS, 1)
             // intermediate row b_row (the unit's first token), the tile's first feature
             uint8_t* hrow = p.out_routed + (size_t)t.b_row * ld_row + t.mt * (BM / 2);
             uint8_t* srow = p.sc_routed + (size_t)t.b_row * ld_sc + t.mt * (BM / 16);
-            for (int c0 = 0; c0 < t.n_valid; c0 += 16, ++chunk) {
+            for (int c0 = 16 * grp; c0 < t.n_valid; c0 += 16 * C::EG, ++chunk) {
                 uint32_t gg[16], uu[16];
                 tmem_ld16(taddr + c0, gg);
                 tmem_ld16(taddr + C::BNX + c0, uu);
                 tmem_ld_wait(gg, uu);
-                uint8_t* b = ep_buf + (chunk & 1) * C::G1_STAGE;
+                uint8_t* b = gstage + (chunk & 1) * C::G1_STAGE;
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
                     const float a = swiglu(__uint_as_float(gg[j]) * f, __uint_as_float(uu[j]) * f,
@@ -450,8 +469,8 @@ __global__ void __launch_bounds__(TileNV<GEMM>::THREADS, 1)
                     if ((lane & 15) == 0) b[16 * 64 + j * 8 + q * 2 + (lane >> 4)] = (uint8_t)s8;
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&ep_bar[chunk & 1]);
-                if (!mbar_wait(&ep_bar[chunk & 1], (uint32_t)(chunk >> 1) & 1u, abort_flag)) {
+                if (lane == 0) mbar_arrive(&gbar[chunk & 1]);
+                if (!mbar_wait(&gbar[chunk & 1], (uint32_t)(chunk >> 1) & 1u, abort_flag)) {
                     ok = false;
                     break;
                 }
@@ -485,11 +504,11 @@ __global__ void __launch_bounds__(TileNV<GEMM>::THREADS, 1)
 
 }  // namespace
 
-template <int GEMM>
+template <int GEMM, int BNX_, int ACCB_>
 cudaError_t launch_nvfp4(const GroupedGemmArgs& a, cudaStream_t st) {
-    using C = TileNV<GEMM>;
+    using C = TileNV<GEMM, BNX_, ACCB_>;
     const cudaError_t attr_err = ensure_smem_limit(
-        reinterpret_cast<const void*>(grouped_gemm_nvfp4_kernel<GEMM>), C::SMEM_BYTES);
+        reinterpret_cast<const void*>(grouped_gemm_nvfp4_kernel<GEMM, BNX_, ACCB_>), C::SMEM_BYTES);
     if (attr_err != cudaSuccess) return attr_err;
     GroupedGemmArgs r = a;
     r.S = 0;  // the shared experts are bf16: not part of this launch
@@ -509,24 +528,30 @@ cudaError_t launch_nvfp4(const GroupedGemmArgs& a, cudaStream_t st) {
     if (!make_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.w_routed, rowsA, K / 2, K / 2, NV_ROW,
                       BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_tmap_2d(&tmSFA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.w_routed_scale, rowsA, K / 16, K / 16,
-                      NV_SF_W, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+                      NV_SF_W, 128, CU_TENSOR_MAP_SWIZZLE_64B))
         return cudaErrorInvalidValue;
     if (a.N == 0) return cudaSuccess;
     if (!make_bmaps(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.b_rows, (uint64_t)a.N, K / 2, NV_ROW) ||
         !make_tmap_2d(&tmSFB, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.b_scale, (uint64_t)a.N, K / 16, K / 16,
-                      NV_SF_W, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+                      NV_SF_W, 128, CU_TENSOR_MAP_SWIZZLE_64B))
         return cudaErrorInvalidValue;
     NVScales s;
     s.w_gscale = a.w_gscale;
     s.a_gscale = a.a_gscale;
     s.out_gscale = a.out_gscale;
-    launch_pdl(grouped_gemm_nvfp4_kernel<GEMM>, grid_for(p), C::THREADS, C::SMEM_BYTES, st, tmA,
+    launch_pdl(grouped_gemm_nvfp4_kernel<GEMM, BNX_, ACCB_>, grid_for(p), C::THREADS, C::SMEM_BYTES, st, tmA,
         tmSFA, tmB, tmSFB, p, s);
     return cudaGetLastError();
 }
 
 cudaError_t launch_gemm_nvfp4(const GroupedGemmArgs& a, cudaStream_t st) {
-    return a.gemm == 1 ? launch_nvfp4<1>(a, st) : launch_nvfp4<2>(a, st);
+    // experts averaging 64 tokens or more: 128-token tiles, single-buffered
+    // accumulators with two epilogue groups (fewer passes over an expert's
+    // weight tiles when it holds a few hundred tokens); fewer: 96-token tiles,
+    // double-buffered
+    const bool wide = a.N >= 64L * a.E;
+    if (a.gemm == 1) return wide ? launch_nvfp4<1, 128, 1>(a, st) : launch_nvfp4<1, 96, 2>(a, st);
+    return wide ? launch_nvfp4<2, 128, 1>(a, st) : launch_nvfp4<2, 96, 2>(a, st);
 }
 
 }  // namespace gemm

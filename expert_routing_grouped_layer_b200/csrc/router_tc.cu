@@ -11,10 +11,13 @@
 // MMAs) measured errors that grow with the number of MMAs and lean one way:
 // the largest logits of the 896-expert layer came out up to 1.8e-4 low
 // (4e-5 rms), enough to reorder experts whose scores differ by 1e-5. Here each
-// 64-wide k-block is accumulated afresh (12 MMAs) and the epilogue warps add
-// the k-blocks' fp32 partial sums into fp64 registers, so only 12 MMAs'
-// accumulation error enters per k-block, with signs that vary across
-// k-blocks, plus one rounding of the final value to fp32.
+// 64-wide k-block is accumulated afresh (12 MMAs) in one of four tensor-memory
+// accumulators, and the epilogue warps add the k-blocks' fp32 partial sums
+// with Kahan's compensated summation, so only 12 MMAs' accumulation error
+// enters per k-block, with signs that vary across k-blocks, plus one rounding
+// of the final value (measured: 2.1e-6 at most, as with fp64 sums, which cost
+// the 896-expert router 0.5 ms in conversions; plain fp32 sums doubled the
+// largest error).
 //
 // Layout: experts are the MMA M operand (128 per tile, the three planes of the
 // same 128 experts are three A tiles of one stage), tokens are N (<= 128).
@@ -34,8 +37,9 @@ constexpr int RT_STAGES = 3;
 constexpr int RT_A_BYTES = BM * BK * 2;
 constexpr int RT_B_BYTES = RT_BN * BK * 2;
 constexpr int RT_STAGE_BYTES = 3 * RT_A_BYTES + RT_B_BYTES;
-constexpr int RT_TMEM_COLS = 2 * RT_BN;
-constexpr int RT_SMEM_BYTES = 1024 + RT_STAGES * RT_STAGE_BYTES + 8 * (2 * RT_STAGES + 5) + 16;
+constexpr int RT_ACCS = 4;  // accumulator buffers (one k-block each)
+constexpr int RT_TMEM_COLS = RT_ACCS * RT_BN;
+constexpr int RT_SMEM_BYTES = 1024 + RT_STAGES * RT_STAGE_BYTES + 8 * (2 * RT_STAGES + 2 * RT_ACCS + 1) + 16;
 constexpr int RT_EPI_WARPS = 8;  // two per TMEM lane quadrant, each 64 token columns
 constexpr int RT_THREADS = 64 + 32 * RT_EPI_WARPS;
 
@@ -129,8 +133,8 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + RT_STAGES * RT_STAGE_BYTES);
     uint64_t* empty = full + RT_STAGES;
     uint64_t* tfull = empty + RT_STAGES;
-    uint64_t* tempty = tfull + 2;
-    uint64_t* mma_done = tempty + 2;
+    uint64_t* tempty = tfull + RT_ACCS;
+    uint64_t* mma_done = tempty + RT_ACCS;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -141,7 +145,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        for (int a = 0; a < 2; ++a) {
+        for (int a = 0; a < RT_ACCS; ++a) {
             mbar_init(&tfull[a], 1);
             mbar_init(&tempty[a], 32 * RT_EPI_WARPS);
         }
@@ -223,7 +227,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
                     mma_commit(&empty[stage]);
                     mma_commit(&tfull[acc]);
                     if (++stage == RT_STAGES) { stage = 0; phase ^= 1; }
-                    if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+                    if (++acc == RT_ACCS) { acc = 0; acc_phase ^= 1; }
                 }
             }
             mma_commit(mma_done);
@@ -234,7 +238,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
     } else {
         // epilogue: warp w reads TMEM lane quadrant w % 4 (experts 32*(w%4) ..) and
         // token columns 64*h .. 64*h+63 of each k-block's accumulator, adding them
-        // into fp64 registers; the unit's sum is rounded once to fp32
+        // into Kahan-compensated fp32 sums; the unit's sum is rounded once
         const int q = warp & 3;
         const int h = (warp - 2) >> 2;
         const int e = q * 32 + lane;  // expert within the M tile
@@ -243,9 +247,12 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
         bool ok = true;
         for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
             const RUnit r = router_unit(p, u);
-            double sum[64];
+            float sum[64], comp[64];
 #pragma unroll
-            for (int j = 0; j < 64; ++j) sum[j] = 0.0;
+            for (int j = 0; j < 64; ++j) {
+                sum[j] = 0.0f;
+                comp[j] = 0.0f;
+            }
             for (int kb = r.kb0; kb < r.kb1; ++kb) {
                 if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) { ok = false; break; }
                 tc_fence_after();
@@ -258,12 +265,17 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
                         tmem_ld16(taddr + c0, v);
                         tmem_ld_wait(v);
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) sum[c0 + j] += (double)__uint_as_float(v[j]);
+                        for (int j = 0; j < 16; ++j) {  // Kahan: comp carries the lost low part
+                            const float y = __uint_as_float(v[j]) - comp[c0 + j];
+                            const float t = sum[c0 + j] + y;
+                            comp[c0 + j] = (t - sum[c0 + j]) - y;
+                            sum[c0 + j] = t;
+                        }
                     }
                 }
                 tc_fence_before();
                 mbar_arrive(&tempty[acc]);
-                if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+                if (++acc == RT_ACCS) { acc = 0; acc_phase ^= 1; }
             }
             if (!ok) break;
             const int eg = r.mt * BM + e;
@@ -271,7 +283,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
                 float* out = p.part + ((size_t)r.ks * p.T + r.t0) * p.E + eg;
 #pragma unroll
                 for (int j = 0; j < 64; ++j)
-                    if (h * 64 + j < r.n_valid) out[(size_t)(h * 64 + j) * p.E] = (float)sum[j];
+                    if (h * 64 + j < r.n_valid) out[(size_t)(h * 64 + j) * p.E] = sum[j] - comp[j];
             }
         }
     }
