@@ -586,18 +586,20 @@ cudaError_t launch_mx(const GroupedGemmArgs& a, cudaStream_t st) {
     return cudaGetLastError();
 }
 
+cudaError_t launch_gemm_mx_pair_down(const GroupedGemmArgs& a, cudaStream_t st);
+
 template <int AFMT>
 cudaError_t launch_mx_tiles(const GroupedGemmArgs& a, cudaStream_t st) {
     // When experts average many tokens: 224-token tiles (gate/up single-buffered
-    // with three epilogue groups, down double-buffered with one weight tile;
-    // at 224 both keep one TMEM scale set per pipeline stage).
+    // with two epilogue groups; the down projection on CTA pairs, gemm_mx_pair.cu,
+    // M = 256 over two SMs each loading half the token tile).
     // Otherwise 112-token tiles with double-buffered accumulators, so the
     // epilogue overlaps the next tile, and two weight tiles (two MMA threads)
     // per unit in both GEMMs.
     const bool wide = a.N >= 128L * a.E;
     if (a.gemm == 1)
         return wide ? launch_mx<1, AFMT, 2, 224, 1>(a, st) : launch_mx<1, AFMT, 2, 112, 2>(a, st);
-    return wide ? launch_mx<2, AFMT, 1, 224, 2>(a, st) : launch_mx<2, AFMT, 2, 112, 2>(a, st);
+    return wide ? launch_gemm_mx_pair_down(a, st) : launch_mx<2, AFMT, 2, 112, 2>(a, st);
 }
 
 cudaError_t launch_gemm_mx(const GroupedGemmArgs& a, cudaStream_t st) {
