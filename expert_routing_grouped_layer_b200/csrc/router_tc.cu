@@ -13,7 +13,8 @@
 // (4e-5 rms), enough to reorder experts whose scores differ by 1e-5. Here each
 // 64-wide k-block is accumulated afresh (12 MMAs) in one of four tensor-memory
 // accumulators, and the epilogue warps add the k-blocks' fp32 partial sums
-// with Kahan's compensated summation, so only 12 MMAs' accumulation error
+// with Kahan's compensated summation (packed fp32x2 arithmetic, two token
+// columns per instruction), so only 12 MMAs' accumulation error
 // enters per k-block, with signs that vary across k-blocks, plus one rounding
 // of the final value (measured: 2.1e-6 at most, as with fp64 sums, which cost
 // the 896-expert router 0.5 ms in conversions; plain fp32 sums doubled the
@@ -247,12 +248,14 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
         bool ok = true;
         for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
             const RUnit r = router_unit(p, u);
-            float sum[64], comp[64];
+            // Kahan sums of two token columns at a time (packed fp32x2 arithmetic)
+            float2 sum[32], comp[32];
 #pragma unroll
-            for (int j = 0; j < 64; ++j) {
-                sum[j] = 0.0f;
-                comp[j] = 0.0f;
+            for (int j = 0; j < 32; ++j) {
+                sum[j] = make_float2(0.0f, 0.0f);
+                comp[j] = make_float2(0.0f, 0.0f);
             }
+            const float2 neg1 = make_float2(-1.0f, -1.0f);
             for (int kb = r.kb0; kb < r.kb1; ++kb) {
                 if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) { ok = false; break; }
                 tc_fence_after();
@@ -265,11 +268,14 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
                         tmem_ld16(taddr + c0, v);
                         tmem_ld_wait(v);
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) {  // Kahan: comp carries the lost low part
-                            const float y = __uint_as_float(v[j]) - comp[c0 + j];
-                            const float t = sum[c0 + j] + y;
-                            comp[c0 + j] = (t - sum[c0 + j]) - y;
-                            sum[c0 + j] = t;
+                        for (int j = 0; j < 8; ++j) {  // Kahan: comp carries the lost low part
+                            const int i = c0 / 2 + j;
+                            const float2 x = make_float2(__uint_as_float(v[2 * j]),
+                                                         __uint_as_float(v[2 * j + 1]));
+                            const float2 y = __ffma2_rn(comp[i], neg1, x);     // x - comp
+                            const float2 t = __fadd2_rn(sum[i], y);            // sum + y
+                            comp[i] = __ffma2_rn(y, neg1, __ffma2_rn(sum[i], neg1, t));  // (t - sum) - y
+                            sum[i] = t;
                         }
                     }
                 }
@@ -282,8 +288,11 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
             if (eg < p.E) {
                 float* out = p.part + ((size_t)r.ks * p.T + r.t0) * p.E + eg;
 #pragma unroll
-                for (int j = 0; j < 64; ++j)
-                    if (h * 64 + j < r.n_valid) out[(size_t)(h * 64 + j) * p.E] = sum[j] - comp[j];
+                for (int j = 0; j < 64; ++j) {
+                    const float hi = (j & 1) ? sum[j / 2].y : sum[j / 2].x;
+                    const float lo = (j & 1) ? comp[j / 2].y : comp[j / 2].x;
+                    if (h * 64 + j < r.n_valid) out[(size_t)(h * 64 + j) * p.E] = hi - lo;
+                }
             }
         }
     }
