@@ -173,20 +173,24 @@ __device__ __forceinline__ void epilogue_f16_gate_up(const KParams& p, const int
 
 // Down epilogue of the f16 path: per unit, wait for the accumulator, read it 16
 // token columns at a time (lane = output feature), restore 2^E (the W2 tile) and
-// 2^e (the token's h row), store bf16, release the buffer.
+// 2^e (the token's h row), and store bf16. Each warp stages its 16 x 32 chunk in
+// its own shared [16 tokens][32 features] tile (two, alternating) and writes
+// every token row's 64 bytes as four 16-byte pieces (two per lane), instead of
+// one 2-byte store per element; then it releases the buffer.
 template <int ACC_COLS, int ACCB>
 __device__ __forceinline__ void epilogue_f16_down(const KParams& p, const int* pref, int total,
                                                   uint32_t tmem_base, uint64_t* tfull, uint64_t* tempty,
                                                   volatile int* abort_flag, int warp, int lane,
                                                   const float* __restrict__ scale_routed,
                                                   const float* __restrict__ scale_shared,
-                                                  const int8_t* __restrict__ row_exp) {
+                                                  const int8_t* __restrict__ row_exp,
+                                                  __nv_bfloat16* wbuf) {
     const int q = warp & 3;
-    const int row = q * 32 + lane;
     const int KS = p.K / 128;
     const int RS = p.a_rows_per_mat / 128;
     int acc = 0;
     uint32_t acc_phase = 0;
+    int chunk = 0;
     for (int u = blockIdx.x; u < total; u += gridDim.x) {
         const Unit t = decode_unit(p, pref, u);
         const bool routed = t.seg < p.E;
@@ -196,19 +200,28 @@ __device__ __forceinline__ void epilogue_f16_down(const KParams& p, const int* p
         if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) break;
         tc_fence_after();
         const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * ACC_COLS;
-        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(t.out) + t.mt * BM + row;
-        for (int c0 = 0; c0 < t.n_valid; c0 += 16) {
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(t.out) + t.mt * BM + q * 32;
+        for (int c0 = 0; c0 < t.n_valid; c0 += 16, ++chunk) {
             uint32_t g[16];
             tmem_ld16(taddr + c0, g);
             // 2^e of this lane's token column (e in [-127, 114]; 2^-127 is subnormal)
             const int ex_l = (lane < 16 && c0 + lane < t.n_valid) ? row_exp[t.b_row + c0 + lane] : 0;
             const float fe_l = ex_l >= -126 ? pow2f(ex_l) : __uint_as_float(0x00400000u);
             tmem_ld_wait(g);
+            __nv_bfloat16* b = wbuf + (chunk & 1) * 16 * 32;
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
+            for (int j = 0; j < 16; ++j) {  // exact power-of-two factors
                 const float fe = __shfl_sync(0xffffffffu, fe_l, j);
-                if (c0 + j < t.n_valid)  // exact power-of-two factors
-                    out[(size_t)(c0 + j) * p.ld_out] = __float2bfloat16_rn(__uint_as_float(g[j]) * fw * fe);
+                b[j * 32 + lane] = __float2bfloat16_rn(__uint_as_float(g[j]) * fw * fe);
+            }
+            __syncwarp();
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int i = lane + 32 * k;  // 16 token rows x 4 pieces of 8 features
+                const int r = i >> 2, pc = i & 3;
+                if (c0 + r < t.n_valid)
+                    *reinterpret_cast<uint4*>(out + (size_t)(c0 + r) * p.ld_out + pc * 8) =
+                        *reinterpret_cast<const uint4*>(b + r * 32 + pc * 8);
             }
         }
         tc_fence_before();
@@ -525,6 +538,8 @@ __device__ __forceinline__ void epilogue_f16_gate_up_staged(
         tc_fence_after();
         const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16);
         __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(t.out) + t.mt * BM;
+        const bool lim = p.swiglu_limit > 0.0f;  // optional limit: min(g, L), clamp(u, -L, L)
+        const float L = p.swiglu_limit;
         for (int c0 = 16 * group; c0 < t.n_valid; c0 += 16 * GROUPS, ++chunk) {
             uint32_t g[16], uu[16];
             tmem_ld16(taddr + c0, g);
@@ -534,13 +549,20 @@ __device__ __forceinline__ void epilogue_f16_gate_up_staged(
             const float fe_l = ex_l >= -126 ? pow2f(ex_l) : __uint_as_float(0x00400000u);
             tmem_ld_wait(g, uu);
             __nv_bfloat16* b = buf2 + (chunk & 1) * 16 * BM;
+            // each step over all 16 token columns, branch-free, so that the
+            // columns' exp / division chains overlap
+            float a[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 const float fe = __shfl_sync(0xffffffffu, fe_l, j);
-                const float gv = __uint_as_float(g[j]) * fg * fe;  // exact power-of-two factors
-                const float uv = __uint_as_float(uu[j]) * fu * fe;
-                b[j * BM + row] = __float2bfloat16_rn(swiglu(gv, uv, p.swiglu_limit));
+                const float g0 = __uint_as_float(g[j]) * fg * fe;  // exact power-of-two factors
+                const float u0 = __uint_as_float(uu[j]) * fu * fe;
+                const float gv = lim ? fminf(g0, L) : g0;
+                const float uv = lim ? fminf(fmaxf(u0, -L), L) : u0;
+                a[j] = __fdividef(gv, 1.0f + __expf(-gv)) * uv;
             }
+#pragma unroll
+            for (int j = 0; j < 16; ++j) b[j * BM + row] = __float2bfloat16_rn(a[j]);
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar2[chunk & 1]);
             if (!mbar_wait(&bar2[chunk & 1], (uint32_t)(chunk >> 1) & 1u, abort_flag)) {
@@ -576,8 +598,9 @@ struct TileTA {
     static constexpr int B_BYTES = BNT * BK * 2;
     static constexpr int MSLOT_BYTES = (B_BYTES + 1023) / 1024 * 1024;
     static constexpr int MSTAGES = MST_;
-    // gate/up: each epilogue group stages 16-token chunks of h, [2][16][128] bf16
-    static constexpr int EPI_BYTES = GEMM == 1 ? EG * 2 * 16 * BM * 2 + 128 : 0;
+    // gate/up: each epilogue group stages 16-token chunks of h, [2][16][128] bf16;
+    // down: each epilogue warp its 16 x 32 chunks of y, [4 warps][2][16][32] bf16
+    static constexpr int EPI_BYTES = (GEMM == 1 ? EG * 2 * 16 * BM * 2 : 4 * 2 * 16 * 32 * 2) + 128;
     static constexpr int FIXED_BYTES =
         1024 + 8 * (2 * 8 + 3 * MSTAGES + 5 + 2 * EG) + 16 + 4 * (MAX_SEG + 1) + EPI_BYTES;
     static constexpr int RSTAGES_FIT = (232448 - FIXED_BYTES - MSTAGES * MSLOT_BYTES) / RSLOT_BYTES;
@@ -782,7 +805,8 @@ __global__ void __launch_bounds__(TileTA<GEMM, BNT_, MST_>::THREADS, 1)
         }
         else
             epilogue_f16_down<C::ACC_COLS, C::ACCB>(p, pref, total, tmem_base, tfull, tempty, abort_flag,
-                                                    warp, lane, scale_routed, scale_shared, row_exp);
+                                                    warp, lane, scale_routed, scale_shared, row_exp,
+                                                    ep_buf + (warp & 3) * 2 * 16 * 32);
     } else {
         // converters, thread = one weight row of its lane quadrant. gate/up: warps
         // 6..9 gate rows, 10..13 up rows, 64 K each; down: warps 6..9 the first

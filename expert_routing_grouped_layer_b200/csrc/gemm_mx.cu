@@ -469,17 +469,20 @@ __global__ void __launch_bounds__(TileMX<GEMM, NA_, BNX_, ACCB_>::THREADS, 1)
                 tmem_ld16(taddr + c0, g);
                 tmem_ld16(taddr + C::BNX + c0, uu);
                 tmem_ld_wait(g, uu);
+                // each step runs over all 16 token columns, branch-free, so the
+                // columns' exp / reduction chains overlap
                 float a[16], wmax[16];
+                const bool lim = p.swiglu_limit > 0.0f;  // optional limit: min(g, L), clamp(u, -L, L)
+                const float L = p.swiglu_limit;
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
-                    float gv = __uint_as_float(g[j]), uv = __uint_as_float(uu[j]);
-                    if (p.swiglu_limit > 0.0f) {  // optional limit: min(g, L), clamp(u, -L, L)
-                        gv = fminf(gv, p.swiglu_limit);
-                        uv = fminf(fmaxf(uv, -p.swiglu_limit), p.swiglu_limit);
-                    }
+                    const float g0 = __uint_as_float(g[j]), u0 = __uint_as_float(uu[j]);
+                    const float gv = lim ? fminf(g0, L) : g0;
+                    const float uv = lim ? fminf(fmaxf(u0, -L), L) : u0;
                     a[j] = __fdividef(gv, 1.0f + __expf(-gv)) * uv;
-                    wmax[j] = warp_max_nonneg(fabsf(a[j]));
                 }
+#pragma unroll
+                for (int j = 0; j < 16; ++j) wmax[j] = warp_max_nonneg(fabsf(a[j]));
                 int e[16];
                 if (AFMT == MOE_A_MXFP8) {
 #pragma unroll
@@ -505,10 +508,13 @@ __global__ void __launch_bounds__(TileMX<GEMM, NA_, BNX_, ACCB_>::THREADS, 1)
                 uint8_t* b = gstage + (chunk & 1) * C::G1_STAGE;
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
-                    const int ej = min(max(e[j], -127), 127);
-                    const float inv = __uint_as_float((uint32_t)(127 - ej) << 23);
+                    e[j] = min(max(e[j], -127), 127);
+                    const float inv = __uint_as_float((uint32_t)(127 - e[j]) << 23);
                     b[j * BM + row] = e4m3_sat(a[j] * inv);
-                    if (lane == 0) b[16 * BM + j * 4 + q] = (uint8_t)(ej + 127);
+                }
+                if (lane == 0) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) b[16 * BM + j * 4 + q] = (uint8_t)(e[j] + 127);
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&gbar[chunk & 1]);

@@ -116,6 +116,16 @@ __device__ __forceinline__ uint32_t word4(const uint4& u, int w) {
 // E2M1 code of v by round to nearest even onto {0, .5, 1, 1.5, 2, 3, 4, 6},
 // saturating: the magnitude code counts the midpoints below |v| (a midpoint
 // itself goes to the even code), the sign bit is v's.
+// SwiGLU with the optional limit, fast division (the fp32 rounding of the
+// quotient is below the E2M1 grid the result is quantised to)
+__device__ __forceinline__ float swiglu_nv(float g, float u, float limit) {
+    if (limit > 0.0f) {
+        g = fminf(g, limit);
+        u = fminf(fmaxf(u, -limit), limit);
+    }
+    return __fdividef(g, 1.0f + __expf(-g)) * u;
+}
+
 __device__ __forceinline__ uint32_t e2m1_code(float v) {
     const float a = fabsf(v);
     const uint32_t c = (a > 0.25f) + (a >= 0.75f) + (a > 1.25f) + (a >= 1.75f) + (a > 2.5f) +
@@ -454,19 +464,36 @@ __global__ void __launch_bounds__(TileNV<GEMM, BNX_, ACCB_>::THREADS, 1)
                 tmem_ld16(taddr + C::BNX + c0, uu);
                 tmem_ld_wait(gg, uu);
                 uint8_t* b = gstage + (chunk & 1) * C::G1_STAGE;
+                // Each step runs over all 16 token columns before the next, with
+                // no branch inside, so the columns' long-latency chains (exp,
+                // division, four shuffles, conversions) overlap instead of
+                // running one column at a time.
+                float a[16], m[16];
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
-                    const float a = swiglu(__uint_as_float(gg[j]) * f, __uint_as_float(uu[j]) * f,
-                                           p.swiglu_limit);
-                    float m = fabsf(a);
+                    a[j] = swiglu_nv(__uint_as_float(gg[j]) * f, __uint_as_float(uu[j]) * f, p.swiglu_limit);
+                    m[j] = fabsf(a[j]);
+                }
 #pragma unroll
-                    for (int off = 8; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-                    const __nv_fp8_storage_t s8 = __nv_cvt_float_to_fp8(m * inv6G, __NV_SATFINITE, __NV_E4M3);
-                    const float sv = __half2float(__nv_cvt_fp8_to_halfraw(s8, __NV_E4M3));
-                    const uint32_t code = sv > 0.0f ? e2m1_code(a / (sv * G)) : 0u;
-                    const uint32_t hi = __shfl_down_sync(0xffffffffu, code, 1);
-                    if ((lane & 1) == 0) b[j * 64 + q * 16 + (lane >> 1)] = (uint8_t)(code | (hi << 4));
-                    if ((lane & 15) == 0) b[16 * 64 + j * 8 + q * 2 + (lane >> 4)] = (uint8_t)s8;
+                for (int off = 8; off > 0; off >>= 1)
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) m[j] = fmaxf(m[j], __shfl_xor_sync(0xffffffffu, m[j], off));
+                uint32_t code[16], s8[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    s8[j] = __nv_cvt_float_to_fp8(m[j] * inv6G, __NV_SATFINITE, __NV_E4M3);
+                    const float sv = __half2float(__nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)s8[j], __NV_E4M3));
+                    code[j] = sv > 0.0f ? e2m1_code(__fdividef(a[j], sv * G)) : 0u;
+                }
+#pragma unroll
+                for (int j = 0; j < 16; ++j) code[j] |= __shfl_down_sync(0xffffffffu, code[j], 1) << 4;
+                if ((lane & 1) == 0) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) b[j * 64 + q * 16 + (lane >> 1)] = (uint8_t)code[j];
+                }
+                if ((lane & 15) == 0) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) b[16 * 64 + j * 8 + q * 2 + (lane >> 4)] = (uint8_t)s8[j];
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&gbar[chunk & 1]);
