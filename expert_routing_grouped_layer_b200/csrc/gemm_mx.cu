@@ -115,8 +115,12 @@ __device__ __forceinline__ int mx_exp(float a) {
     return f == 0 ? -127 : max(f - 135, -127);
 }
 
-__device__ __forceinline__ uint8_t e4m3_sat(float v) {
-    return (uint8_t)(__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3));
+// Two floats to E4M3 (saturating, nearest-even) in one conversion: byte 0 = a,
+// byte 1 = b (the instruction puts its first source in the upper byte).
+__device__ __forceinline__ uint32_t e4m3x2_sat(float a, float b) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(b), "f"(a));
+    return r;
 }
 
 // Word w (0..3) of a 16-byte vector.
@@ -507,10 +511,13 @@ __global__ void __launch_bounds__(TileMX<GEMM, NA_, BNX_, ACCB_>::THREADS, 1)
                 }
                 uint8_t* b = gstage + (chunk & 1) * C::G1_STAGE;
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
+                for (int j = 0; j < 16; j += 2) {
                     e[j] = min(max(e[j], -127), 127);
-                    const float inv = __uint_as_float((uint32_t)(127 - e[j]) << 23);
-                    b[j * BM + row] = e4m3_sat(a[j] * inv);
+                    e[j + 1] = min(max(e[j + 1], -127), 127);
+                    const uint32_t pr = e4m3x2_sat(a[j] * __uint_as_float((uint32_t)(127 - e[j]) << 23),
+                                                   a[j + 1] * __uint_as_float((uint32_t)(127 - e[j + 1]) << 23));
+                    b[j * BM + row] = (uint8_t)pr;
+                    b[(j + 1) * BM + row] = (uint8_t)(pr >> 8);
                 }
                 if (lane == 0) {
 #pragma unroll

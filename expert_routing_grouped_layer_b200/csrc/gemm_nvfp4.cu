@@ -126,11 +126,31 @@ __device__ __forceinline__ float swiglu_nv(float g, float u, float limit) {
     return __fdividef(g, 1.0f + __expf(-g)) * u;
 }
 
-__device__ __forceinline__ uint32_t e2m1_code(float v) {
-    const float a = fabsf(v);
-    const uint32_t c = (a > 0.25f) + (a >= 0.75f) + (a > 1.25f) + (a >= 1.75f) + (a > 2.5f) +
-                       (a >= 3.5f) + (a > 5.0f);
-    return c | (signbit(v) ? 8u : 0u);
+// Two floats to E4M3 (saturating, nearest-even) in one conversion: byte 0 = a,
+// byte 1 = b (the instruction puts its first source in the upper byte).
+__device__ __forceinline__ uint32_t e4m3x2_sat(float a, float b) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(b), "f"(a));
+    return r;
+}
+
+// Value of a non-negative finite E4M3 code c (0..0x7E), exactly: normal codes
+// are (1 + m/8) 2^(e-7), i.e. the fp32 bits (c << 20) + (120 << 23); subnormal
+// ones (e = 0) are m 2^-9 = (1 + m/8) 2^-6 - 2^-6.
+__device__ __forceinline__ float e4m3_value(uint32_t c) {
+    const float nrm = __uint_as_float((c << 20) + (120u << 23));
+    const float sub = __uint_as_float((c << 20) + (121u << 23)) - 0x1p-6f;
+    return (c >> 3) ? nrm : sub;
+}
+
+// E2M1 code of a / d (d > 0) by comparing |a| with the rounding thresholds
+// scaled by d (ties to even: 0.25 -> 0, 0.75 -> 1, 1.25 -> 1, 1.75 -> 2,
+// 2.5 -> 2, 3.5 -> 4, 5 -> 4)
+__device__ __forceinline__ uint32_t e2m1_code_div(float a, float d) {
+    const float x = fabsf(a);
+    const uint32_t c = (x > 0.25f * d) + (x >= 0.75f * d) + (x > 1.25f * d) + (x >= 1.75f * d) +
+                       (x > 2.5f * d) + (x >= 3.5f * d) + (x > 5.0f * d);
+    return c | (signbit(a) ? 8u : 0u);
 }
 
 __device__ __forceinline__ bool warp_wait_nv(uint64_t* bar, uint32_t parity, volatile int* abort,
@@ -480,10 +500,15 @@ __global__ void __launch_bounds__(TileNV<GEMM, BNX_, ACCB_>::THREADS, 1)
                     for (int j = 0; j < 16; ++j) m[j] = fmaxf(m[j], __shfl_xor_sync(0xffffffffu, m[j], off));
                 uint32_t code[16], s8[16];
 #pragma unroll
+                for (int j = 0; j < 16; j += 2) {
+                    const uint32_t pr = e4m3x2_sat(m[j] * inv6G, m[j + 1] * inv6G);
+                    s8[j] = pr & 0xFFu;
+                    s8[j + 1] = pr >> 8;
+                }
+#pragma unroll
                 for (int j = 0; j < 16; ++j) {
-                    s8[j] = __nv_cvt_float_to_fp8(m[j] * inv6G, __NV_SATFINITE, __NV_E4M3);
-                    const float sv = __half2float(__nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)s8[j], __NV_E4M3));
-                    code[j] = sv > 0.0f ? e2m1_code(__fdividef(a[j], sv * G)) : 0u;
+                    const float sv = e4m3_value(s8[j]);
+                    code[j] = sv > 0.0f ? e2m1_code_div(a[j], sv * G) : 0u;
                 }
 #pragma unroll
                 for (int j = 0; j < 16; ++j) code[j] |= __shfl_down_sync(0xffffffffu, code[j], 1) << 4;
