@@ -392,52 +392,44 @@ __global__ void __launch_bounds__(TileMX<GEMM, NA_, BNX_, ACCB_>::THREADS, 1)
     } else if (GEMM == 2) {
         // down epilogue: NA accumulators of BNX columns, lane = output feature.
         // Group grp takes the 16-token chunks grp, grp + EG, ... Per chunk each
-        // warp converts its 32 features to bf16 into the group's shared
-        // [16 tokens][128 features] tile (two, alternating), the group's four
-        // warps meet at an mbarrier, and warp q writes token rows 4q..4q+3 as
-        // 256 contiguous bytes each, 16 bytes per lane.
+        // warp converts its 32 features to bf16 into its own shared [16 tokens]
+        // [32 features] tile (two, alternating) and writes each token row's 64
+        // bytes of them as four 16-byte pieces, two per lane; no barrier between
+        // warps.
         const int q = warp & 3;
         const int grp = (warp - 2) >> 2;
-        const int row = q * 32 + lane;
-        __nv_bfloat16* gbuf = ep_buf + grp * 2 * 16 * BM;
-        uint64_t* gbar = ep_bar + 2 * grp;
+        __nv_bfloat16* wbuf = ep_buf + (warp - 2) * 2 * 16 * 32;
         int acc = 0;
         uint32_t acc_phase = 0;
         int chunk = 0;
-        bool ok = true;
-        for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+        for (int u = blockIdx.x; u < total; u += gridDim.x) {
             const Unit t = decode_unit(p, pref, u);
             if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) break;
             tc_fence_after();
 #pragma unroll 1
-            for (int w = 0; w < C::NA && ok; ++w) {
+            for (int w = 0; w < C::NA; ++w) {
                 const uint32_t taddr =
                     tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::ACC_COLS + w * C::BNX;
-                __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(t.out) + t.mt * p.tile_rows + w * BM;
+                __nv_bfloat16* out =
+                    reinterpret_cast<__nv_bfloat16*>(t.out) + t.mt * p.tile_rows + w * BM + q * 32;
                 for (int c0 = 16 * grp; c0 < t.n_valid; c0 += 16 * C::EG, ++chunk) {
                     uint32_t g[16];
                     tmem_ld16(taddr + c0, g);
                     tmem_ld_wait(g);
-                    __nv_bfloat16* buf = gbuf + (chunk & 1) * 16 * BM;
+                    __nv_bfloat16* buf = wbuf + (chunk & 1) * 16 * 32;
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) buf[j * BM + row] = __float2bfloat16_rn(__uint_as_float(g[j]));
+                    for (int j = 0; j < 16; ++j) buf[j * 32 + lane] = __float2bfloat16_rn(__uint_as_float(g[j]));
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&gbar[chunk & 1]);
-                    if (!mbar_wait(&gbar[chunk & 1], (uint32_t)(chunk >> 1) & 1u, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
-                        const int r = 4 * q + 2 * h + (lane >> 4);  // token row of the chunk
-                        const int col = (lane & 15) * 8;            // first of 8 features
+                        const int i2 = lane + 32 * h;  // 16 token rows x 4 pieces of 8 features
+                        const int r = i2 >> 2, pc = i2 & 3;
                         if (c0 + r < t.n_valid)
-                            *reinterpret_cast<uint4*>(out + (size_t)(c0 + r) * p.ld_out + col) =
-                                *reinterpret_cast<const uint4*>(buf + r * BM + col);
+                            *reinterpret_cast<uint4*>(out + (size_t)(c0 + r) * p.ld_out + pc * 8) =
+                                *reinterpret_cast<const uint4*>(buf + r * 32 + pc * 8);
                     }
                 }
             }
-            if (!ok) break;
             tc_fence_before();
             mbar_arrive(&tempty[acc]);
             if (++acc == C::ACCB) { acc = 0; acc_phase ^= 1; }

@@ -45,9 +45,10 @@ struct TileP {
     static constexpr int BNX = 224;
     static constexpr int BHALF = BNX / 2;
     static constexpr int ACCB = 2;
-    static constexpr int SCALE_WARP = 6;  // warps: 0 TMA, 1 MMA, 2-5 epilogue, 6-9 scales
-    static constexpr int THREADS = 32 * 10;
-    static constexpr int EPI_BYTES = 2 * 16 * BM * 2 + 128;  // two [16 tokens][128] bf16 chunks
+    static constexpr int SCALE_WARP = 6;  // warps: 0 TMA, 1 MMA, 2-5 and 10-13 epilogue, 6-9 scales
+    static constexpr int EPI_WARPS = 8;   // two groups of four, alternate 16-token chunks
+    static constexpr int THREADS = 32 * 14;
+    static constexpr int EPI_BYTES = EPI_WARPS * 2 * 16 * 32 * 2 + 128;  // per warp two [16][32] bf16 chunks
     static constexpr int SFB_ROWS = (BNX + 127) / 128 * 128;
     static constexpr int SFB_ATOMS = SFB_ROWS / 128;
     static constexpr int NOPS = 1 + SFB_ATOMS;  // scale operands: the weight rows, the token rows
@@ -199,8 +200,7 @@ __global__ void __launch_bounds__(TileP::THREADS, 1)
     uint64_t* mma_done = tempty + 2;
     uint64_t* sf_full = mma_done + 1;
     uint64_t* sf_empty = sf_full + 2;
-    uint64_t* ep_bar = sf_empty + 2;  // [parity]: the epilogue warps' staged chunk
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ep_bar + 2);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_empty + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* pref = reinterpret_cast<int*>(tmem_slot + 4);
     __nv_bfloat16* ep_buf = reinterpret_cast<__nv_bfloat16*>(
@@ -219,14 +219,13 @@ __global__ void __launch_bounds__(TileP::THREADS, 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull[a], 1);
-            mbar_init(&tempty[a], 2 * 128);  // both SMs' epilogues (leader's copy used)
+            mbar_init(&tempty[a], 2 * 32 * C::EPI_WARPS);  // both SMs' epilogues (leader's copy used)
         }
         mbar_init(mma_done, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sf_full[i], 1);
             mbar_init(&sf_empty[i], 4);
         }
-        for (int i = 0; i < 2; ++i) mbar_init(&ep_bar[i], 4);
         *abort_flag = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tmA_routed);
@@ -418,47 +417,42 @@ __global__ void __launch_bounds__(TileP::THREADS, 1)
                 ++g;
             }
         }
-    } else if (warp >= 2 && warp < 6) {
-        // this SM's 128 output features of the pair's 256, bf16: per 16-token chunk
-        // each warp converts its 32 features into the shared [16 tokens][128] tile
-        // (two, alternating), the four warps meet at an mbarrier, and warp q
-        // writes token rows 4q..4q+3 with 16-byte stores (as in gemm_mx.cu)
+    } else if ((warp >= 2 && warp < 6) || warp >= 10) {
+        // this SM's 128 output features of the pair's 256, bf16. Group grp (warps
+        // 2-5 or 10-13) takes the 16-token chunks grp, grp + 2, ...; per chunk each
+        // warp converts its 32 features into its own shared [16 tokens][32] tile
+        // (two, alternating) and writes each token row's 64 bytes of them as four
+        // 16-byte pieces, two per lane; no barrier between warps.
         const int q = warp & 3;
-        const int row = q * 32 + lane;
+        const int grp = warp >= 10 ? 1 : 0;
+        __nv_bfloat16* wbuf = ep_buf + (warp < 6 ? warp - 2 : warp - 6) * 2 * 16 * 32;
         int acc = 0;
         uint32_t acc_phase = 0;
         int chunk = 0;
-        bool ok = true;
-        for (int u = pair; u < total && ok; u += npairs) {
+        for (int u = pair; u < total; u += npairs) {
             const Unit t = decode_unit(p, pref, u);
             if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::ACC_COLS;
             __nv_bfloat16* out =
-                reinterpret_cast<__nv_bfloat16*>(t.out) + t.mt * p.tile_rows + (int)rank * BM;
-            for (int c0 = 0; c0 < t.n_valid; c0 += 16, ++chunk) {
+                reinterpret_cast<__nv_bfloat16*>(t.out) + t.mt * p.tile_rows + (int)rank * BM + q * 32;
+            for (int c0 = 16 * grp; c0 < t.n_valid; c0 += 32, ++chunk) {
                 uint32_t gq[16];
                 tmem_ld16(taddr + c0, gq);
                 tmem_ld_wait(gq);
-                __nv_bfloat16* buf = ep_buf + (chunk & 1) * 16 * BM;
+                __nv_bfloat16* buf = wbuf + (chunk & 1) * 16 * 32;
 #pragma unroll
-                for (int j = 0; j < 16; ++j) buf[j * BM + row] = __float2bfloat16_rn(__uint_as_float(gq[j]));
+                for (int j = 0; j < 16; ++j) buf[j * 32 + lane] = __float2bfloat16_rn(__uint_as_float(gq[j]));
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&ep_bar[chunk & 1]);
-                if (!mbar_wait(&ep_bar[chunk & 1], (uint32_t)(chunk >> 1) & 1u, abort_flag)) {
-                    ok = false;
-                    break;
-                }
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    const int r = 4 * q + 2 * h + (lane >> 4);
-                    const int col = (lane & 15) * 8;
+                    const int i = lane + 32 * h;  // 16 token rows x 4 pieces of 8 features
+                    const int r = i >> 2, pc = i & 3;
                     if (c0 + r < t.n_valid)
-                        *reinterpret_cast<uint4*>(out + (size_t)(c0 + r) * p.ld_out + col) =
-                            *reinterpret_cast<const uint4*>(buf + r * BM + col);
+                        *reinterpret_cast<uint4*>(out + (size_t)(c0 + r) * p.ld_out + pc * 8) =
+                            *reinterpret_cast<const uint4*>(buf + r * 32 + pc * 8);
                 }
             }
-            if (!ok) break;
             tc_fence_before();
             if (rank == 0) mbar_arrive(&tempty[acc]);
             else mbar_arrive_remote(peer_addr(&tempty[acc], 0));
