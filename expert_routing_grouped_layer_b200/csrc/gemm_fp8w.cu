@@ -609,7 +609,10 @@ struct TileTA {
     static constexpr int A_COL = ACCB * ACC_COLS;   // A stage s at A_COL + s * A_STAGE_COLS
     static constexpr int A_STAGE_COLS = 32 * NA;    // 64 K of 16-bit values per weight tile
     static constexpr int TMEM_COLS = 512;
-    static_assert(A_COL + 2 * A_STAGE_COLS <= TMEM_COLS, "tensor memory budget");
+    // converted weight stages in tensor memory: as many as fit, up to the MMA ring's depth
+    static constexpr int ASTAGES_FIT = (TMEM_COLS - A_COL) / A_STAGE_COLS;
+    static constexpr int ASTAGES = ASTAGES_FIT < MST_ ? ASTAGES_FIT : MST_;
+    static_assert(ASTAGES >= 2, "tensor memory budget");
     static constexpr int RING_BYTES = MSTAGES * MSLOT_BYTES + RSTAGES * RSLOT_BYTES;
     static constexpr int BAR_BYTES = 8 * (2 * RSTAGES + 3 * MSTAGES + 5 + 2 * EG) + 16;
     static constexpr int SMEM_BYTES = 1024 + RING_BYTES + BAR_BYTES + 4 * (MAX_SEG + 1) + EPI_BYTES;
@@ -745,7 +748,7 @@ __global__ void __launch_bounds__(TileTA<GEMM, BNT_, MST_>::THREADS, 1)
                     if (!mbar_wait(&b_full[stage], phase, abort_flag) ||
                         !mbar_wait(&cvt_full[stage], phase, abort_flag)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t a0 = tmem_base + C::A_COL + C::A_STAGE_COLS * (g & 1);
+                    const uint32_t a0 = tmem_base + C::A_COL + C::A_STAGE_COLS * (g % C::ASTAGES);
                     const uint32_t sb = smem_u32(mring + stage * C::MSLOT_BYTES);
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
@@ -811,8 +814,8 @@ __global__ void __launch_bounds__(TileTA<GEMM, BNT_, MST_>::THREADS, 1)
         // converters, thread = one weight row of its lane quadrant. gate/up: warps
         // 6..9 gate rows, 10..13 up rows, 64 K each; down: warps 6..9 the first
         // 32 K of a row, 10..13 the last 32. The TMEM stage of MMA stage g was
-        // last read by stage g - 2, whose completion (its slot's empty barrier)
-        // is awaited first.
+        // last read by stage g - ASTAGES, whose completion (its slot's empty
+        // barrier) is awaited first.
         const int tile = (warp - 6) >> 2;  // gate/up: which tile; down: which half of the row
         const int row = (warp & 3) * 32 + lane;
         const uint32_t lane_cols = tmem_base + ((uint32_t)((warp & 3) * 32) << 16) + C::A_COL +
@@ -842,8 +845,8 @@ __global__ void __launch_bounds__(TileTA<GEMM, BNT_, MST_>::THREADS, 1)
                 }
                 const int h = kb & 1;  // half of the staged 128-K tile
                 if (h == 0 && !mbar_wait(&raw_full[rstage], rphase, abort_flag)) { ok = false; break; }
-                if (g >= 2) {
-                    const int gp = g - 2;
+                if (g >= C::ASTAGES) {
+                    const int gp = g - C::ASTAGES;
                     if (!mbar_wait(&m_empty[gp % C::MSTAGES], (uint32_t)(gp / C::MSTAGES) & 1u, abort_flag)) {
                         ok = false;
                         break;
@@ -863,7 +866,7 @@ __global__ void __launch_bounds__(TileTA<GEMM, BNT_, MST_>::THREADS, 1)
                         v[8 * c + 4] = hi.x; v[8 * c + 5] = hi.y; v[8 * c + 6] = hi.z; v[8 * c + 7] = hi.w;
                     }
                     if (h == 1) mbar_arrive(&raw_empty[rstage]);
-                    tmem_st32(lane_cols + C::A_STAGE_COLS * (g & 1), v);
+                    tmem_st32(lane_cols + C::A_STAGE_COLS * (g % C::ASTAGES), v);
                 } else {
                     const uint8_t* src = rring + rstage * C::RSLOT_BYTES + row * 128;
                     uint32_t v[16];
@@ -877,7 +880,7 @@ __global__ void __launch_bounds__(TileTA<GEMM, BNT_, MST_>::THREADS, 1)
                         v[8 * i + 4] = hi.x; v[8 * i + 5] = hi.y; v[8 * i + 6] = hi.z; v[8 * i + 7] = hi.w;
                     }
                     if (h == 1) mbar_arrive(&raw_empty[rstage]);
-                    tmem_st16(lane_cols + C::A_STAGE_COLS * (g & 1), v);
+                    tmem_st16(lane_cols + C::A_STAGE_COLS * (g % C::ASTAGES), v);
                 }
                 tmem_st_wait();
                 tc_fence_before();
