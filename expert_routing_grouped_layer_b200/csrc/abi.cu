@@ -35,13 +35,13 @@ cudaError_t ensure_smem_limit(const void* kernel, int bytes) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     static std::mutex mu;
-    static std::map<std::pair<const void*, int>, cudaError_t> done;
+    static std::map<std::pair<const void*, int>, int> limit;  // largest size set per (kernel, device)
     std::lock_guard<std::mutex> lock(mu);
     const auto key = std::make_pair(kernel, dev);
-    const auto it = done.find(key);
-    if (it != done.end()) return it->second;
+    const auto it = limit.find(key);
+    if (it != limit.end() && it->second >= bytes) return cudaSuccess;
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    done.emplace(key, e);
+    if (e == cudaSuccess) limit[key] = bytes;
     return e;
 }
 

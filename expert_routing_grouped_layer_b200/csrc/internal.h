@@ -40,8 +40,9 @@ struct WsLayout {
 };
 
 bool config_valid(const moe_config* c);
-// Raises a kernel's opt-in dynamic shared-memory limit on the current device,
-// once per (kernel, device) pair; later calls return the first call's result.
+// Raises a kernel's opt-in dynamic shared-memory limit on the current device to
+// at least `bytes`; the size set per (kernel, device) pair is cached, so a call
+// at or below it does nothing. A failed call leaves the cached size as it was.
 cudaError_t ensure_smem_limit(const void* kernel, int bytes);
 // Status of a launch error: MOE_ERR_UNSUPPORTED for an operation the device or
 // driver does not support, MOE_ERR_CUDA for any other failure.
