@@ -590,13 +590,16 @@ cudaError_t launch_nvfp4(const GroupedGemmArgs& a, cudaStream_t st) {
 }
 
 cudaError_t launch_gemm_nvfp4(const GroupedGemmArgs& a, cudaStream_t st) {
-    // experts averaging 64 tokens or more: 128-token tiles, single-buffered
-    // accumulators with two epilogue groups (fewer passes over an expert's
-    // weight tiles when it holds a few hundred tokens); fewer: 96-token tiles,
-    // double-buffered
-    const bool wide = a.N >= 64L * a.E;
-    if (a.gemm == 1) return wide ? launch_nvfp4<1, 128, 1>(a, st) : launch_nvfp4<1, 96, 2>(a, st);
-    return wide ? launch_nvfp4<2, 128, 1>(a, st) : launch_nvfp4<2, 96, 2>(a, st);
+    // 128-token tiles with single-buffered accumulators and two epilogue groups
+    // (fewer passes over an expert's weight tiles), or 96-token tiles with
+    // double-buffered accumulators (the epilogue overlaps the next tile). The
+    // gate/up epilogue (SwiGLU and NVFP4 quantisation) is the heavier one, so
+    // gate/up goes wide only from 128 tokens per expert on average, the down
+    // projection from 64. Measured at ~85 tokens per expert: narrow gate/up
+    // 1.48 -> 1.32 ms; narrow down 0.72 -> 0.77 ms.
+    if (a.gemm == 1)
+        return a.N >= 128L * a.E ? launch_nvfp4<1, 128, 1>(a, st) : launch_nvfp4<1, 96, 2>(a, st);
+    return a.N >= 64L * a.E ? launch_nvfp4<2, 128, 1>(a, st) : launch_nvfp4<2, 96, 2>(a, st);
 }
 
 }  // namespace gemm
