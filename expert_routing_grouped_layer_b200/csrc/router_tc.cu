@@ -320,14 +320,32 @@ static bool make_tmap_planes(CUtensorMap* tm, const void* planes, uint64_t Epad,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// K splits: the count that minimises the estimated time, (waves of units) x
+// (k-blocks per unit) plus the partial-sum slabs' round trip through memory
+// (T x E x 8 bytes per split, costed at ~4 MB per k-block time: measured, two
+// splits of the 16384-token, 896-expert router were 5% slower than one). Units of one split are equally long, so a grid a little above a
+// multiple of the SM count pays a whole extra wave: splitting the 8192-token,
+// 384-expert router into three gives four waves of a third as long instead of
+// two full ones. At least 4 k-blocks per split; a plan depends on (T, E, H) and
+// the SM count only.
 RouterPlan router_plan(int T, int E, int H) {
     RouterPlan r;
     r.Epad = (E + BM - 1) / BM * BM;
     const int KB = H / BK;
-    const int base = (r.Epad / BM) * ((T + RT_BN - 1) / RT_BN);
-    int s = (num_sms() + base - 1) / base;
-    s = std::max(1, std::min(s, KB / 4));  // at least 4 k-blocks per split
-    r.kbps = (KB + s - 1) / s;
+    const long base = (long)(r.Epad / BM) * ((T + RT_BN - 1) / RT_BN);
+    const long sms = num_sms();
+    const double slab_kb = (double)T * E * 8.0 / 4.0e6;  // one split's slab round trip, in k-block times
+    int best = 1;
+    double best_cost = 1e300;
+    for (int s = 1; s <= std::max(1, KB / 4); ++s) {
+        const int kbps = (KB + s - 1) / s;
+        const int splits = (KB + kbps - 1) / kbps;
+        if (splits != s) continue;  // same plan as a smaller count
+        const long waves = (base * s + sms - 1) / sms;
+        const double cost = (double)waves * kbps + (s > 1 ? s * slab_kb : 0.0);
+        if (cost < best_cost - 1e-9) { best_cost = cost; best = s; }
+    }
+    r.kbps = (KB + best - 1) / best;
     r.splits = (KB + r.kbps - 1) / r.kbps;  // no empty split
     return r;
 }
