@@ -41,6 +41,27 @@ L2_FLUSH_BYTES = 256 << 20  # > 2x the 126 MB L2
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+def router_splits(T, E, H, n_sms):
+    """K splits of the router GEMM, as the library plans them: the count that
+    minimises (waves of units) x (k-blocks per unit) plus T*E*8 bytes per split
+    costed at 4 MB per k-block time, at least 4 k-blocks per split."""
+    epad = (E + 127) // 128 * 128
+    kb = H // 64
+    base = (epad // 128) * ((T + 127) // 128)
+    slab = T * E * 8.0 / 4.0e6
+    best, best_cost = 1, float("inf")
+    for s in range(1, max(1, kb // 4) + 1):
+        kbps = (kb + s - 1) // s
+        if (kb + kbps - 1) // kbps != s:
+            continue
+        waves = (base * s + n_sms - 1) // n_sms
+        cost = waves * kbps + (s * slab if s > 1 else 0.0)
+        if cost < best_cost - 1e-9:
+            best, best_cost = s, cost
+    kbps = (kb + best - 1) // best
+    return (kb + kbps - 1) // kbps
+
+
 def launches_per_step(cfg, T, n_sms):
     """Kernels one layer step launches, mirroring the library's launch rules:
     router plane split, router GEMM, its split-K reduction when K is split;
@@ -51,12 +72,7 @@ def launches_per_step(cfg, T, n_sms):
     of h); down; combine."""
     E, H = cfg.n_routed_experts, cfg.hidden
     N = T * cfg.num_experts_per_tok
-    epad = (E + 127) // 128 * 128
-    kb = H // 64
-    base = (epad // 128) * ((T + 127) // 128)
-    s = max(1, min((n_sms + base - 1) // base, kb // 4))
-    kbps = (kb + s - 1) // s
-    splits = (kb + kbps - 1) // kbps
+    splits = router_splits(T, E, H, n_sms)
     router = 2 + (1 if splits > 1 else 0)
     permute = 1 if N <= 4096 else 3
     fp8w = cfg.wfmt == "fp8_e4m3_b128x128" and cfg.afmt == "bf16"

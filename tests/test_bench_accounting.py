@@ -71,12 +71,13 @@ def test_clock_log_path():
     assert bench.clock_log_path("c.csv", 3) == "c.csv"
 
 
-@pytest.mark.parametrize("name,count", [("k2_decode_bf16", 9), ("k2_prefill_fp8w", 12),
+@pytest.mark.parametrize("name,count", [("k2_decode_bf16", 9), ("k2_prefill_fp8w", 13),
                                         ("v4_fp4", 12), ("mx896", 11), ("k2_nvfp4", 14)])
 def test_launch_count_matches_the_launch_lists(name, count):
     """The kernels one step of each workload launches on a 148-SM B200, as the
-    ncu launch lists of the four workloads show them (one-kernel permutation up
-    to 4096 pairs; two-pass packs; the FP8-weight h repack)."""
+    ncu launch lists of the five workloads show them (one-kernel permutation up
+    to 4096 pairs; two-pass packs; the FP8-weight h repack; the router's
+    split-K reduction for the 8192- and 4096-token layers)."""
     cfg = W.CONFIGS[name]
     assert bench.launches_per_step(cfg, cfg.T, 148) == count
 
@@ -118,3 +119,13 @@ def test_both_arms_build_the_config_from_one_function():
     assert "cfgd[" not in src
     d = bench.workload_config(W.CONFIGS["mx896"], 1)
     assert d["T"] == 16384 and d["experts"] == 896 and d["weights"] == "mxfp4"
+
+
+@pytest.mark.parametrize("T,E,H,splits", [(128, 384, 7168, 28), (8192, 384, 7168, 3),
+                                          (4096, 384, 7168, 3), (16384, 896, 7168, 1),
+                                          (64, 16, 256, 1), (700, 8, 512, 2)])
+def test_router_split_plan(T, E, H, splits):
+    """The router's K-split counts on 148 SMs, as measured best: every decode unit
+    its own 4 k-blocks; three splits where one would leave a mostly idle second
+    wave; none for the 896-expert layer (two measured slower)."""
+    assert bench.router_splits(T, E, H, 148) == splits
