@@ -41,14 +41,14 @@ namespace {
 template <bool WIDE_B>
 using BParam = typename std::conditional<WIDE_B, BMaps, CUtensorMap>::type;
 
-template <int GEMM, bool WIDE_B>
+template <int GEMM, bool WIDE_B, int NA>
 __global__ void __launch_bounds__(192, 1)
     grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA_routed,
                              const __grid_constant__ CUtensorMap tmA_shared,
                              const __grid_constant__ BParam<WIDE_B> tmB, const KParams p) {
     pdl_wait();
     pdl_trigger();
-    using C = Tile<GEMM>;
+    using C = Tile<GEMM, NA>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -86,7 +86,7 @@ __global__ void __launch_bounds__(192, 1)
         tmem_relinquish();
     }
     // tile schedule: pref[s] = first unit of segment s
-    const int MT = p.M / BM;
+    const int MT = p.M / p.tile_rows;
     if (warp == 1) build_schedule(p, pref, MT, lane);
     tc_fence_before();
     __syncthreads();
@@ -112,7 +112,7 @@ __global__ void __launch_bounds__(192, 1)
                     uint8_t* st = smem + stage * C::STAGE_BYTES;
                     mbar_arrive_expect_tx(&full[stage], tx);
                     tma_load_2d(st, tmA, kb * BK, t.a_row, &full[stage]);
-                    if (GEMM == 1)
+                    if (C::NA == 2)  // gate/up: the up tile; down: the next 128-row block
                         tma_load_2d(st + C::A_BYTES, tmA, kb * BK, t.a_row + p.a_up_offset, &full[stage]);
                     uint8_t* sb = st + C::NA * C::A_BYTES;
                     if constexpr (WIDE_B) {
@@ -163,7 +163,7 @@ __global__ void __launch_bounds__(192, 1)
                         const uint32_t acc_flag = (kb | kk) != 0;
                         const uint64_t bd = sdesc_kmajor_sw128(sb + kk * 32);
                         mma_bf16(d0, sdesc_kmajor_sw128(st + kk * 32), bd, idesc, acc_flag);
-                        if (GEMM == 1)
+                        if (C::NA == 2)
                             mma_bf16(d0 + BN, sdesc_kmajor_sw128(st + C::A_BYTES + kk * 32), bd, idesc,
                                      acc_flag);
                     }
@@ -181,8 +181,8 @@ __global__ void __launch_bounds__(192, 1)
             if (*abort_flag) status_or(p.status, MOE_DEV_TIMEOUT);
         }
     } else {
-        epilogue_loop<GEMM, C::ACC_COLS>(p, pref, total, tmem_base, tfull, tempty, abort_flag,
-                                         warp, lane);
+        epilogue_loop<GEMM, C::ACC_COLS, 2, (GEMM == 2 ? NA : 1)>(p, pref, total, tmem_base, tfull,
+                                                                  tempty, abort_flag, warp, lane);
     }
 
     tc_fence_before();
@@ -196,15 +196,20 @@ __global__ void __launch_bounds__(192, 1)
 
 }  // namespace
 
-template <int GEMM, bool WIDE_B>
+template <int GEMM, bool WIDE_B, int NA>
 cudaError_t launch_bf16(const GroupedGemmArgs& a, cudaStream_t st) {
-    using C = Tile<GEMM>;
+    using C = Tile<GEMM, NA>;
     const cudaError_t attr_err = ensure_smem_limit(
-        reinterpret_cast<const void*>(grouped_gemm_bf16_kernel<GEMM, WIDE_B>), C::SMEM_BYTES);
+        reinterpret_cast<const void*>(grouped_gemm_bf16_kernel<GEMM, WIDE_B, NA>), C::SMEM_BYTES);
     if (attr_err != cudaSuccess) return attr_err;
 
     uint64_t b_rows;
-    const KParams p = make_params(a, GEMM, &b_rows);
+    KParams p = make_params(a, GEMM, &b_rows);
+    if (GEMM == 2 && NA == 2) {  // two consecutive 128-row blocks of W2 per unit
+        if (p.M % (2 * BM)) return cudaErrorInvalidValue;
+        p.tile_rows = 2 * BM;
+        p.a_up_offset = BM;
+    }
     const int E = a.E, S = a.S;
     CUtensorMap tmAr, tmAs;
     BParam<WIDE_B> tmB;
@@ -223,15 +228,19 @@ cudaError_t launch_bf16(const GroupedGemmArgs& a, cudaStream_t st) {
         if (!make_tmap_bf16(&tmB, a.b_rows, b_rows, p.K, B_BOX)) return cudaErrorInvalidValue;
     }
     const int grid = grid_for(p);
-    launch_pdl(grouped_gemm_bf16_kernel<GEMM, WIDE_B>, grid, 192, C::SMEM_BYTES, st, tmAr, tmAs, tmB, p);
+    launch_pdl(grouped_gemm_bf16_kernel<GEMM, WIDE_B, NA>, grid, 192, C::SMEM_BYTES, st, tmAr, tmAs, tmB, p);
     return cudaGetLastError();
 }
 
 cudaError_t launch_gemm_bf16(const GroupedGemmArgs& a, cudaStream_t st) {
     // wide token boxes for many tokens per expert (at least 64 on average)
     const bool wide = (long)(a.N + (long)a.S * a.T) >= 64L * (a.E + a.S);
-    if (a.gemm == 1) return wide ? launch_bf16<1, true>(a, st) : launch_bf16<1, false>(a, st);
-    return wide ? launch_bf16<2, true>(a, st) : launch_bf16<2, false>(a, st);
+    if (a.gemm == 1) return wide ? launch_bf16<1, true, 2>(a, st) : launch_bf16<1, false, 2>(a, st);
+    // down: two 128-row blocks of W2 per unit (twice the weight bytes per stage and
+    // half the units) when H allows it
+    if (a.H % (2 * BM) == 0)
+        return wide ? launch_bf16<2, true, 2>(a, st) : launch_bf16<2, false, 2>(a, st);
+    return wide ? launch_bf16<2, true, 1>(a, st) : launch_bf16<2, false, 1>(a, st);
 }
 
 }  // namespace gemm

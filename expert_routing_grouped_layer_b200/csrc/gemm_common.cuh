@@ -25,13 +25,15 @@ constexpr int BK = 64;    // bf16 elements in one 128-byte swizzled row
 constexpr int B_BOX = 16; // token rows per TMA box
 constexpr int MAX_SEG = 1024 + 4;
 
-template <int GEMM>
+// NA_: weight tiles per stage sharing the token tile (GEMM1: gate and up;
+// GEMM2: one 128-row block, or two consecutive ones)
+template <int GEMM, int NA_ = (GEMM == 1 ? 2 : 1)>
 struct Tile {
-    static constexpr int NA = (GEMM == 1) ? 2 : 1;  // A tiles per stage (gate + up)
+    static constexpr int NA = NA_;
     static constexpr int A_BYTES = BM * BK * 2;
     static constexpr int B_BYTES = BN * BK * 2;
     static constexpr int STAGE_BYTES = NA * A_BYTES + B_BYTES;
-    static constexpr int STAGES = (GEMM == 1) ? 4 : 6;
+    static constexpr int STAGES = (NA == 2) ? 4 : 6;
     static constexpr int ACC_COLS = NA * BN;        // TMEM columns of one accumulator set
     static constexpr int TMEM_COLS = 2 * ACC_COLS;  // double-buffered
     static constexpr int BAR_BYTES = 8 * (2 * STAGES + 5) + 16;
@@ -140,7 +142,9 @@ __device__ __forceinline__ void build_schedule(const KParams& p, int* pref, int 
 // Epilogue warps (4 of them, one per TMEM lane quadrant): per unit, wait for
 // the accumulator, read it 16 columns at a time (lane = output feature,
 // column = token), apply SwiGLU for GEMM1, store bf16, release the buffer.
-template <int GEMM, int ACC_COLS, int ACCB = 2>
+// GEMM2 units may hold ND consecutive 128-row blocks (accumulators BN columns
+// apart).
+template <int GEMM, int ACC_COLS, int ACCB = 2, int ND = 1>
 __device__ __forceinline__ void epilogue_loop(const KParams& p, const int* pref, int total,
                                               uint32_t tmem_base, uint64_t* tfull,
                                               uint64_t* tempty, volatile int* abort_flag,
@@ -153,8 +157,11 @@ __device__ __forceinline__ void epilogue_loop(const KParams& p, const int* pref,
         const Unit t = decode_unit(p, pref, u);
         if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) break;
         tc_fence_after();
-        const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * ACC_COLS;
-        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(t.out) + t.mt * BM + row;
+        const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + acc * ACC_COLS;
+#pragma unroll 1
+        for (int w = 0; w < (GEMM == 1 ? 1 : ND); ++w) {
+        const uint32_t taddr = tbase + w * BN;
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(t.out) + t.mt * p.tile_rows + w * BM + row;
         for (int c0 = 0; c0 < t.n_valid; c0 += 16) {
             uint32_t g[16];
             tmem_ld16(taddr + c0, g);
@@ -177,6 +184,7 @@ __device__ __forceinline__ void epilogue_loop(const KParams& p, const int* pref,
                     if (c0 + j < t.n_valid)
                         out[(size_t)(c0 + j) * p.ld_out] = __float2bfloat16_rn(__uint_as_float(g[j]));
             }
+        }
         }
         tc_fence_before();
         mbar_arrive(&tempty[acc]);
